@@ -1,0 +1,251 @@
+"""The oracle: a plain float64 CPU implementation of one denoising step of
+block discrete-diffusion decoding.
+
+TEST INFRASTRUCTURE. Only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import it.
+The product library (``block_discrete_diffusion_dd_b200``) never imports,
+links or calls anything here, and this package imports nothing from it.
+
+The arithmetic lives in ``dd_oracle.c`` (plain C, float64, one OpenMP loop
+over independent rows); this module only marshals numpy arrays and runs the
+step loop of a block in plain Python.
+
+Sources: "DiffusionGemma Technical Report" (paperfeed review), sections "The
+mechanism: an AR model turned inside out" and "Training"; Salmon et al.,
+"Parallel random numbers: as easy as 1, 2, 3" (SC'11) for Philox4x32-10.
+
+Parity status per function (what pins it; tests/test_oracle_*.py):
+  philox4x32_10 / words     -- torch's independent CPU Philox engine
+                               (ATen PhiloxRNGEngine), bit-exact; uniformity.
+  canvas_attn               -- float64 torch SDPA, pure-Python brute force,
+                               closed forms, permutation/zero-prefix/GQA
+                               invariants.
+  sample_renoise            -- chi-square of Gumbel-max vs softmax, scipy
+                               log-softmax/entropy, spike and constant-logit
+                               closed forms, binomial re-noise rate,
+                               chi-square uniformity of replacements.
+  init_canvas               -- chi-square uniformity; shares the replacement
+                               rule pinned above.
+  denoise_block             -- a loop of the two pinned functions (plain
+                               Python), checked for step0-restart identity.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "dd_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+BF16 = 0
+F32 = 1
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile dd_oracle.c with gcc (float64, no FMA contraction, OpenMP)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fopenmp",
+               "-fPIC", "-shared", "-o", _LIB + ".tmp", _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(_LIB + ".tmp", _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    build()
+    lib = ctypes.CDLL(_LIB)
+    P = ctypes.c_void_p
+    i32, i64, u32, u64, f64, f32 = (ctypes.c_int, ctypes.c_int64, ctypes.c_uint32,
+                                    ctypes.c_uint64, ctypes.c_double, ctypes.c_float)
+    lib.oracle_word.restype = u32
+    lib.oracle_word.argtypes = [u64, u32, u32, u32, u32]
+    lib.oracle_uniform.restype = f64
+    lib.oracle_uniform.argtypes = [u32]
+    lib.oracle_words.restype = None
+    lib.oracle_words.argtypes = [u64, u32, u32, P, P, i64, P]
+    lib.oracle_philox_blocks.restype = None
+    lib.oracle_philox_blocks.argtypes = [P, P, i64, P]
+    lib.oracle_canvas_attn.restype = i32
+    lib.oracle_canvas_attn.argtypes = [i32, i32, i32, i32, i32, f64, i32, P, P, P, P, P, P, P, i32,
+                                       P, P, i32]
+    lib.oracle_sample_renoise.restype = i32
+    lib.oracle_sample_renoise.argtypes = [P, i32, i64, i64, i64, P, i64, f64, f32, u64, u32, u32,
+                                          P, P, P, P, P, P, P, i32]
+    lib.oracle_init_canvas.restype = None
+    lib.oracle_init_canvas.argtypes = [P, i64, i64, u64, u32]
+    _lib = lib
+    return lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _raw(x):
+    """(numpy array, dtype code) from a torch tensor or numpy array.
+
+    bf16 tensors are passed as their raw 16-bit patterns; the C side upcasts
+    them exactly.  Anything else must already be float32.
+    """
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            x = x.detach().cpu().contiguous()
+            if x.dtype == torch.bfloat16:
+                return np.ascontiguousarray(x.view(torch.int16).numpy().view(np.uint16)), BF16
+            if x.dtype == torch.float32:
+                return np.ascontiguousarray(x.numpy()), F32
+            raise TypeError(f"oracle: unsupported tensor dtype {x.dtype}")
+    except ImportError:  # pragma: no cover - torch is always present here
+        pass
+    x = np.asarray(x)
+    if x.dtype == np.uint16:
+        return np.ascontiguousarray(x), BF16
+    if x.dtype == np.float32:
+        return np.ascontiguousarray(x), F32
+    raise TypeError(f"oracle: unsupported array dtype {x.dtype}")
+
+
+# ---------------------------------------------------------------- Philox
+
+def philox4x32_10(ctrs, keys):
+    """Philox4x32-10 blocks: ctrs [n,4] uint32, keys [n,2] uint32 -> [n,4]."""
+    lib = _load()
+    c = np.ascontiguousarray(ctrs, dtype=np.uint32).reshape(-1, 4)
+    k = np.ascontiguousarray(keys, dtype=np.uint32).reshape(-1, 2)
+    assert c.shape[0] == k.shape[0]
+    out = np.empty_like(c)
+    lib.oracle_philox_blocks(_ptr(c), _ptr(k), c.shape[0], _ptr(out))
+    return out
+
+
+def words(seed: int, stream: int, step: int, rows, vs):
+    """32-bit words for counter (v >> 2, row, step, stream), word v & 3."""
+    lib = _load()
+    r = np.ascontiguousarray(rows, dtype=np.uint32).ravel()
+    v = np.ascontiguousarray(vs, dtype=np.uint32).ravel()
+    assert r.shape == v.shape
+    out = np.empty_like(r)
+    lib.oracle_words(seed, stream, step, _ptr(r), _ptr(v), r.size, _ptr(out))
+    return out
+
+
+def uniform(x: int) -> float:
+    return _load().oracle_uniform(int(x))
+
+
+# ------------------------------------------------------- canvas attention
+
+def canvas_attn(q, kc, vc, kp, vp, cu_prefix, scale=None, positions=None, threads=0):
+    """float64 attention over [prefix_b || canvas_b] for every (b, i, h).
+
+    Shapes: q [B,C,Hq,D]; kc, vc [B,C,Hkv,D]; kp, vp [sum L_b, Hkv, D];
+    cu_prefix [B+1] int.  positions: optional list of canvas positions to
+    compute (others are NaN).  Returns (out [B,C,Hq,D], lse [B,Hq,C]).
+    """
+    lib = _load()
+    qa, dt = _raw(q)
+    kca, dt2 = _raw(kc)
+    vca, dt3 = _raw(vc)
+    kpa, dt4 = _raw(kp)
+    vpa, dt5 = _raw(vp)
+    if len({dt, dt2, dt3, dt4, dt5}) != 1:
+        raise TypeError("oracle: mixed input dtypes")
+    B, C, Hq, D = qa.shape
+    Hkv = kca.shape[2]
+    cu = np.ascontiguousarray(np.asarray(cu_prefix, dtype=np.int32))
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    out = np.full((B, C, Hq, D), np.nan, dtype=np.float64)
+    lse = np.full((B, Hq, C), np.nan, dtype=np.float64)
+    if positions is None:
+        pos, npos = None, -1
+    else:
+        pos = np.ascontiguousarray(np.asarray(positions, dtype=np.int32))
+        npos = pos.size
+    rc = lib.oracle_canvas_attn(B, C, Hq, Hkv, D, float(scale), dt, _ptr(qa), _ptr(kca),
+                                _ptr(vca), _ptr(kpa), _ptr(vpa), _ptr(cu), _ptr(pos), npos,
+                                _ptr(out), _ptr(lse), int(threads))
+    if rc != 0:
+        raise ValueError("oracle_canvas_attn: bad arguments")
+    return out, lse
+
+
+# ------------------------------------------------------------------ sampler
+
+def sample_renoise(logits, tau, rate, seed, step, row_offset=0, rows=None, row_stride=None,
+                   vocab=None, n_rows=None, threads=0):
+    """One sampler step (Gumbel-max, confidence, entropy, re-noise).
+
+    logits: [R, V] (bf16 or f32).  rows: optional local row indices to compute.
+    row_stride/vocab/n_rows override the shape (row_stride 0 broadcasts one
+    row to n_rows rows).  Returns a dict of numpy arrays indexed like `rows`.
+    """
+    lib = _load()
+    la, dt = _raw(logits)
+    if vocab is None:
+        vocab = la.shape[-1]
+    if row_stride is None:
+        row_stride = la.shape[-1]
+    if n_rows is None:
+        n_rows = la.size // la.shape[-1]
+    if rows is None:
+        sel, nsel = None, -1
+        n = n_rows
+    else:
+        sel = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+        nsel = sel.size
+        n = nsel
+    res = {
+        "tokens": np.empty(n, np.int32), "pred": np.empty(n, np.int32),
+        "conf": np.empty(n, np.float64), "entropy": np.empty(n, np.float64),
+        "renoised": np.empty(n, np.uint8), "gap": np.empty(n, np.float64),
+        "best": np.empty(n, np.float64),
+    }
+    rc = lib.oracle_sample_renoise(
+        _ptr(la), dt, int(n_rows), int(vocab), int(row_stride), _ptr(sel), int(nsel), float(tau),
+        float(np.float32(rate)), int(seed), int(step), int(row_offset), _ptr(res["tokens"]),
+        _ptr(res["pred"]), _ptr(res["conf"]), _ptr(res["entropy"]), _ptr(res["renoised"]),
+        _ptr(res["gap"]), _ptr(res["best"]), int(threads))
+    if rc != 0:
+        raise ValueError("oracle_sample_renoise: bad arguments")
+    return res
+
+
+def init_canvas(rows: int, vocab: int, seed: int, row_offset: int = 0):
+    lib = _load()
+    out = np.empty(rows, np.int32)
+    lib.oracle_init_canvas(_ptr(out), rows, vocab, seed, row_offset)
+    return out
+
+
+# --------------------------------------------------------- the block loop
+
+def denoise_block(steps, q_steps, kc_steps, vc_steps, kp, vp, cu_prefix, logits_steps, rates,
+                  temperatures, seed, step0=0, scale=None, positions=None, sample_rows=None,
+                  threads=0):
+    """The step loop of one block: for s in 0..S-1, attention of step s and
+    the sampler of step s (Philox step = step0 + s).  The sampler does not
+    read the previous canvas: each step's canvas is its pred-or-replacement.
+
+    Returns (attn_out list, lse list, per-step sampler dicts).
+    """
+    outs, lses, samp = [], [], []
+    for s in range(steps):
+        if q_steps is not None:
+            o, l = canvas_attn(q_steps[s], kc_steps[s], vc_steps[s], kp, vp, cu_prefix, scale,
+                               positions, threads)
+            outs.append(o)
+            lses.append(l)
+        samp.append(sample_renoise(logits_steps[s], temperatures[s], rates[s], seed, step0 + s,
+                                   0, sample_rows, threads=threads))
+    return outs, lses, samp

@@ -1,0 +1,171 @@
+"""Seeded synthetic inputs for the denoise-step workloads.
+
+This module holds shapes, distributions and seeds only: none of the method's
+arithmetic.  Both sides of every parity check (the CUDA library and the
+float64 oracle) consume the tensors it makes, so it imports neither.
+
+The five workloads mirror the shapes the method runs at ("DiffusionGemma
+Technical Report", paperfeed review: 256-token canvas; 262,144-entry vocabulary
+in "The numbers, honestly"; ~12 passes per block in "The mechanism"):
+
+  tiny_fp32      B=1, Hq=2, Hkv=1, D=64, prefix 128, canvas 256, fp32, scale
+                 1/8; sampler 256 x 1024 fp32 logits ~ N(0, 2^2), tau 1,
+                 rate 0.5.
+  b1_L4096       B=1, Hq=16, Hkv=8, D=128, prefix 4096, bf16; logits
+                 256 x 262144 ~ N(0, 3^2) + 8 at one uniform index per row,
+                 rate 0.3.
+  long_L65536    as b1_L4096 with prefix 65536, rate 0.1.
+  ragged_b8      B=8, prefix lengths numpy default_rng(0).integers(512, 16385,
+                 8), logits 2048 x 262144, rate 0.2.
+  block12_L8192  B=1, prefix 8192, 12 steps, fresh canvas Q/K/V and logits
+                 per step keyed on (seed, step), rate_s = 0.9 (11 - s) / 11,
+                 tau 1.
+
+Every tensor is drawn in float32 from a torch.Generator seeded with a hash
+of (seed, workload, tensor name, step), then rounded to bf16 (round to
+nearest even) where the workload is bf16.  The generator's device is the
+caller's choice; the same device always gives the same bits.
+"""
+from __future__ import annotations
+
+import dataclasses
+import hashlib
+from typing import List, Optional
+
+import numpy as np
+import torch
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    name: str
+    batch: int
+    canvas: int
+    heads_q: int
+    heads_kv: int
+    head_dim: int
+    prefix_lens: tuple
+    dtype: str            # "f32" or "bf16"
+    vocab: int
+    logit_std: float
+    spike: float           # added at one uniform index per row (0: none)
+    rates: tuple           # one per step
+    temperatures: tuple    # one per step
+    steps: int = 1
+    seed: int = 0
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / float(np.sqrt(self.head_dim))
+
+    @property
+    def rows(self) -> int:
+        return self.batch * self.canvas
+
+    @property
+    def torch_dtype(self):
+        return torch.float32 if self.dtype == "f32" else torch.bfloat16
+
+    @property
+    def cu_prefix(self) -> np.ndarray:
+        return np.concatenate([[0], np.cumsum(self.prefix_lens)]).astype(np.int32)
+
+    def attn_flops(self) -> int:
+        """Algorithmic attention FLOPs of one step: 4 Hq C (L_b + C) D per row b."""
+        return sum(4 * self.heads_q * self.canvas * (L + self.canvas) * self.head_dim
+                   for L in self.prefix_lens)
+
+    def logit_bytes(self) -> int:
+        return self.rows * self.vocab * (4 if self.dtype == "f32" else 2)
+
+
+def _ragged_lens():
+    return tuple(int(x) for x in np.random.default_rng(0).integers(512, 16385, 8))
+
+
+WORKLOADS = {
+    "tiny_fp32": Workload("tiny_fp32", 1, 256, 2, 1, 64, (128,), "f32", 1024, 2.0, 0.0,
+                          (0.5,), (1.0,)),
+    "b1_L4096": Workload("b1_L4096", 1, 256, 16, 8, 128, (4096,), "bf16", 262144, 3.0, 8.0,
+                         (0.3,), (1.0,)),
+    "long_L65536": Workload("long_L65536", 1, 256, 16, 8, 128, (65536,), "bf16", 262144, 3.0,
+                            8.0, (0.1,), (1.0,)),
+    "ragged_b8": Workload("ragged_b8", 8, 256, 16, 8, 128, _ragged_lens(), "bf16", 262144, 3.0,
+                          8.0, (0.2,), (1.0,)),
+    "block12_L8192": Workload("block12_L8192", 1, 256, 16, 8, 128, (8192,), "bf16", 262144, 3.0,
+                              8.0, tuple(float(np.float32(0.9 * (11 - s) / 11)) for s in range(12)),
+                              (1.0,) * 12, steps=12),
+}
+
+
+def scaled(w: Workload, **changes) -> Workload:
+    """A copy of a workload with some fields replaced (smaller parity cases)."""
+    return dataclasses.replace(w, **changes)
+
+
+def _seed_for(w: Workload, tensor: str, step: int) -> int:
+    h = hashlib.sha256(f"{w.seed}/{w.name}/{tensor}/{step}".encode()).hexdigest()
+    return int(h[:15], 16)
+
+
+def _gen(w: Workload, tensor: str, step: int, device) -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed(_seed_for(w, tensor, step))
+    return g
+
+
+def _normal(w, tensor, step, shape, std, device):
+    g = _gen(w, tensor, step, device)
+    x = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+    if std != 1.0:
+        x.mul_(std)
+    return x.to(w.torch_dtype)
+
+
+def canvas_qkv(w: Workload, step: int = 0, device="cpu", q_gain: float = 1.0):
+    """Q [B,C,Hq,D], Kc, Vc [B,C,Hkv,D] for one step, i.i.d. N(0,1).
+
+    q_gain > 1 scales Q before rounding (a sharper softmax that exercises the
+    running-max rescale path)."""
+    B, C, Hq, Hkv, D = w.batch, w.canvas, w.heads_q, w.heads_kv, w.head_dim
+    q = _normal(w, "q", step, (B, C, Hq, D), q_gain, device)
+    kc = _normal(w, "kc", step, (B, C, Hkv, D), 1.0, device)
+    vc = _normal(w, "vc", step, (B, C, Hkv, D), 1.0, device)
+    return q, kc, vc
+
+
+def prefix_kv(w: Workload, device="cpu"):
+    """Packed prefix cache Kp, Vp [sum L_b, Hkv, D] and cu_prefix [B+1]."""
+    n = int(sum(w.prefix_lens))
+    kp = _normal(w, "kp", 0, (n, w.heads_kv, w.head_dim), 1.0, device)
+    vp = _normal(w, "vp", 0, (n, w.heads_kv, w.head_dim), 1.0, device)
+    return kp, vp, torch.from_numpy(w.cu_prefix)
+
+
+def logits(w: Workload, step: int = 0, device="cpu", rows: Optional[int] = None):
+    """Logits [R, V]: N(0, std^2) plus `spike` at one uniform index per row."""
+    R = w.rows if rows is None else rows
+    g = _gen(w, "logits", step, device)
+    x = torch.randn((R, w.vocab), generator=g, device=device, dtype=torch.float32)
+    x.mul_(w.logit_std)
+    if w.spike:
+        gi = _gen(w, "spike", step, device)
+        idx = torch.randint(0, w.vocab, (R,), generator=gi, device=device)
+        x[torch.arange(R, device=device), idx] += w.spike
+    return x.to(w.torch_dtype)
+
+
+def all_steps(w: Workload, device="cpu"):
+    """Per-step canvas Q/K/V and logits for every step of the workload."""
+    qs, kcs, vcs, ls = [], [], [], []
+    for s in range(w.steps):
+        q, kc, vc = canvas_qkv(w, s, device)
+        qs.append(q)
+        kcs.append(kc)
+        vcs.append(vc)
+        ls.append(logits(w, s, device))
+    return torch.stack(qs), torch.stack(kcs), torch.stack(vcs), torch.stack(ls)
+
+
+def names() -> List[str]:
+    return list(WORKLOADS)
