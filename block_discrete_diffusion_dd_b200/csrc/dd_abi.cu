@@ -1,0 +1,364 @@
+// dd_abi.cu -- the extern "C" boundary of libdd (declared in include/dd.h):
+// argument validation (always before any launch), launch planning, workspace
+// carving, error reporting and the block loop.  All device work happens in
+// the kernels of dd_sampler.cu, dd_attn_tc.cu and dd_attn_simt.cu.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "dd.h"
+#include "dd_internal.h"
+
+namespace dd {
+
+namespace {
+thread_local std::string g_last_error;
+thread_local uint64_t g_launches = 0;
+
+constexpr size_t kHeaderBytes = 256;  // device error word + padding
+
+dd_status fail(dd_status st, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+dd_status fail(dd_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+dd_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(DD_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t elem_size(dd_dtype t) { return t == DD_BF16 ? 2 : 4; }
+
+// Validates the geometry and the host prefix offsets; fills total prefix.
+dd_status check_attn_desc(const dd_attn_desc* d, const int32_t* cu_host, int64_t* total) {
+  if (!d) return fail(DD_ERR_INVALID_ARG, "desc is NULL");
+  if (d->batch < 0 || d->canvas < 1 || d->heads_q < 1 || d->heads_kv < 1)
+    return fail(DD_ERR_INVALID_ARG, "bad geometry B=%d C=%d Hq=%d Hkv=%d", d->batch, d->canvas,
+                d->heads_q, d->heads_kv);
+  if (d->heads_q % d->heads_kv != 0)
+    return fail(DD_ERR_INVALID_ARG, "heads_q (%d) is not a multiple of heads_kv (%d)",
+                d->heads_q, d->heads_kv);
+  if (d->dtype != DD_BF16 && d->dtype != DD_F32)
+    return fail(DD_ERR_INVALID_ARG, "unknown dtype %d", (int)d->dtype);
+  if (d->head_dim != 64 && d->head_dim != 128)
+    return fail(DD_ERR_UNSUPPORTED, "head_dim %d (supported: 64, 128)", d->head_dim);
+  if (!std::isfinite(d->scale) || d->scale <= 0.f)
+    return fail(DD_ERR_INVALID_ARG, "scale must be finite and > 0");
+  if (d->batch > 0 && !cu_host) return fail(DD_ERR_INVALID_ARG, "cu_prefix_host is NULL");
+  if ((int64_t)d->batch * d->canvas > INT32_MAX)
+    return fail(DD_ERR_UNSUPPORTED, "batch * canvas exceeds 2^31");
+  int64_t tot = 0;
+  if (d->batch > 0) {
+    if (cu_host[0] != 0) return fail(DD_ERR_INVALID_ARG, "cu_prefix[0] must be 0");
+    for (int b = 0; b < d->batch; ++b)
+      if (cu_host[b + 1] < cu_host[b])
+        return fail(DD_ERR_INVALID_ARG, "cu_prefix decreases at %d", b);
+    tot = cu_host[d->batch];
+  }
+  *total = tot;
+  return DD_OK;
+}
+
+AttnArgs make_attn_args(const dd_attn_desc* d, int64_t total, const int32_t* cu_host) {
+  AttnArgs a{};
+  a.cu_prefix_host = cu_host;
+  a.B = d->batch;
+  a.C = d->canvas;
+  a.Hq = d->heads_q;
+  a.Hkv = d->heads_kv;
+  a.D = d->head_dim;
+  a.scale = d->scale;
+  a.bf16 = d->dtype == DD_BF16;
+  a.total_prefix = total;
+  return a;
+}
+
+size_t attn_ws_bytes(const AttnArgs& a) {
+  // pointers are unknown at query time: plan for the tensor-core path when
+  // the geometry allows it (its scratch is the larger of the two)
+  AttnArgs t = a;
+  const void* fake = reinterpret_cast<const void*>(static_cast<uintptr_t>(256));
+  t.q = t.kc = t.vc = t.kp = t.vp = fake;
+  if (a.B > 0 && attn_tc_supported(t)) return kHeaderBytes + attn_tc_scratch_bytes(t);
+  return kHeaderBytes + attn_simt_scratch_bytes(t);
+}
+
+size_t sample_ws_bytes(int rows, int vocab) {
+  return kHeaderBytes + (size_t)rows * (size_t)sampler_nchunk(vocab) * sizeof(ChunkRecord);
+}
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// Block-loop workspace: the attention and sampler scratch share one region
+// (they run one after the other on the stream), followed by a confidence
+// buffer used when the caller passes no conf_steps.
+size_t block_ws_layout(const dd_attn_desc* desc, int64_t total, const int32_t* cu_prefix_host,
+                       int vocab, size_t* conf_off) {
+  const size_t a = attn_ws_bytes(make_attn_args(desc, total, cu_prefix_host));
+  const size_t s = sample_ws_bytes(desc->batch * desc->canvas, vocab);
+  const size_t shared = align256(a > s ? a : s);
+  if (conf_off) *conf_off = shared;
+  return shared + align256((size_t)desc->batch * desc->canvas * sizeof(float));
+}
+
+dd_status run_attn(const dd_attn_desc* d, const void* q, const void* kc, const void* vc,
+                   const void* kp, const void* vp, const int32_t* cu, const int32_t* cu_host,
+                   void* out, float* lse, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  int64_t total = 0;
+  dd_status st = check_attn_desc(d, cu_host, &total);
+  if (st != DD_OK) return st;
+  if (d->batch == 0) return DD_OK;
+  if (!q || !kc || !vc || !out || !cu) return fail(DD_ERR_INVALID_ARG, "NULL tensor pointer");
+  if (total > 0 && (!kp || !vp)) return fail(DD_ERR_INVALID_ARG, "NULL prefix pointer");
+  if (!aligned16(q) || !aligned16(kc) || !aligned16(vc) || !aligned16(out) ||
+      (total > 0 && (!aligned16(kp) || !aligned16(vp))))
+    return fail(DD_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u))
+    return fail(DD_ERR_WORKSPACE, "workspace must be non-NULL and 256-byte aligned");
+  AttnArgs a = make_attn_args(d, total, cu_host);
+  a.q = q;
+  a.kc = kc;
+  a.vc = vc;
+  a.kp = total > 0 ? kp : kc;
+  a.vp = total > 0 ? vp : vc;
+  a.cu_prefix = cu;
+  a.cu_prefix_host = cu_host;
+  a.out = out;
+  a.lse = lse;
+  a.err = static_cast<uint32_t*>(ws);
+  a.scratch = static_cast<uint8_t*>(ws) + kHeaderBytes;
+  const bool tc = attn_tc_supported(a);
+  const size_t need = kHeaderBytes + (tc ? attn_tc_scratch_bytes(a) : attn_simt_scratch_bytes(a));
+  if (ws_bytes < need)
+    return fail(DD_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", ws_bytes, need);
+  a.scratch_bytes = ws_bytes - kHeaderBytes;
+  cudaError_t e = tc ? launch_attn_tc(a, stream) : launch_attn_simt(a, stream);
+  if (e != cudaSuccess) return cuda_fail(e, tc ? "canvas attention (tcgen05)" : "canvas attention");
+  return DD_OK;
+}
+
+dd_status run_sampler(const void* logits, dd_dtype dtype, int rows, int vocab, int64_t row_stride,
+                      const dd_sample_params* p, int32_t* tokens, int32_t* pred, float* conf,
+                      float* entropy, uint8_t* renoised, void* ws, size_t ws_bytes,
+                      cudaStream_t stream) {
+  if (!p) return fail(DD_ERR_INVALID_ARG, "params is NULL");
+  if (dtype != DD_BF16 && dtype != DD_F32)
+    return fail(DD_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+  if (rows < 0 || vocab < 1) return fail(DD_ERR_INVALID_ARG, "rows=%d vocab=%d", rows, vocab);
+  if (row_stride < vocab)
+    return fail(DD_ERR_INVALID_ARG, "row_stride (%lld) < vocab (%d)", (long long)row_stride,
+                vocab);
+  if (!std::isfinite(p->temperature) || p->temperature <= 0.f)
+    return fail(DD_ERR_INVALID_ARG, "temperature must be finite and > 0");
+  if (!(p->renoise_rate >= 0.f && p->renoise_rate <= 1.f))
+    return fail(DD_ERR_INVALID_ARG, "renoise_rate must lie in [0, 1]");
+  if ((uint64_t)rows + p->row_offset > (1ull << 32))
+    return fail(DD_ERR_INVALID_ARG, "row_offset + rows exceeds 2^32");
+  if (rows == 0) return DD_OK;
+  if (!logits || !tokens || !conf) return fail(DD_ERR_INVALID_ARG, "NULL required pointer");
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u))
+    return fail(DD_ERR_WORKSPACE, "workspace must be non-NULL and 256-byte aligned");
+  const size_t need = sample_ws_bytes(rows, vocab);
+  if (ws_bytes < need)
+    return fail(DD_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", ws_bytes, need);
+  if ((int64_t)rows * sampler_nchunk(vocab) > INT32_MAX)
+    return fail(DD_ERR_UNSUPPORTED, "rows * chunks exceeds 2^31");
+  SamplerArgs a{};
+  a.logits = logits;
+  a.bf16 = dtype == DD_BF16;
+  a.rows = rows;
+  a.vocab = vocab;
+  a.row_stride = row_stride;
+  a.inv_tau = 1.0f / p->temperature;
+  a.rate = p->renoise_rate;
+  a.seed = p->seed;
+  a.step = p->step;
+  a.row_offset = p->row_offset;
+  a.tokens = tokens;
+  a.pred = pred;
+  a.conf = conf;
+  a.entropy = entropy;
+  a.renoised = renoised;
+  a.recs = reinterpret_cast<ChunkRecord*>(static_cast<uint8_t*>(ws) + kHeaderBytes);
+  cudaError_t e = launch_sampler(a, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "sampler");
+  return DD_OK;
+}
+
+}  // namespace
+
+void note_launch() { ++g_launches; }
+
+}  // namespace dd
+
+using namespace dd;
+
+extern "C" {
+
+size_t dd_canvas_attn_workspace(const dd_attn_desc* desc, const int32_t* cu_prefix_host) {
+  int64_t total = 0;
+  if (check_attn_desc(desc, cu_prefix_host, &total) != DD_OK) return 0;
+  return attn_ws_bytes(make_attn_args(desc, total, cu_prefix_host));
+}
+
+dd_status dd_canvas_attn(const dd_attn_desc* desc, const void* q, const void* k_canvas,
+                         const void* v_canvas, const void* k_prefix, const void* v_prefix,
+                         const int32_t* cu_prefix, const int32_t* cu_prefix_host, void* out,
+                         float* lse, void* workspace, size_t workspace_bytes, dd_stream_t stream) {
+  g_last_error.clear();
+  return run_attn(desc, q, k_canvas, v_canvas, k_prefix, v_prefix, cu_prefix, cu_prefix_host, out,
+                  lse, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t dd_sample_renoise_workspace(int rows, int vocab, dd_dtype dtype) {
+  if (rows < 0 || vocab < 1 || (dtype != DD_BF16 && dtype != DD_F32)) return 0;
+  return sample_ws_bytes(rows, vocab);
+}
+
+dd_status dd_sample_renoise(const void* logits, dd_dtype dtype, int rows, int vocab,
+                            int64_t row_stride, const dd_sample_params* params,
+                            int32_t* tokens_out, int32_t* pred_out, float* conf_out,
+                            float* entropy_out, uint8_t* renoised_out, void* workspace,
+                            size_t workspace_bytes, dd_stream_t stream) {
+  g_last_error.clear();
+  return run_sampler(logits, dtype, rows, vocab, row_stride, params, tokens_out, pred_out,
+                     conf_out, entropy_out, renoised_out, workspace, workspace_bytes,
+                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+dd_status dd_init_canvas(int32_t* canvas, int rows, int vocab, uint64_t seed, uint32_t row_offset,
+                         dd_stream_t stream) {
+  g_last_error.clear();
+  if (rows < 0 || vocab < 1) return fail(DD_ERR_INVALID_ARG, "rows=%d vocab=%d", rows, vocab);
+  if ((uint64_t)rows + row_offset > (1ull << 32))
+    return fail(DD_ERR_INVALID_ARG, "row_offset + rows exceeds 2^32");
+  if (rows == 0) return DD_OK;
+  if (!canvas) return fail(DD_ERR_INVALID_ARG, "canvas is NULL");
+  cudaError_t e = launch_init_canvas(canvas, rows, vocab, seed, row_offset,
+                                     reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "init canvas");
+  return DD_OK;
+}
+
+size_t dd_denoise_block_workspace(const dd_attn_desc* desc, const int32_t* cu_prefix_host,
+                                  int vocab) {
+  int64_t total = 0;
+  if (vocab < 1 || check_attn_desc(desc, cu_prefix_host, &total) != DD_OK) return 0;
+  return block_ws_layout(desc, total, cu_prefix_host, vocab, nullptr);
+}
+
+dd_status dd_denoise_block(const dd_attn_desc* desc, int steps, const void* q_steps,
+                           const void* kc_steps, const void* vc_steps, const void* k_prefix,
+                           const void* v_prefix, const int32_t* cu_prefix,
+                           const int32_t* cu_prefix_host, void* attn_out,
+                           const void* logits_steps, int vocab, const float* rate_host,
+                           const float* temperature_host, uint64_t seed, uint32_t step0,
+                           int32_t* canvas, int32_t* canvas_history, float* conf_steps,
+                           void* workspace, size_t workspace_bytes, dd_stream_t stream) {
+  g_last_error.clear();
+  int64_t total = 0;
+  dd_status st = check_attn_desc(desc, cu_prefix_host, &total);
+  if (st != DD_OK) return st;
+  if (steps < 0) return fail(DD_ERR_INVALID_ARG, "steps < 0");
+  if (steps > 0 && (!rate_host || !temperature_host))
+    return fail(DD_ERR_INVALID_ARG, "rate_host / temperature_host is NULL");
+  if (!canvas) return fail(DD_ERR_INVALID_ARG, "canvas is NULL");
+  if ((uint64_t)step0 + (uint64_t)steps > (1ull << 32))
+    return fail(DD_ERR_INVALID_ARG, "step0 + steps exceeds 2^32");
+  const int B = desc->batch, C = desc->canvas, Hq = desc->heads_q, Hkv = desc->heads_kv;
+  const int D = desc->head_dim;
+  const int rows = B * C;
+  const size_t es = elem_size(desc->dtype);
+  const size_t q_step = (size_t)rows * Hq * D * es;
+  const size_t kv_step = (size_t)rows * Hkv * D * es;
+  const size_t lg_step = (size_t)rows * (size_t)vocab * es;
+  if (vocab < 1) return fail(DD_ERR_INVALID_ARG, "vocab=%d", vocab);
+  size_t conf_off = 0;
+  const size_t need = block_ws_layout(desc, total, cu_prefix_host, vocab, &conf_off);
+  if (!workspace) return fail(DD_ERR_WORKSPACE, "workspace is NULL");
+  if (workspace_bytes < need)
+    return fail(DD_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", workspace_bytes, need);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  for (int i = 0; i < steps; ++i) {
+    st = run_attn(desc, static_cast<const uint8_t*>(q_steps) + i * q_step,
+                  static_cast<const uint8_t*>(kc_steps) + i * kv_step,
+                  static_cast<const uint8_t*>(vc_steps) + i * kv_step, k_prefix, v_prefix,
+                  cu_prefix, cu_prefix_host, static_cast<uint8_t*>(attn_out) + i * q_step,
+                  nullptr, workspace, workspace_bytes, s);
+    if (st != DD_OK) return st;
+    dd_sample_params sp;
+    sp.temperature = temperature_host[i];
+    sp.renoise_rate = rate_host[i];
+    sp.seed = seed;
+    sp.step = step0 + (uint32_t)i;
+    sp.row_offset = 0;
+    int32_t* tok = canvas_history ? canvas_history + (size_t)i * rows : canvas;
+    float* conf = conf_steps ? conf_steps + (size_t)i * rows
+                             : reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + conf_off);
+    st = run_sampler(static_cast<const uint8_t*>(logits_steps) + i * lg_step, desc->dtype, rows,
+                     vocab, vocab, &sp, tok, nullptr, conf, nullptr, nullptr, workspace,
+                     conf_off, s);
+    if (st != DD_OK) return st;
+    if (canvas_history && i == steps - 1) {
+      cudaError_t e = cudaMemcpyAsync(canvas, tok, (size_t)rows * sizeof(int32_t),
+                                      cudaMemcpyDeviceToDevice, s);
+      if (e != cudaSuccess) return cuda_fail(e, "canvas copy");
+    }
+  }
+  return DD_OK;
+}
+
+dd_status dd_workspace_init(void* workspace, size_t workspace_bytes, dd_stream_t stream) {
+  g_last_error.clear();
+  if (!workspace || workspace_bytes < kHeaderBytes)
+    return fail(DD_ERR_WORKSPACE, "workspace must hold at least %zu bytes", kHeaderBytes);
+  cudaError_t e =
+      cudaMemsetAsync(workspace, 0, kHeaderBytes, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "workspace init");
+  return DD_OK;
+}
+
+dd_status dd_query_device_error(void* workspace, dd_stream_t stream) {
+  g_last_error.clear();
+  if (!workspace) return fail(DD_ERR_INVALID_ARG, "workspace is NULL");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint32_t word = 0;
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e == cudaSuccess) e = cudaMemcpy(&word, workspace, sizeof word, cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemset(workspace, 0, sizeof word);
+  if (e != cudaSuccess) return cuda_fail(e, "query device error");
+  if (word & kDevErrTimeout)
+    return fail(DD_ERR_DEVICE_TIMEOUT, "a kernel pipeline wait exceeded its time limit");
+  if (word & kDevErrBounds)
+    return fail(DD_ERR_DEVICE_BOUNDS, "device-side index check failed (inconsistent cu_prefix?)");
+  return DD_OK;
+}
+
+const char* dd_status_string(dd_status s) {
+  switch (s) {
+    case DD_OK: return "ok";
+    case DD_ERR_INVALID_ARG: return "invalid argument";
+    case DD_ERR_UNSUPPORTED: return "unsupported configuration";
+    case DD_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case DD_ERR_CUDA: return "CUDA error";
+    case DD_ERR_DEVICE_TIMEOUT: return "device pipeline wait timed out";
+    case DD_ERR_DEVICE_BOUNDS: return "device index check failed";
+  }
+  return "unknown status";
+}
+
+const char* dd_last_error(void) { return g_last_error.c_str(); }
+
+uint64_t dd_launch_count(void) { return g_launches; }
+void dd_reset_launch_count(void) { g_launches = 0; }
+
+}  // extern "C"

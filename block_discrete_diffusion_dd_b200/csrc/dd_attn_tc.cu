@@ -1,0 +1,603 @@
+// dd_attn_tc.cu -- canvas attention on the 5th-generation tensor cores
+// (tcgen05.mma, accumulators in tensor memory, operands staged by TMA).
+//
+// Definition ("DiffusionGemma Technical Report", paperfeed review, "The
+// mechanism"): canvas queries attend bidirectionally to the canvas and to
+// the causally encoded cache.  For batch row b and kv head g, the
+// Hq/Hkv query heads that share g are packed with the canvas positions into
+// M = C * (Hq/Hkv) query rows (row r = position * group + head-in-group);
+// they all see the same key range [prefix_b || canvas_b] under one unmasked
+// softmax.
+//
+// Work unit (one CTA): (b, g, 128-row query tile t, split s of the key
+// tiles).  The key range of b is cut into 128-key tiles -- prefix tiles
+// first, then canvas tiles, each read through its own tensor map so a tile
+// never straddles the prefix/canvas boundary; the last tile of each part is
+// masked by key index.  Splits are balanced on the host so that one wave of
+// CTAs covers the SMs; a second kernel merges the splits by their
+// log-sum-exp.
+//
+// Inside a CTA (7 warps):
+//   warps 0-3  softmax: one query row per thread (= one TMEM lane); read S
+//              from TMEM, online softmax in fp32 (log2 domain, lazy rescale
+//              of O only when the running max grows by more than 2^8), write
+//              P as bf16 into shared memory in the 128B-swizzled K-major
+//              layout the MMA reads;
+//   warp 4     TMA producer for Q and K (2-stage ring);
+//   warp 5     TMA producer for V (2-stage ring);
+//   warp 6     allocates 512 TMEM columns (S double buffer + O) and issues
+//              the MMAs from one thread: S_j = Q K_j^T into S[j%2], then
+//              O += P_{j-1} V_{j-1}, so the tensor core works on tile j while
+//              the softmax warps work on tile j-1.
+// Every mbarrier wait is bounded in time; on expiry the CTA latches an
+// error word, drains its own asynchronous work and frees its TMEM.
+#include <mutex>
+
+#include "dd_device.cuh"
+#include "dd_internal.h"
+
+namespace dd {
+namespace {
+
+constexpr int BM = 128;  // query rows per tile
+constexpr int BN = 128;  // keys per tile
+constexpr int HD = 128;  // head dim
+constexpr int kThreads = 7 * 32;
+constexpr int kWarpK = 4, kWarpV = 5, kWarpMMA = 6;
+constexpr uint32_t kHalfBytes = 128 * 64 * 2;    // 128 rows x 128 bytes
+constexpr uint32_t kTileBytes = 2 * kHalfBytes;  // 128 x 128 bf16
+constexpr uint32_t kOffQ = 0;
+constexpr uint32_t kOffK = kTileBytes;
+constexpr uint32_t kOffV = 3 * kTileBytes;
+constexpr uint32_t kOffP = 5 * kTileBytes;
+constexpr uint32_t kOffBar = 7 * kTileBytes;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per wait
+constexpr float kLazyRescale = 8.0f;              // log2 units
+
+struct Barriers {
+  uint64_t q_full;
+  uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
+  uint64_t s_full[2], p_full[2], pv_done[2];
+  uint64_t mma_final;
+  uint32_t tmem_base;
+  int abort;
+  int unit_b, unit_g, unit_t, unit_s, unit_valid;
+};
+
+constexpr uint32_t kSmemBytes = kOffBar + sizeof(Barriers) + 1024;
+
+struct TcParams {
+  int B, C, Hq, Hkv, group, T, chunk;
+  float scale_log2;
+  const int32_t* cu_prefix;
+  float* part_o;    // [units][BM][HD]
+  float* part_lse;  // [units][BM]   log2 units
+  uint32_t* err;
+};
+
+__device__ __forceinline__ int cdiv(int a, int b) { return (a + b - 1) / b; }
+
+// Resolve blockIdx.x -> (b, g, t, s) by walking the batch rows.
+__device__ void resolve_unit(const TcParams& p, Barriers* bars) {
+  int u = blockIdx.x;
+  const int nc = cdiv(p.C, BN);
+  int valid = 0, b = 0, g = 0, t = 0, s = 0;
+  for (int bb = 0; bb < p.B; ++bb) {
+    const int L = p.cu_prefix[bb + 1] - p.cu_prefix[bb];
+    const int ntiles = cdiv(L, BN) + nc;
+    const int nsplit = cdiv(ntiles, p.chunk);
+    const int units = p.Hkv * p.T * nsplit;
+    if (u < units) {
+      s = u % nsplit;
+      t = (u / nsplit) % p.T;
+      g = u / (nsplit * p.T);
+      b = bb;
+      valid = 1;
+      break;
+    }
+    u -= units;
+  }
+  bars->unit_b = b;
+  bars->unit_g = g;
+  bars->unit_t = t;
+  bars->unit_s = s;
+  bars->unit_valid = valid;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
+                   const __grid_constant__ CUtensorMap tmKp,
+                   const __grid_constant__ CUtensorMap tmVp,
+                   const __grid_constant__ CUtensorMap tmKc,
+                   const __grid_constant__ CUtensorMap tmVc, const TcParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  Barriers* bars = reinterpret_cast<Barriers*>(smem + kOffBar);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  volatile int* abort_flag = &bars->abort;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars->k_full[i], 1);
+      mbar_init(&bars->k_empty[i], 1);
+      mbar_init(&bars->v_full[i], 1);
+      mbar_init(&bars->v_empty[i], 1);
+      mbar_init(&bars->s_full[i], 1);
+      mbar_init(&bars->p_full[i], 4);
+      mbar_init(&bars->pv_done[i], 1);
+    }
+    mbar_init(&bars->mma_final, 1);
+    bars->abort = 0;
+    fence_mbar_init();
+    resolve_unit(p, bars);
+  }
+  if (warp == kWarpMMA) {
+    tmem_alloc(&bars->tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  const uint32_t tmem = bars->tmem_base;
+  const int b = bars->unit_b, g = bars->unit_g, t = bars->unit_t, s = bars->unit_s;
+  const bool unit_ok = bars->unit_valid != 0;
+  const int p0 = unit_ok ? p.cu_prefix[b] : 0;
+  const int L = unit_ok ? p.cu_prefix[b + 1] - p0 : 0;
+  const int np = cdiv(L, BN), nc = cdiv(p.C, BN);
+  const int ntiles = np + nc;
+  const int k_begin = s * p.chunk;
+  const int n = unit_ok ? min(p.chunk, ntiles - k_begin) : 0;
+
+  if (warp == kWarpK) {
+    if (lane == 0 && n > 0) {
+    prefetch_tensormap(&tmQ);
+    prefetch_tensormap(&tmKp);
+    prefetch_tensormap(&tmKc);
+    mbar_arrive_expect_tx(&bars->q_full, kTileBytes);
+    const int qpos = b * p.C + t * (BM / p.group);
+    tma_load_3d(smem + kOffQ, &tmQ, &bars->q_full, 0, g * p.group, qpos);
+    tma_load_3d(smem + kOffQ + kHalfBytes, &tmQ, &bars->q_full, 64, g * p.group, qpos);
+    int issued = 0;
+    for (int j = 0; j < n; ++j) {
+      const int st = j & 1, rd = j >> 1;
+      if (rd > 0 &&
+          !mbar_wait_bounded(&bars->k_empty[st], (rd - 1) & 1, abort_flag, kWaitLimitNs))
+        break;
+      const int k = k_begin + j;
+      const CUtensorMap* map = k < np ? &tmKp : &tmKc;
+      const int row0 = k < np ? p0 + k * BN : b * p.C + (k - np) * BN;
+      uint8_t* dst = smem + kOffK + st * kTileBytes;
+      mbar_arrive_expect_tx(&bars->k_full[st], kTileBytes);
+      tma_load_3d(dst, map, &bars->k_full[st], 0, g, row0);
+      tma_load_3d(dst + kHalfBytes, map, &bars->k_full[st], 64, g, row0);
+      issued = j + 1;
+    }
+    // drain: loads still in flight must land before the CTA exits
+    for (int j = max(0, issued - 2); j < issued; ++j)
+      mbar_wait_bounded(&bars->k_full[j & 1], (j >> 1) & 1, nullptr, kWaitLimitNs);
+    mbar_wait_bounded(&bars->q_full, 0, nullptr, kWaitLimitNs);
+    }
+    __syncwarp();
+  } else if (warp == kWarpV) {
+    if (lane == 0 && n > 0) {
+    prefetch_tensormap(&tmVp);
+    prefetch_tensormap(&tmVc);
+    int issued = 0;
+    for (int j = 0; j < n; ++j) {
+      const int st = j & 1, rd = j >> 1;
+      if (rd > 0 &&
+          !mbar_wait_bounded(&bars->v_empty[st], (rd - 1) & 1, abort_flag, kWaitLimitNs))
+        break;
+      const int k = k_begin + j;
+      const CUtensorMap* map = k < np ? &tmVp : &tmVc;
+      const int row0 = k < np ? p0 + k * BN : b * p.C + (k - np) * BN;
+      uint8_t* dst = smem + kOffV + st * kTileBytes;
+      mbar_arrive_expect_tx(&bars->v_full[st], kTileBytes);
+      tma_load_3d(dst, map, &bars->v_full[st], 0, g, row0);
+      tma_load_3d(dst + kHalfBytes, map, &bars->v_full[st], 64, g, row0);
+      issued = j + 1;
+    }
+    for (int j = max(0, issued - 2); j < issued; ++j)
+      mbar_wait_bounded(&bars->v_full[j & 1], (j >> 1) & 1, nullptr, kWaitLimitNs);
+    }
+    __syncwarp();
+  } else if (warp == kWarpMMA) {
+    if (lane == 0 && n > 0) {
+    constexpr uint32_t idS = idesc_bf16_f32(BM, BN, 0, 0);
+    constexpr uint32_t idPV = idesc_bf16_f32(BM, HD, 0, 1);
+    const uint32_t sQ = smem_u32(smem + kOffQ);
+    const uint32_t sK = smem_u32(smem + kOffK);
+    const uint32_t sV = smem_u32(smem + kOffV);
+    const uint32_t sP = smem_u32(smem + kOffP);
+    bool ok = mbar_wait_bounded(&bars->q_full, 0, abort_flag, kWaitLimitNs);
+    tc_fence_after();
+    for (int j = 0; ok && j <= n; ++j) {
+      if (j < n) {
+        const int st = j & 1;
+        if (!mbar_wait_bounded(&bars->k_full[st], (j >> 1) & 1, abort_flag, kWaitLimitNs)) break;
+        if (j >= 2 &&
+            !mbar_wait_bounded(&bars->p_full[st], ((j - 2) >> 1) & 1, abort_flag, kWaitLimitNs))
+          break;
+        tc_fence_after();
+        const uint32_t dS = tmem + (uint32_t)(st * BN);
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+          tc_mma_ss(dS, smem_desc_sw128(sQ + off, 16, 1024),
+                    smem_desc_sw128(sK + st * kTileBytes + off, 16, 1024), idS, kk > 0);
+        }
+        tc_commit(&bars->s_full[st]);
+        tc_commit(&bars->k_empty[st]);
+      }
+      if (j >= 1) {
+        const int jj = j - 1, st = jj & 1;
+        if (!mbar_wait_bounded(&bars->p_full[st], (jj >> 1) & 1, abort_flag, kWaitLimitNs)) break;
+        if (!mbar_wait_bounded(&bars->v_full[st], (jj >> 1) & 1, abort_flag, kWaitLimitNs)) break;
+        tc_fence_after();
+        const uint32_t dO = tmem + 2u * BN;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          const uint32_t offA = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+          const uint32_t offB = kk * 16 * 128;
+          tc_mma_ss(dO, smem_desc_sw128(sP + st * kTileBytes + offA, 16, 1024),
+                    smem_desc_sw128(sV + st * kTileBytes + offB, kHalfBytes, 1024), idPV,
+                    (jj > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc_commit(&bars->pv_done[st]);
+        tc_commit(&bars->v_empty[st]);
+      }
+    }
+    // every MMA issued above has completed before TMEM is released
+    tc_commit(&bars->mma_final);
+    mbar_wait_bounded(&bars->mma_final, 0, nullptr, kWaitLimitNs);
+    }
+    __syncwarp();
+  } else if (warp < 4 && n > 0) {
+    // ------------------------------------------------------------ softmax
+    const int r = warp * 32 + lane;                       // query row in tile
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;  // TMEM lane field
+    uint8_t* sP = smem + kOffP;
+    float m_ref = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n && ok; ++j) {
+      const int st = j & 1;
+      const int k = k_begin + j;
+      const int n_valid = k < np ? min(BN, L - k * BN) : min(BN, p.C - (k - np) * BN);
+      // wait outcomes are made warp-uniform: tcgen05.ld/st are .sync.aligned
+      if (!__all_sync(0xffffffffu,
+                      mbar_wait_bounded(&bars->s_full[st], (j >> 1) & 1, abort_flag,
+                                        kWaitLimitNs))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float sv[BN];
+#pragma unroll
+      for (int c4 = 0; c4 < BN / 32; ++c4) {
+        uint32_t raw[32];
+        tmem_ld32(tmem + lane_base + (uint32_t)(st * BN + c4 * 32), raw);
+#pragma unroll
+        for (int c = 0; c < 32; ++c) sv[c4 * 32 + c] = __uint_as_float(raw[c]);
+      }
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < BN; ++c) {
+        if (c >= n_valid) sv[c] = -INFINITY;
+        mx = fmaxf(mx, sv[c]);
+      }
+      mx *= p.scale_log2;
+      // P buffer st was last read by PV_{j-2}
+      if (j >= 2 &&
+          !__all_sync(0xffffffffu, mbar_wait_bounded(&bars->pv_done[st], ((j - 2) >> 1) & 1,
+                                                     abort_flag, kWaitLimitNs))) {
+        ok = false;
+        break;
+      }
+      // lazy rescale (warp-uniform decision so tcgen05.ld/st stay converged)
+      const bool need = __any_sync(0xffffffffu, mx > m_ref + kLazyRescale);
+      if (need) {
+        const float m_new = fmaxf(m_ref, mx);
+        const float alpha = ex2_approx(m_ref - m_new);  // 0 when m_ref = -inf
+        l *= alpha;
+        if (j >= 1) {
+          const int pj = j - 1;
+          if (!__all_sync(0xffffffffu, mbar_wait_bounded(&bars->pv_done[pj & 1], (pj >> 1) & 1,
+                                                         abort_flag, kWaitLimitNs))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int c4 = 0; c4 < HD / 32; ++c4) {
+            uint32_t raw[32];
+            const uint32_t ta = tmem + lane_base + (uint32_t)(2 * BN + c4 * 32);
+            tmem_ld32(ta, raw);
+#pragma unroll
+            for (int c = 0; c < 32; ++c) raw[c] = __float_as_uint(__uint_as_float(raw[c]) * alpha);
+            tmem_st32(ta, raw);
+          }
+          tmem_wait_st();
+        }
+        m_ref = m_new;
+      }
+      // P = 2^(s * scale_log2 - m_ref) as bf16, 128B-swizzled K-major rows
+      float lsum = 0.f;
+      uint8_t* prow = sP + st * kTileBytes + r * 128;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) {
+          uint32_t w[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int c = h * 64 + cc * 8 + 2 * e;
+            const float pa = ex2_approx(fmaf(sv[c], p.scale_log2, -m_ref));
+            const float pb = ex2_approx(fmaf(sv[c + 1], p.scale_log2, -m_ref));
+            lsum += pa + pb;
+            w[e] = pack_bf16x2(pa, pb);
+          }
+          const int phys = cc ^ (r & 7);
+          *reinterpret_cast<uint4*>(prow + h * kHalfBytes + phys * 16) =
+              make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      }
+      l += lsum;
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->p_full[st]);
+    }
+    // epilogue: O / l and the log2-domain LSE of this split
+    if (ok) {
+      const int last = n - 1;
+      ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->pv_done[last & 1], (last >> 1) & 1,
+                                                     abort_flag, kWaitLimitNs));
+    }
+    if (ok) {
+      tc_fence_after();
+      const float inv = 1.f / l;
+      float* orow = p.part_o + ((size_t)blockIdx.x * BM + r) * HD;
+#pragma unroll
+      for (int c4 = 0; c4 < HD / 32; ++c4) {
+        uint32_t raw[32];
+        tmem_ld32(tmem + lane_base + (uint32_t)(2 * BN + c4 * 32), raw);
+#pragma unroll
+        for (int c = 0; c < 32; c += 4)
+          *reinterpret_cast<float4*>(orow + c4 * 32 + c) =
+              make_float4(__uint_as_float(raw[c]) * inv, __uint_as_float(raw[c + 1]) * inv,
+                          __uint_as_float(raw[c + 2]) * inv, __uint_as_float(raw[c + 3]) * inv);
+      }
+      p.part_lse[(size_t)blockIdx.x * BM + r] = m_ref + __log2f(l);
+    }
+  }
+
+  if (*abort_flag && threadIdx.x == 0) atomicOr(p.err, kDevErrTimeout);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kWarpMMA) tmem_dealloc(tmem, kTmemCols);
+}
+
+// Merge the splits of every (b, g, t) query tile: lse = log2 sum 2^lse_s,
+// O = sum_s 2^(lse_s - lse) O_s.  One warp per query row.
+template <typename TOut>
+__global__ void __launch_bounds__(256)
+    attn_combine_kernel(const TcParams p, int total_units, TOut* __restrict__ out,
+                        float* __restrict__ lse_out) {
+  const int nc = cdiv(p.C, BN);
+  int q = blockIdx.x;  // (b, g, t) group
+  int b = -1, nsplit = 0, ubase = 0;
+  for (int bb = 0; bb < p.B; ++bb) {
+    const int L = p.cu_prefix[bb + 1] - p.cu_prefix[bb];
+    const int ns = cdiv(cdiv(L, BN) + nc, p.chunk);
+    const int groups = p.Hkv * p.T;
+    if (q < groups) {
+      b = bb;
+      nsplit = ns;
+      break;
+    }
+    q -= groups;
+    ubase += groups * ns;
+  }
+  if (b < 0) return;
+  const int g = q / p.T, t = q % p.T;
+  const int u0 = ubase + q * nsplit;
+  if (u0 + nsplit > total_units) {
+    if (threadIdx.x == 0) atomicOr(p.err, kDevErrBounds);
+    return;
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int M = p.C * p.group;
+  for (int r = warp; r < BM; r += 8) {
+    const int pr = t * BM + r;
+    if (pr >= M) break;
+    float mx = -INFINITY;
+    for (int s = 0; s < nsplit; ++s) mx = fmaxf(mx, p.part_lse[(size_t)(u0 + s) * BM + r]);
+    float wsum = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s = 0; s < nsplit; ++s) {
+      const float w = exp2f(p.part_lse[(size_t)(u0 + s) * BM + r] - mx);
+      wsum += w;
+      const float4 o =
+          *reinterpret_cast<const float4*>(p.part_o + ((size_t)(u0 + s) * BM + r) * HD + lane * 4);
+      acc.x = fmaf(w, o.x, acc.x);
+      acc.y = fmaf(w, o.y, acc.y);
+      acc.z = fmaf(w, o.z, acc.z);
+      acc.w = fmaf(w, o.w, acc.w);
+    }
+    const float inv = 1.f / wsum;
+    const int i = pr / p.group, h = g * p.group + (pr - i * p.group);
+    TOut* orow = out + (((size_t)b * p.C + i) * p.Hq + h) * HD + lane * 4;
+    if constexpr (sizeof(TOut) == 2) {
+      uint2 v;
+      v.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+      v.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+      *reinterpret_cast<uint2*>(orow) = v;
+    } else {
+      *reinterpret_cast<float4*>(orow) =
+          make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+    }
+    if (lse_out && lane == 0)
+      lse_out[((size_t)b * p.Hq + h) * p.C + i] = (mx + __log2f(wsum)) * 0.6931471805599453f;
+  }
+}
+
+// ----------------------------------------------------------------- host
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// 3-D map over a [rows, heads, 128] bf16 tensor, box (64, box_heads, box_rows),
+// 128-byte swizzle; rows outside [0, rows) read as zero.
+bool encode_map(CUtensorMap* m, const void* base, int64_t rows, int heads, int box_heads,
+                int box_rows) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)HD, (cuuint64_t)heads, (cuuint64_t)rows};
+  const cuuint64_t strides[2] = {(cuuint64_t)HD * 2, (cuuint64_t)heads * HD * 2};
+  const cuuint32_t box[3] = {64, (cuuint32_t)box_heads, (cuuint32_t)box_rows};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+int num_sms() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+struct Plan {
+  int T, chunk, units, groups;
+};
+
+// Choose the split size (key tiles per CTA) that minimises the makespan
+// waves(units) * chunk over the SMs.
+Plan make_plan(const AttnArgs& a) {
+  Plan pl{};
+  const int group = a.Hq / a.Hkv;
+  pl.T = (a.C * group + BM - 1) / BM;
+  const int nc = (a.C + BN - 1) / BN;
+  int max_tiles = 1;
+  for (int b = 0; b < a.B; ++b) {
+    const int L = a.cu_prefix_host[b + 1] - a.cu_prefix_host[b];
+    max_tiles = std::max(max_tiles, (L + BN - 1) / BN + nc);
+  }
+  const int sms = num_sms();
+  double best_cost = 1e300;
+  for (int chunk = 1; chunk <= max_tiles; ++chunk) {
+    int64_t units = 0;
+    for (int b = 0; b < a.B; ++b) {
+      const int L = a.cu_prefix_host[b + 1] - a.cu_prefix_host[b];
+      const int ntiles = (L + BN - 1) / BN + nc;
+      units += (int64_t)a.Hkv * pl.T * ((ntiles + chunk - 1) / chunk);
+    }
+    const int64_t waves = (units + sms - 1) / sms;
+    // each split also costs its share of the merge pass (~ a quarter tile)
+    const double cost = (double)waves * chunk + 0.25 * (double)units / sms;
+    if (cost < best_cost - 1e-9) {
+      best_cost = cost;
+      pl.chunk = chunk;
+      pl.units = (int)units;
+    }
+  }
+  pl.groups = a.B * a.Hkv * pl.T;
+  return pl;
+}
+
+}  // namespace
+
+bool attn_tc_supported(const AttnArgs& a) {
+  if (!a.bf16 || a.D != HD) return false;
+  const int group = a.Hq / a.Hkv;
+  if (group < 1 || BM % group != 0) return false;
+  // TMA: 16-byte aligned bases (rows of 256 bytes are always aligned)
+  const uintptr_t mask = 15;
+  if ((reinterpret_cast<uintptr_t>(a.q) | reinterpret_cast<uintptr_t>(a.kc) |
+       reinterpret_cast<uintptr_t>(a.vc) | reinterpret_cast<uintptr_t>(a.kp) |
+       reinterpret_cast<uintptr_t>(a.vp)) & mask)
+    return false;
+  return true;
+}
+
+size_t attn_tc_scratch_bytes(const AttnArgs& a) {
+  const Plan pl = make_plan(a);
+  return (size_t)pl.units * BM * (HD + 1) * sizeof(float) + 256;
+}
+
+cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t stream) {
+  static std::once_flag attr_once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once, [] {
+    attr_err = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)kSmemBytes);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+
+  const Plan pl = make_plan(a);
+  const int group = a.Hq / a.Hkv;
+  CUtensorMap mQ, mKp, mVp, mKc, mVc;
+  bool ok = encode_map(&mQ, a.q, (int64_t)a.B * a.C, a.Hq, group, BM / group) &&
+            encode_map(&mKc, a.kc, (int64_t)a.B * a.C, a.Hkv, 1, BN) &&
+            encode_map(&mVc, a.vc, (int64_t)a.B * a.C, a.Hkv, 1, BN);
+  if (a.total_prefix > 0) {
+    ok = ok && encode_map(&mKp, a.kp, a.total_prefix, a.Hkv, 1, BN) &&
+         encode_map(&mVp, a.vp, a.total_prefix, a.Hkv, 1, BN);
+  } else {  // no prefix rows anywhere: the prefix maps are never read
+    mKp = mKc;
+    mVp = mVc;
+  }
+  if (!ok) return cudaErrorInvalidValue;
+
+  TcParams tp;
+  tp.B = a.B;
+  tp.C = a.C;
+  tp.Hq = a.Hq;
+  tp.Hkv = a.Hkv;
+  tp.group = group;
+  tp.T = pl.T;
+  tp.chunk = pl.chunk;
+  tp.scale_log2 = a.scale * 1.4426950408889634f;
+  tp.cu_prefix = a.cu_prefix;
+  uint8_t* scratch = static_cast<uint8_t*>(a.scratch);
+  tp.part_o = reinterpret_cast<float*>(scratch);
+  tp.part_lse = reinterpret_cast<float*>(scratch + (size_t)pl.units * BM * HD * sizeof(float));
+  tp.err = a.err;
+
+  attn_tc_kernel<<<pl.units, kThreads, kSmemBytes, stream>>>(mQ, mKp, mVp, mKc, mVc, tp);
+  note_launch();
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  attn_combine_kernel<__nv_bfloat16><<<pl.groups, 256, 0, stream>>>(
+      tp, pl.units, static_cast<__nv_bfloat16*>(a.out), a.lse);
+  note_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace dd

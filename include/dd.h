@@ -1,0 +1,215 @@
+/*
+ * dd.h -- C ABI of libdd: one denoising step of block discrete-diffusion
+ * decoding on an NVIDIA B200 (sm_100a).
+ *
+ * What the step computes ("DiffusionGemma Technical Report", paperfeed
+ * review, section "The mechanism: an AR model turned inside out"):
+ *   - a 256-token canvas whose queries attend bidirectionally to the whole
+ *     canvas and to a causally encoded prefix KV cache;
+ *   - a sampler that turns each position's temperature-scaled logits into a
+ *     new token, a confidence and an entropy, then re-corrupts positions to
+ *     uniformly random vocabulary tokens (multinomial noise, not [MASK]);
+ *   - about 12 such passes per 256-token block.
+ *
+ * Conventions for every entry point:
+ *   - Ownership: the caller owns every buffer.  libdd never allocates device
+ *     or pinned memory; scratch space is the caller's `workspace`.
+ *   - Pointers are DEVICE pointers unless the name ends in `_host`.
+ *   - Tensors are dense row-major ("C order"), last dimension fastest, with
+ *     the shapes given below.  Device pointers must be 16-byte aligned.
+ *   - Every call is asynchronous on `stream` (0 = the legacy default stream)
+ *     and makes no host synchronisation, except dd_query_device_error.
+ *   - Errors: arguments are validated on the host BEFORE any launch.  Invalid
+ *     shapes/pointers return DD_ERR_INVALID_ARG, shapes without a kernel
+ *     return DD_ERR_UNSUPPORTED, a too-small workspace DD_ERR_WORKSPACE, a
+ *     failed launch DD_ERR_CUDA.  dd_last_error() then holds a message
+ *     (thread-local).  Nothing aborts or throws across this boundary.
+ *   - Device-side faults that kernels detect themselves (a pipeline wait that
+ *     exceeded its time limit) are latched in the first 16 bytes of the
+ *     workspace and read back by dd_query_device_error.  A workspace must be
+ *     cleared once with dd_workspace_init before first use.
+ *   - There is no CPU fallback: if the CUDA kernels cannot run, calls fail.
+ */
+#ifndef DD_H_
+#define DD_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define DD_API __attribute__((visibility("default")))
+#else
+#define DD_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* dd_stream_t; /* == cudaStream_t */
+
+typedef enum {
+  DD_OK = 0,
+  DD_ERR_INVALID_ARG = 1,
+  DD_ERR_UNSUPPORTED = 2,
+  DD_ERR_WORKSPACE = 3,
+  DD_ERR_CUDA = 4,
+  DD_ERR_DEVICE_TIMEOUT = 5,
+  DD_ERR_DEVICE_BOUNDS = 6
+} dd_status;
+
+typedef enum { DD_BF16 = 0, DD_F32 = 1 } dd_dtype;
+
+/* Geometry of one canvas-attention call.
+ *   batch     B >= 1 canvases (batch rows)
+ *   canvas    C >= 1 positions per canvas (256 in the method)
+ *   heads_q   Hq query heads; heads_kv Hkv kv heads, Hq % Hkv == 0.  Query
+ *             head h reads kv head h / (Hq / Hkv) (grouped-query attention;
+ *             the pages do not state the head mapping, this is the usual one).
+ *   head_dim  D in {64, 128}
+ *   scale     softmax scale (1/sqrt(D) in every workload here)
+ *   dtype     DD_BF16 (tensor cores, fp32 accumulation) or DD_F32 (fp32 FMA) */
+typedef struct {
+  int batch, canvas, heads_q, heads_kv, head_dim;
+  float scale;
+  dd_dtype dtype;
+} dd_attn_desc;
+
+/* Workspace bytes that dd_canvas_attn needs for this geometry and these
+ * prefix lengths (cu_prefix_host: [B+1] host array, see dd_canvas_attn).
+ * Returns 0 if the arguments are invalid. */
+DD_API size_t dd_canvas_attn_workspace(const dd_attn_desc* desc, const int32_t* cu_prefix_host);
+
+/* Bidirectional canvas attention over [prefix KV || canvas KV]
+ * ("DiffusionGemma Technical Report", "The mechanism": the canvas is refined
+ * with full bidirectional attention inside the canvas while attending to the
+ * causally encoded cache).  For batch row b, position i, query head h with
+ * g = h / (Hq/Hkv), the keys are the L_b prefix rows of b followed by the C
+ * canvas rows of b, all unmasked, under ONE softmax:
+ *   O[b,i,h,:] = sum_j softmax_j(scale * <q, k_j>) v_j
+ * Arguments (element type = desc->dtype):
+ *   q            [B, C, Hq, D]
+ *   k_canvas     [B, C, Hkv, D]     v_canvas  same
+ *   k_prefix     [sum_b L_b, Hkv, D] packed; rows cu_prefix[b]..cu_prefix[b+1]-1
+ *   v_prefix     same
+ *   cu_prefix    device int32 [B+1], cu_prefix[0] = 0, non-decreasing;
+ *                L_b = cu_prefix[b+1] - cu_prefix[b] may be 0
+ *   cu_prefix_host  host copy of the same values (used to plan the launch;
+ *                the two must agree, which is not checked on the device)
+ *   out          [B, C, Hq, D], element type = desc->dtype
+ *   lse          optional fp32 [B, Hq, C]: natural-log sum of exp of scores
+ *   workspace    >= dd_canvas_attn_workspace(...) bytes, 256-byte aligned */
+DD_API dd_status dd_canvas_attn(const dd_attn_desc* desc, const void* q, const void* k_canvas,
+                         const void* v_canvas, const void* k_prefix, const void* v_prefix,
+                         const int32_t* cu_prefix, const int32_t* cu_prefix_host, void* out,
+                         float* lse, void* workspace, size_t workspace_bytes, dd_stream_t stream);
+
+/* Sampler parameters for one step.
+ *   temperature   tau > 0; logits are divided by it (the method anneals it
+ *                 0.8 -> 0.4 over the steps; the caller passes each step's)
+ *   renoise_rate  probability in [0,1] that a position is re-noised
+ *   seed          Philox4x32-10 key
+ *   step          Philox counter word 2 (the denoising step)
+ *   row_offset    global index of row 0 of this call (Philox counter word 1
+ *                 is row_offset + local row), so that a batch split across
+ *                 calls draws the same numbers as one call. */
+typedef struct {
+  float temperature;
+  float renoise_rate;
+  uint64_t seed;
+  uint32_t step;
+  uint32_t row_offset;
+} dd_sample_params;
+
+/* Workspace bytes that dd_sample_renoise needs (0 on invalid arguments). */
+DD_API size_t dd_sample_renoise_workspace(int rows, int vocab, dd_dtype dtype);
+
+/* One sampler + re-noise step over `rows` positions ("DiffusionGemma
+ * Technical Report", "The mechanism": temperature-scaled logits give
+ * per-position entropies; positions not kept are re-noised to uniformly
+ * random vocabulary tokens; "Training": each token is corrupted
+ * independently with a probability).  For global row r and vocab index v,
+ * with z = logit / tau and Philox4x32-10 words x(stream, v) under key = seed,
+ * counter (v >> 2, r, step, stream), word v & 3:
+ *   pred      = argmax_v z_v - ln(-ln U(x(0, v))),  U(x) = (2 (x >> 9) + 1) 2^-24
+ *               (Gumbel-max: a draw from softmax(z); lowest v on exact ties)
+ *   conf      = softmax(z)[pred]
+ *   entropy   = -sum_v p_v ln p_v, p = softmax(z)
+ *   renoised  = U(x(1, 0)) < renoise_rate   (fp32 compare)
+ *   token     = renoised ? (x(2, 0) * V) >> 32 : pred
+ * Arguments:
+ *   logits       [rows, V] of `dtype` with `row_stride` elements between rows
+ *                (row_stride >= V)
+ *   tokens_out   int32 [rows] (required)
+ *   pred_out     int32 [rows] or NULL
+ *   conf_out     fp32 [rows] (required)
+ *   entropy_out  fp32 [rows] or NULL
+ *   renoised_out uint8 [rows] or NULL
+ *   workspace    >= dd_sample_renoise_workspace(rows, V, dtype) bytes */
+DD_API dd_status dd_sample_renoise(const void* logits, dd_dtype dtype, int rows, int vocab,
+                            int64_t row_stride, const dd_sample_params* params,
+                            int32_t* tokens_out, int32_t* pred_out, float* conf_out,
+                            float* entropy_out, uint8_t* renoised_out, void* workspace,
+                            size_t workspace_bytes, dd_stream_t stream);
+
+/* Canvas initialisation to uniformly random vocabulary tokens ("The
+ * mechanism": a canvas of noise): canvas[r] = (x * V) >> 32 with x the word
+ * for key = seed, counter (0, row_offset + r, 0, 3), word 0.
+ *   canvas  int32 [rows] */
+DD_API dd_status dd_init_canvas(int32_t* canvas, int rows, int vocab, uint64_t seed, uint32_t row_offset,
+                         dd_stream_t stream);
+
+/* Workspace bytes for dd_denoise_block (the larger of the two steps' needs). */
+DD_API size_t dd_denoise_block_workspace(const dd_attn_desc* desc, const int32_t* cu_prefix_host,
+                                  int vocab);
+
+/* The inner loop of one block: `steps` denoising passes ("about 12 forward
+ * passes per 256-token block", "The mechanism").  Step s (0-based) runs
+ * dd_canvas_attn on the step's canvas Q/K/V and dd_sample_renoise on the
+ * step's logits with Philox step = step0 + s, temperature_host[s] and
+ * rate_host[s]; the canvas after step s is its tokens.  Steps are
+ * independent of the previous canvas (the model that would map the canvas
+ * to Q/K/V and logits is outside this library), so restarting at step0 = k
+ * reproduces steps k.. exactly.
+ * Arguments (R = B*C rows, element type = desc->dtype):
+ *   q_steps        [S, B, C, Hq, D];  kc_steps, vc_steps [S, B, C, Hkv, D]
+ *   k_prefix, v_prefix, cu_prefix, cu_prefix_host: as dd_canvas_attn
+ *   attn_out       [S, B, C, Hq, D]
+ *   logits_steps   [S, R, V] (dtype as desc->dtype)
+ *   rate_host, temperature_host   host fp32 [S]
+ *   canvas         int32 [R]: the canvas after the last step
+ *   canvas_history int32 [S, R] or NULL: every step's canvas
+ *   conf_steps     fp32 [S, R] or NULL: every step's confidences
+ *   workspace      >= dd_denoise_block_workspace(...) bytes */
+DD_API dd_status dd_denoise_block(const dd_attn_desc* desc, int steps, const void* q_steps,
+                           const void* kc_steps, const void* vc_steps, const void* k_prefix,
+                           const void* v_prefix, const int32_t* cu_prefix,
+                           const int32_t* cu_prefix_host, void* attn_out,
+                           const void* logits_steps, int vocab, const float* rate_host,
+                           const float* temperature_host, uint64_t seed, uint32_t step0,
+                           int32_t* canvas, int32_t* canvas_history, float* conf_steps,
+                           void* workspace, size_t workspace_bytes, dd_stream_t stream);
+
+/* Clears the error word at the start of a workspace (async on stream). */
+DD_API dd_status dd_workspace_init(void* workspace, size_t workspace_bytes, dd_stream_t stream);
+
+/* Synchronises `stream`, reads the workspace's latched device error and
+ * clears it.  Returns DD_OK, DD_ERR_DEVICE_TIMEOUT or DD_ERR_DEVICE_BOUNDS. */
+DD_API dd_status dd_query_device_error(void* workspace, dd_stream_t stream);
+
+/* Static description of a status code. */
+DD_API const char* dd_status_string(dd_status status);
+
+/* Detail of the last failure on this host thread ("" if none). */
+DD_API const char* dd_last_error(void);
+
+/* Number of kernels the library launched on this host thread since the last
+ * call to dd_reset_launch_count (for launch accounting in benchmarks). */
+DD_API uint64_t dd_launch_count(void);
+DD_API void dd_reset_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DD_H_ */

@@ -1,0 +1,148 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every symbol include/dd.h declares, answers workspace queries, and rejects
+invalid arguments before any launch (no CUDA call is reached)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import block_discrete_diffusion_dd_b200 as dd
+from block_discrete_diffusion_dd_b200 import build as libbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    libbuild.build()
+    return dd.load()
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "dd.h")).read()
+    return sorted(set(re.findall(r"^DD_API[^(]*?\b(dd_\w+)\s*\(", text, re.M)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = _declared()
+    assert len(names) >= 12
+    assert set(names) == set(dd.EXPORTS)
+    for n in names:
+        assert getattr(lib, n) is not None
+    # and nothing else with the dd_ prefix is exported
+    out = os.popen(f"nm -D --defined-only {dd.LIB_PATH}").read()
+    exported = sorted(set(re.findall(r" T (dd_\w+)$", out, re.M)))
+    assert exported == names
+
+
+def test_status_strings(lib):
+    for code in range(7):
+        assert dd.status_string(code)
+    assert dd.status_string(99) == "unknown status"
+
+
+def _desc(B=1, C=256, Hq=16, Hkv=8, D=128, dtype=dd.DD_BF16, scale=None):
+    return dd.AttnDesc(B, C, Hq, Hkv, D, scale if scale is not None else D ** -0.5, dtype)
+
+
+def _cu(lens):
+    return np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+
+
+def test_workspace_queries(lib):
+    d = _desc()
+    n = dd.canvas_attn_workspace_bytes(d, _cu([4096]))
+    assert n > 256
+    assert dd.canvas_attn_workspace_bytes(_desc(Hq=6, Hkv=4), _cu([4096])) == 0  # Hq % Hkv
+    assert dd.canvas_attn_workspace_bytes(_desc(D=96), _cu([4096])) == 0         # head_dim
+    assert dd.canvas_attn_workspace_bytes(_desc(B=2), np.array([0, 5, 3], np.int32)) == 0
+    s = dd.sample_workspace_bytes(256, 262144)
+    assert s >= 256 + 256 * 32
+    assert lib.dd_sample_renoise_workspace(-1, 10, 0) == 0
+    assert lib.dd_sample_renoise_workspace(4, 0, 0) == 0
+    b = dd.denoise_block_workspace_bytes(d, _cu([4096]), 262144)
+    assert b >= max(n, s)
+
+
+FAKE = ctypes.c_void_p(1 << 20)  # never dereferenced: validation fails first
+
+
+def _sample(lib, rows=4, vocab=16, stride=16, temp=1.0, rate=0.5, dtype=0, tokens=FAKE,
+            conf=FAKE, ws=FAKE, ws_bytes=1 << 20, logits=FAKE, row_offset=0):
+    p = dd.SampleParams(temp, rate, 0, 0, row_offset)
+    return lib.dd_sample_renoise(logits, dtype, rows, vocab, stride, ctypes.byref(p), tokens, None,
+                                 conf, None, None, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(rows=-1), 1), (dict(vocab=0), 1), (dict(stride=8), 1), (dict(temp=0.0), 1),
+    (dict(temp=float("nan")), 1), (dict(rate=1.5), 1), (dict(rate=-0.1), 1), (dict(dtype=7), 1),
+    (dict(tokens=None), 1), (dict(conf=None), 1), (dict(logits=None), 1),
+    (dict(ws=None), 3), (dict(ws_bytes=16), 3), (dict(ws=ctypes.c_void_p((1 << 20) + 8)), 3),
+    (dict(rows=2, row_offset=0xFFFFFFFF), 1),
+])
+def test_sampler_rejects_bad_arguments(lib, kw, code):
+    assert _sample(lib, **kw) == code
+    assert dd.last_error()
+
+
+def test_sampler_zero_rows_is_a_no_op(lib):
+    assert _sample(lib, rows=0, tokens=None, conf=None, logits=None, ws=None) == 0
+
+
+def _attn(lib, desc, cu, ws_bytes=1 << 30, ptr=FAKE, ws=FAKE, cu_dev=FAKE, kp=FAKE):
+    return lib.dd_canvas_attn(ctypes.byref(desc), ptr, ptr, ptr, kp, kp, cu_dev,
+                              cu.ctypes.data_as(ctypes.c_void_p), ptr, None, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("desc,cu,code", [
+    (_desc(Hq=6, Hkv=4), _cu([16]), 1),
+    (_desc(D=96), _cu([16]), 2),
+    (_desc(C=0), _cu([16]), 1),
+    (_desc(scale=0.0), _cu([16]), 1),
+    (_desc(dtype=5), _cu([16]), 1),
+    (_desc(B=2), np.array([0, 9, 3], np.int32), 1),
+    (_desc(B=2), np.array([1, 9, 30], np.int32), 1),
+])
+def test_attention_rejects_bad_arguments(lib, desc, cu, code):
+    assert _attn(lib, desc, cu) == code
+    assert dd.last_error()
+
+
+def test_attention_rejects_null_and_misaligned(lib):
+    d = _desc()
+    cu = _cu([16])
+    assert _attn(lib, d, cu, ptr=None) == 1
+    assert _attn(lib, d, cu, kp=None) == 1                       # prefix rows exist
+    assert _attn(lib, d, cu, ptr=ctypes.c_void_p((1 << 20) + 2)) == 1
+    assert _attn(lib, d, cu, ws=None) == 3
+    assert _attn(lib, d, cu, ws_bytes=300) == 3
+    assert _attn(lib, _desc(B=0), cu[:1]) == 0                   # empty batch: no-op
+
+
+def test_block_rejects_bad_arguments(lib):
+    d = _desc()
+    cu = _cu([16])
+    r = np.zeros(1, np.float32)
+    args = [ctypes.byref(d), 1, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+            cu.ctypes.data_as(ctypes.c_void_p), FAKE, FAKE, 1024,
+            r.ctypes.data_as(ctypes.c_void_p), r.ctypes.data_as(ctypes.c_void_p), 0, 0, FAKE,
+            None, None, FAKE, 16, None]
+    assert lib.dd_denoise_block(*args) == 3                      # workspace too small
+    bad = list(args)
+    bad[1] = -1
+    assert lib.dd_denoise_block(*bad) == 1
+    bad = list(args)
+    bad[12] = None
+    assert lib.dd_denoise_block(*bad) == 1
+    bad = list(args)
+    bad[16] = None
+    assert lib.dd_denoise_block(*bad) == 1
+
+
+def test_init_canvas_rejects_bad_arguments(lib):
+    assert lib.dd_init_canvas(None, 4, 10, 0, 0, None) == 1
+    assert lib.dd_init_canvas(FAKE, 4, 0, 0, 0, None) == 1
+    assert lib.dd_init_canvas(None, 0, 10, 0, 0, None) == 0
