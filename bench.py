@@ -1,0 +1,466 @@
+#!/usr/bin/env python3
+"""Benchmark of one denoising step of block discrete-diffusion decoding.
+
+A step = canvas attention over [prefix KV || canvas KV] (tcgen05 kernel +
+split merge) followed by the vocabulary-wide sampler and re-noise (chunk
+pass + row merge): every step of the hot path, through the C ABI
+(dd_canvas_attn, dd_sample_renoise).  Default workload: batch 1, 16 query /
+8 kv heads, head_dim 128, prefix 4096, canvas 256, vocabulary 262144, bf16.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints ONE JSON line (rank 0).  `value` is canvas-steps/s over all ranks
+(each rank runs its own independent canvases: no collective on the data
+path), from CUDA events on the launch stream, max over ranks.  Inputs are
+rotated among 3 sets of ~152 MB each (> 126 MB L2) so no step reads the
+previous step's inputs from L2.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = "denoise steps/s per 256-token canvas"
+UNIT = "canvas-steps/s"
+N_SETS = 3
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p["bf16_tflops_sustained"]), \
+            "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi samples every 100 ms in a background thread."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.samples = []
+        self.proc = None
+        self.gpu = gpu_index
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.gpu)], stdout=subprocess.PIPE,
+                stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.time(), [x.strip() for x in line.split(",")]))
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self, t0, t1):
+        sel = [s for t, s in self.samples if t0 <= t <= t1] or [s for _, s in self.samples[-3:]]
+        if not sel:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(s[0]) for s in sel if s[0].replace(".", "").isdigit()]
+        mx = [float(s[1]) for s in sel if s[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for s in sel for n, v in zip(names, s[4:8]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(sel)}
+
+
+def _dist():
+    n = int(os.environ.get("WORLD_SIZE", "1"))
+    if n > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        return dist, dist.get_rank(), n, int(os.environ.get("LOCAL_RANK", "0"))
+    return None, 0, 1, 0
+
+
+def _max_over_ranks(dist, x: float) -> float:
+    if dist is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _barrier(dist):
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def make_inputs(w, rank: int, dev):
+    """N_SETS independent input sets on the device (seeded per rank and set)."""
+    sets = []
+    for s in range(N_SETS):
+        ws = workloads.scaled(w, seed=w.seed + 1000 * rank + s)
+        q, kc, vc = workloads.canvas_qkv(ws, 0, device=dev)
+        kp, vp, cu = workloads.prefix_kv(ws, device=dev)
+        lg = workloads.logits(ws, 0, device=dev)
+        sets.append({"q": q, "kc": kc, "vc": vc, "kp": kp, "vp": vp, "cu": cu.to(dev),
+                     "cu_host": cu.numpy(), "logits": lg})
+    return sets
+
+
+def run_ours(args, w, dist, rank, world, local_rank):
+    import block_discrete_diffusion_dd_b200 as dd
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    sets = make_inputs(w, rank, dev)
+    R, V = w.rows, w.vocab
+    desc = dd.attn_desc(sets[0]["q"], sets[0]["kc"], w.scale)
+    ws_attn = dd.new_workspace(dd.canvas_attn_workspace_bytes(desc, sets[0]["cu_host"]), dev)
+    ws_samp = dd.new_workspace(dd.sample_workspace_bytes(R, V, w.torch_dtype), dev)
+    attn_out = torch.empty_like(sets[0]["q"])
+    outs = {"tokens": torch.empty(R, dtype=torch.int32, device=dev),
+            "pred": None, "entropy": torch.empty(R, dtype=torch.float32, device=dev),
+            "conf": torch.empty(R, dtype=torch.float32, device=dev),
+            "renoised": torch.empty(R, dtype=torch.uint8, device=dev)}
+    rate, tau = w.rates[0], w.temperatures[0]
+
+    def attn(i):
+        s = sets[i % N_SETS]
+        dd.canvas_attn(s["q"], s["kc"], s["vc"], s["kp"], s["vp"], s["cu"], s["cu_host"],
+                       scale=w.scale, out=attn_out, workspace=ws_attn)
+
+    def samp(i):
+        s = sets[i % N_SETS]
+        dd.sample_renoise(s["logits"], tau, rate, w.seed + rank, i, row_offset=0, outputs=outs,
+                          workspace=ws_samp)
+
+    def step(i):
+        attn(i)
+        samp(i)
+
+    # eager warm-up (first calls set kernel attributes), then CUDA graphs
+    # per input set: the whole step, and the whole step with timing events
+    # between the attention and the sampler calls
+    for i in range(N_SETS):
+        step(i)
+    dd.query_device_error(ws_attn)
+    side = torch.cuda.Stream(device=dev)
+    side.wait_stream(stream)
+    graphs, timed = [], []
+    with torch.cuda.stream(side):
+        for i in range(N_SETS):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=side):
+                step(i)
+            graphs.append(g)
+            ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)]
+            g2 = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g2, stream=side):
+                ev[0].record()
+                attn(i)
+                ev[1].record()
+                samp(i)
+                ev[2].record()
+            timed.append((g2, ev))
+    launches_per_step = _launches_per_step(dd, step)
+    stream.wait_stream(side)
+    for i in range(args.warmup):
+        graphs[i % N_SETS].replay()
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(local_rank if world > 1 else torch.cuda.current_device())
+    clocks.start()
+    time.sleep(0.3)
+    # the whole-job number: K steps between one event pair
+    _barrier(dist)
+    t_wall0 = time.time()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        graphs[i % N_SETS].replay()
+    e1.record(stream)
+    _barrier(dist)
+    t_wall1 = time.time()
+    launches = launches_per_step * args.steps
+    ms_total = _max_over_ranks(dist, e0.elapsed_time(e1))
+    # per-kernel durations inside whole steps (events between the calls)
+    n2 = max(N_SETS, min(args.steps, 300))
+    ta, ts = [], []
+    for i in range(n2):
+        g2, ev = timed[i % N_SETS]
+        g2.replay()
+        torch.cuda.synchronize()
+        ta.append(ev[0].elapsed_time(ev[1]))
+        ts.append(ev[1].elapsed_time(ev[2]))
+    per = {"attn": _max_over_ranks(dist, statistics.mean(ta) / 1e3),
+           "samp": _max_over_ranks(dist, statistics.mean(ts) / 1e3)}
+    time.sleep(0.2)
+    clocks.stop()
+    dd.query_device_error(ws_attn)
+    t_attn, t_samp = per["attn"], per["samp"]
+    del graphs, timed
+
+    # end to end: host buffers, copies inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, w, sets[0], dd, dev, stream, desc, dist)
+
+    ms_per_step = ms_total / args.steps
+    value = world * w.batch * args.steps / (ms_total / 1e3)
+    hbm, tf_burst, tf_sus, src = _peaks()
+    samp_bytes = w.logit_bytes() + R * (4 + 4 + 4 + 1)
+    samp_gbs = samp_bytes / t_samp / 1e9
+    attn_tf = w.attn_flops() / t_attn / 1e12
+    traffic = _profile_traffic()
+    res = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "batch_per_gpu": w.batch, "canvas": w.canvas,
+                   "heads_q": w.heads_q, "heads_kv": w.heads_kv, "head_dim": w.head_dim,
+                   "prefix": list(w.prefix_lens), "vocab": w.vocab, "renoise_rate": w.rates[0],
+                   "temperature": w.temperatures[0],
+                   "l2": f"{N_SETS} rotating input sets of "
+                         f"{(w.logit_bytes() + 2 * sets[0]['kp'].numel() * 2) / 1e6:.0f} MB "
+                         "(> 126 MB L2)",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": {"bound": "hbm", "kernel": "sampler (chunk pass + row merge)",
+                     "achieved": samp_gbs, "peak": hbm, "unit": "GB/s", "frac": samp_gbs / hbm,
+                     "traffic": traffic.get("sampler"), "peak_source": src,
+                     "algorithmic_bytes": samp_bytes, "ms": t_samp * 1e3},
+        "roofline_attn": {"bound": "tensor", "kernel": "canvas attention (tcgen05 + merge)",
+                          "achieved": attn_tf, "peak": tf_burst, "unit": "TFLOP/s",
+                          "frac": attn_tf / tf_burst, "frac_of_sustained": attn_tf / tf_sus,
+                          "flops": w.attn_flops(), "ms": t_attn * 1e3,
+                          "traffic": traffic.get("attention"), "peak_source": src},
+        "e2e": e2e,
+        "gpu_launches": int(launches),
+        "clocks": clocks.summary(t_wall0, t_wall1),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu:
+        res["cpu_baseline"] = cpu_baseline(w, sets[0], frac=args.cpu_sample)
+    return res
+
+
+def _launches_per_step(dd, step) -> int:
+    """Kernels one step launches (counted by the library on this thread)."""
+    dd.reset_launch_count()
+    step(0)
+    torch.cuda.synchronize()
+    return dd.launch_count()
+
+
+def run_e2e(args, w, s, dd, dev, stream, desc, dist):
+    """Same step through the C ABI with inputs in pinned host memory: every
+    step copies its inputs host->device and reads tokens + confidences back."""
+    names = ["q", "kc", "vc", "kp", "vp", "logits"]
+    host = {k: s[k].cpu().pin_memory() for k in names}
+    host["cu"] = s["cu"].cpu().pin_memory()
+    devb = {k: torch.empty_like(s[k]) for k in names}
+    devb["cu"] = torch.empty_like(s["cu"])
+    ws_attn = dd.new_workspace(dd.canvas_attn_workspace_bytes(desc, s["cu_host"]), dev)
+    ws_samp = dd.new_workspace(dd.sample_workspace_bytes(w.rows, w.vocab, w.torch_dtype), dev)
+    attn_out = torch.empty_like(s["q"])
+    outs = {"tokens": torch.empty(w.rows, dtype=torch.int32, device=dev), "pred": None,
+            "entropy": None, "conf": torch.empty(w.rows, dtype=torch.float32, device=dev),
+            "renoised": None}
+    tok_h = torch.empty(w.rows, dtype=torch.int32).pin_memory()
+    conf_h = torch.empty(w.rows, dtype=torch.float32).pin_memory()
+    h2d = sum(host[k].numel() * host[k].element_size() for k in host)
+    d2h = tok_h.numel() * 4 + conf_h.numel() * 4
+
+    def step(i):
+        for k in host:
+            devb[k].copy_(host[k], non_blocking=True)
+        dd.canvas_attn(devb["q"], devb["kc"], devb["vc"], devb["kp"], devb["vp"], devb["cu"],
+                       s["cu_host"], scale=w.scale, out=attn_out, workspace=ws_attn,
+                       stream=stream)
+        dd.sample_renoise(devb["logits"], w.temperatures[0], w.rates[0], w.seed, i,
+                          outputs=outs, workspace=ws_samp, stream=stream)
+        tok_h.copy_(outs["tokens"], non_blocking=True)
+        conf_h.copy_(outs["conf"], non_blocking=True)
+
+    n = max(3, min(args.steps, args.e2e_steps))
+    for i in range(3):
+        step(i)
+    _barrier(dist)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for i in range(n):
+        step(i)
+    b.record(stream)
+    _barrier(dist)
+    ms = _max_over_ranks(dist, a.elapsed_time(b))
+    world = dist.get_world_size() if dist is not None else 1
+    return {"value": world * w.batch * n / (ms / 1e3), "unit": UNIT, "steps": n,
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "ms_per_step": ms / n}
+
+
+def _profile_traffic() -> dict:
+    """DRAM bytes per launch from the committed ncu summary (None if absent
+    or taken on an older build of the kernel)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            t = json.load(f)
+        return {k: v.get("bytes_per_launch") for k, v in t.items() if v.get("current", False)}
+    except Exception:
+        return {}
+
+
+def cpu_baseline(w, s, frac: float):
+    """The oracle, as it stands, on this host's cores, on a bounded sample of
+    one step (a fraction `frac` of the canvas positions for attention and of
+    the rows for the sampler), scaled to a whole step."""
+    import oracle
+    oracle.build()
+    npos = max(1, int(round(w.canvas * frac)))
+    rows = max(1, int(round(w.rows * frac)))
+    pos = np.linspace(0, w.canvas - 1, npos).astype(np.int32)
+    sel = np.linspace(0, w.rows - 1, rows).astype(np.int64)
+    q, kc, vc, kp, vp = (s[k].cpu() for k in ("q", "kc", "vc", "kp", "vp"))
+    lg = s["logits"].cpu()
+    t0 = time.perf_counter()
+    oracle.canvas_attn(q, kc, vc, kp, vp, s["cu_host"], w.scale, positions=pos)
+    t1 = time.perf_counter()
+    oracle.sample_renoise(lg, w.temperatures[0], w.rates[0], w.seed, 0, rows=sel)
+    t2 = time.perf_counter()
+    step_s = (t1 - t0) * (w.canvas / npos) + (t2 - t1) * (w.rows / rows)
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    return {"value": w.batch / step_s, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{npos}/{w.canvas} canvas positions (all heads) for attention and "
+                      f"{rows}/{w.rows} sampler rows of one step, float64, scaled to a step",
+            "seconds": t2 - t0}
+
+
+def run_reference(args, w, dist, rank, world):
+    """The reference arm: the oracle timed on host cores, each step a bounded
+    sample of the workload scaled to a whole step."""
+    if rank != 0:
+        return None
+    import oracle
+    oracle.build()
+    frac = args.ref_sample
+    s = {}
+    ws0 = workloads.scaled(w)
+    s["q"], s["kc"], s["vc"] = workloads.canvas_qkv(ws0, 0)
+    s["kp"], s["vp"], cu = workloads.prefix_kv(ws0)
+    s["cu_host"] = cu.numpy()
+    lg = workloads.logits(ws0, 0)
+    # size the per-step sample so the whole run stays within ~2 minutes
+    budget = 120.0 / (args.warmup + args.steps)
+    t0 = time.perf_counter()
+    oracle.canvas_attn(s["q"], s["kc"], s["vc"], s["kp"], s["vp"], s["cu_host"], w.scale,
+                       positions=np.arange(max(1, int(w.canvas * frac)), dtype=np.int32))
+    oracle.sample_renoise(lg, w.temperatures[0], w.rates[0], w.seed, 0,
+                          rows=np.arange(max(1, int(w.rows * frac))))
+    probe = time.perf_counter() - t0
+    if probe > budget:
+        frac = max(frac * budget / probe, 1.0 / w.canvas)
+    npos = max(1, int(round(w.canvas * frac)))
+    rows = max(1, int(round(w.rows * frac)))
+    times = []
+    for i in range(args.warmup + args.steps):
+        off = (i * 7) % w.canvas
+        pos = ((np.arange(npos) * (w.canvas // npos) + off) % w.canvas).astype(np.int32)
+        sel = ((np.arange(rows) * (w.rows // rows) + off) % w.rows).astype(np.int64)
+        t0 = time.perf_counter()
+        oracle.canvas_attn(s["q"], s["kc"], s["vc"], s["kp"], s["vp"], s["cu_host"], w.scale,
+                           positions=pos)
+        t1 = time.perf_counter()
+        oracle.sample_renoise(lg, w.temperatures[0], w.rates[0], w.seed, i, rows=sel)
+        t2 = time.perf_counter()
+        if i >= args.warmup:
+            times.append((t1 - t0) * (w.canvas / npos) + (t2 - t1) * (w.rows / rows))
+    step_s = statistics.mean(times)
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    value = w.batch / step_s
+    sample = (f"{npos}/{w.canvas} canvas positions (all heads) and {rows}/{w.rows} sampler rows "
+              "per step, float64 oracle, scaled to a whole step")
+    return {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": w.name, "batch_per_gpu": w.batch, "canvas": w.canvas,
+                       "heads_q": w.heads_q, "heads_kv": w.heads_kv, "head_dim": w.head_dim,
+                       "prefix": list(w.prefix_lens), "vocab": w.vocab,
+                       "parallelism": "host cores (rank 0 only)"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="b1_L4096", choices=list(workloads.WORKLOADS))
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--cpu-sample", type=float, default=0.125)
+    ap.add_argument("--ref-sample", type=float, default=1.0 / 32)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    w = workloads.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        res = run_reference(args, w, None, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    from block_discrete_diffusion_dd_b200 import build as libbuild
+    if not os.path.exists(libbuild.LIB):
+        libbuild.build()
+    dist, rank, world, local_rank = _dist()
+    if world != args.gpus and rank == 0:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
+    res = run_ours(args, w, dist, rank, world, local_rank)
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

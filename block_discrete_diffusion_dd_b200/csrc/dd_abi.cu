@@ -92,8 +92,9 @@ size_t attn_ws_bytes(const AttnArgs& a) {
   return kHeaderBytes + attn_simt_scratch_bytes(t);
 }
 
-size_t sample_ws_bytes(int rows, int vocab) {
-  return kHeaderBytes + (size_t)rows * (size_t)sampler_nchunk(vocab) * sizeof(ChunkRecord);
+size_t sample_ws_bytes(int rows, int vocab, dd_dtype dtype) {
+  return kHeaderBytes +
+         (size_t)rows * (size_t)sampler_nchunk(vocab, dtype == DD_BF16) * sizeof(ChunkRecord);
 }
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -104,7 +105,7 @@ size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 size_t block_ws_layout(const dd_attn_desc* desc, int64_t total, const int32_t* cu_prefix_host,
                        int vocab, size_t* conf_off) {
   const size_t a = attn_ws_bytes(make_attn_args(desc, total, cu_prefix_host));
-  const size_t s = sample_ws_bytes(desc->batch * desc->canvas, vocab);
+  const size_t s = sample_ws_bytes(desc->batch * desc->canvas, vocab, desc->dtype);
   const size_t shared = align256(a > s ? a : s);
   if (conf_off) *conf_off = shared;
   return shared + align256((size_t)desc->batch * desc->canvas * sizeof(float));
@@ -157,8 +158,8 @@ dd_status run_sampler(const void* logits, dd_dtype dtype, int rows, int vocab, i
   if (row_stride < vocab)
     return fail(DD_ERR_INVALID_ARG, "row_stride (%lld) < vocab (%d)", (long long)row_stride,
                 vocab);
-  if (!std::isfinite(p->temperature) || p->temperature <= 0.f)
-    return fail(DD_ERR_INVALID_ARG, "temperature must be finite and > 0");
+  if (!std::isfinite(p->temperature) || p->temperature < 1e-3f)
+    return fail(DD_ERR_INVALID_ARG, "temperature must be finite and >= 1e-3");
   if (!(p->renoise_rate >= 0.f && p->renoise_rate <= 1.f))
     return fail(DD_ERR_INVALID_ARG, "renoise_rate must lie in [0, 1]");
   if ((uint64_t)rows + p->row_offset > (1ull << 32))
@@ -167,10 +168,10 @@ dd_status run_sampler(const void* logits, dd_dtype dtype, int rows, int vocab, i
   if (!logits || !tokens || !conf) return fail(DD_ERR_INVALID_ARG, "NULL required pointer");
   if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u))
     return fail(DD_ERR_WORKSPACE, "workspace must be non-NULL and 256-byte aligned");
-  const size_t need = sample_ws_bytes(rows, vocab);
+  const size_t need = sample_ws_bytes(rows, vocab, dtype);
   if (ws_bytes < need)
     return fail(DD_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", ws_bytes, need);
-  if ((int64_t)rows * sampler_nchunk(vocab) > INT32_MAX)
+  if ((int64_t)rows * sampler_nchunk(vocab, dtype == DD_BF16) > INT32_MAX)
     return fail(DD_ERR_UNSUPPORTED, "rows * chunks exceeds 2^31");
   SamplerArgs a{};
   a.logits = logits;
@@ -189,6 +190,7 @@ dd_status run_sampler(const void* logits, dd_dtype dtype, int rows, int vocab, i
   a.entropy = entropy;
   a.renoised = renoised;
   a.recs = reinterpret_cast<ChunkRecord*>(static_cast<uint8_t*>(ws) + kHeaderBytes);
+  a.err = static_cast<uint32_t*>(ws);
   cudaError_t e = launch_sampler(a, stream);
   if (e != cudaSuccess) return cuda_fail(e, "sampler");
   return DD_OK;
@@ -221,7 +223,7 @@ dd_status dd_canvas_attn(const dd_attn_desc* desc, const void* q, const void* k_
 
 size_t dd_sample_renoise_workspace(int rows, int vocab, dd_dtype dtype) {
   if (rows < 0 || vocab < 1 || (dtype != DD_BF16 && dtype != DD_F32)) return 0;
-  return sample_ws_bytes(rows, vocab);
+  return sample_ws_bytes(rows, vocab, dtype);
 }
 
 dd_status dd_sample_renoise(const void* logits, dd_dtype dtype, int rows, int vocab,

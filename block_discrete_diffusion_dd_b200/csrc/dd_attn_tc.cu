@@ -276,18 +276,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       float sv[BN];
+      {
+        uint32_t raw[BN];
+        tmem_ld128(tmem + lane_base + (uint32_t)(st * BN), raw);
 #pragma unroll
-      for (int c4 = 0; c4 < BN / 32; ++c4) {
-        uint32_t raw[32];
-        tmem_ld32(tmem + lane_base + (uint32_t)(st * BN + c4 * 32), raw);
-#pragma unroll
-        for (int c = 0; c < 32; ++c) sv[c4 * 32 + c] = __uint_as_float(raw[c]);
+        for (int c = 0; c < BN; ++c) sv[c] = __uint_as_float(raw[c]);
       }
       float mx = -INFINITY;
+      if (n_valid == BN) {
 #pragma unroll
-      for (int c = 0; c < BN; ++c) {
-        if (c >= n_valid) sv[c] = -INFINITY;
-        mx = fmaxf(mx, sv[c]);
+        for (int c = 0; c < BN; ++c) mx = fmaxf(mx, sv[c]);
+      } else {  // ragged last tile of the prefix or of the canvas
+#pragma unroll
+        for (int c = 0; c < BN; ++c) {
+          if (c >= n_valid) sv[c] = -INFINITY;
+          mx = fmaxf(mx, sv[c]);
+        }
       }
       mx *= p.scale_log2;
       // P buffer st was last read by PV_{j-2}
@@ -383,13 +387,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // Merge the splits of every (b, g, t) query tile: lse = log2 sum 2^lse_s,
-// O = sum_s 2^(lse_s - lse) O_s.  One warp per query row.
+// O = sum_s 2^(lse_s - lse) O_s.  One warp per query row (8 rows per CTA,
+// 16 CTAs per 128-row tile); lane s holds split s's weight.
+constexpr int kCombineRowsPerCta = 8;
+
 template <typename TOut>
 __global__ void __launch_bounds__(256)
     attn_combine_kernel(const TcParams p, int total_units, TOut* __restrict__ out,
                         float* __restrict__ lse_out) {
   const int nc = cdiv(p.C, BN);
-  int q = blockIdx.x;  // (b, g, t) group
+  constexpr int kBlocksPerTile = BM / kCombineRowsPerCta;
+  int q = blockIdx.x / kBlocksPerTile;  // (b, g, t) group
+  const int rbase = (blockIdx.x % kBlocksPerTile) * kCombineRowsPerCta;
   int b = -1, nsplit = 0, ubase = 0;
   for (int bb = 0; bb < p.B; ++bb) {
     const int L = p.cu_prefix[bb + 1] - p.cu_prefix[bb];
@@ -411,39 +420,51 @@ __global__ void __launch_bounds__(256)
     return;
   }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int M = p.C * p.group;
-  for (int r = warp; r < BM; r += 8) {
-    const int pr = t * BM + r;
-    if (pr >= M) break;
-    float mx = -INFINITY;
-    for (int s = 0; s < nsplit; ++s) mx = fmaxf(mx, p.part_lse[(size_t)(u0 + s) * BM + r]);
-    float wsum = 0.f;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s = 0; s < nsplit; ++s) {
-      const float w = exp2f(p.part_lse[(size_t)(u0 + s) * BM + r] - mx);
-      wsum += w;
-      const float4 o =
-          *reinterpret_cast<const float4*>(p.part_o + ((size_t)(u0 + s) * BM + r) * HD + lane * 4);
+  const int r = rbase + warp;
+  const int pr = t * BM + r;
+  if (pr >= p.C * p.group) return;
+  // split weights, 32 splits per pass
+  float mx = -INFINITY;
+  for (int s0 = 0; s0 < nsplit; s0 += 32) {
+    const int s = s0 + lane;
+    if (s < nsplit) mx = fmaxf(mx, p.part_lse[(size_t)(u0 + s) * BM + r]);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  float wsum = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s0 = 0; s0 < nsplit; s0 += 32) {
+    const int s = s0 + lane;
+    const float wl = s < nsplit ? exp2f(p.part_lse[(size_t)(u0 + s) * BM + r] - mx) : 0.f;
+    float ws = wl;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) ws += __shfl_xor_sync(0xffffffffu, ws, off);
+    wsum += ws;
+    const int n = min(32, nsplit - s0);
+    for (int j = 0; j < n; ++j) {
+      const float w = __shfl_sync(0xffffffffu, wl, j);
+      const float4 o = *reinterpret_cast<const float4*>(
+          p.part_o + ((size_t)(u0 + s0 + j) * BM + r) * HD + lane * 4);
       acc.x = fmaf(w, o.x, acc.x);
       acc.y = fmaf(w, o.y, acc.y);
       acc.z = fmaf(w, o.z, acc.z);
       acc.w = fmaf(w, o.w, acc.w);
     }
-    const float inv = 1.f / wsum;
-    const int i = pr / p.group, h = g * p.group + (pr - i * p.group);
-    TOut* orow = out + (((size_t)b * p.C + i) * p.Hq + h) * HD + lane * 4;
-    if constexpr (sizeof(TOut) == 2) {
-      uint2 v;
-      v.x = pack_bf16x2(acc.x * inv, acc.y * inv);
-      v.y = pack_bf16x2(acc.z * inv, acc.w * inv);
-      *reinterpret_cast<uint2*>(orow) = v;
-    } else {
-      *reinterpret_cast<float4*>(orow) =
-          make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-    }
-    if (lse_out && lane == 0)
-      lse_out[((size_t)b * p.Hq + h) * p.C + i] = (mx + __log2f(wsum)) * 0.6931471805599453f;
   }
+  const float inv = 1.f / wsum;
+  const int i = pr / p.group, h = g * p.group + (pr - i * p.group);
+  TOut* orow = out + (((size_t)b * p.C + i) * p.Hq + h) * HD + lane * 4;
+  if constexpr (sizeof(TOut) == 2) {
+    uint2 v;
+    v.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+    v.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+    *reinterpret_cast<uint2*>(orow) = v;
+  } else {
+    *reinterpret_cast<float4*>(orow) =
+        make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+  }
+  if (lse_out && lane == 0)
+    lse_out[((size_t)b * p.Hq + h) * p.C + i] = (mx + __log2f(wsum)) * 0.6931471805599453f;
 }
 
 // ----------------------------------------------------------------- host
@@ -594,7 +615,7 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t stream) {
   note_launch();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  attn_combine_kernel<__nv_bfloat16><<<pl.groups, 256, 0, stream>>>(
+  attn_combine_kernel<__nv_bfloat16><<<pl.groups * (BM / kCombineRowsPerCta), 256, 0, stream>>>(
       tp, pl.units, static_cast<__nv_bfloat16*>(a.out), a.lse);
   note_launch();
   return cudaGetLastError();

@@ -30,9 +30,10 @@ struct SamplerArgs {
   float* entropy;
   uint8_t* renoised;
   ChunkRecord* recs;
+  uint32_t* err;  // device error word
 };
 
-int sampler_nchunk(int vocab);
+int sampler_nchunk(int vocab, bool bf16);
 cudaError_t launch_sampler(const SamplerArgs& a, cudaStream_t stream);
 cudaError_t launch_init_canvas(int32_t* canvas, int rows, int vocab, uint64_t seed,
                                uint32_t row_offset, cudaStream_t stream);

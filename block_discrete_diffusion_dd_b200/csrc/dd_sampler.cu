@@ -19,8 +19,6 @@ namespace dd {
 namespace {
 
 constexpr int kSampleThreads = 256;
-constexpr int kItemsPerThread = 4;  // 8 logits per item
-constexpr int kChunk = kSampleThreads * kItemsPerThread * 8;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -84,137 +82,161 @@ __device__ __forceinline__ void warp_merge(SampState& s) {
   }
 }
 
-// Loads of 8 consecutive logits as fp32.
-template <typename T, bool kVec>
-struct Load8;
+// Exact Gumbel score z - ln(-ln U) in fp32.  -ln U is taken as
+// -log1p(-(1 - U)) for U >= 1/2, where 1 - U is exact, so it stays accurate
+// as U approaches 1.
+__device__ __forceinline__ float gumbel_score(float z, uint32_t w) {
+  const float U = uniform24(w);
+  const float lnU = U < 0.5f ? logf(U) : log1pf(-(1.0f - U));
+  return z - logf(-lnU);
+}
 
-template <>
-struct Load8<__nv_bfloat16, true> {
-  uint4 raw;
-  __device__ __forceinline__ void issue(const __nv_bfloat16* p, int64_t, int64_t) {
-    raw = __ldcs(reinterpret_cast<const uint4*>(p));
-  }
-  __device__ __forceinline__ void get(float (&x)[8]) const {
-    x[0] = bf16lo(raw.x); x[1] = bf16hi(raw.x);
-    x[2] = bf16lo(raw.y); x[3] = bf16hi(raw.y);
-    x[4] = bf16lo(raw.z); x[5] = bf16hi(raw.z);
-    x[6] = bf16lo(raw.w); x[7] = bf16hi(raw.w);
-  }
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+  return v;
+}
+
+// Logits below this are treated as this value (exp underflows to 0 either
+// way); it keeps -inf entries and padding out of 0 * inf products.
+constexpr float kFloorLogit = -1e30f;
+
+// Per-thread running state (log2 units for the softmax sums; packed pairs
+// so that two entries update with one f32x2 instruction).
+struct Run {
+  float m;
+  float2 s2, t2;
+  float best;
+  int idx;
 };
 
-template <>
-struct Load8<float, true> {
-  float4 a, b;
-  __device__ __forceinline__ void issue(const float* p, int64_t, int64_t) {
-    a = __ldcs(reinterpret_cast<const float4*>(p));
-    b = __ldcs(reinterpret_cast<const float4*>(p) + 1);
+// One item = 8 consecutive vocabulary entries x[0..7] starting at v0 (all
+// finite: -inf and padding arrive as kFloorLogit); bm = max of x.
+// best_w is the warp-wide running best Gumbel score; `seed` marks the first
+// item, where the threshold is seeded with the exact score of each lane's
+// largest entry.  Control flow is warp-uniform apart from the rare exact
+// path, so the shuffles inside are safe.
+__device__ __forceinline__ void process8(Run& st, float& best_w, const float (&x)[8], float bm,
+                                         int64_t v0, bool seed, const PhiloxKey& key,
+                                         uint32_t grow, uint32_t step, float c2, float inv_tau) {
+  const float ym = bm * c2;
+  if (ym > st.m) {
+    const float s = st.s2.x + st.s2.y, t = st.t2.x + st.t2.y;
+    if (s > 0.f) {
+      const float f = ex2_approx(st.m - ym);
+      st.t2 = make_float2(f * fmaf(s, st.m - ym, t), 0.f);
+      st.s2 = make_float2(s * f, 0.f);
+    }
+    st.m = ym;
   }
-  __device__ __forceinline__ void get(float (&x)[8]) const {
-    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
-    x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+  const float2 c22 = make_float2(c2, c2);
+  const float2 nm = make_float2(-st.m, -st.m);
+  float p[8];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float2 d = __ffma2_rn(make_float2(x[2 * j], x[2 * j + 1]), c22, nm);
+    p[2 * j] = ex2_approx(d.x);
+    p[2 * j + 1] = ex2_approx(d.y);
+    const float2 pp = make_float2(p[2 * j], p[2 * j + 1]);
+    st.s2 = __fadd2_rn(st.s2, pp);
+    st.t2 = __ffma2_rn(pp, d, st.t2);
   }
-};
-
-// Scalar path for unaligned rows or a vocabulary that is not a multiple of
-// 8: entries at or beyond `vocab` read as -inf and never win.
-template <typename T>
-struct Load8<T, false> {
-  float v[8];
-  __device__ __forceinline__ void issue(const T* p, int64_t v0, int64_t vocab) {
+  // Gumbel words for the 8 entries: two Philox blocks.
+  const uint32_t q0 = (uint32_t)(v0 >> 2);
+  const uint4 wa = philox4x32_10(make_uint4(q0, grow, step, 0u), key);
+  const uint4 wb = philox4x32_10(make_uint4(q0 + 1u, grow, step, 0u), key);
+  const uint32_t w[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+  if (seed) {
+    if (bm > kFloorLogit) {
+      int j = 7;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = (v0 + i < vocab) ? (float)p[i] : -INFINITY;
-  }
-  __device__ __forceinline__ void get(float (&x)[8]) const {
+      for (int i = 6; i >= 0; --i) j = (x[i] == bm) ? i : j;
+      float xj = x[0];
+      uint32_t wj = w[0];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) x[i] = v[i];
-  }
-};
-
-template <typename T, bool kVec>
-__global__ void __launch_bounds__(kSampleThreads)
-    sample_chunk_kernel(const T* __restrict__ logits, int64_t row_stride, int vocab, int nchunk,
-                        float inv_tau, uint64_t seed, uint32_t step, uint32_t row_offset,
-                        ChunkRecord* __restrict__ recs) {
-  const int row = blockIdx.x / nchunk;
-  const int chunk = blockIdx.x - row * nchunk;
-  const T* rowp = logits + (int64_t)row * row_stride;
-  const int64_t c0 = (int64_t)chunk * kChunk;
-
-  Load8<T, kVec> ld[kItemsPerThread];
-  int64_t vbase[kItemsPerThread];
-#pragma unroll
-  for (int k = 0; k < kItemsPerThread; ++k) {
-    vbase[k] = c0 + (int64_t)(k * kSampleThreads + threadIdx.x) * 8;
-    if (vbase[k] < vocab) ld[k].issue(rowp + vbase[k], vbase[k], vocab);
-  }
-
-  const PhiloxKey key = philox_key(seed);
-  const uint32_t grow = row_offset + (uint32_t)row;
-  const float c2 = inv_tau * kLog2e;
-
-  SampState st{-INFINITY, 0.f, 0.f, -INFINITY, 0x7fffffff};
-  float Kp = 1e30f;  // (1 + 2^-8) e^(m ln 2 - best), clamped
-
-#pragma unroll
-  for (int k = 0; k < kItemsPerThread; ++k) {
-    if (vbase[k] >= vocab) continue;
-    float x[8];
-    ld[k].get(x);
-    float bm = x[0];
-#pragma unroll
-    for (int i = 1; i < 8; ++i) bm = fmaxf(bm, x[i]);
-    const float ym = bm * c2;
-    if (ym > st.m) {
-      if (st.s > 0.f) {
-        const float f = ex2_approx(st.m - ym);
-        st.t = f * fmaf(st.s, st.m - ym, st.t);
-        st.s *= f;
+      for (int i = 1; i < 8; ++i) {
+        xj = (j == i) ? x[i] : xj;
+        wj = (j == i) ? w[i] : wj;
       }
-      st.m = ym;
-      Kp = fminf(ex2_approx(st.m - st.best * kLog2e) * 1.00390625f, 1e30f);
+      const float sc = gumbel_score(xj * inv_tau, wj);
+      if (sc > st.best) {
+        st.best = sc;
+        st.idx = (int)(v0 + j);
+      }
     }
-    float p[8];
+    best_w = warp_max(st.best);
+  }
+  // Exponential-race prune: the score z - ln E (E = -ln U) can beat best_w
+  // only if E < e^(z - best_w); since E >= 1 - U, an entry with
+  // 1 - U >= e^(z - best_w) (1 + 2^-8) is skipped without a logarithm.  With
+  // U' = 1 + (x >> 9) 2^-23 = U + 1 - 2^-24 the test reads
+  // U' > 2 - 2^-23 - p Kp,  Kp = (1 + 2^-8) e^(m ln 2 - best_w).
+  const float Kp = fminf(ex2_approx(st.m - best_w * kLog2e) * 1.00390625f, 1e30f);
+  const float2 kk = make_float2(-Kp, -Kp);
+  const float2 cc = make_float2(1.99999988079071044921875f, 1.99999988079071044921875f);
+  float thr[8];
+  bool any = false;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float2 t = __ffma2_rn(make_float2(p[2 * j], p[2 * j + 1]), kk, cc);
+    thr[2 * j] = t.x;
+    thr[2 * j + 1] = t.y;
+    any |= __uint_as_float(0x3F800000u | (w[2 * j] >> 9)) > t.x;
+    any |= __uint_as_float(0x3F800000u | (w[2 * j + 1] >> 9)) > t.y;
+  }
+  if (any) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const float d = fmaf(x[i], c2, -st.m);
-      p[i] = ex2_approx(d);
-      st.s += p[i];
-      st.t = fmaf(p[i], d, st.t);
-    }
-    // Gumbel words for the 8 entries: two Philox blocks.
-    const uint32_t q0 = (uint32_t)(vbase[k] >> 2);
-    const uint4 wa = philox4x32_10(make_uint4(q0, grow, step, 0u), key);
-    const uint4 wb = philox4x32_10(make_uint4(q0 + 1u, grow, step, 0u), key);
-    const uint32_t w[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
-    // Exponential-race prune: the score z - ln E (E = -ln U) can only beat
-    // `best` if E < e^(z - best); since E >= 1 - U, entries with
-    // 1 - U >= e^(z - best) are skipped without any logarithm.  The test is
-    // U' > 2 - 2^-23 - p Kp with U' = 1 + (x >> 9) 2^-23 (conservative).
-    bool any = false;
-    float thr[8], f[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      f[i] = __uint_as_float(0x3F800000u | (w[i] >> 9));
-      thr[i] = fmaf(-p[i], Kp, 1.99999988079071044921875f);
-      any |= f[i] > thr[i];
-    }
-    if (any) {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        if (f[i] > thr[i] && x[i] != -INFINITY) {
-          const float U = uniform24(w[i]);
-          const float E = -logf(U);
-          const float sc = x[i] * inv_tau - logf(E);
-          if (sc > st.best) {
-            st.best = sc;
-            st.idx = (int)(vbase[k] + i);
-          }
+      if (__uint_as_float(0x3F800000u | (w[i] >> 9)) > thr[i]) {
+        const float sc = gumbel_score(x[i] * inv_tau, w[i]);
+        const int v = (int)(v0 + i);
+        if (sc > st.best || (sc == st.best && v < st.idx)) {
+          st.best = sc;
+          st.idx = v;
         }
       }
-      Kp = fminf(ex2_approx(st.m - st.best * kLog2e) * 1.00390625f, 1e30f);
     }
   }
+  best_w = warp_max(st.best);
+}
 
+// bf16 pairs in a 32-bit word, floored at kFloorLogit (max.bf16x2 is exact).
+__device__ __forceinline__ uint32_t floor_bf16x2(uint32_t w) {
+  uint32_t r;
+  // 0xF149 is the bf16 value -9.96e29 (>= kFloorLogit after widening)
+  asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(w), "r"(0xF149F149u));
+  return r;
+}
+__device__ __forceinline__ uint32_t max_bf16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+__device__ __forceinline__ void unpack8(uint4 raw, float (&x)[8], float& bm) {
+  raw.x = floor_bf16x2(raw.x);
+  raw.y = floor_bf16x2(raw.y);
+  raw.z = floor_bf16x2(raw.z);
+  raw.w = floor_bf16x2(raw.w);
+  const uint32_t mx = max_bf16x2(max_bf16x2(raw.x, raw.y), max_bf16x2(raw.z, raw.w));
+  bm = fmaxf(bf16lo(mx), bf16hi(mx));
+  x[0] = bf16lo(raw.x); x[1] = bf16hi(raw.x);
+  x[2] = bf16lo(raw.y); x[3] = bf16hi(raw.y);
+  x[4] = bf16lo(raw.z); x[5] = bf16hi(raw.z);
+  x[6] = bf16lo(raw.w); x[7] = bf16hi(raw.w);
+}
+
+__device__ __forceinline__ void unpack8(float4 a, float4 b, float (&x)[8], float& bm) {
+  x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+  x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) x[i] = fmaxf(x[i], kFloorLogit);
+  bm = fmaxf(fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3])), fmaxf(fmaxf(x[4], x[5]), fmaxf(x[6], x[7])));
+}
+
+// Reduce the CTA's states and write its chunk record.
+__device__ __forceinline__ void write_record(const Run& r, ChunkRecord* rec) {
+  SampState st{r.m, r.s2.x + r.s2.y, r.t2.x + r.t2.y, r.best, r.idx};
   warp_merge(st);
   __shared__ SampState red[kSampleThreads / 32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -226,15 +248,111 @@ __global__ void __launch_bounds__(kSampleThreads)
                       : SampState{-INFINITY, 0.f, 0.f, -INFINITY, 0x7fffffff};
     warp_merge(s);
     if (lane == 0) {
-      ChunkRecord r;
-      r.m = s.m;
-      r.s = s.s;
-      r.t = s.t;
-      r.best = s.best;
-      r.idx = s.idx;
-      recs[(int64_t)row * nchunk + chunk] = r;
+      ChunkRecord out;
+      out.m = s.m;
+      out.s = s.s;
+      out.t = s.t;
+      out.best = s.best;
+      out.idx = s.idx;
+      *rec = out;
     }
   }
+}
+
+constexpr uint32_t kStageBytes = 32768;  // logits per CTA (one bulk copy)
+
+template <typename T>
+constexpr int chunk_elems() { return (int)(kStageBytes / sizeof(T)); }
+
+// Vector path: rows 16-byte aligned and V % 8 == 0.  Thread 0 fetches the
+// CTA's 32 KB slice of the row with one bulk asynchronous copy into shared
+// memory; all 256 threads then stream it 8 entries at a time.
+template <typename T>
+__global__ void __launch_bounds__(kSampleThreads, 4)
+    sample_chunk_bulk_kernel(const T* __restrict__ logits, int64_t row_stride, int vocab,
+                             int nchunk, float inv_tau, uint64_t seed, uint32_t step,
+                             uint32_t row_offset, ChunkRecord* __restrict__ recs,
+                             uint32_t* __restrict__ err) {
+  constexpr int kElems = chunk_elems<T>();
+  constexpr int kItems = kElems / (kSampleThreads * 8);
+  __shared__ __align__(128) uint8_t buf[kStageBytes];
+  __shared__ uint64_t bar;
+  const int row = blockIdx.x / nchunk;
+  const int chunk = blockIdx.x - row * nchunk;
+  const int64_t c0 = (int64_t)chunk * kElems;
+  const int n = (int)min((int64_t)kElems, (int64_t)vocab - c0);
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(&bar, (uint32_t)(n * sizeof(T)));
+    bulk_load(buf, logits + (int64_t)row * row_stride + c0, (uint32_t)(n * sizeof(T)), &bar);
+  }
+  const PhiloxKey key = philox_key(seed);
+  const uint32_t grow = row_offset + (uint32_t)row;
+  const float c2 = inv_tau * kLog2e;
+  Run st{-INFINITY, make_float2(0.f, 0.f), make_float2(0.f, 0.f), -INFINITY, 0x7fffffff};
+  float best_w = -INFINITY;
+  if (!mbar_wait_bounded(&bar, 0, nullptr, 1000000000ull)) {
+    // never observed: the copy is plain memory traffic; report and drain
+    if (threadIdx.x == 0) atomicOr(err, kDevErrTimeout);
+    mbar_wait_bounded(&bar, 0, nullptr, 4000000000ull);
+    return;
+  }
+#pragma unroll 1
+  for (int k = 0; k < kItems; ++k) {
+    const int e = (k * kSampleThreads + threadIdx.x) * 8;
+    float x[8], bm;
+    if (e < n) {
+      if constexpr (sizeof(T) == 2) {
+        unpack8(*reinterpret_cast<const uint4*>(buf + e * 2), x, bm);
+      } else {
+        const float4* q = reinterpret_cast<const float4*>(buf + e * 4);
+        unpack8(q[0], q[1], x, bm);
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) x[i] = kFloorLogit;
+      bm = kFloorLogit;
+    }
+    process8(st, best_w, x, bm, c0 + e, k == 0, key, grow, step, c2, inv_tau);
+  }
+  write_record(st, recs + (int64_t)row * nchunk + chunk);
+}
+
+// Scalar path for unaligned rows or V % 8 != 0: direct loads with bounds
+// checks; entries at or beyond V read as kFloorLogit and never win.
+template <typename T>
+__global__ void __launch_bounds__(kSampleThreads)
+    sample_chunk_scalar_kernel(const T* __restrict__ logits, int64_t row_stride, int vocab,
+                               int nchunk, float inv_tau, uint64_t seed, uint32_t step,
+                               uint32_t row_offset, ChunkRecord* __restrict__ recs) {
+  constexpr int kElems = chunk_elems<T>();
+  constexpr int kItems = kElems / (kSampleThreads * 8);
+  const int row = blockIdx.x / nchunk;
+  const int chunk = blockIdx.x - row * nchunk;
+  const int64_t c0 = (int64_t)chunk * kElems;
+  const T* rowp = logits + (int64_t)row * row_stride;
+  const PhiloxKey key = philox_key(seed);
+  const uint32_t grow = row_offset + (uint32_t)row;
+  const float c2 = inv_tau * kLog2e;
+  Run st{-INFINITY, make_float2(0.f, 0.f), make_float2(0.f, 0.f), -INFINITY, 0x7fffffff};
+  float best_w = -INFINITY;
+#pragma unroll 1
+  for (int k = 0; k < kItems; ++k) {
+    const int64_t v0 = c0 + (int64_t)(k * kSampleThreads + threadIdx.x) * 8;
+    float x[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      x[i] = (v0 + i < vocab) ? fmaxf((float)rowp[v0 + i], kFloorLogit) : kFloorLogit;
+    float bm = x[0];
+#pragma unroll
+    for (int i = 1; i < 8; ++i) bm = fmaxf(bm, x[i]);
+    process8(st, best_w, x, bm, v0, k == 0, key, grow, step, c2, inv_tau);
+  }
+  write_record(st, recs + (int64_t)row * nchunk + chunk);
 }
 
 template <typename T>
@@ -283,17 +401,18 @@ __global__ void init_canvas_kernel(int32_t* __restrict__ canvas, int rows, int v
 
 template <typename T>
 cudaError_t launch_sampler_t(const SamplerArgs& a, cudaStream_t stream) {
-  const int nchunk = sampler_nchunk(a.vocab);
+  const int nchunk = (a.vocab + chunk_elems<T>() - 1) / chunk_elems<T>();
   const T* lg = static_cast<const T*>(a.logits);
   const size_t esz = sizeof(T);
   const bool vec = ((reinterpret_cast<uintptr_t>(lg) & 15u) == 0) &&
                    (((size_t)a.row_stride * esz) % 16 == 0) && (a.vocab % 8 == 0);
   const int64_t grid = (int64_t)a.rows * nchunk;
   if (vec)
-    sample_chunk_kernel<T, true><<<(unsigned)grid, kSampleThreads, 0, stream>>>(
-        lg, a.row_stride, a.vocab, nchunk, a.inv_tau, a.seed, a.step, a.row_offset, a.recs);
+    sample_chunk_bulk_kernel<T><<<(unsigned)grid, kSampleThreads, 0, stream>>>(
+        lg, a.row_stride, a.vocab, nchunk, a.inv_tau, a.seed, a.step, a.row_offset, a.recs,
+        a.err);
   else
-    sample_chunk_kernel<T, false><<<(unsigned)grid, kSampleThreads, 0, stream>>>(
+    sample_chunk_scalar_kernel<T><<<(unsigned)grid, kSampleThreads, 0, stream>>>(
         lg, a.row_stride, a.vocab, nchunk, a.inv_tau, a.seed, a.step, a.row_offset, a.recs);
   note_launch();
   cudaError_t e = cudaGetLastError();
@@ -307,7 +426,10 @@ cudaError_t launch_sampler_t(const SamplerArgs& a, cudaStream_t stream) {
 
 }  // namespace
 
-int sampler_nchunk(int vocab) { return (vocab + kChunk - 1) / kChunk; }
+int sampler_nchunk(int vocab, bool bf16) {
+  const int ce = bf16 ? chunk_elems<__nv_bfloat16>() : chunk_elems<float>();
+  return (vocab + ce - 1) / ce;
+}
 
 cudaError_t launch_sampler(const SamplerArgs& a, cudaStream_t stream) {
   if (a.bf16) return launch_sampler_t<__nv_bfloat16>(a, stream);

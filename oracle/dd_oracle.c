@@ -263,7 +263,8 @@ int oracle_sample_renoise(const void* logits, int dtype, int64_t rows, int64_t v
       double ent = 0.0;
       for (int64_t v = 0; v < vocab; ++v) {
         const double lp = z[v] - lse;
-        ent -= exp(lp) * lp;
+        const double p = exp(lp);
+        if (p > 0.0) ent -= p * lp; /* 0 ln 0 = 0 (entries with logit -inf) */
       }
 
       /* re-noise */
