@@ -9,26 +9,28 @@
 // they all see the same key range [prefix_b || canvas_b] under one unmasked
 // softmax.
 //
-// Work unit (one CTA): (b, g, 128-row query tile t, split s of the key
-// tiles).  The key range of b is cut into 128-key tiles -- prefix tiles
+// Work unit (one CTA): (b, g, pair of 128-row query tiles, split s of the
+// key tiles).  The key range of b is cut into 64-key tiles -- prefix tiles
 // first, then canvas tiles, each read through its own tensor map so a tile
 // never straddles the prefix/canvas boundary; the last tile of each part is
-// masked by key index.  Splits are balanced on the host so that one wave of
-// CTAs covers the SMs; a second kernel merges the splits by their
+// masked by key index.  Splits are balanced on the host so that whole waves
+// of CTAs cover the SMs; a second kernel merges the splits by their
 // log-sum-exp.
 //
-// Inside a CTA (7 warps):
-//   warps 0-3  softmax: one query row per thread (= one TMEM lane); read S
-//              from TMEM, online softmax in fp32 (log2 domain, lazy rescale
-//              of O only when the running max grows by more than 2^8), write
-//              P as bf16 into shared memory in the 128B-swizzled K-major
-//              layout the MMA reads;
-//   warp 4     TMA producer for Q and K (2-stage ring);
-//   warp 5     TMA producer for V (2-stage ring);
-//   warp 6     allocates 512 TMEM columns (S double buffer + O) and issues
-//              the MMAs from one thread: S_j = Q K_j^T into S[j%2], then
-//              O += P_{j-1} V_{j-1}, so the tensor core works on tile j while
-//              the softmax warps work on tile j-1.
+// Inside a CTA (11 warps) two 128-row query tiles share every key tile:
+//   warps 0-3  softmax for query tile 0, warps 4-7 for query tile 1: one
+//              query row per thread (= one TMEM lane); read S from TMEM,
+//              online softmax in fp32 (log2 domain; O is rescaled only when
+//              the running max grows by more than 2^8), write P as bf16 into
+//              shared memory in the 128B-swizzled K-major layout the MMA
+//              reads;
+//   warp 8     TMA producer for Q and K (3-stage ring of 64-key tiles);
+//   warp 9     TMA producer for V (3-stage ring);
+//   warp 10    allocates 512 TMEM columns (per query tile: S double buffer
+//              of 64 columns and O of 128) and issues every MMA from one
+//              thread: S = Q K_j^T for both query tiles, then O += P V_{j-1},
+//              so the tensor core computes tile j while the softmax warps
+//              work on tile j-1.
 // Every mbarrier wait is bounded in time; on expiry the CTA latches an
 // error word, drains its own asynchronous work and frees its TMEM.
 #include <mutex>
@@ -40,69 +42,81 @@ namespace dd {
 namespace {
 
 constexpr int BM = 128;  // query rows per tile
-constexpr int BN = 128;  // keys per tile
+constexpr int BN = 64;   // keys per tile
 constexpr int HD = 128;  // head dim
-constexpr int kThreads = 7 * 32;
-constexpr int kWarpK = 4, kWarpV = 5, kWarpMMA = 6;
-constexpr uint32_t kHalfBytes = 128 * 64 * 2;    // 128 rows x 128 bytes
-constexpr uint32_t kTileBytes = 2 * kHalfBytes;  // 128 x 128 bf16
+constexpr int kQT = 2;   // query tiles per CTA
+constexpr int kStages = 3;
+constexpr int kWarpK = 8, kWarpV = 9, kWarpMMA = 10;
+constexpr int kThreads = 11 * 32;
+constexpr uint32_t kQHalf = BM * 64 * 2;      // 128 rows x 128 bytes
+constexpr uint32_t kQTile = 2 * kQHalf;       // 128 x 128 bf16
+constexpr uint32_t kKHalf = BN * 64 * 2;      // 64 rows x 128 bytes
+constexpr uint32_t kKTile = 2 * kKHalf;       // 64 x 128 bf16
+constexpr uint32_t kPTile = BM * BN * 2;      // 128 rows x 128 bytes
 constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffK = kTileBytes;
-constexpr uint32_t kOffV = 3 * kTileBytes;
-constexpr uint32_t kOffP = 5 * kTileBytes;
-constexpr uint32_t kOffBar = 7 * kTileBytes;
+constexpr uint32_t kOffK = kOffQ + kQT * kQTile;
+constexpr uint32_t kOffV = kOffK + kStages * kKTile;
+constexpr uint32_t kOffP = kOffV + kStages * kKTile;
+constexpr uint32_t kOffBar = kOffP + kQT * 2 * kPTile;
 constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemO = kQT * 2 * BN;     // O columns start after the S buffers
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per wait
 constexpr float kLazyRescale = 8.0f;              // log2 units
 
 struct Barriers {
   uint64_t q_full;
-  uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
-  uint64_t s_full[2], p_full[2], pv_done[2];
+  uint64_t k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
+  uint64_t s_full[kQT][2], p_full[kQT][2], pv_done[kQT][2];
   uint64_t mma_final;
   uint32_t tmem_base;
   int abort;
-  int unit_b, unit_g, unit_t, unit_s, unit_valid;
+  int unit_b, unit_g, unit_tp, unit_s, unit_valid, unit_nsplit, unit_slot0;
 };
 
 constexpr uint32_t kSmemBytes = kOffBar + sizeof(Barriers) + 1024;
+static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 struct TcParams {
   int B, C, Hq, Hkv, group, T, chunk;
   float scale_log2;
   const int32_t* cu_prefix;
-  float* part_o;    // [units][BM][HD]
-  float* part_lse;  // [units][BM]   log2 units
+  float* part_o;    // [slots][BM][HD], slot = (b, g, t, split)
+  float* part_lse;  // [slots][BM]   log2 units
   uint32_t* err;
 };
 
 __device__ __forceinline__ int cdiv(int a, int b) { return (a + b - 1) / b; }
 
-// Resolve blockIdx.x -> (b, g, t, s) by walking the batch rows.
+// blockIdx.x -> (b, g, query-tile pair tp, split s) by walking the batch
+// rows; slot0 = partial slot of (b, g, 2 tp, s).
 __device__ void resolve_unit(const TcParams& p, Barriers* bars) {
   int u = blockIdx.x;
   const int nc = cdiv(p.C, BN);
-  int valid = 0, b = 0, g = 0, t = 0, s = 0;
+  const int TP = cdiv(p.T, kQT);
+  int valid = 0, b = 0, g = 0, tp = 0, s = 0, nsplit = 1, slots = 0;
   for (int bb = 0; bb < p.B; ++bb) {
     const int L = p.cu_prefix[bb + 1] - p.cu_prefix[bb];
-    const int ntiles = cdiv(L, BN) + nc;
-    const int nsplit = cdiv(ntiles, p.chunk);
-    const int units = p.Hkv * p.T * nsplit;
+    const int ns = cdiv(cdiv(L, BN) + nc, p.chunk);
+    const int units = p.Hkv * TP * ns;
     if (u < units) {
-      s = u % nsplit;
-      t = (u / nsplit) % p.T;
-      g = u / (nsplit * p.T);
+      s = u % ns;
+      tp = (u / ns) % TP;
+      g = u / (ns * TP);
       b = bb;
+      nsplit = ns;
       valid = 1;
       break;
     }
     u -= units;
+    slots += p.Hkv * p.T * ns;
   }
   bars->unit_b = b;
   bars->unit_g = g;
-  bars->unit_t = t;
+  bars->unit_tp = tp;
   bars->unit_s = s;
   bars->unit_valid = valid;
+  bars->unit_nsplit = nsplit;
+  bars->unit_slot0 = slots + (g * p.T + tp * kQT) * nsplit + s;
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -120,15 +134,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kStages; ++i) {
       mbar_init(&bars->k_full[i], 1);
       mbar_init(&bars->k_empty[i], 1);
       mbar_init(&bars->v_full[i], 1);
       mbar_init(&bars->v_empty[i], 1);
-      mbar_init(&bars->s_full[i], 1);
-      mbar_init(&bars->p_full[i], 4);
-      mbar_init(&bars->pv_done[i], 1);
     }
+    for (int q = 0; q < kQT; ++q)
+      for (int i = 0; i < 2; ++i) {
+        mbar_init(&bars->s_full[q][i], 1);
+        mbar_init(&bars->p_full[q][i], 4);
+        mbar_init(&bars->pv_done[q][i], 1);
+      }
     mbar_init(&bars->mma_final, 1);
     bars->abort = 0;
     fence_mbar_init();
@@ -143,134 +160,162 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
 
   const uint32_t tmem = bars->tmem_base;
-  const int b = bars->unit_b, g = bars->unit_g, t = bars->unit_t, s = bars->unit_s;
+  const int b = bars->unit_b, g = bars->unit_g, tp = bars->unit_tp, s = bars->unit_s;
   const bool unit_ok = bars->unit_valid != 0;
+  const int nsplit = bars->unit_nsplit, slot0 = bars->unit_slot0;
   const int p0 = unit_ok ? p.cu_prefix[b] : 0;
   const int L = unit_ok ? p.cu_prefix[b + 1] - p0 : 0;
   const int np = cdiv(L, BN), nc = cdiv(p.C, BN);
   const int ntiles = np + nc;
   const int k_begin = s * p.chunk;
   const int n = unit_ok ? min(p.chunk, ntiles - k_begin) : 0;
+  const int nq = min(kQT, p.T - tp * kQT);  // query tiles in this CTA (1 or 2)
 
   if (warp == kWarpK) {
     if (lane == 0 && n > 0) {
-    prefetch_tensormap(&tmQ);
-    prefetch_tensormap(&tmKp);
-    prefetch_tensormap(&tmKc);
-    mbar_arrive_expect_tx(&bars->q_full, kTileBytes);
-    const int qpos = b * p.C + t * (BM / p.group);
-    tma_load_3d(smem + kOffQ, &tmQ, &bars->q_full, 0, g * p.group, qpos);
-    tma_load_3d(smem + kOffQ + kHalfBytes, &tmQ, &bars->q_full, 64, g * p.group, qpos);
-    int issued = 0;
-    for (int j = 0; j < n; ++j) {
-      const int st = j & 1, rd = j >> 1;
-      if (rd > 0 &&
-          !mbar_wait_bounded(&bars->k_empty[st], (rd - 1) & 1, abort_flag, kWaitLimitNs))
-        break;
-      const int k = k_begin + j;
-      const CUtensorMap* map = k < np ? &tmKp : &tmKc;
-      const int row0 = k < np ? p0 + k * BN : b * p.C + (k - np) * BN;
-      uint8_t* dst = smem + kOffK + st * kTileBytes;
-      mbar_arrive_expect_tx(&bars->k_full[st], kTileBytes);
-      tma_load_3d(dst, map, &bars->k_full[st], 0, g, row0);
-      tma_load_3d(dst + kHalfBytes, map, &bars->k_full[st], 64, g, row0);
-      issued = j + 1;
-    }
-    // drain: loads still in flight must land before the CTA exits
-    for (int j = max(0, issued - 2); j < issued; ++j)
-      mbar_wait_bounded(&bars->k_full[j & 1], (j >> 1) & 1, nullptr, kWaitLimitNs);
-    mbar_wait_bounded(&bars->q_full, 0, nullptr, kWaitLimitNs);
+      prefetch_tensormap(&tmQ);
+      prefetch_tensormap(&tmKp);
+      prefetch_tensormap(&tmKc);
+      mbar_arrive_expect_tx(&bars->q_full, nq * kQTile);
+      for (int q = 0; q < nq; ++q) {
+        const int qpos = b * p.C + (tp * kQT + q) * (BM / p.group);
+        uint8_t* dst = smem + kOffQ + q * kQTile;
+        tma_load_3d(dst, &tmQ, &bars->q_full, 0, g * p.group, qpos);
+        tma_load_3d(dst + kQHalf, &tmQ, &bars->q_full, 64, g * p.group, qpos);
+      }
+      int issued = 0;
+      for (int j = 0; j < n; ++j) {
+        const int st = j % kStages, rd = j / kStages;
+        if (rd > 0 &&
+            !mbar_wait_bounded(&bars->k_empty[st], (rd - 1) & 1, abort_flag, kWaitLimitNs))
+          break;
+        const int k = k_begin + j;
+        const CUtensorMap* map = k < np ? &tmKp : &tmKc;
+        const int row0 = k < np ? p0 + k * BN : b * p.C + (k - np) * BN;
+        uint8_t* dst = smem + kOffK + st * kKTile;
+        mbar_arrive_expect_tx(&bars->k_full[st], kKTile);
+        tma_load_3d(dst, map, &bars->k_full[st], 0, g, row0);
+        tma_load_3d(dst + kKHalf, map, &bars->k_full[st], 64, g, row0);
+        issued = j + 1;
+      }
+      // drain: loads still in flight must land before the CTA exits
+      for (int j = max(0, issued - kStages); j < issued; ++j)
+        mbar_wait_bounded(&bars->k_full[j % kStages], (j / kStages) & 1, nullptr, kWaitLimitNs);
+      mbar_wait_bounded(&bars->q_full, 0, nullptr, kWaitLimitNs);
     }
     __syncwarp();
   } else if (warp == kWarpV) {
     if (lane == 0 && n > 0) {
-    prefetch_tensormap(&tmVp);
-    prefetch_tensormap(&tmVc);
-    int issued = 0;
-    for (int j = 0; j < n; ++j) {
-      const int st = j & 1, rd = j >> 1;
-      if (rd > 0 &&
-          !mbar_wait_bounded(&bars->v_empty[st], (rd - 1) & 1, abort_flag, kWaitLimitNs))
-        break;
-      const int k = k_begin + j;
-      const CUtensorMap* map = k < np ? &tmVp : &tmVc;
-      const int row0 = k < np ? p0 + k * BN : b * p.C + (k - np) * BN;
-      uint8_t* dst = smem + kOffV + st * kTileBytes;
-      mbar_arrive_expect_tx(&bars->v_full[st], kTileBytes);
-      tma_load_3d(dst, map, &bars->v_full[st], 0, g, row0);
-      tma_load_3d(dst + kHalfBytes, map, &bars->v_full[st], 64, g, row0);
-      issued = j + 1;
-    }
-    for (int j = max(0, issued - 2); j < issued; ++j)
-      mbar_wait_bounded(&bars->v_full[j & 1], (j >> 1) & 1, nullptr, kWaitLimitNs);
+      prefetch_tensormap(&tmVp);
+      prefetch_tensormap(&tmVc);
+      int issued = 0;
+      for (int j = 0; j < n; ++j) {
+        const int st = j % kStages, rd = j / kStages;
+        if (rd > 0 &&
+            !mbar_wait_bounded(&bars->v_empty[st], (rd - 1) & 1, abort_flag, kWaitLimitNs))
+          break;
+        const int k = k_begin + j;
+        const CUtensorMap* map = k < np ? &tmVp : &tmVc;
+        const int row0 = k < np ? p0 + k * BN : b * p.C + (k - np) * BN;
+        uint8_t* dst = smem + kOffV + st * kKTile;
+        mbar_arrive_expect_tx(&bars->v_full[st], kKTile);
+        tma_load_3d(dst, map, &bars->v_full[st], 0, g, row0);
+        tma_load_3d(dst + kKHalf, map, &bars->v_full[st], 64, g, row0);
+        issued = j + 1;
+      }
+      for (int j = max(0, issued - kStages); j < issued; ++j)
+        mbar_wait_bounded(&bars->v_full[j % kStages], (j / kStages) & 1, nullptr, kWaitLimitNs);
     }
     __syncwarp();
   } else if (warp == kWarpMMA) {
     if (lane == 0 && n > 0) {
-    constexpr uint32_t idS = idesc_bf16_f32(BM, BN, 0, 0);
-    constexpr uint32_t idPV = idesc_bf16_f32(BM, HD, 0, 1);
-    const uint32_t sQ = smem_u32(smem + kOffQ);
-    const uint32_t sK = smem_u32(smem + kOffK);
-    const uint32_t sV = smem_u32(smem + kOffV);
-    const uint32_t sP = smem_u32(smem + kOffP);
-    bool ok = mbar_wait_bounded(&bars->q_full, 0, abort_flag, kWaitLimitNs);
-    tc_fence_after();
-    for (int j = 0; ok && j <= n; ++j) {
-      if (j < n) {
-        const int st = j & 1;
-        if (!mbar_wait_bounded(&bars->k_full[st], (j >> 1) & 1, abort_flag, kWaitLimitNs)) break;
-        if (j >= 2 &&
-            !mbar_wait_bounded(&bars->p_full[st], ((j - 2) >> 1) & 1, abort_flag, kWaitLimitNs))
-          break;
-        tc_fence_after();
-        const uint32_t dS = tmem + (uint32_t)(st * BN);
+      constexpr uint32_t idS = idesc_bf16_f32(BM, BN, 0, 0);
+      constexpr uint32_t idPV = idesc_bf16_f32(BM, HD, 0, 1);
+      const uint32_t sQ = smem_u32(smem + kOffQ);
+      const uint32_t sK = smem_u32(smem + kOffK);
+      const uint32_t sV = smem_u32(smem + kOffV);
+      const uint32_t sP = smem_u32(smem + kOffP);
+      bool ok = mbar_wait_bounded(&bars->q_full, 0, abort_flag, kWaitLimitNs);
+      tc_fence_after();
+      for (int j = 0; ok && j <= n; ++j) {
+        if (j < n) {
+          const int st = j % kStages, sb = j & 1;
+          if (!mbar_wait_bounded(&bars->k_full[st], (j / kStages) & 1, abort_flag,
+                                 kWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+          for (int q = 0; q < nq; ++q) {
+            // S buffer sb of query tile q was last read by the softmax of tile j-2
+            if (j >= 2 && !mbar_wait_bounded(&bars->p_full[q][sb], ((j - 2) >> 1) & 1,
+                                              abort_flag, kWaitLimitNs)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t dS = tmem + (uint32_t)((q * 2 + sb) * BN);
 #pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-          tc_mma_ss(dS, smem_desc_sw128(sQ + off, 16, 1024),
-                    smem_desc_sw128(sK + st * kTileBytes + off, 16, 1024), idS, kk > 0);
+            for (int kk = 0; kk < HD / 16; ++kk) {
+              const uint32_t offQ = q * kQTile + (kk >> 2) * kQHalf + (kk & 3) * 32;
+              const uint32_t offK = st * kKTile + (kk >> 2) * kKHalf + (kk & 3) * 32;
+              tc_mma_ss(dS, smem_desc_sw128(sQ + offQ, 16, 1024),
+                        smem_desc_sw128(sK + offK, 16, 1024), idS, kk > 0);
+            }
+            tc_commit(&bars->s_full[q][sb]);
+          }
+          if (!ok) break;
+          tc_commit(&bars->k_empty[st]);
         }
-        tc_commit(&bars->s_full[st]);
-        tc_commit(&bars->k_empty[st]);
-      }
-      if (j >= 1) {
-        const int jj = j - 1, st = jj & 1;
-        if (!mbar_wait_bounded(&bars->p_full[st], (jj >> 1) & 1, abort_flag, kWaitLimitNs)) break;
-        if (!mbar_wait_bounded(&bars->v_full[st], (jj >> 1) & 1, abort_flag, kWaitLimitNs)) break;
-        tc_fence_after();
-        const uint32_t dO = tmem + 2u * BN;
+        if (j >= 1) {
+          const int jj = j - 1, st = jj % kStages, pb = jj & 1;
+          if (!mbar_wait_bounded(&bars->v_full[st], (jj / kStages) & 1, abort_flag,
+                                 kWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+          for (int q = 0; q < nq; ++q) {
+            if (!mbar_wait_bounded(&bars->p_full[q][pb], (jj >> 1) & 1, abort_flag,
+                                   kWaitLimitNs)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t dO = tmem + kTmemO + (uint32_t)(q * HD);
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint32_t offA = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-          const uint32_t offB = kk * 16 * 128;
-          tc_mma_ss(dO, smem_desc_sw128(sP + st * kTileBytes + offA, 16, 1024),
-                    smem_desc_sw128(sV + st * kTileBytes + offB, kHalfBytes, 1024), idPV,
-                    (jj > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < BN / 16; ++kk) {
+              const uint32_t offP = (q * 2 + pb) * kPTile + kk * 32;
+              const uint32_t offV = st * kKTile + kk * 16 * 128;
+              tc_mma_ss(dO, smem_desc_sw128(sP + offP, 16, 1024),
+                        smem_desc_sw128(sV + offV, kKHalf, 1024), idPV,
+                        (jj > 0 || kk > 0) ? 1u : 0u);
+            }
+            tc_commit(&bars->pv_done[q][pb]);
+          }
+          if (!ok) break;
+          tc_commit(&bars->v_empty[st]);
         }
-        tc_commit(&bars->pv_done[st]);
-        tc_commit(&bars->v_empty[st]);
       }
-    }
-    // every MMA issued above has completed before TMEM is released
-    tc_commit(&bars->mma_final);
-    mbar_wait_bounded(&bars->mma_final, 0, nullptr, kWaitLimitNs);
+      // every MMA issued above has completed before TMEM is released
+      tc_commit(&bars->mma_final);
+      mbar_wait_bounded(&bars->mma_final, 0, nullptr, kWaitLimitNs);
     }
     __syncwarp();
-  } else if (warp < 4 && n > 0) {
+  } else if (warp < 4 * kQT && n > 0 && (warp >> 2) < nq) {
     // ------------------------------------------------------------ softmax
-    const int r = warp * 32 + lane;                       // query row in tile
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;  // TMEM lane field
-    uint8_t* sP = smem + kOffP;
+    const int q = warp >> 2, wl = warp & 3;
+    const int r = wl * 32 + lane;                         // query row in tile q
+    const uint32_t lane_base = (uint32_t)(wl * 32) << 16;  // TMEM lane field
+    uint8_t* sPq = smem + kOffP + q * 2 * kPTile;
+    const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < n && ok; ++j) {
-      const int st = j & 1;
+      const int sb = j & 1;
       const int k = k_begin + j;
       const int n_valid = k < np ? min(BN, L - k * BN) : min(BN, p.C - (k - np) * BN);
       // wait outcomes are made warp-uniform: tcgen05.ld/st are .sync.aligned
-      if (!__all_sync(0xffffffffu,
-                      mbar_wait_bounded(&bars->s_full[st], (j >> 1) & 1, abort_flag,
-                                        kWaitLimitNs))) {
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(&bars->s_full[q][sb], (j >> 1) & 1,
+                                                     abort_flag, kWaitLimitNs))) {
         ok = false;
         break;
       }
@@ -278,39 +323,39 @@ __global__ void __launch_bounds__(kThreads, 1)
       float sv[BN];
       {
         uint32_t raw[BN];
-        tmem_ld128(tmem + lane_base + (uint32_t)(st * BN), raw);
+        tmem_ld64(tmem + lane_base + (uint32_t)((q * 2 + sb) * BN), raw);
 #pragma unroll
         for (int c = 0; c < BN; ++c) sv[c] = __uint_as_float(raw[c]);
       }
-      float mx = -INFINITY;
-      if (n_valid == BN) {
+      if (n_valid < BN) {  // ragged last tile of the prefix or of the canvas
 #pragma unroll
-        for (int c = 0; c < BN; ++c) mx = fmaxf(mx, sv[c]);
-      } else {  // ragged last tile of the prefix or of the canvas
-#pragma unroll
-        for (int c = 0; c < BN; ++c) {
+        for (int c = 0; c < BN; ++c)
           if (c >= n_valid) sv[c] = -INFINITY;
-          mx = fmaxf(mx, sv[c]);
-        }
       }
-      mx *= p.scale_log2;
-      // P buffer st was last read by PV_{j-2}
+      float mx0 = sv[0], mx1 = sv[1];
+#pragma unroll
+      for (int c = 2; c < BN; c += 2) {
+        mx0 = fmaxf(mx0, sv[c]);
+        mx1 = fmaxf(mx1, sv[c + 1]);
+      }
+      const float mx = fmaxf(mx0, mx1) * p.scale_log2;
+      // P buffer sb was last read by PV of tile j-2
       if (j >= 2 &&
-          !__all_sync(0xffffffffu, mbar_wait_bounded(&bars->pv_done[st], ((j - 2) >> 1) & 1,
+          !__all_sync(0xffffffffu, mbar_wait_bounded(&bars->pv_done[q][sb], ((j - 2) >> 1) & 1,
                                                      abort_flag, kWaitLimitNs))) {
         ok = false;
         break;
       }
       // lazy rescale (warp-uniform decision so tcgen05.ld/st stay converged)
-      const bool need = __any_sync(0xffffffffu, mx > m_ref + kLazyRescale);
-      if (need) {
+      if (__any_sync(0xffffffffu, mx > m_ref + kLazyRescale)) {
         const float m_new = fmaxf(m_ref, mx);
         const float alpha = ex2_approx(m_ref - m_new);  // 0 when m_ref = -inf
         l *= alpha;
         if (j >= 1) {
           const int pj = j - 1;
-          if (!__all_sync(0xffffffffu, mbar_wait_bounded(&bars->pv_done[pj & 1], (pj >> 1) & 1,
-                                                         abort_flag, kWaitLimitNs))) {
+          if (!__all_sync(0xffffffffu,
+                          mbar_wait_bounded(&bars->pv_done[q][pj & 1], (pj >> 1) & 1, abort_flag,
+                                            kWaitLimitNs))) {
             ok = false;
             break;
           }
@@ -318,7 +363,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int c4 = 0; c4 < HD / 32; ++c4) {
             uint32_t raw[32];
-            const uint32_t ta = tmem + lane_base + (uint32_t)(2 * BN + c4 * 32);
+            const uint32_t ta = tmem + lane_base + kTmemO + (uint32_t)(q * HD + c4 * 32);
             tmem_ld32(ta, raw);
 #pragma unroll
             for (int c = 0; c < 32; ++c) raw[c] = __float_as_uint(__uint_as_float(raw[c]) * alpha);
@@ -328,54 +373,54 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         m_ref = m_new;
       }
-      // P = 2^(s * scale_log2 - m_ref) as bf16, 128B-swizzled K-major rows
-      float lsum = 0.f;
-      uint8_t* prow = sP + st * kTileBytes + r * 128;
+      // P = 2^(s * scale_log2 - m_ref) as bf16, one 128-byte swizzled row
+      const float2 nm = make_float2(-m_ref, -m_ref);
+      float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                       make_float2(0.f, 0.f)};
+      uint8_t* prow = sPq + sb * kPTile + r * 128;
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
+      for (int cc = 0; cc < BN / 8; ++cc) {
+        uint32_t w[4];
 #pragma unroll
-        for (int cc = 0; cc < 8; ++cc) {
-          uint32_t w[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int c = h * 64 + cc * 8 + 2 * e;
-            const float pa = ex2_approx(fmaf(sv[c], p.scale_log2, -m_ref));
-            const float pb = ex2_approx(fmaf(sv[c + 1], p.scale_log2, -m_ref));
-            lsum += pa + pb;
-            w[e] = pack_bf16x2(pa, pb);
-          }
-          const int phys = cc ^ (r & 7);
-          *reinterpret_cast<uint4*>(prow + h * kHalfBytes + phys * 16) =
-              make_uint4(w[0], w[1], w[2], w[3]);
+        for (int e = 0; e < 4; ++e) {
+          const int c = cc * 8 + 2 * e;
+          const float2 d = __ffma2_rn(make_float2(sv[c], sv[c + 1]), sl2, nm);
+          const float2 pp = make_float2(ex2_approx(d.x), ex2_approx(d.y));
+          acc[e] = __fadd2_rn(acc[e], pp);
+          w[e] = pack_bf16x2(pp.x, pp.y);
         }
+        *reinterpret_cast<uint4*>(prow + ((cc ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
       }
-      l += lsum;
+      const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
+      const float2 a = __fadd2_rn(a01, a23);
+      l += a.x + a.y;
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->p_full[st]);
+      if (lane == 0) mbar_arrive(&bars->p_full[q][sb]);
     }
     // epilogue: O / l and the log2-domain LSE of this split
     if (ok) {
       const int last = n - 1;
-      ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->pv_done[last & 1], (last >> 1) & 1,
-                                                     abort_flag, kWaitLimitNs));
+      ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->pv_done[q][last & 1],
+                                                     (last >> 1) & 1, abort_flag, kWaitLimitNs));
     }
     if (ok) {
       tc_fence_after();
       const float inv = 1.f / l;
-      float* orow = p.part_o + ((size_t)blockIdx.x * BM + r) * HD;
+      const size_t slot = (size_t)slot0 + (size_t)q * nsplit;
+      float* orow = p.part_o + (slot * BM + r) * HD;
 #pragma unroll
       for (int c4 = 0; c4 < HD / 32; ++c4) {
         uint32_t raw[32];
-        tmem_ld32(tmem + lane_base + (uint32_t)(2 * BN + c4 * 32), raw);
+        tmem_ld32(tmem + lane_base + kTmemO + (uint32_t)(q * HD + c4 * 32), raw);
 #pragma unroll
         for (int c = 0; c < 32; c += 4)
           *reinterpret_cast<float4*>(orow + c4 * 32 + c) =
               make_float4(__uint_as_float(raw[c]) * inv, __uint_as_float(raw[c + 1]) * inv,
                           __uint_as_float(raw[c + 2]) * inv, __uint_as_float(raw[c + 3]) * inv);
       }
-      p.part_lse[(size_t)blockIdx.x * BM + r] = m_ref + __log2f(l);
+      p.part_lse[slot * BM + r] = m_ref + __log2f(l);
     }
   }
 
@@ -515,15 +560,17 @@ int num_sms() {
 }
 
 struct Plan {
-  int T, chunk, units, groups;
+  int T, chunk, units, slots, groups;
 };
 
 // Choose the split size (key tiles per CTA) that minimises the makespan
-// waves(units) * chunk over the SMs.
+// waves(units) * chunk over the SMs, plus a small charge per split for the
+// merge pass.
 Plan make_plan(const AttnArgs& a) {
   Plan pl{};
   const int group = a.Hq / a.Hkv;
   pl.T = (a.C * group + BM - 1) / BM;
+  const int TP = (pl.T + kQT - 1) / kQT;
   const int nc = (a.C + BN - 1) / BN;
   int max_tiles = 1;
   for (int b = 0; b < a.B; ++b) {
@@ -533,19 +580,20 @@ Plan make_plan(const AttnArgs& a) {
   const int sms = num_sms();
   double best_cost = 1e300;
   for (int chunk = 1; chunk <= max_tiles; ++chunk) {
-    int64_t units = 0;
+    int64_t units = 0, slots = 0;
     for (int b = 0; b < a.B; ++b) {
       const int L = a.cu_prefix_host[b + 1] - a.cu_prefix_host[b];
-      const int ntiles = (L + BN - 1) / BN + nc;
-      units += (int64_t)a.Hkv * pl.T * ((ntiles + chunk - 1) / chunk);
+      const int ns = ((L + BN - 1) / BN + nc + chunk - 1) / chunk;
+      units += (int64_t)a.Hkv * TP * ns;
+      slots += (int64_t)a.Hkv * pl.T * ns;
     }
     const int64_t waves = (units + sms - 1) / sms;
-    // each split also costs its share of the merge pass (~ a quarter tile)
-    const double cost = (double)waves * chunk + 0.25 * (double)units / sms;
+    const double cost = (double)waves * (chunk + 2) + 0.25 * (double)units / sms;
     if (cost < best_cost - 1e-9) {
       best_cost = cost;
       pl.chunk = chunk;
       pl.units = (int)units;
+      pl.slots = (int)slots;
     }
   }
   pl.groups = a.B * a.Hkv * pl.T;
@@ -569,7 +617,7 @@ bool attn_tc_supported(const AttnArgs& a) {
 
 size_t attn_tc_scratch_bytes(const AttnArgs& a) {
   const Plan pl = make_plan(a);
-  return (size_t)pl.units * BM * (HD + 1) * sizeof(float) + 256;
+  return (size_t)pl.slots * BM * (HD + 1) * sizeof(float) + 256;
 }
 
 cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t stream) {
@@ -608,7 +656,7 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t stream) {
   tp.cu_prefix = a.cu_prefix;
   uint8_t* scratch = static_cast<uint8_t*>(a.scratch);
   tp.part_o = reinterpret_cast<float*>(scratch);
-  tp.part_lse = reinterpret_cast<float*>(scratch + (size_t)pl.units * BM * HD * sizeof(float));
+  tp.part_lse = reinterpret_cast<float*>(scratch + (size_t)pl.slots * BM * HD * sizeof(float));
   tp.err = a.err;
 
   attn_tc_kernel<<<pl.units, kThreads, kSmemBytes, stream>>>(mQ, mKp, mVp, mKc, mVc, tp);
@@ -616,7 +664,7 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t stream) {
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   attn_combine_kernel<__nv_bfloat16><<<pl.groups * (BM / kCombineRowsPerCta), 256, 0, stream>>>(
-      tp, pl.units, static_cast<__nv_bfloat16*>(a.out), a.lse);
+      tp, pl.slots, static_cast<__nv_bfloat16*>(a.out), a.lse);
   note_launch();
   return cudaGetLastError();
 }

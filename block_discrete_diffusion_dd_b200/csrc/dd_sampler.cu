@@ -97,9 +97,11 @@ __device__ __forceinline__ float warp_max(float v) {
   return v;
 }
 
-// Logits below this are treated as this value (exp underflows to 0 either
-// way); it keeps -inf entries and padding out of 0 * inf products.
-constexpr float kFloorLogit = -1e30f;
+// Logits below -2^15 are treated as -2^15: exp underflows to 0 either way
+// (unless the whole row lies below it), and -inf entries and padding stay
+// out of 0 * inf products.  A power of two keeps x * c2 exact, so a thread
+// that has seen only padding gets d = 0 exactly.
+constexpr float kFloorLogit = -32768.0f;
 
 // Per-thread running state (log2 units for the softmax sums; packed pairs
 // so that two entries update with one f32x2 instruction).
@@ -171,7 +173,10 @@ __device__ __forceinline__ void process8(Run& st, float& best_w, const float (&x
   // 1 - U >= e^(z - best_w) (1 + 2^-8) is skipped without a logarithm.  With
   // U' = 1 + (x >> 9) 2^-23 = U + 1 - 2^-24 the test reads
   // U' > 2 - 2^-23 - p Kp,  Kp = (1 + 2^-8) e^(m ln 2 - best_w).
-  const float Kp = fminf(ex2_approx(st.m - best_w * kLog2e) * 1.00390625f, 1e30f);
+  // best_w = -inf only in a warp that holds padding alone: nothing to test
+  const float Kp = best_w == -INFINITY
+                       ? 0.f
+                       : fminf(ex2_approx(st.m - best_w * kLog2e) * 1.00390625f, 1e30f);
   const float2 kk = make_float2(-Kp, -Kp);
   const float2 cc = make_float2(1.99999988079071044921875f, 1.99999988079071044921875f);
   float thr[8];
@@ -203,8 +208,8 @@ __device__ __forceinline__ void process8(Run& st, float& best_w, const float (&x
 // bf16 pairs in a 32-bit word, floored at kFloorLogit (max.bf16x2 is exact).
 __device__ __forceinline__ uint32_t floor_bf16x2(uint32_t w) {
   uint32_t r;
-  // 0xF149 is the bf16 value -9.96e29 (>= kFloorLogit after widening)
-  asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(w), "r"(0xF149F149u));
+  // 0xC700 is the bf16 value -32768 = kFloorLogit
+  asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(w), "r"(0xC700C700u));
   return r;
 }
 __device__ __forceinline__ uint32_t max_bf16x2(uint32_t a, uint32_t b) {
@@ -262,7 +267,7 @@ __device__ __forceinline__ void write_record(const Run& r, ChunkRecord* rec) {
 constexpr uint32_t kStageBytes = 32768;  // logits per CTA (one bulk copy)
 
 template <typename T>
-constexpr int chunk_elems() { return (int)(kStageBytes / sizeof(T)); }
+__host__ __device__ constexpr int chunk_elems() { return (int)(kStageBytes / sizeof(T)); }
 
 // Vector path: rows 16-byte aligned and V % 8 == 0.  Thread 0 fetches the
 // CTA's 32 KB slice of the row with one bulk asynchronous copy into shared
