@@ -29,7 +29,7 @@ EXPORTS = (
     "dd_canvas_attn_workspace", "dd_canvas_attn", "dd_sample_renoise_workspace",
     "dd_sample_renoise", "dd_init_canvas", "dd_denoise_block_workspace", "dd_denoise_block",
     "dd_workspace_init", "dd_query_device_error", "dd_status_string", "dd_last_error",
-    "dd_launch_count", "dd_reset_launch_count",
+    "dd_launch_count", "dd_reset_launch_count", "dd_sample_renoise_noalloc",
 )
 
 
@@ -75,6 +75,9 @@ def load() -> ctypes.CDLL:
     lib.dd_sample_renoise.restype = i32
     lib.dd_sample_renoise.argtypes = [P, i32, i32, i32, i64, ctypes.POINTER(SampleParams), P, P, P,
                                       P, P, P, sz, P]
+    lib.dd_sample_renoise_noalloc.restype = i32
+    lib.dd_sample_renoise_noalloc.argtypes = [P, i32, i32, i32, i64, ctypes.POINTER(SampleParams),
+                                              P, P, P, P, P, P]
     lib.dd_init_canvas.restype = i32
     lib.dd_init_canvas.argtypes = [P, i32, i32, u64, u32, P]
     lib.dd_denoise_block_workspace.restype = sz
@@ -198,6 +201,31 @@ def sample_renoise(logits: torch.Tensor, temperature: float, rate: float, seed: 
                                  ctypes.byref(prm), _ptr(o["tokens"]), _ptr(o.get("pred")),
                                  _ptr(o["conf"]), _ptr(o.get("entropy")), _ptr(o.get("renoised")),
                                  _ptr(workspace), workspace.numel(), _stream(stream)))
+    return o
+
+
+def sample_renoise_noalloc(logits: torch.Tensor, temperature: float, rate: float, seed: int,
+                           step: int, row_offset: int = 0, outputs: Optional[dict] = None,
+                           stream=None) -> dict:
+    """dd_sample_renoise_noalloc: the sampler step with the library's static
+    scratch instead of a workspace (for callers that must not allocate).
+    Calls must not overlap on the GPU; see include/dd.h."""
+    lib = load()
+    R, V = logits.shape[0], logits.shape[-1]
+    dev = logits.device
+    o = outputs if outputs is not None else {
+        "tokens": torch.empty(R, dtype=torch.int32, device=dev),
+        "pred": torch.empty(R, dtype=torch.int32, device=dev),
+        "conf": torch.empty(R, dtype=torch.float32, device=dev),
+        "entropy": torch.empty(R, dtype=torch.float32, device=dev),
+        "renoised": torch.empty(R, dtype=torch.uint8, device=dev),
+    }
+    prm = SampleParams(float(temperature), float(rate), int(seed), int(step), int(row_offset))
+    _check(lib.dd_sample_renoise_noalloc(_ptr(logits), _dtype_code(logits), R, V,
+                                         logits.stride(0), ctypes.byref(prm), _ptr(o["tokens"]),
+                                         _ptr(o.get("pred")), _ptr(o["conf"]),
+                                         _ptr(o.get("entropy")), _ptr(o.get("renoised")),
+                                         _stream(stream)))
     return o
 
 

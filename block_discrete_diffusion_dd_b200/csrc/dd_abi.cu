@@ -200,6 +200,22 @@ dd_status run_sampler(const void* logits, dd_dtype dtype, int rows, int vocab, i
 
 void note_launch() { ++g_launches; }
 
+// Entry for callers that bring their own scratch region (dd_noalloc.cu):
+// the same validation and kernels as dd_sample_renoise.
+dd_status sample_with_scratch(const void* logits, dd_dtype dtype, int rows, int vocab,
+                              int64_t row_stride, const dd_sample_params* p, int32_t* tokens,
+                              int32_t* pred, float* conf, float* entropy, uint8_t* renoised,
+                              void* scratch, size_t scratch_bytes, cudaStream_t stream) {
+  g_last_error.clear();
+  return run_sampler(logits, dtype, rows, vocab, row_stride, p, tokens, pred, conf, entropy,
+                     renoised, scratch, scratch_bytes, stream);
+}
+
+dd_status set_error(dd_status st, const char* msg) {
+  g_last_error = msg;
+  return st;
+}
+
 }  // namespace dd
 
 using namespace dd;

@@ -190,6 +190,31 @@ DD_API dd_status dd_denoise_block(const dd_attn_desc* desc, int steps, const voi
                            int32_t* canvas, int32_t* canvas_history, float* conf_steps,
                            void* workspace, size_t workspace_bytes, dd_stream_t stream);
 
+/* dd_sample_renoise without a workspace, for callers that may not allocate
+ * device memory (code inside another framework's memory pool or fixed
+ * budget, plugin or callback code handed only its input and output
+ * pointers, latency-critical loops that cannot accept cudaMalloc's device
+ * synchronisation).  The paper has no counterpart: this is a deployment
+ * variant of the same sampler step.
+ * Arguments and results: exactly as dd_sample_renoise, minus the workspace.
+ * Scratch: a static device array of 2 MiB that the library holds on every
+ * GPU it is loaded on until the process exits.  A call needs
+ * dd_sample_renoise_workspace(rows, vocab, dtype) bytes of it (512 bytes per
+ * row at V = 262144 in bf16, so up to 4095 rows); larger calls return
+ * DD_ERR_UNSUPPORTED before touching the GPU.  The function allocates
+ * nothing: no cudaMalloc, cudaFree or allocating library call.
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress), so make that first call before any stream capture.
+ * Every call shares the array: calls that overlap on the GPU (two streams,
+ * or two host threads) race and may return wrong results.  Device-side
+ * timeouts are latched in the array but not reported by this entry point;
+ * use dd_sample_renoise and dd_query_device_error to observe them. */
+DD_API dd_status dd_sample_renoise_noalloc(const void* logits, dd_dtype dtype, int rows, int vocab,
+                                           int64_t row_stride, const dd_sample_params* params,
+                                           int32_t* tokens_out, int32_t* pred_out,
+                                           float* conf_out, float* entropy_out,
+                                           uint8_t* renoised_out, dd_stream_t stream);
+
 /* Clears the error word at the start of a workspace (async on stream). */
 DD_API dd_status dd_workspace_init(void* workspace, size_t workspace_bytes, dd_stream_t stream);
 
