@@ -103,8 +103,10 @@ __device__ __forceinline__ float warp_max(float v) {
 // that has seen only padding gets d = 0 exactly.
 constexpr float kFloorLogit = -32768.0f;
 
-// Per-thread running state (log2 units for the softmax sums; packed pairs
-// so that two entries update with one f32x2 instruction).
+// Per-thread running state.  Softmax sums in log2 units relative to a lazy
+// reference m (raised only when an entry exceeds it by more than 2^8, so the
+// terms stay below 256), kept as packed pairs so two entries update with one
+// f32x2 instruction; best = best Gumbel score (natural units), idx its index.
 struct Run {
   float m;
   float2 s2, t2;
@@ -112,97 +114,24 @@ struct Run {
   int idx;
 };
 
-// One item = 8 consecutive vocabulary entries x[0..7] starting at v0 (all
-// finite: -inf and padding arrive as kFloorLogit); bm = max of x.
-// best_w is the warp-wide running best Gumbel score; `seed` marks the first
-// item, where the threshold is seeded with the exact score of each lane's
-// largest entry.  Control flow is warp-uniform apart from the rare exact
-// path, so the shuffles inside are safe.
-__device__ __forceinline__ void process8(Run& st, float& best_w, const float (&x)[8], float bm,
-                                         int64_t v0, bool seed, const PhiloxKey& key,
-                                         uint32_t grow, uint32_t step, float c2, float inv_tau) {
-  const float ym = bm * c2;
-  if (ym > st.m) {
-    const float s = st.s2.x + st.s2.y, t = st.t2.x + st.t2.y;
-    if (s > 0.f) {
-      const float f = ex2_approx(st.m - ym);
-      st.t2 = make_float2(f * fmaf(s, st.m - ym, t), 0.f);
-      st.s2 = make_float2(s * f, 0.f);
-    }
-    st.m = ym;
+constexpr float kLazy = 8.0f;  // log2 headroom of the lazy reference
+
+// Raise the lazy reference of `st` to ym, rescaling its sums.
+__device__ __forceinline__ void raise_ref(Run& st, float ym) {
+  const float s = st.s2.x + st.s2.y, t = st.t2.x + st.t2.y;
+  if (s > 0.f) {
+    const float f = ex2_approx(st.m - ym);
+    st.t2 = make_float2(f * fmaf(s, st.m - ym, t), 0.f);
+    st.s2 = make_float2(s * f, 0.f);
   }
-  const float2 c22 = make_float2(c2, c2);
-  const float2 nm = make_float2(-st.m, -st.m);
-  float p[8];
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const float2 d = __ffma2_rn(make_float2(x[2 * j], x[2 * j + 1]), c22, nm);
-    p[2 * j] = ex2_approx(d.x);
-    p[2 * j + 1] = ex2_approx(d.y);
-    const float2 pp = make_float2(p[2 * j], p[2 * j + 1]);
-    st.s2 = __fadd2_rn(st.s2, pp);
-    st.t2 = __ffma2_rn(pp, d, st.t2);
-  }
-  // Gumbel words for the 8 entries: two Philox blocks.
-  const uint32_t q0 = (uint32_t)(v0 >> 2);
-  const uint4 wa = philox4x32_10(make_uint4(q0, grow, step, 0u), key);
-  const uint4 wb = philox4x32_10(make_uint4(q0 + 1u, grow, step, 0u), key);
-  const uint32_t w[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
-  if (seed) {
-    if (bm > kFloorLogit) {
-      int j = 7;
-#pragma unroll
-      for (int i = 6; i >= 0; --i) j = (x[i] == bm) ? i : j;
-      float xj = x[0];
-      uint32_t wj = w[0];
-#pragma unroll
-      for (int i = 1; i < 8; ++i) {
-        xj = (j == i) ? x[i] : xj;
-        wj = (j == i) ? w[i] : wj;
-      }
-      const float sc = gumbel_score(xj * inv_tau, wj);
-      if (sc > st.best) {
-        st.best = sc;
-        st.idx = (int)(v0 + j);
-      }
-    }
-    best_w = warp_max(st.best);
-  }
-  // Exponential-race prune: the score z - ln E (E = -ln U) can beat best_w
-  // only if E < e^(z - best_w); since E >= 1 - U, an entry with
-  // 1 - U >= e^(z - best_w) (1 + 2^-8) is skipped without a logarithm.  With
-  // U' = 1 + (x >> 9) 2^-23 = U + 1 - 2^-24 the test reads
-  // U' > 2 - 2^-23 - p Kp,  Kp = (1 + 2^-8) e^(m ln 2 - best_w).
-  // best_w = -inf only in a warp that holds padding alone: nothing to test
-  const float Kp = best_w == -INFINITY
-                       ? 0.f
-                       : fminf(ex2_approx(st.m - best_w * kLog2e) * 1.00390625f, 1e30f);
-  const float2 kk = make_float2(-Kp, -Kp);
-  const float2 cc = make_float2(1.99999988079071044921875f, 1.99999988079071044921875f);
-  float thr[8];
-  bool any = false;
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const float2 t = __ffma2_rn(make_float2(p[2 * j], p[2 * j + 1]), kk, cc);
-    thr[2 * j] = t.x;
-    thr[2 * j + 1] = t.y;
-    any |= __uint_as_float(0x3F800000u | (w[2 * j] >> 9)) > t.x;
-    any |= __uint_as_float(0x3F800000u | (w[2 * j + 1] >> 9)) > t.y;
-  }
-  if (any) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      if (__uint_as_float(0x3F800000u | (w[i] >> 9)) > thr[i]) {
-        const float sc = gumbel_score(x[i] * inv_tau, w[i]);
-        const int v = (int)(v0 + i);
-        if (sc > st.best || (sc == st.best && v < st.idx)) {
-          st.best = sc;
-          st.idx = v;
-        }
-      }
-    }
-  }
-  best_w = warp_max(st.best);
+  st.m = ym;
+}
+
+// Prune threshold factor Kp = (1 + 2^-8) e^(m ln 2 - best_w), clamped; 0 in
+// a warp that holds padding alone (best_w = -inf).
+__device__ __forceinline__ float prune_factor(float m, float best_w) {
+  return best_w == -INFINITY ? 0.f
+                             : fminf(ex2_approx(m - best_w * kLog2e) * 1.00390625f, 1e30f);
 }
 
 // bf16 pairs in a 32-bit word, floored at kFloorLogit (max.bf16x2 is exact).
@@ -239,28 +168,56 @@ __device__ __forceinline__ void unpack8(float4 a, float4 b, float (&x)[8], float
   bm = fmaxf(fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3])), fmaxf(fmaxf(x[4], x[5]), fmaxf(x[6], x[7])));
 }
 
-// Reduce the CTA's states and write its chunk record.
+// Reduce the CTA's states and write its chunk record.  Within a warp: the
+// common reference M first, then every lane rescales its sums to M and the
+// sums and the argmax (lowest index on equal scores) reduce by butterflies,
+// a fixed tree, so the result does not depend on scheduling.
+__device__ __forceinline__ SampState warp_reduce(const Run& r) {
+  float M = r.m;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+  float s = r.s2.x + r.s2.y, t = r.t2.x + r.t2.y;
+  if (s > 0.f) {
+    const float f = ex2_approx(r.m - M);
+    t = f * fmaf(s, r.m - M, t);
+    s *= f;
+  } else {
+    s = 0.f;
+    t = 0.f;
+  }
+  float best = r.best;
+  int idx = r.idx;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    s += __shfl_xor_sync(0xffffffffu, s, off);
+    t += __shfl_xor_sync(0xffffffffu, t, off);
+    const float ob = __shfl_xor_sync(0xffffffffu, best, off);
+    const int oi = __shfl_xor_sync(0xffffffffu, idx, off);
+    if (ob > best || (ob == best && oi < idx)) {
+      best = ob;
+      idx = oi;
+    }
+  }
+  return SampState{M, s, t, best, idx};
+}
+
 __device__ __forceinline__ void write_record(const Run& r, ChunkRecord* rec) {
-  SampState st{r.m, r.s2.x + r.s2.y, r.t2.x + r.t2.y, r.best, r.idx};
-  warp_merge(st);
+  const SampState st = warp_reduce(r);
   __shared__ SampState red[kSampleThreads / 32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (lane == 0) red[warp] = st;
   __syncthreads();
-  if (warp == 0) {
-    SampState s = lane < kSampleThreads / 32
-                      ? red[lane]
-                      : SampState{-INFINITY, 0.f, 0.f, -INFINITY, 0x7fffffff};
-    warp_merge(s);
-    if (lane == 0) {
-      ChunkRecord out;
-      out.m = s.m;
-      out.s = s.s;
-      out.t = s.t;
-      out.best = s.best;
-      out.idx = s.idx;
-      *rec = out;
-    }
+  if (threadIdx.x == 0) {
+    SampState a = red[0];
+#pragma unroll
+    for (int w = 1; w < kSampleThreads / 32; ++w) merge_state(a, red[w]);
+    ChunkRecord out;
+    out.m = a.m;
+    out.s = a.s;
+    out.t = a.t;
+    out.best = a.best;
+    out.idx = a.idx;
+    *rec = out;
   }
 }
 
@@ -268,6 +225,88 @@ constexpr uint32_t kStageBytes = 32768;  // logits per CTA (one bulk copy)
 
 template <typename T>
 __host__ __device__ constexpr int chunk_elems() { return (int)(kStageBytes / sizeof(T)); }
+
+// One item = 8 consecutive entries x[0..7] (floored, finite) starting at v0,
+// with bm = their max.  `src` points at the item's first entry (in shared
+// memory, or in global memory on the scalar path) and is re-read only on the
+// rare exact path.
+template <typename T>
+__device__ __forceinline__ void process_item(Run& st, float& best_w, float& Kp, const float (&x)[8],
+                                             float bm, uint32_t v0, bool seed, const T* src,
+                                             const PhiloxKey& key, uint32_t grow, uint32_t step,
+                                             float c2, float inv_tau) {
+  const float ym = bm * c2;
+  if (ym > st.m + kLazy) {  // rare after the first item
+    raise_ref(st, ym);
+    Kp = prune_factor(st.m, best_w);
+  }
+  const float2 c22 = make_float2(c2, c2);
+  const float2 nm = make_float2(-st.m, -st.m);
+  float2 p[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float2 d = __ffma2_rn(make_float2(x[2 * j], x[2 * j + 1]), c22, nm);
+    p[j] = make_float2(ex2_approx(d.x), ex2_approx(d.y));
+    st.s2 = __fadd2_rn(st.s2, p[j]);
+    st.t2 = __ffma2_rn(p[j], d, st.t2);
+  }
+  // Gumbel words for the 8 entries: two Philox blocks.
+  const uint4 wa = philox4x32_10(make_uint4(v0 >> 2, grow, step, 0u), key);
+  const uint4 wb = philox4x32_10(make_uint4((v0 >> 2) + 1u, grow, step, 0u), key);
+  bool changed = false;
+  if (seed) {
+    // seed the threshold with the exact score of this lane's largest entry
+    if (bm > kFloorLogit) {
+      int j = 7;
+#pragma unroll
+      for (int i = 6; i >= 0; --i) j = (x[i] == bm) ? i : j;
+      const uint4 wq = j < 4 ? wa : wb;
+      const uint32_t i4 = (uint32_t)j & 3u;
+      const uint32_t wj = i4 == 0 ? wq.x : i4 == 1 ? wq.y : i4 == 2 ? wq.z : wq.w;
+      st.best = gumbel_score(bm * inv_tau, wj);
+      st.idx = (int)(v0 + (uint32_t)j);
+    }
+    // the seeded threshold applies to this item's own test below
+    best_w = warp_max(st.best);
+    Kp = prune_factor(st.m, best_w);
+  }
+  // Exponential-race prune: the score z - ln E (E = -ln U) can beat best_w
+  // only if E < e^(z - best_w); since E >= 1 - U, an entry with
+  // 1 - U >= e^(z - best_w) (1 + 2^-8) is skipped without a logarithm.  With
+  // U' = 1 + (x >> 9) 2^-23 = U + 1 - 2^-24 the test reads
+  // U' > 2 - 2^-23 - p Kp.
+  const float2 kk = make_float2(-Kp, -Kp);
+  const float2 cc = make_float2(1.99999988079071044921875f, 1.99999988079071044921875f);
+  const uint32_t w[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+  uint32_t cmask = 0;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float2 t = __ffma2_rn(p[j], kk, cc);
+    cmask |= (__uint_as_float(0x3F800000u | (w[2 * j] >> 9)) > t.x) ? (1u << (2 * j)) : 0u;
+    cmask |= (__uint_as_float(0x3F800000u | (w[2 * j + 1] >> 9)) > t.y) ? (2u << (2 * j)) : 0u;
+  }
+  // rare exact path: one entry at a time (the logit re-read, its word
+  // selected from the two blocks above), so the code below exists once
+  while (cmask) {
+    const int i = __ffs(cmask) - 1;
+    cmask &= cmask - 1;
+    const float xi = fmaxf((float)src[i], kFloorLogit);
+    const uint32_t v = v0 + (uint32_t)i;
+    const uint4 wq = i < 4 ? wa : wb;
+    const int i4 = i & 3;
+    const uint32_t wi = i4 == 0 ? wq.x : i4 == 1 ? wq.y : i4 == 2 ? wq.z : wq.w;
+    const float sc = gumbel_score(xi * inv_tau, wi);
+    if (sc > st.best || (sc == st.best && (int)v < st.idx)) {
+      st.best = sc;
+      st.idx = (int)v;
+      changed = true;
+    }
+  }
+  if (__any_sync(0xffffffffu, changed)) {
+    best_w = warp_max(st.best);
+    Kp = prune_factor(st.m, best_w);
+  }
+}
 
 // Vector path: rows 16-byte aligned and V % 8 == 0.  Thread 0 fetches the
 // CTA's 32 KB slice of the row with one bulk asynchronous copy into shared
@@ -284,8 +323,8 @@ __global__ void __launch_bounds__(kSampleThreads, 4)
   __shared__ uint64_t bar;
   const int row = blockIdx.x / nchunk;
   const int chunk = blockIdx.x - row * nchunk;
-  const int64_t c0 = (int64_t)chunk * kElems;
-  const int n = (int)min((int64_t)kElems, (int64_t)vocab - c0);
+  const int c0 = chunk * kElems;
+  const int n = min(kElems, vocab - c0);
   if (threadIdx.x == 0) {
     mbar_init(&bar, 1);
     fence_mbar_init();
@@ -299,16 +338,17 @@ __global__ void __launch_bounds__(kSampleThreads, 4)
   const uint32_t grow = row_offset + (uint32_t)row;
   const float c2 = inv_tau * kLog2e;
   Run st{-INFINITY, make_float2(0.f, 0.f), make_float2(0.f, 0.f), -INFINITY, 0x7fffffff};
-  float best_w = -INFINITY;
+  float best_w = -INFINITY, Kp = 0.f;
   if (!mbar_wait_bounded(&bar, 0, nullptr, 1000000000ull)) {
     // never observed: the copy is plain memory traffic; report and drain
     if (threadIdx.x == 0) atomicOr(err, kDevErrTimeout);
     mbar_wait_bounded(&bar, 0, nullptr, 4000000000ull);
     return;
   }
+  const T* tb = reinterpret_cast<const T*>(buf);
 #pragma unroll 1
   for (int k = 0; k < kItems; ++k) {
-    const int e = (k * kSampleThreads + threadIdx.x) * 8;
+    const int e = (k * kSampleThreads + (int)threadIdx.x) * 8;
     float x[8], bm;
     if (e < n) {
       if constexpr (sizeof(T) == 2) {
@@ -322,13 +362,15 @@ __global__ void __launch_bounds__(kSampleThreads, 4)
       for (int i = 0; i < 8; ++i) x[i] = kFloorLogit;
       bm = kFloorLogit;
     }
-    process8(st, best_w, x, bm, c0 + e, k == 0, key, grow, step, c2, inv_tau);
+    process_item<T>(st, best_w, Kp, x, bm, (uint32_t)(c0 + e), k == 0, tb + e, key, grow, step,
+                    c2, inv_tau);
   }
   write_record(st, recs + (int64_t)row * nchunk + chunk);
 }
 
 // Scalar path for unaligned rows or V % 8 != 0: direct loads with bounds
-// checks; entries at or beyond V read as kFloorLogit and never win.
+// checks; entries at or beyond V read as kFloorLogit and never win (their p
+// is 0, so the prune never selects them and they are never re-read).
 template <typename T>
 __global__ void __launch_bounds__(kSampleThreads)
     sample_chunk_scalar_kernel(const T* __restrict__ logits, int64_t row_stride, int vocab,
@@ -338,16 +380,16 @@ __global__ void __launch_bounds__(kSampleThreads)
   constexpr int kItems = kElems / (kSampleThreads * 8);
   const int row = blockIdx.x / nchunk;
   const int chunk = blockIdx.x - row * nchunk;
-  const int64_t c0 = (int64_t)chunk * kElems;
+  const int c0 = chunk * kElems;
   const T* rowp = logits + (int64_t)row * row_stride;
   const PhiloxKey key = philox_key(seed);
   const uint32_t grow = row_offset + (uint32_t)row;
   const float c2 = inv_tau * kLog2e;
   Run st{-INFINITY, make_float2(0.f, 0.f), make_float2(0.f, 0.f), -INFINITY, 0x7fffffff};
-  float best_w = -INFINITY;
+  float best_w = -INFINITY, Kp = 0.f;
 #pragma unroll 1
   for (int k = 0; k < kItems; ++k) {
-    const int64_t v0 = c0 + (int64_t)(k * kSampleThreads + threadIdx.x) * 8;
+    const int v0 = c0 + (k * kSampleThreads + (int)threadIdx.x) * 8;
     float x[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i)
@@ -355,7 +397,8 @@ __global__ void __launch_bounds__(kSampleThreads)
     float bm = x[0];
 #pragma unroll
     for (int i = 1; i < 8; ++i) bm = fmaxf(bm, x[i]);
-    process8(st, best_w, x, bm, v0, k == 0, key, grow, step, c2, inv_tau);
+    process_item<T>(st, best_w, Kp, x, bm, (uint32_t)v0, k == 0, rowp + v0, key, grow, step,
+                    c2, inv_tau);
   }
   write_record(st, recs + (int64_t)row * nchunk + chunk);
 }
