@@ -330,16 +330,32 @@ def run_e2e(args, w, s, dd, dev, stream, desc, dist):
             "ms_per_step": ms / n}
 
 
-def _profile_traffic() -> dict:
-    """DRAM bytes per launch from the committed ncu summary (None if absent
-    or taken on an older build of the kernel)."""
-    path = os.path.join(ROOT, "profiles", "traffic.json")
+def _source_sha(name: str) -> str:
+    import hashlib
+    path = os.path.join(ROOT, "block_discrete_diffusion_dd_b200", "csrc", name)
     try:
-        with open(path) as f:
-            t = json.load(f)
-        return {k: v.get("bytes_per_launch") for k, v in t.items() if v.get("current", False)}
-    except Exception:
-        return {}
+        with open(path, "rb") as f:
+            return hashlib.sha256(f.read()).hexdigest()[:16]
+    except OSError:
+        return ""
+
+
+def _profile_traffic() -> dict:
+    """DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum)
+    from the committed ncu summary profiles/traffic.txt.  A line reads
+    `<kernel> <bytes per launch> <source file> <sha256/16 of that source>`;
+    a figure taken on another version of the kernel source reads as None."""
+    out = {}
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.txt")) as f:
+            for line in f:
+                parts = line.split()
+                if len(parts) == 4 and not line.startswith("#"):
+                    kernel, nbytes, src, sha = parts
+                    out[kernel] = float(nbytes) if _source_sha(src) == sha else None
+    except OSError:
+        pass
+    return out
 
 
 def cpu_baseline(w, s, frac: float):

@@ -10,27 +10,30 @@
 // softmax.
 //
 // Work unit (one CTA): (b, g, pair of 128-row query tiles, split s of the
-// key tiles).  The key range of b is cut into 64-key tiles -- prefix tiles
+// key tiles).  The key range of b is cut into 128-key tiles -- prefix tiles
 // first, then canvas tiles, each read through its own tensor map so a tile
 // never straddles the prefix/canvas boundary; the last tile of each part is
 // masked by key index.  Splits are balanced on the host so that whole waves
 // of CTAs cover the SMs; a second kernel merges the splits by their
 // log-sum-exp.
 //
-// Inside a CTA (11 warps) two 128-row query tiles share every key tile:
-//   warps 0-3  softmax for query tile 0, warps 4-7 for query tile 1: one
-//              query row per thread (= one TMEM lane); read S from TMEM,
-//              online softmax in fp32 (log2 domain; O is rescaled only when
-//              the running max grows by more than 2^8), write P as bf16 into
-//              shared memory in the 128B-swizzled K-major layout the MMA
-//              reads;
-//   warp 8     TMA producer for Q and K (3-stage ring of 64-key tiles);
-//   warp 9     TMA producer for V (3-stage ring);
-//   warp 10    allocates 512 TMEM columns (per query tile: S double buffer
-//              of 64 columns and O of 128) and issues every MMA from one
-//              thread: S = Q K_j^T for both query tiles, then O += P V_{j-1},
-//              so the tensor core computes tile j while the softmax warps
-//              work on tile j-1.
+// Inside a CTA (10 warps) the two query tiles share every key tile:
+//   warps 0-3 / 4-7  softmax of query tile 0 / 1: one query row per thread
+//              (= one TMEM lane).  Each reads S (fp32, 128 columns) from
+//              TMEM, runs the online softmax in fp32 (log2 domain; O is
+//              rescaled only when the running max grows by more than 2^8)
+//              and writes P back as bf16 into the first 64 columns of the
+//              same TMEM region, where the P.V MMA reads it directly;
+//   warp 8     TMA producer: Q, then K and V tiles (2-stage rings of 128
+//              keys) in the order the MMAs consume them;
+//   warp 9     allocates all 512 TMEM columns (per query tile: S/P 128, O
+//              128) and issues every MMA from one thread, in the order
+//              PV_0(j), S_0(j+1), PV_1(j), S_1(j+1): each softmax warpgroup
+//              works while the tensor core runs the other tile's MMAs.
+// The tensor core executes one thread's MMAs in issue order, so:
+//   - S_q(j+1) overwrites P_q(j) only after PV_q(j) has read it;
+//   - when S_q(j) is complete, PV_q(j-1) is complete too, so the softmax
+//     may rescale O_q at that point without a further wait.
 // Every mbarrier wait is bounded in time; on expiry the CTA latches an
 // error word, drains its own asynchronous work and frees its TMEM.
 #include <mutex>
@@ -42,31 +45,27 @@ namespace dd {
 namespace {
 
 constexpr int BM = 128;  // query rows per tile
-constexpr int BN = 64;   // keys per tile
+constexpr int BN = 128;  // keys per tile
 constexpr int HD = 128;  // head dim
 constexpr int kQT = 2;   // query tiles per CTA
-constexpr int kStages = 3;
-constexpr int kWarpK = 8, kWarpV = 9, kWarpMMA = 10;
-constexpr int kThreads = 11 * 32;
-constexpr uint32_t kQHalf = BM * 64 * 2;      // 128 rows x 128 bytes
-constexpr uint32_t kQTile = 2 * kQHalf;       // 128 x 128 bf16
-constexpr uint32_t kKHalf = BN * 64 * 2;      // 64 rows x 128 bytes
-constexpr uint32_t kKTile = 2 * kKHalf;       // 64 x 128 bf16
-constexpr uint32_t kPTile = BM * BN * 2;      // 128 rows x 128 bytes
+constexpr int kStages = 2;
+constexpr int kWarpTMA = 8, kWarpMMA = 9;
+constexpr int kThreads = 10 * 32;
+constexpr uint32_t kHalf = 128 * 64 * 2;  // 128 rows x 128 bytes
+constexpr uint32_t kTile = 2 * kHalf;     // 128 x 128 bf16
 constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffK = kOffQ + kQT * kQTile;
-constexpr uint32_t kOffV = kOffK + kStages * kKTile;
-constexpr uint32_t kOffP = kOffV + kStages * kKTile;
-constexpr uint32_t kOffBar = kOffP + kQT * 2 * kPTile;
+constexpr uint32_t kOffK = kOffQ + kQT * kTile;
+constexpr uint32_t kOffV = kOffK + kStages * kTile;
+constexpr uint32_t kOffBar = kOffV + kStages * kTile;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemO = kQT * 2 * BN;     // O columns start after the S buffers
+constexpr uint32_t kTmemO = kQT * BN;     // O columns start after the S/P regions
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per wait
 constexpr float kLazyRescale = 8.0f;              // log2 units
 
 struct Barriers {
   uint64_t q_full;
   uint64_t k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
-  uint64_t s_full[kQT][2], p_full[kQT][2], pv_done[kQT][2];
+  uint64_t s_full[kQT], p_full[kQT], o_done[kQT];
   uint64_t mma_final;
   uint32_t tmem_base;
   int abort;
@@ -119,6 +118,39 @@ __device__ void resolve_unit(const TcParams& p, Barriers* bars) {
   bars->unit_slot0 = slots + (g * p.T + tp * kQT) * nsplit + s;
 }
 
+// S_q = Q_q K^T into the S/P region of query tile q (K-major operands).
+__device__ __forceinline__ void issue_s(uint32_t tmem, uint32_t sQ, uint32_t sK, int q, int st) {
+  constexpr uint32_t idS = idesc_bf16_f32(BM, BN, 0, 0);
+  const uint32_t dS = tmem + (uint32_t)(q * BN);
+#pragma unroll
+  for (int kk = 0; kk < HD / 16; ++kk) {
+    const uint32_t offQ = q * kTile + (kk >> 2) * kHalf + (kk & 3) * 32;
+    const uint32_t offK = st * kTile + (kk >> 2) * kHalf + (kk & 3) * 32;
+    tc_mma_ss(dS, smem_desc_sw128(sQ + offQ, 16, 1024), smem_desc_sw128(sK + offK, 16, 1024), idS,
+              kk > 0);
+  }
+}
+
+// One 128-key tile of K (v = 0) or V (v = 1) into ring stage j % kStages.
+__device__ __forceinline__ bool load_kv(Barriers* bars, uint8_t* smem, int j, int v, int k_begin,
+                                        int np, int p0, int b, int C, int g,
+                                        const CUtensorMap* tmKp, const CUtensorMap* tmVp,
+                                        const CUtensorMap* tmKc, const CUtensorMap* tmVc,
+                                        volatile int* abort_flag) {
+  const int st = j % kStages, rd = j / kStages;
+  uint64_t* empty = v ? &bars->v_empty[st] : &bars->k_empty[st];
+  uint64_t* full = v ? &bars->v_full[st] : &bars->k_full[st];
+  if (rd > 0 && !mbar_wait_bounded(empty, (rd - 1) & 1, abort_flag, kWaitLimitNs)) return false;
+  const int k = k_begin + j;
+  const CUtensorMap* map = k < np ? (v ? tmVp : tmKp) : (v ? tmVc : tmKc);
+  const int row0 = k < np ? p0 + k * BN : b * C + (k - np) * BN;
+  uint8_t* dst = smem + (v ? kOffV : kOffK) + st * kTile;
+  mbar_arrive_expect_tx(full, kTile);
+  tma_load_3d(dst, map, full, 0, g, row0);
+  tma_load_3d(dst + kHalf, map, full, 64, g, row0);
+  return true;
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                    const __grid_constant__ CUtensorMap tmKp,
@@ -140,12 +172,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->v_full[i], 1);
       mbar_init(&bars->v_empty[i], 1);
     }
-    for (int q = 0; q < kQT; ++q)
-      for (int i = 0; i < 2; ++i) {
-        mbar_init(&bars->s_full[q][i], 1);
-        mbar_init(&bars->p_full[q][i], 4);
-        mbar_init(&bars->pv_done[q][i], 1);
-      }
+    for (int q = 0; q < kQT; ++q) {
+      mbar_init(&bars->s_full[q], 1);
+      mbar_init(&bars->p_full[q], 4);
+      mbar_init(&bars->o_done[q], 1);
+    }
     mbar_init(&bars->mma_final, 1);
     bars->abort = 0;
     fence_mbar_init();
@@ -171,130 +202,102 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n = unit_ok ? min(p.chunk, ntiles - k_begin) : 0;
   const int nq = min(kQT, p.T - tp * kQT);  // query tiles in this CTA (1 or 2)
 
-  if (warp == kWarpK) {
+  if (warp == kWarpTMA) {
     if (lane == 0 && n > 0) {
       prefetch_tensormap(&tmQ);
       prefetch_tensormap(&tmKp);
       prefetch_tensormap(&tmKc);
-      mbar_arrive_expect_tx(&bars->q_full, nq * kQTile);
-      for (int q = 0; q < nq; ++q) {
-        const int qpos = b * p.C + (tp * kQT + q) * (BM / p.group);
-        uint8_t* dst = smem + kOffQ + q * kQTile;
-        tma_load_3d(dst, &tmQ, &bars->q_full, 0, g * p.group, qpos);
-        tma_load_3d(dst + kQHalf, &tmQ, &bars->q_full, 64, g * p.group, qpos);
-      }
-      int issued = 0;
-      for (int j = 0; j < n; ++j) {
-        const int st = j % kStages, rd = j / kStages;
-        if (rd > 0 &&
-            !mbar_wait_bounded(&bars->k_empty[st], (rd - 1) & 1, abort_flag, kWaitLimitNs))
-          break;
-        const int k = k_begin + j;
-        const CUtensorMap* map = k < np ? &tmKp : &tmKc;
-        const int row0 = k < np ? p0 + k * BN : b * p.C + (k - np) * BN;
-        uint8_t* dst = smem + kOffK + st * kKTile;
-        mbar_arrive_expect_tx(&bars->k_full[st], kKTile);
-        tma_load_3d(dst, map, &bars->k_full[st], 0, g, row0);
-        tma_load_3d(dst + kKHalf, map, &bars->k_full[st], 64, g, row0);
-        issued = j + 1;
-      }
-      // drain: loads still in flight must land before the CTA exits
-      for (int j = max(0, issued - kStages); j < issued; ++j)
-        mbar_wait_bounded(&bars->k_full[j % kStages], (j / kStages) & 1, nullptr, kWaitLimitNs);
-      mbar_wait_bounded(&bars->q_full, 0, nullptr, kWaitLimitNs);
-    }
-    __syncwarp();
-  } else if (warp == kWarpV) {
-    if (lane == 0 && n > 0) {
       prefetch_tensormap(&tmVp);
       prefetch_tensormap(&tmVc);
-      int issued = 0;
-      for (int j = 0; j < n; ++j) {
-        const int st = j % kStages, rd = j / kStages;
-        if (rd > 0 &&
-            !mbar_wait_bounded(&bars->v_empty[st], (rd - 1) & 1, abort_flag, kWaitLimitNs))
-          break;
-        const int k = k_begin + j;
-        const CUtensorMap* map = k < np ? &tmVp : &tmVc;
-        const int row0 = k < np ? p0 + k * BN : b * p.C + (k - np) * BN;
-        uint8_t* dst = smem + kOffV + st * kKTile;
-        mbar_arrive_expect_tx(&bars->v_full[st], kKTile);
-        tma_load_3d(dst, map, &bars->v_full[st], 0, g, row0);
-        tma_load_3d(dst + kKHalf, map, &bars->v_full[st], 64, g, row0);
-        issued = j + 1;
+      mbar_arrive_expect_tx(&bars->q_full, nq * kTile);
+      for (int q = 0; q < nq; ++q) {
+        const int qpos = b * p.C + (tp * kQT + q) * (BM / p.group);
+        uint8_t* dst = smem + kOffQ + q * kTile;
+        tma_load_3d(dst, &tmQ, &bars->q_full, 0, g * p.group, qpos);
+        tma_load_3d(dst + kHalf, &tmQ, &bars->q_full, 64, g * p.group, qpos);
       }
-      for (int j = max(0, issued - kStages); j < issued; ++j)
+      // in the order the MMAs consume them: K0, then V_j, K_{j+1}
+      int kiss = 0, viss = 0;
+      if (load_kv(bars, smem, 0, 0, k_begin, np, p0, b, p.C, g, &tmKp, &tmVp, &tmKc, &tmVc,
+                  abort_flag)) {
+        kiss = 1;
+        for (int j = 0; j < n; ++j) {
+          if (!load_kv(bars, smem, j, 1, k_begin, np, p0, b, p.C, g, &tmKp, &tmVp, &tmKc, &tmVc,
+                       abort_flag))
+            break;
+          viss = j + 1;
+          if (j + 1 < n) {
+            if (!load_kv(bars, smem, j + 1, 0, k_begin, np, p0, b, p.C, g, &tmKp, &tmVp, &tmKc,
+                         &tmVc, abort_flag))
+              break;
+            kiss = j + 2;
+          }
+        }
+      }
+      // drain: loads still in flight must land before the CTA exits
+      for (int j = max(0, kiss - kStages); j < kiss; ++j)
+        mbar_wait_bounded(&bars->k_full[j % kStages], (j / kStages) & 1, nullptr, kWaitLimitNs);
+      for (int j = max(0, viss - kStages); j < viss; ++j)
         mbar_wait_bounded(&bars->v_full[j % kStages], (j / kStages) & 1, nullptr, kWaitLimitNs);
+      mbar_wait_bounded(&bars->q_full, 0, nullptr, kWaitLimitNs);
     }
     __syncwarp();
   } else if (warp == kWarpMMA) {
     if (lane == 0 && n > 0) {
-      constexpr uint32_t idS = idesc_bf16_f32(BM, BN, 0, 0);
       constexpr uint32_t idPV = idesc_bf16_f32(BM, HD, 0, 1);
       const uint32_t sQ = smem_u32(smem + kOffQ);
       const uint32_t sK = smem_u32(smem + kOffK);
       const uint32_t sV = smem_u32(smem + kOffV);
-      const uint32_t sP = smem_u32(smem + kOffP);
-      bool ok = mbar_wait_bounded(&bars->q_full, 0, abort_flag, kWaitLimitNs);
+      bool ok = mbar_wait_bounded(&bars->q_full, 0, abort_flag, kWaitLimitNs) &&
+                mbar_wait_bounded(&bars->k_full[0], 0, abort_flag, kWaitLimitNs);
       tc_fence_after();
-      for (int j = 0; ok && j <= n; ++j) {
-        if (j < n) {
-          const int st = j % kStages, sb = j & 1;
-          if (!mbar_wait_bounded(&bars->k_full[st], (j / kStages) & 1, abort_flag,
-                                 kWaitLimitNs)) {
-            ok = false;
-            break;
-          }
-          for (int q = 0; q < nq; ++q) {
-            // S buffer sb of query tile q was last read by the softmax of tile j-2
-            if (j >= 2 && !mbar_wait_bounded(&bars->p_full[q][sb], ((j - 2) >> 1) & 1,
-                                              abort_flag, kWaitLimitNs)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint32_t dS = tmem + (uint32_t)((q * 2 + sb) * BN);
-#pragma unroll
-            for (int kk = 0; kk < HD / 16; ++kk) {
-              const uint32_t offQ = q * kQTile + (kk >> 2) * kQHalf + (kk & 3) * 32;
-              const uint32_t offK = st * kKTile + (kk >> 2) * kKHalf + (kk & 3) * 32;
-              tc_mma_ss(dS, smem_desc_sw128(sQ + offQ, 16, 1024),
-                        smem_desc_sw128(sK + offK, 16, 1024), idS, kk > 0);
-            }
-            tc_commit(&bars->s_full[q][sb]);
-          }
-          if (!ok) break;
-          tc_commit(&bars->k_empty[st]);
+      if (ok) {
+        for (int q = 0; q < nq; ++q) {
+          issue_s(tmem, sQ, sK, q, 0);
+          tc_commit(&bars->s_full[q]);
         }
-        if (j >= 1) {
-          const int jj = j - 1, st = jj % kStages, pb = jj & 1;
-          if (!mbar_wait_bounded(&bars->v_full[st], (jj / kStages) & 1, abort_flag,
-                                 kWaitLimitNs)) {
-            ok = false;
-            break;
-          }
-          for (int q = 0; q < nq; ++q) {
-            if (!mbar_wait_bounded(&bars->p_full[q][pb], (jj >> 1) & 1, abort_flag,
-                                   kWaitLimitNs)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint32_t dO = tmem + kTmemO + (uint32_t)(q * HD);
-#pragma unroll
-            for (int kk = 0; kk < BN / 16; ++kk) {
-              const uint32_t offP = (q * 2 + pb) * kPTile + kk * 32;
-              const uint32_t offV = st * kKTile + kk * 16 * 128;
-              tc_mma_ss(dO, smem_desc_sw128(sP + offP, 16, 1024),
-                        smem_desc_sw128(sV + offV, kKHalf, 1024), idPV,
-                        (jj > 0 || kk > 0) ? 1u : 0u);
-            }
-            tc_commit(&bars->pv_done[q][pb]);
-          }
-          if (!ok) break;
-          tc_commit(&bars->v_empty[st]);
-        }
+        tc_commit(&bars->k_empty[0]);
       }
+      for (int j = 0; ok && j < n; ++j) {
+        const int vst = j % kStages;
+        const bool more = j + 1 < n;
+        const int kst = (j + 1) % kStages;
+        if (!mbar_wait_bounded(&bars->v_full[vst], (j / kStages) & 1, abort_flag, kWaitLimitNs)) {
+          ok = false;
+          break;
+        }
+        for (int q = 0; q < nq; ++q) {
+          if (!mbar_wait_bounded(&bars->p_full[q], j & 1, abort_flag, kWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          // O_q += P_q(j) V_j, P_q from TMEM (8 columns per 16 keys)
+          const uint32_t dO = tmem + kTmemO + (uint32_t)(q * HD);
+          const uint32_t aP = tmem + (uint32_t)(q * BN);
+#pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk) {
+            const uint32_t offV = vst * kTile + kk * 16 * 128;
+            tc_mma_ts(dO, aP + (uint32_t)(kk * 8), smem_desc_sw128(sV + offV, kHalf, 1024), idPV,
+                      (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          if (more) {
+            if (q == 0 && !mbar_wait_bounded(&bars->k_full[kst], ((j + 1) / kStages) & 1,
+                                             abort_flag, kWaitLimitNs)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_s(tmem, sQ, sK, q, kst);
+            tc_commit(&bars->s_full[q]);
+          }
+        }
+        if (!ok) break;
+        tc_commit(&bars->v_empty[vst]);
+        if (more) tc_commit(&bars->k_empty[kst]);
+      }
+      if (ok)
+        for (int q = 0; q < nq; ++q) tc_commit(&bars->o_done[q]);
       // every MMA issued above has completed before TMEM is released
       tc_commit(&bars->mma_final);
       mbar_wait_bounded(&bars->mma_final, 0, nullptr, kWaitLimitNs);
@@ -305,17 +308,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q = warp >> 2, wl = warp & 3;
     const int r = wl * 32 + lane;                         // query row in tile q
     const uint32_t lane_base = (uint32_t)(wl * 32) << 16;  // TMEM lane field
-    uint8_t* sPq = smem + kOffP + q * 2 * kPTile;
+    const uint32_t tS = tmem + lane_base + (uint32_t)(q * BN);
+    const uint32_t tO = tmem + lane_base + kTmemO + (uint32_t)(q * HD);
     const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < n && ok; ++j) {
-      const int sb = j & 1;
       const int k = k_begin + j;
       const int n_valid = k < np ? min(BN, L - k * BN) : min(BN, p.C - (k - np) * BN);
       // wait outcomes are made warp-uniform: tcgen05.ld/st are .sync.aligned
-      if (!__all_sync(0xffffffffu, mbar_wait_bounded(&bars->s_full[q][sb], (j >> 1) & 1,
-                                                     abort_flag, kWaitLimitNs))) {
+      if (!__all_sync(0xffffffffu,
+                      mbar_wait_bounded(&bars->s_full[q], j & 1, abort_flag, kWaitLimitNs))) {
         ok = false;
         break;
       }
@@ -323,7 +326,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       float sv[BN];
       {
         uint32_t raw[BN];
-        tmem_ld64(tmem + lane_base + (uint32_t)((q * 2 + sb) * BN), raw);
+        tmem_ld128(tS, raw);
 #pragma unroll
         for (int c = 0; c < BN; ++c) sv[c] = __uint_as_float(raw[c]);
       }
@@ -339,72 +342,54 @@ __global__ void __launch_bounds__(kThreads, 1)
         mx1 = fmaxf(mx1, sv[c + 1]);
       }
       const float mx = fmaxf(mx0, mx1) * p.scale_log2;
-      // P buffer sb was last read by PV of tile j-2
-      if (j >= 2 &&
-          !__all_sync(0xffffffffu, mbar_wait_bounded(&bars->pv_done[q][sb], ((j - 2) >> 1) & 1,
-                                                     abort_flag, kWaitLimitNs))) {
-        ok = false;
-        break;
-      }
-      // lazy rescale (warp-uniform decision so tcgen05.ld/st stay converged)
+      // lazy rescale (warp-uniform decision so tcgen05.ld/st stay converged);
+      // PV_q(j-1) is complete because S_q(j) is
       if (__any_sync(0xffffffffu, mx > m_ref + kLazyRescale)) {
         const float m_new = fmaxf(m_ref, mx);
         const float alpha = ex2_approx(m_ref - m_new);  // 0 when m_ref = -inf
         l *= alpha;
         if (j >= 1) {
-          const int pj = j - 1;
-          if (!__all_sync(0xffffffffu,
-                          mbar_wait_bounded(&bars->pv_done[q][pj & 1], (pj >> 1) & 1, abort_flag,
-                                            kWaitLimitNs))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
+          // 8 columns at a time: the S row stays live in registers meanwhile
+#pragma unroll 1
+          for (int c8 = 0; c8 < HD / 8; ++c8) {
+            uint32_t raw[8];
+            tmem_ld8(tO + (uint32_t)(c8 * 8), raw);
 #pragma unroll
-          for (int c4 = 0; c4 < HD / 32; ++c4) {
-            uint32_t raw[32];
-            const uint32_t ta = tmem + lane_base + kTmemO + (uint32_t)(q * HD + c4 * 32);
-            tmem_ld32(ta, raw);
-#pragma unroll
-            for (int c = 0; c < 32; ++c) raw[c] = __float_as_uint(__uint_as_float(raw[c]) * alpha);
-            tmem_st32(ta, raw);
+            for (int c = 0; c < 8; ++c) raw[c] = __float_as_uint(__uint_as_float(raw[c]) * alpha);
+            tmem_st8(tO + (uint32_t)(c8 * 8), raw);
           }
-          tmem_wait_st();
         }
         m_ref = m_new;
       }
-      // P = 2^(s * scale_log2 - m_ref) as bf16, one 128-byte swizzled row
+      // P = 2^(s * scale_log2 - m_ref) as bf16 pairs into TMEM columns 0..63
       const float2 nm = make_float2(-m_ref, -m_ref);
       float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                        make_float2(0.f, 0.f)};
-      uint8_t* prow = sPq + sb * kPTile + r * 128;
 #pragma unroll
-      for (int cc = 0; cc < BN / 8; ++cc) {
-        uint32_t w[4];
+      for (int h = 0; h < BN / 16; ++h) {  // 16 keys -> 8 packed columns per store
+        uint32_t w[8];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int c = cc * 8 + 2 * e;
+        for (int e = 0; e < 8; ++e) {
+          const int c = h * 16 + 2 * e;
           const float2 d = __ffma2_rn(make_float2(sv[c], sv[c + 1]), sl2, nm);
           const float2 pp = make_float2(ex2_approx(d.x), ex2_approx(d.y));
-          acc[e] = __fadd2_rn(acc[e], pp);
+          acc[e & 3] = __fadd2_rn(acc[e & 3], pp);
           w[e] = pack_bf16x2(pp.x, pp.y);
         }
-        *reinterpret_cast<uint4*>(prow + ((cc ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+        tmem_st8(tS + (uint32_t)(h * 8), w);
       }
       const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
       const float2 a = __fadd2_rn(a01, a23);
       l += a.x + a.y;
-      fence_proxy_async_smem();
+      tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->p_full[q][sb]);
+      if (lane == 0) mbar_arrive(&bars->p_full[q]);
     }
     // epilogue: O / l and the log2-domain LSE of this split
-    if (ok) {
-      const int last = n - 1;
-      ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->pv_done[q][last & 1],
-                                                     (last >> 1) & 1, abort_flag, kWaitLimitNs));
-    }
+    if (ok)
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait_bounded(&bars->o_done[q], 0, abort_flag, kWaitLimitNs));
     if (ok) {
       tc_fence_after();
       const float inv = 1.f / l;
@@ -413,7 +398,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int c4 = 0; c4 < HD / 32; ++c4) {
         uint32_t raw[32];
-        tmem_ld32(tmem + lane_base + kTmemO + (uint32_t)(q * HD + c4 * 32), raw);
+        tmem_ld32(tO + (uint32_t)(c4 * 32), raw);
 #pragma unroll
         for (int c = 0; c < 32; c += 4)
           *reinterpret_cast<float4*>(orow + c4 * 32 + c) =
