@@ -45,6 +45,51 @@ __device__ __forceinline__ uint4 philox4x32_10(uint4 c, const PhiloxKey& k) {
   return c;
 }
 
+// Philox4x32-10 for counters (c, y, z, w) whose last three words are fixed
+// (one row, one step, one stream) and only c varies.  Round 1 multiplies
+// words 0 and 2; with z fixed its product is fixed, and round 2's product of
+// word 0 is then fixed as well, so those two products (and the xors that
+// use only fixed words) are computed once.  Same outputs as philox4x32_10.
+struct PhiloxRow {
+  uint32_t r1_y0, r1_y1;     // round-1 outputs 0 and 1 (fixed)
+  uint32_t r2_hi0k, r2_lo0;  // round 2: hi(M0 * r1_y0) ^ k1[1], lo(M0 * r1_y0)
+  uint32_t r2_k0y1;          // r1_y1 ^ k0[1]
+};
+
+__device__ __forceinline__ PhiloxRow philox_row(uint32_t y, uint32_t z, uint32_t w,
+                                                const PhiloxKey& k) {
+  PhiloxRow h;
+  const uint64_t p1 = (uint64_t)0xCD9E8D57u * z;
+  h.r1_y0 = (uint32_t)(p1 >> 32) ^ y ^ k.k0[0];
+  h.r1_y1 = (uint32_t)p1;
+  const uint64_t q0 = (uint64_t)0xD2511F53u * h.r1_y0;
+  h.r2_hi0k = (uint32_t)(q0 >> 32) ^ k.k1[1];
+  h.r2_lo0 = (uint32_t)q0;
+  h.r2_k0y1 = h.r1_y1 ^ k.k0[1];
+  (void)w;
+  return h;
+}
+
+// w is folded into round 1 here (word 3 enters only through hi(M0 c) ^ w).
+__device__ __forceinline__ uint4 philox4x32_10_row(uint32_t c, uint32_t w, const PhiloxRow& h,
+                                                   const PhiloxKey& k) {
+  // round 1: word 0 varies
+  const uint64_t p0 = (uint64_t)0xD2511F53u * c;
+  const uint32_t x2 = (uint32_t)(p0 >> 32) ^ w ^ k.k1[0];
+  const uint32_t x3 = (uint32_t)p0;
+  // round 2: the product of word 0 (= r1_y0) is fixed
+  const uint64_t p1 = (uint64_t)0xCD9E8D57u * x2;
+  uint4 x = make_uint4((uint32_t)(p1 >> 32) ^ h.r2_k0y1, (uint32_t)p1, h.r2_hi0k ^ x3, h.r2_lo0);
+#pragma unroll
+  for (int r = 2; r < 10; ++r) {
+    const uint64_t a = (uint64_t)0xD2511F53u * x.x;
+    const uint64_t b = (uint64_t)0xCD9E8D57u * x.z;
+    x = make_uint4((uint32_t)(b >> 32) ^ x.y ^ k.k0[r], (uint32_t)b,
+                   (uint32_t)(a >> 32) ^ x.w ^ k.k1[r], (uint32_t)a);
+  }
+  return x;
+}
+
 // Single-block helper for the per-row streams (counter word 0 = 0, word 0).
 __device__ __forceinline__ uint32_t philox_word0(uint64_t seed, uint32_t row, uint32_t step,
                                                  uint32_t stream) {

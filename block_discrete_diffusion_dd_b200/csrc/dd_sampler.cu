@@ -226,19 +226,37 @@ constexpr uint32_t kStageBytes = 32768;  // logits per CTA (one bulk copy)
 template <typename T>
 __host__ __device__ constexpr int chunk_elems() { return (int)(kStageBytes / sizeof(T)); }
 
+// Gumbel scores order like floats; as ints for atomicMax on shared memory.
+__device__ __forceinline__ int ord_float(float f) {
+  const int b = __float_as_int(f);
+  return b ^ ((b >> 31) & 0x7fffffff);
+}
+__device__ __forceinline__ float unord_float(int o) {
+  return __int_as_float(o ^ ((o >> 31) & 0x7fffffff));
+}
+
 // One item = 8 consecutive entries x[0..7] (floored, finite) starting at v0,
 // with bm = their max.  `src` points at the item's first entry (in shared
 // memory, or in global memory on the scalar path) and is re-read only on the
-// rare exact path.
+// rare exact path.  best_w is the warp's view of the best Gumbel score so far;
+// cta_best holds the best over the whole CTA (ordered int), which every warp
+// adopts when it is higher than its own.
 template <typename T>
 __device__ __forceinline__ void process_item(Run& st, float& best_w, float& Kp, const float (&x)[8],
                                              float bm, uint32_t v0, bool seed, const T* src,
-                                             const PhiloxKey& key, uint32_t grow, uint32_t step,
-                                             float c2, float inv_tau) {
+                                             const PhiloxKey& key, const PhiloxRow& prow,
+                                             float c2, float inv_tau, int* cta_best) {
   const float ym = bm * c2;
   if (ym > st.m + kLazy) {  // rare after the first item
     raise_ref(st, ym);
     Kp = prune_factor(st.m, best_w);
+  }
+  {
+    const float cb = unord_float(*reinterpret_cast<volatile int*>(cta_best));
+    if (cb > best_w) {
+      best_w = cb;
+      Kp = prune_factor(st.m, best_w);
+    }
   }
   const float2 c22 = make_float2(c2, c2);
   const float2 nm = make_float2(-st.m, -st.m);
@@ -251,8 +269,8 @@ __device__ __forceinline__ void process_item(Run& st, float& best_w, float& Kp, 
     st.t2 = __ffma2_rn(p[j], d, st.t2);
   }
   // Gumbel words for the 8 entries: two Philox blocks.
-  const uint4 wa = philox4x32_10(make_uint4(v0 >> 2, grow, step, 0u), key);
-  const uint4 wb = philox4x32_10(make_uint4((v0 >> 2) + 1u, grow, step, 0u), key);
+  const uint4 wa = philox4x32_10_row(v0 >> 2, 0u, prow, key);
+  const uint4 wb = philox4x32_10_row((v0 >> 2) + 1u, 0u, prow, key);
   bool changed = false;
   if (seed) {
     // seed the threshold with the exact score of this lane's largest entry
@@ -267,7 +285,8 @@ __device__ __forceinline__ void process_item(Run& st, float& best_w, float& Kp, 
       st.idx = (int)(v0 + (uint32_t)j);
     }
     // the seeded threshold applies to this item's own test below
-    best_w = warp_max(st.best);
+    best_w = fmaxf(best_w, warp_max(st.best));
+    if ((threadIdx.x & 31) == 0) atomicMax(cta_best, ord_float(best_w));
     Kp = prune_factor(st.m, best_w);
   }
   // Exponential-race prune: the score z - ln E (E = -ln U) can beat best_w
@@ -278,32 +297,42 @@ __device__ __forceinline__ void process_item(Run& st, float& best_w, float& Kp, 
   const float2 kk = make_float2(-Kp, -Kp);
   const float2 cc = make_float2(1.99999988079071044921875f, 1.99999988079071044921875f);
   const uint32_t w[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
-  uint32_t cmask = 0;
+  float thr[8];
+  bool any = false;
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     const float2 t = __ffma2_rn(p[j], kk, cc);
-    cmask |= (__uint_as_float(0x3F800000u | (w[2 * j] >> 9)) > t.x) ? (1u << (2 * j)) : 0u;
-    cmask |= (__uint_as_float(0x3F800000u | (w[2 * j + 1] >> 9)) > t.y) ? (2u << (2 * j)) : 0u;
+    thr[2 * j] = t.x;
+    thr[2 * j + 1] = t.y;
+    any |= __uint_as_float(0x3F800000u | (w[2 * j] >> 9)) > t.x;
+    any |= __uint_as_float(0x3F800000u | (w[2 * j + 1] >> 9)) > t.y;
   }
-  // rare exact path: one entry at a time (the logit re-read, its word
-  // selected from the two blocks above), so the code below exists once
-  while (cmask) {
-    const int i = __ffs(cmask) - 1;
-    cmask &= cmask - 1;
-    const float xi = fmaxf((float)src[i], kFloorLogit);
-    const uint32_t v = v0 + (uint32_t)i;
-    const uint4 wq = i < 4 ? wa : wb;
-    const int i4 = i & 3;
-    const uint32_t wi = i4 == 0 ? wq.x : i4 == 1 ? wq.y : i4 == 2 ? wq.z : wq.w;
-    const float sc = gumbel_score(xi * inv_tau, wi);
-    if (sc > st.best || (sc == st.best && (int)v < st.idx)) {
-      st.best = sc;
-      st.idx = (int)v;
-      changed = true;
+  if (any) {
+    // rare exact path: one entry at a time (the logit re-read, its word
+    // selected from the two blocks above), so the code below exists once
+    uint32_t cmask = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      cmask |= (__uint_as_float(0x3F800000u | (w[i] >> 9)) > thr[i]) ? (1u << i) : 0u;
+    while (cmask) {
+      const int i = __ffs(cmask) - 1;
+      cmask &= cmask - 1;
+      const float xi = fmaxf((float)src[i], kFloorLogit);
+      const uint32_t v = v0 + (uint32_t)i;
+      const uint4 wq = i < 4 ? wa : wb;
+      const int i4 = i & 3;
+      const uint32_t wi = i4 == 0 ? wq.x : i4 == 1 ? wq.y : i4 == 2 ? wq.z : wq.w;
+      const float sc = gumbel_score(xi * inv_tau, wi);
+      if (sc > st.best || (sc == st.best && (int)v < st.idx)) {
+        st.best = sc;
+        st.idx = (int)v;
+        changed = true;
+      }
     }
   }
   if (__any_sync(0xffffffffu, changed)) {
-    best_w = warp_max(st.best);
+    best_w = fmaxf(best_w, warp_max(st.best));
+    if ((threadIdx.x & 31) == 0) atomicMax(cta_best, ord_float(best_w));
     Kp = prune_factor(st.m, best_w);
   }
 }
@@ -321,6 +350,7 @@ __global__ void __launch_bounds__(kSampleThreads, 4)
   constexpr int kItems = kElems / (kSampleThreads * 8);
   __shared__ __align__(128) uint8_t buf[kStageBytes];
   __shared__ uint64_t bar;
+  __shared__ int cta_best;
   const int row = blockIdx.x / nchunk;
   const int chunk = blockIdx.x - row * nchunk;
   const int c0 = chunk * kElems;
@@ -328,6 +358,7 @@ __global__ void __launch_bounds__(kSampleThreads, 4)
   if (threadIdx.x == 0) {
     mbar_init(&bar, 1);
     fence_mbar_init();
+    cta_best = ord_float(-INFINITY);
   }
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -336,6 +367,7 @@ __global__ void __launch_bounds__(kSampleThreads, 4)
   }
   const PhiloxKey key = philox_key(seed);
   const uint32_t grow = row_offset + (uint32_t)row;
+  const PhiloxRow prow = philox_row(grow, step, 0u, key);
   const float c2 = inv_tau * kLog2e;
   Run st{-INFINITY, make_float2(0.f, 0.f), make_float2(0.f, 0.f), -INFINITY, 0x7fffffff};
   float best_w = -INFINITY, Kp = 0.f;
@@ -362,8 +394,8 @@ __global__ void __launch_bounds__(kSampleThreads, 4)
       for (int i = 0; i < 8; ++i) x[i] = kFloorLogit;
       bm = kFloorLogit;
     }
-    process_item<T>(st, best_w, Kp, x, bm, (uint32_t)(c0 + e), k == 0, tb + e, key, grow, step,
-                    c2, inv_tau);
+    process_item<T>(st, best_w, Kp, x, bm, (uint32_t)(c0 + e), k == 0, tb + e, key, prow, c2,
+                    inv_tau, &cta_best);
   }
   write_record(st, recs + (int64_t)row * nchunk + chunk);
 }
@@ -384,9 +416,13 @@ __global__ void __launch_bounds__(kSampleThreads)
   const T* rowp = logits + (int64_t)row * row_stride;
   const PhiloxKey key = philox_key(seed);
   const uint32_t grow = row_offset + (uint32_t)row;
+  const PhiloxRow prow = philox_row(grow, step, 0u, key);
   const float c2 = inv_tau * kLog2e;
   Run st{-INFINITY, make_float2(0.f, 0.f), make_float2(0.f, 0.f), -INFINITY, 0x7fffffff};
   float best_w = -INFINITY, Kp = 0.f;
+  __shared__ int cta_best;
+  if (threadIdx.x == 0) cta_best = ord_float(-INFINITY);
+  __syncthreads();
 #pragma unroll 1
   for (int k = 0; k < kItems; ++k) {
     const int v0 = c0 + (k * kSampleThreads + (int)threadIdx.x) * 8;
@@ -397,8 +433,8 @@ __global__ void __launch_bounds__(kSampleThreads)
     float bm = x[0];
 #pragma unroll
     for (int i = 1; i < 8; ++i) bm = fmaxf(bm, x[i]);
-    process_item<T>(st, best_w, Kp, x, bm, (uint32_t)v0, k == 0, rowp + v0, key, grow, step,
-                    c2, inv_tau);
+    process_item<T>(st, best_w, Kp, x, bm, (uint32_t)v0, k == 0, rowp + v0, key, prow, c2,
+                    inv_tau, &cta_best);
   }
   write_record(st, recs + (int64_t)row * nchunk + chunk);
 }
