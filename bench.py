@@ -358,29 +358,39 @@ def _profile_traffic() -> dict:
     return out
 
 
-def cpu_baseline(w, s, frac: float):
+def cpu_baseline(w, s, frac: float, budget_s: float = 10.0):
     """The oracle, as it stands, on this host's cores, on a bounded sample of
-    one step (a fraction `frac` of the canvas positions for attention and of
-    the rows for the sampler), scaled to a whole step."""
+    the workload: slices of `frac` of the canvas positions (attention, all
+    heads) and of the rows (sampler), repeated over different positions and
+    rows for about `budget_s` seconds, scaled to whole steps."""
     import oracle
     oracle.build()
     npos = max(1, int(round(w.canvas * frac)))
     rows = max(1, int(round(w.rows * frac)))
-    pos = np.linspace(0, w.canvas - 1, npos).astype(np.int32)
-    sel = np.linspace(0, w.rows - 1, rows).astype(np.int64)
     q, kc, vc, kp, vp = (s[k].cpu() for k in ("q", "kc", "vc", "kp", "vp"))
     lg = s["logits"].cpu()
-    t0 = time.perf_counter()
-    oracle.canvas_attn(q, kc, vc, kp, vp, s["cu_host"], w.scale, positions=pos)
-    t1 = time.perf_counter()
-    oracle.sample_renoise(lg, w.temperatures[0], w.rates[0], w.seed, 0, rows=sel)
-    t2 = time.perf_counter()
-    step_s = (t1 - t0) * (w.canvas / npos) + (t2 - t1) * (w.rows / rows)
+    t_attn = t_samp = 0.0
+    reps = 0
+    t_start = time.perf_counter()
+    while reps == 0 or time.perf_counter() - t_start < budget_s:
+        off = (reps * 37) % w.canvas
+        pos = ((np.arange(npos) * (w.canvas // npos) + off) % w.canvas).astype(np.int32)
+        sel = ((np.arange(rows) * (w.rows // rows) + off) % w.rows).astype(np.int64)
+        t0 = time.perf_counter()
+        oracle.canvas_attn(q, kc, vc, kp, vp, s["cu_host"], w.scale, positions=pos)
+        t1 = time.perf_counter()
+        oracle.sample_renoise(lg, w.temperatures[0], w.rates[0], w.seed, reps, rows=sel)
+        t2 = time.perf_counter()
+        t_attn += t1 - t0
+        t_samp += t2 - t1
+        reps += 1
+    step_s = (t_attn * (w.canvas / npos) + t_samp * (w.rows / rows)) / reps
     cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
     return {"value": w.batch / step_s, "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": f"{npos}/{w.canvas} canvas positions (all heads) for attention and "
-                      f"{rows}/{w.rows} sampler rows of one step, float64, scaled to a step",
-            "seconds": t2 - t0}
+            "sample": f"{reps} x ({npos}/{w.canvas} canvas positions, all heads, for attention "
+                      f"+ {rows}/{w.rows} sampler rows), float64, {t_attn + t_samp:.1f} s of "
+                      "wall time on all host cores, scaled to whole steps",
+            "seconds": t_attn + t_samp}
 
 
 def run_reference(args, w, dist, rank, world):
