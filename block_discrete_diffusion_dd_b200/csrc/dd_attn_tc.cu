@@ -17,16 +17,19 @@
 // of CTAs cover the SMs; a second kernel merges the splits by their
 // log-sum-exp.
 //
-// Inside a CTA (10 warps) the two query tiles share every key tile:
-//   warps 0-3 / 4-7  softmax of query tile 0 / 1: one query row per thread
-//              (= one TMEM lane).  Each reads S (fp32, 128 columns) from
-//              TMEM, runs the online softmax in fp32 (log2 domain; O is
-//              rescaled only when the running max grows by more than 2^8)
-//              and writes P back as bf16 into the first 64 columns of the
-//              same TMEM region, where the P.V MMA reads it directly;
-//   warp 8     TMA producer: Q, then K and V tiles (2-stage rings of 128
+// Inside a CTA (18 warps) the two query tiles share every key tile:
+//   warps 0-7 / 8-15  softmax of query tile 0 / 1.  A query row (= one TMEM
+//              lane) is shared by two threads in two warps, one per half of
+//              the 128 key columns; they meet once per tile in shared
+//              memory to agree on the row max.  Each half reads its 64 S
+//              columns (fp32) from TMEM, runs the online softmax in fp32
+//              (log2 domain; O is rescaled only when the running max grows
+//              by more than 2^8) and writes its half of P back as bf16 into
+//              its own half of the same TMEM region (columns 0-31 and
+//              64-95), where the P.V MMA reads it directly;
+//   warp 16    TMA producer: Q, then K and V tiles (2-stage rings of 128
 //              keys) in the order the MMAs consume them;
-//   warp 9     allocates all 512 TMEM columns (per query tile: S/P 128, O
+//   warp 17    allocates all 512 TMEM columns (per query tile: S/P 128, O
 //              128) and issues every MMA from one thread, in the order
 //              PV_0(j), S_0(j+1), PV_1(j), S_1(j+1): each softmax warpgroup
 //              works while the tensor core runs the other tile's MMAs.
@@ -49,23 +52,32 @@ constexpr int BN = 128;  // keys per tile
 constexpr int HD = 128;  // head dim
 constexpr int kQT = 2;   // query tiles per CTA
 constexpr int kStages = 2;
-constexpr int kWarpTMA = 8, kWarpMMA = 9;
-constexpr int kThreads = 10 * 32;
+constexpr int kSoftmaxWarps = 8 * kQT;  // two warps per 32 query rows
+constexpr int kWarpTMA = kSoftmaxWarps, kWarpMMA = kSoftmaxWarps + 1;
+constexpr int kThreads = (kSoftmaxWarps + 2) * 32;
 constexpr uint32_t kHalf = 128 * 64 * 2;  // 128 rows x 128 bytes
 constexpr uint32_t kTile = 2 * kHalf;     // 128 x 128 bf16
 constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffK = kOffQ + kQT * kTile;
 constexpr uint32_t kOffV = kOffK + kStages * kTile;
-constexpr uint32_t kOffBar = kOffV + kStages * kTile;
+constexpr uint32_t kOffX = kOffV + kStages * kTile;  // row-max exchange [q][slot][half][row]
+constexpr uint32_t kOffBar = kOffX + kQT * 2 * 2 * BM * 4;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemO = kQT * BN;     // O columns start after the S/P regions
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per wait
 constexpr float kLazyRescale = 8.0f;              // log2 units
+#ifndef DD_POLY_PAIRS
+#define DD_POLY_PAIRS 0
+#endif
+// Of every 8 pairs of softmax exponentials, this many are evaluated by a
+// polynomial on the FMA pipe instead of the MUFU unit (balances the pipes).
+constexpr int kPolyPairs = DD_POLY_PAIRS;
 
 struct Barriers {
   uint64_t q_full;
   uint64_t k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
   uint64_t s_full[kQT], p_full[kQT], o_done[kQT];
+  uint64_t xch[kQT][4];  // per (query tile, 32-row group): the two column halves meet
   uint64_t mma_final;
   uint32_t tmem_base;
   int abort;
@@ -118,16 +130,23 @@ __device__ void resolve_unit(const TcParams& p, Barriers* bars) {
   bars->unit_slot0 = slots + (g * p.T + tp * kQT) * nsplit + s;
 }
 
+// Shared-memory descriptors are built once per CTA; an operand at byte
+// offset `off` from a 1024-aligned base has the base descriptor plus off/16
+// in its start-address field (bits 0-13; every address here is below 2^18,
+// so the field never carries).
+__device__ __forceinline__ uint64_t desc_at(uint64_t base, uint32_t off) {
+  return base + (uint64_t)(off >> 4);
+}
+
 // S_q = Q_q K^T into the S/P region of query tile q (K-major operands).
-__device__ __forceinline__ void issue_s(uint32_t tmem, uint32_t sQ, uint32_t sK, int q, int st) {
+__device__ __forceinline__ void issue_s(uint32_t tmem, uint64_t dQ, uint64_t dK, int q, int st) {
   constexpr uint32_t idS = idesc_bf16_f32(BM, BN, 0, 0);
   const uint32_t dS = tmem + (uint32_t)(q * BN);
+  const uint64_t aq = desc_at(dQ, q * kTile), bk = desc_at(dK, st * kTile);
 #pragma unroll
   for (int kk = 0; kk < HD / 16; ++kk) {
-    const uint32_t offQ = q * kTile + (kk >> 2) * kHalf + (kk & 3) * 32;
-    const uint32_t offK = st * kTile + (kk >> 2) * kHalf + (kk & 3) * 32;
-    tc_mma_ss(dS, smem_desc_sw128(sQ + offQ, 16, 1024), smem_desc_sw128(sK + offK, 16, 1024), idS,
-              kk > 0);
+    const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
+    tc_mma_ss(dS, desc_at(aq, off), desc_at(bk, off), idS, kk > 0);
   }
 }
 
@@ -174,8 +193,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int q = 0; q < kQT; ++q) {
       mbar_init(&bars->s_full[q], 1);
-      mbar_init(&bars->p_full[q], 4);
+      mbar_init(&bars->p_full[q], 8);
       mbar_init(&bars->o_done[q], 1);
+      for (int i = 0; i < 4; ++i) mbar_init(&bars->xch[q][i], 2);
     }
     mbar_init(&bars->mma_final, 1);
     bars->abort = 0;
@@ -245,15 +265,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kWarpMMA) {
     if (lane == 0 && n > 0) {
       constexpr uint32_t idPV = idesc_bf16_f32(BM, HD, 0, 1);
-      const uint32_t sQ = smem_u32(smem + kOffQ);
-      const uint32_t sK = smem_u32(smem + kOffK);
-      const uint32_t sV = smem_u32(smem + kOffV);
+      const uint64_t dQ = smem_desc_sw128(smem_u32(smem + kOffQ), 16, 1024);
+      const uint64_t dK = smem_desc_sw128(smem_u32(smem + kOffK), 16, 1024);
+      const uint64_t dV = smem_desc_sw128(smem_u32(smem + kOffV), kHalf, 1024);
       bool ok = mbar_wait_bounded(&bars->q_full, 0, abort_flag, kWaitLimitNs) &&
                 mbar_wait_bounded(&bars->k_full[0], 0, abort_flag, kWaitLimitNs);
       tc_fence_after();
       if (ok) {
         for (int q = 0; q < nq; ++q) {
-          issue_s(tmem, sQ, sK, q, 0);
+          issue_s(tmem, dQ, dK, q, 0);
           tc_commit(&bars->s_full[q]);
         }
         tc_commit(&bars->k_empty[0]);
@@ -275,12 +295,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           // O_q += P_q(j) V_j, P_q from TMEM (8 columns per 16 keys)
           const uint32_t dO = tmem + kTmemO + (uint32_t)(q * HD);
           const uint32_t aP = tmem + (uint32_t)(q * BN);
+          const uint64_t bv = desc_at(dV, vst * kTile);
+          // keys 0-63 are packed in columns 0-31, keys 64-127 in 64-95
 #pragma unroll
-          for (int kk = 0; kk < BN / 16; ++kk) {
-            const uint32_t offV = vst * kTile + kk * 16 * 128;
-            tc_mma_ts(dO, aP + (uint32_t)(kk * 8), smem_desc_sw128(sV + offV, kHalf, 1024), idPV,
-                      (j > 0 || kk > 0) ? 1u : 0u);
-          }
+          for (int kk = 0; kk < BN / 16; ++kk)
+            tc_mma_ts(dO, aP + (uint32_t)((kk >> 2) * (BN / 2) + (kk & 3) * 8),
+                      desc_at(bv, kk * 16 * 128), idPV, (j > 0 || kk > 0) ? 1u : 0u);
           if (more) {
             if (q == 0 && !mbar_wait_bounded(&bars->k_full[kst], ((j + 1) / kStages) & 1,
                                              abort_flag, kWaitLimitNs)) {
@@ -288,7 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               break;
             }
             tc_fence_after();
-            issue_s(tmem, sQ, sK, q, kst);
+            issue_s(tmem, dQ, dK, q, kst);
             tc_commit(&bars->s_full[q]);
           }
         }
@@ -303,17 +323,61 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait_bounded(&bars->mma_final, 0, nullptr, kWaitLimitNs);
     }
     __syncwarp();
-  } else if (warp < 4 * kQT && n > 0 && (warp >> 2) < nq) {
+  } else if (warp < kSoftmaxWarps && n > 0 && (warp >> 3) < nq) {
     // ------------------------------------------------------------ softmax
-    const int q = warp >> 2, wl = warp & 3;
+    const int q = warp >> 3, h = (warp >> 2) & 1, wl = warp & 3;
     const int r = wl * 32 + lane;                         // query row in tile q
     const uint32_t lane_base = (uint32_t)(wl * 32) << 16;  // TMEM lane field
     const uint32_t tS = tmem + lane_base + (uint32_t)(q * BN);
-    const uint32_t tO = tmem + lane_base + kTmemO + (uint32_t)(q * HD);
+    const uint32_t tO = tmem + lane_base + kTmemO + (uint32_t)(q * HD + h * (HD / 2));
+    float* xch = reinterpret_cast<float*>(smem + kOffX) + q * (2 * 2 * BM);
+    uint64_t* xbar = &bars->xch[q][wl];
     const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int j = 0; j < n && ok; ++j) {
+    // exchange a per-row value with the other column half (phase `ph`):
+    // post it, then (possibly after other work) wait for the partner's
+    auto post = [&](float v, int ph) {
+      xch[(ph & 1) * (2 * BM) + h * BM + r] = v;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(xbar);
+    };
+    auto take = [&](int ph) -> float {
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(xbar, ph & 1, abort_flag, kWaitLimitNs))) {
+        ok = false;
+        return -INFINITY;
+      }
+      return xch[(ph & 1) * (2 * BM) + (h ^ 1) * BM + r];
+    };
+    // P = 2^(s * scale_log2 - mref) as bf16 pairs into packed columns
+    // [h*64, h*64 + 32) of the S/P region: inside this half's own S columns,
+    // so it never overwrites S the other half has yet to read; returns the
+    // partial row sum
+    auto emit_p = [&](const float (&sv)[BN / 2], float mref) -> float {
+      const float2 nm = make_float2(-mref, -mref);
+      float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                       make_float2(0.f, 0.f)};
+#pragma unroll
+      for (int hh = 0; hh < BN / 32; ++hh) {  // 16 keys -> 8 packed columns per store
+        uint32_t w[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int c = hh * 16 + 2 * e;
+          const float2 d = __ffma2_rn(make_float2(sv[c], sv[c + 1]), sl2, nm);
+          // kPolyPairs of every 8 pairs take the FMA-pipe exponential
+          const float2 pp = e < kPolyPairs ? exp2_poly2(d)
+                                           : make_float2(ex2_approx(d.x), ex2_approx(d.y));
+          acc[e & 3] = __fadd2_rn(acc[e & 3], pp);
+          w[e] = pack_bf16x2(pp.x, pp.y);
+        }
+        tmem_st8(tS + (uint32_t)(h * (BN / 2) + hh * 8), w);
+      }
+      const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
+      const float2 a = __fadd2_rn(a01, a23);
+      return a.x + a.y;
+    };
+    int j = 0;
+    for (; j < n && ok; ++j) {
       const int k = k_begin + j;
       const int n_valid = k < np ? min(BN, L - k * BN) : min(BN, p.C - (k - np) * BN);
       // wait outcomes are made warp-uniform: tcgen05.ld/st are .sync.aligned
@@ -323,80 +387,83 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      float sv[BN];
+      float sv[BN / 2];
       {
-        uint32_t raw[BN];
-        tmem_ld128(tS, raw);
+        uint32_t raw[BN / 2];
+        tmem_ld64(tS + (uint32_t)(h * (BN / 2)), raw);
 #pragma unroll
-        for (int c = 0; c < BN; ++c) sv[c] = __uint_as_float(raw[c]);
+        for (int c = 0; c < BN / 2; ++c) sv[c] = __uint_as_float(raw[c]);
       }
-      if (n_valid < BN) {  // ragged last tile of the prefix or of the canvas
+      const int nv = n_valid - h * (BN / 2);  // valid columns in this half
+      if (nv < BN / 2) {  // ragged last tile of the prefix or of the canvas
 #pragma unroll
-        for (int c = 0; c < BN; ++c)
-          if (c >= n_valid) sv[c] = -INFINITY;
+        for (int c = 0; c < BN / 2; ++c)
+          if (c >= nv) sv[c] = -INFINITY;
       }
       float mx0 = sv[0], mx1 = sv[1];
 #pragma unroll
-      for (int c = 2; c < BN; c += 2) {
+      for (int c = 2; c < BN / 2; c += 2) {
         mx0 = fmaxf(mx0, sv[c]);
         mx1 = fmaxf(mx1, sv[c + 1]);
       }
-      const float mx = fmaxf(mx0, mx1) * p.scale_log2;
-      // lazy rescale (warp-uniform decision so tcgen05.ld/st stay converged);
-      // PV_q(j-1) is complete because S_q(j) is
-      if (__any_sync(0xffffffffu, mx > m_ref + kLazyRescale)) {
-        const float m_new = fmaxf(m_ref, mx);
-        const float alpha = ex2_approx(m_ref - m_new);  // 0 when m_ref = -inf
-        l *= alpha;
-        if (j >= 1) {
-          // 8 columns at a time: the S row stays live in registers meanwhile
+      const float mh = fmaxf(mx0, mx1);
+      post(mh, j);
+      float lt;
+      if (j == 0) {
+        // first tile: the reference is the row max itself
+        const float mx = fmaxf(mh, take(j)) * p.scale_log2;
+        if (!ok) break;
+        m_ref = mx;
+        lt = emit_p(sv, m_ref);
+      } else {
+        // later tiles: P with the current reference first; the row max
+        // (the partner's post has usually arrived by then) decides, rarely,
+        // that the reference must rise by more than 2^8 and P be redone
+        lt = emit_p(sv, m_ref);
+        const float mx = fmaxf(mh, take(j)) * p.scale_log2;
+        if (!ok) break;
+        // lazy rescale (warp-uniform decision so tcgen05.ld/st stay
+        // converged; both halves see the same row maxima, so they decide
+        // alike); PV_q(j-1) is complete because S_q(j) is
+        if (__any_sync(0xffffffffu, mx > m_ref + kLazyRescale)) {
+          const float m_new = fmaxf(m_ref, mx);
+          const float alpha = ex2_approx(m_ref - m_new);
+          l *= alpha;
 #pragma unroll 1
-          for (int c8 = 0; c8 < HD / 8; ++c8) {
+          for (int c8 = 0; c8 < HD / 16; ++c8) {
             uint32_t raw[8];
             tmem_ld8(tO + (uint32_t)(c8 * 8), raw);
 #pragma unroll
             for (int c = 0; c < 8; ++c) raw[c] = __float_as_uint(__uint_as_float(raw[c]) * alpha);
             tmem_st8(tO + (uint32_t)(c8 * 8), raw);
           }
+          m_ref = m_new;
+          lt = emit_p(sv, m_ref);
         }
-        m_ref = m_new;
       }
-      // P = 2^(s * scale_log2 - m_ref) as bf16 pairs into TMEM columns 0..63
-      const float2 nm = make_float2(-m_ref, -m_ref);
-      float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                       make_float2(0.f, 0.f)};
-#pragma unroll
-      for (int h = 0; h < BN / 16; ++h) {  // 16 keys -> 8 packed columns per store
-        uint32_t w[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int c = h * 16 + 2 * e;
-          const float2 d = __ffma2_rn(make_float2(sv[c], sv[c + 1]), sl2, nm);
-          const float2 pp = make_float2(ex2_approx(d.x), ex2_approx(d.y));
-          acc[e & 3] = __fadd2_rn(acc[e & 3], pp);
-          w[e] = pack_bf16x2(pp.x, pp.y);
-        }
-        tmem_st8(tS + (uint32_t)(h * 8), w);
-      }
-      const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
-      const float2 a = __fadd2_rn(a01, a23);
-      l += a.x + a.y;
+      l += lt;
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->p_full[q]);
     }
-    // epilogue: O / l and the log2-domain LSE of this split
+    // epilogue: O / l and the log2-domain LSE of this split; the halves add
+    // their partial row sums
     if (ok)
       ok = __all_sync(0xffffffffu,
                       mbar_wait_bounded(&bars->o_done[q], 0, abort_flag, kWaitLimitNs));
+    float lrow = l;
+    if (ok) {
+      post(l, n);
+      lrow = l + take(n);
+    }
     if (ok) {
       tc_fence_after();
-      const float inv = 1.f / l;
+      const float inv = 1.f / lrow;
       const size_t slot = (size_t)slot0 + (size_t)q * nsplit;
-      float* orow = p.part_o + (slot * BM + r) * HD;
+      float* orow = p.part_o + (slot * BM + r) * HD + h * (HD / 2);
 #pragma unroll
-      for (int c4 = 0; c4 < HD / 32; ++c4) {
+      for (int c4 = 0; c4 < HD / 64; ++c4) {
         uint32_t raw[32];
         tmem_ld32(tO + (uint32_t)(c4 * 32), raw);
 #pragma unroll
@@ -405,7 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               make_float4(__uint_as_float(raw[c]) * inv, __uint_as_float(raw[c + 1]) * inv,
                           __uint_as_float(raw[c + 2]) * inv, __uint_as_float(raw[c + 3]) * inv);
       }
-      p.part_lse[slot * BM + r] = m_ref + __log2f(l);
+      if (h == 0) p.part_lse[slot * BM + r] = m_ref + __log2f(lrow);
     }
   }
 
