@@ -64,6 +64,8 @@ constexpr uint32_t kOffX = kOffV + kStages * kTile;  // row-max exchange [q][slo
 constexpr uint32_t kOffBar = kOffX + kQT * 2 * 2 * BM * 4;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemO = kQT * BN;     // O columns start after the S/P regions
+constexpr int kStageStride = HD + 4;       // padded fp32 row of the O staging area
+static_assert(kQT * BM * kStageStride * 4 <= kOffX, "O staging fits the operand buffers");
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per wait
 constexpr float kLazyRescale = 8.0f;              // log2 units
 #ifndef DD_POLY_PAIRS
@@ -78,6 +80,7 @@ struct Barriers {
   uint64_t k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
   uint64_t s_full[kQT], p_full[kQT], o_done[kQT];
   uint64_t xch[kQT][4];  // per (query tile, 32-row group): the two column halves meet
+  uint64_t staged[kQT];  // per query tile: all 8 warps have staged their O rows
   uint64_t mma_final;
   uint32_t tmem_base;
   int abort;
@@ -196,6 +199,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->p_full[q], 8);
       mbar_init(&bars->o_done[q], 1);
       for (int i = 0; i < 4; ++i) mbar_init(&bars->xch[q][i], 2);
+      mbar_init(&bars->staged[q], 8);
     }
     mbar_init(&bars->mma_final, 1);
     bars->abort = 0;
@@ -458,21 +462,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       lrow = l + take(n);
     }
     if (ok) {
+      // O / l staged row-wise in shared memory (free now: every MMA has
+      // completed), then copied out in whole 512-byte rows
       tc_fence_after();
       const float inv = 1.f / lrow;
-      const size_t slot = (size_t)slot0 + (size_t)q * nsplit;
-      float* orow = p.part_o + (slot * BM + r) * HD + h * (HD / 2);
+      float* stage = reinterpret_cast<float*>(smem) + q * (BM * kStageStride);
+      float* srow = stage + r * kStageStride + h * (HD / 2);
 #pragma unroll
       for (int c4 = 0; c4 < HD / 64; ++c4) {
         uint32_t raw[32];
         tmem_ld32(tO + (uint32_t)(c4 * 32), raw);
 #pragma unroll
         for (int c = 0; c < 32; c += 4)
-          *reinterpret_cast<float4*>(orow + c4 * 32 + c) =
+          *reinterpret_cast<float4*>(srow + c4 * 32 + c) =
               make_float4(__uint_as_float(raw[c]) * inv, __uint_as_float(raw[c + 1]) * inv,
                           __uint_as_float(raw[c + 2]) * inv, __uint_as_float(raw[c + 3]) * inv);
       }
+      const size_t slot = (size_t)slot0 + (size_t)q * nsplit;
       if (h == 0) p.part_lse[slot * BM + r] = m_ref + __log2f(lrow);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->staged[q]);
+      if (__all_sync(0xffffffffu,
+                     mbar_wait_bounded(&bars->staged[q], 0, abort_flag, kWaitLimitNs))) {
+        float* dst = p.part_o + slot * BM * HD;
+        const int wq = warp & 7;  // warp index within this query tile's 8
+        for (int row = wq; row < BM; row += 8)
+          *reinterpret_cast<float4*>(dst + row * HD + lane * 4) =
+              *reinterpret_cast<const float4*>(stage + row * kStageStride + lane * 4);
+      }
     }
   }
 
