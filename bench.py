@@ -244,6 +244,7 @@ def run_ours(args, w, dist, rank, world, local_rank):
     samp_gbs = samp_bytes / t_samp / 1e9
     attn_tf = w.attn_flops() / t_attn / 1e12
     traffic = _profile_traffic()
+    clk = clocks.summary(t_wall0, t_wall1)
     res = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
@@ -256,10 +257,11 @@ def run_ours(args, w, dist, rank, world, local_rank):
                          f"{(w.logit_bytes() + 2 * sets[0]['kp'].numel() * 2) / 1e6:.0f} MB "
                          "(> 126 MB L2)",
                    "parallelism": f"replicas x{world}"},
-        "roofline": {"bound": "hbm", "kernel": "sampler (chunk pass + row merge)",
+        "roofline": {"bound": "hbm", "kernel": "sampler (scan pass + row merge)",
                      "achieved": samp_gbs, "peak": hbm, "unit": "GB/s", "frac": samp_gbs / hbm,
                      "traffic": traffic.get("sampler"), "peak_source": src,
-                     "algorithmic_bytes": samp_bytes, "ms": t_samp * 1e3},
+                     "algorithmic_bytes": samp_bytes, "ms": t_samp * 1e3,
+                     "alu_ceiling": _sampler_alu_ceiling(samp_gbs, clk.get("sm_mhz"))},
         "roofline_attn": {"bound": "tensor", "kernel": "canvas attention (tcgen05 + merge)",
                           "achieved": attn_tf, "peak": tf_burst, "unit": "TFLOP/s",
                           "frac": attn_tf / tf_burst, "frac_of_sustained": attn_tf / tf_sus,
@@ -267,11 +269,30 @@ def run_ours(args, w, dist, rank, world, local_rank):
                           "traffic": traffic.get("attention"), "peak_source": src},
         "e2e": e2e,
         "gpu_launches": int(launches),
-        "clocks": clocks.summary(t_wall0, t_wall1),
+        "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu:
         res["cpu_baseline"] = cpu_baseline(w, sets[0], frac=args.cpu_sample)
     return res
+
+
+# The sampler's arithmetic ceiling: per warp-item of 256 logits the scan
+# issues 2 Philox4x32-10 blocks x 18 IMAD.WIDE (two of the 20 products per
+# block are row-invariant and hoisted) plus 16 packed fp32 ops, all on the
+# FMA-heavy pipe of an SM sub-partition; the ncu counters of the scan kernel
+# (heavy-pipe cycles per IMAD) put an IMAD.WIDE at 4 cycles of that pipe and
+# a packed fp32 op at 2.  B200: 148 SMs x 4 sub-partitions.
+SAMPLER_HEAVY_CYCLES_PER_ITEM = 36 * 4 + 16 * 2
+B200_SUBPARTITIONS = 148 * 4
+
+
+def _sampler_alu_ceiling(achieved_gbs, sm_mhz):
+    if not sm_mhz:
+        return None
+    items_per_s = B200_SUBPARTITIONS * sm_mhz * 1e6 / SAMPLER_HEAVY_CYCLES_PER_ITEM
+    ceiling = items_per_s * 256 * 2 / 1e9  # GB/s of bf16 logits
+    return {"bound": "alu", "unit": "GB/s", "peak": ceiling, "frac": achieved_gbs / ceiling,
+            "sm_mhz": sm_mhz, "heavy_cycles_per_256_logits": SAMPLER_HEAVY_CYCLES_PER_ITEM}
 
 
 def _launches_per_step(dd, step) -> int:

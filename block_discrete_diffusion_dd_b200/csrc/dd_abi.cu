@@ -92,23 +92,29 @@ size_t attn_ws_bytes(const AttnArgs& a) {
   return kHeaderBytes + attn_simt_scratch_bytes(t);
 }
 
-size_t sample_ws_bytes(int rows, int vocab, dd_dtype dtype) {
-  return kHeaderBytes +
-         (size_t)rows * (size_t)sampler_nchunk(vocab, dtype == DD_BF16) * sizeof(ChunkRecord);
-}
-
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
-// Block-loop workspace: the attention and sampler scratch share one region
-// (they run one after the other on the stream), followed by a confidence
-// buffer used when the caller passes no conf_steps.
+// Sampler workspace: header, then the persistent state (ticket counter and
+// row keys, kept zero between calls), then the per-chunk records.
+size_t sample_ws_bytes(int rows, int vocab, dd_dtype dtype) {
+  (void)dtype;
+  return kHeaderBytes + align256(sampler_state_bytes(rows)) + sampler_record_bytes(rows, vocab);
+}
+
+// Block-loop workspace: the attention scratch and the sampler records share
+// one region (they run one after the other on the stream); the sampler's
+// persistent state and a confidence buffer (used when the caller passes no
+// conf_steps) follow it.
 size_t block_ws_layout(const dd_attn_desc* desc, int64_t total, const int32_t* cu_prefix_host,
-                       int vocab, size_t* conf_off) {
+                       int vocab, size_t* state_off, size_t* conf_off) {
+  const int rows = desc->batch * desc->canvas;
   const size_t a = attn_ws_bytes(make_attn_args(desc, total, cu_prefix_host));
-  const size_t s = sample_ws_bytes(desc->batch * desc->canvas, vocab, desc->dtype);
+  const size_t s = kHeaderBytes + sampler_record_bytes(rows, vocab);
   const size_t shared = align256(a > s ? a : s);
-  if (conf_off) *conf_off = shared;
-  return shared + align256((size_t)desc->batch * desc->canvas * sizeof(float));
+  const size_t cf = shared + align256(sampler_state_bytes(rows));
+  if (state_off) *state_off = shared;
+  if (conf_off) *conf_off = cf;
+  return cf + align256((size_t)rows * sizeof(float));
 }
 
 dd_status run_attn(const dd_attn_desc* d, const void* q, const void* kc, const void* vc,
@@ -147,10 +153,12 @@ dd_status run_attn(const dd_attn_desc* d, const void* q, const void* kc, const v
   return DD_OK;
 }
 
+// `state` is the sampler's persistent state, or nullptr for the standalone
+// layout (state after the header, records after the state).
 dd_status run_sampler(const void* logits, dd_dtype dtype, int rows, int vocab, int64_t row_stride,
                       const dd_sample_params* p, int32_t* tokens, int32_t* pred, float* conf,
                       float* entropy, uint8_t* renoised, void* ws, size_t ws_bytes,
-                      cudaStream_t stream) {
+                      cudaStream_t stream, void* state = nullptr) {
   if (!p) return fail(DD_ERR_INVALID_ARG, "params is NULL");
   if (dtype != DD_BF16 && dtype != DD_F32)
     return fail(DD_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
@@ -168,11 +176,13 @@ dd_status run_sampler(const void* logits, dd_dtype dtype, int rows, int vocab, i
   if (!logits || !tokens || !conf) return fail(DD_ERR_INVALID_ARG, "NULL required pointer");
   if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u))
     return fail(DD_ERR_WORKSPACE, "workspace must be non-NULL and 256-byte aligned");
-  const size_t need = sample_ws_bytes(rows, vocab, dtype);
+  const size_t need = state ? kHeaderBytes + sampler_record_bytes(rows, vocab)
+                            : sample_ws_bytes(rows, vocab, dtype);
   if (ws_bytes < need)
     return fail(DD_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", ws_bytes, need);
-  if ((int64_t)rows * sampler_nchunk(vocab, dtype == DD_BF16) > INT32_MAX)
-    return fail(DD_ERR_UNSUPPORTED, "rows * chunks exceeds 2^31");
+  if ((uint64_t)rows * (uint64_t)((vocab + 2047) / 2048) > 0xffffffffull)
+    return fail(DD_ERR_UNSUPPORTED, "rows * chunks exceeds 2^32");
+  uint8_t* const body = static_cast<uint8_t*>(ws) + kHeaderBytes;
   SamplerArgs a{};
   a.logits = logits;
   a.bf16 = dtype == DD_BF16;
@@ -189,7 +199,8 @@ dd_status run_sampler(const void* logits, dd_dtype dtype, int rows, int vocab, i
   a.conf = conf;
   a.entropy = entropy;
   a.renoised = renoised;
-  a.recs = reinterpret_cast<ChunkRecord*>(static_cast<uint8_t*>(ws) + kHeaderBytes);
+  a.state = state ? state : body;
+  a.recs = state ? body : body + align256(sampler_state_bytes(rows));
   a.err = static_cast<uint32_t*>(ws);
   cudaError_t e = launch_sampler(a, stream);
   if (e != cudaSuccess) return cuda_fail(e, "sampler");
@@ -271,7 +282,7 @@ size_t dd_denoise_block_workspace(const dd_attn_desc* desc, const int32_t* cu_pr
                                   int vocab) {
   int64_t total = 0;
   if (vocab < 1 || check_attn_desc(desc, cu_prefix_host, &total) != DD_OK) return 0;
-  return block_ws_layout(desc, total, cu_prefix_host, vocab, nullptr);
+  return block_ws_layout(desc, total, cu_prefix_host, vocab, nullptr, nullptr);
 }
 
 dd_status dd_denoise_block(const dd_attn_desc* desc, int steps, const void* q_steps,
@@ -300,8 +311,8 @@ dd_status dd_denoise_block(const dd_attn_desc* desc, int steps, const void* q_st
   const size_t kv_step = (size_t)rows * Hkv * D * es;
   const size_t lg_step = (size_t)rows * (size_t)vocab * es;
   if (vocab < 1) return fail(DD_ERR_INVALID_ARG, "vocab=%d", vocab);
-  size_t conf_off = 0;
-  const size_t need = block_ws_layout(desc, total, cu_prefix_host, vocab, &conf_off);
+  size_t state_off = 0, conf_off = 0;
+  const size_t need = block_ws_layout(desc, total, cu_prefix_host, vocab, &state_off, &conf_off);
   if (!workspace) return fail(DD_ERR_WORKSPACE, "workspace is NULL");
   if (workspace_bytes < need)
     return fail(DD_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", workspace_bytes, need);
@@ -311,7 +322,7 @@ dd_status dd_denoise_block(const dd_attn_desc* desc, int steps, const void* q_st
                   static_cast<const uint8_t*>(kc_steps) + i * kv_step,
                   static_cast<const uint8_t*>(vc_steps) + i * kv_step, k_prefix, v_prefix,
                   cu_prefix, cu_prefix_host, static_cast<uint8_t*>(attn_out) + i * q_step,
-                  nullptr, workspace, workspace_bytes, s);
+                  nullptr, workspace, state_off, s);
     if (st != DD_OK) return st;
     dd_sample_params sp;
     sp.temperature = temperature_host[i];
@@ -324,7 +335,7 @@ dd_status dd_denoise_block(const dd_attn_desc* desc, int steps, const void* q_st
                              : reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + conf_off);
     st = run_sampler(static_cast<const uint8_t*>(logits_steps) + i * lg_step, desc->dtype, rows,
                      vocab, vocab, &sp, tok, nullptr, conf, nullptr, nullptr, workspace,
-                     conf_off, s);
+                     state_off, s, static_cast<uint8_t*>(workspace) + state_off);
     if (st != DD_OK) return st;
     if (canvas_history && i == steps - 1) {
       cudaError_t e = cudaMemcpyAsync(canvas, tok, (size_t)rows * sizeof(int32_t),
@@ -340,7 +351,7 @@ dd_status dd_workspace_init(void* workspace, size_t workspace_bytes, dd_stream_t
   if (!workspace || workspace_bytes < kHeaderBytes)
     return fail(DD_ERR_WORKSPACE, "workspace must hold at least %zu bytes", kHeaderBytes);
   cudaError_t e =
-      cudaMemsetAsync(workspace, 0, kHeaderBytes, reinterpret_cast<cudaStream_t>(stream));
+      cudaMemsetAsync(workspace, 0, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "workspace init");
   return DD_OK;
 }

@@ -20,7 +20,7 @@ struct PhiloxKey {
   uint32_t k0[10], k1[10];  // hoisted round keys
 };
 
-__device__ __forceinline__ PhiloxKey philox_key(uint64_t seed) {
+__host__ __device__ __forceinline__ PhiloxKey philox_key(uint64_t seed) {
   PhiloxKey k;
   uint32_t a = (uint32_t)seed, b = (uint32_t)(seed >> 32);
 #pragma unroll

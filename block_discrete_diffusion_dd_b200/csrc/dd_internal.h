@@ -8,14 +8,6 @@
 
 namespace dd {
 
-// Per-(row, vocabulary chunk) partial record written by the sampler's first
-// pass (32 bytes, one per CTA).
-struct alignas(32) ChunkRecord {
-  float m, s, t, best;
-  int idx;
-  int pad[3];
-};
-
 struct SamplerArgs {
   const void* logits;
   bool bf16;
@@ -29,11 +21,22 @@ struct SamplerArgs {
   float* conf;
   float* entropy;
   uint8_t* renoised;
-  ChunkRecord* recs;
+  void* recs;     // per-chunk softmax partials, sampler_record_bytes()
+  void* state;    // ticket counter and row keys, sampler_state_bytes(); zero
+                  // before the first call, and left zero by every call
   uint32_t* err;  // device error word
 };
 
-int sampler_nchunk(int vocab, bool bf16);
+// The sampler's persistent state: a ticket counter (first 256 bytes) and one
+// 64-bit argmax key per row.  Zero between calls (the merge kernel clears it).
+struct SamplerState {
+  uint32_t* ticket;
+  unsigned long long* row_key;
+};
+SamplerState sampler_state(void* state);
+size_t sampler_state_bytes(int rows);
+// Per-chunk partial records (16 bytes per chunk of 2048 entries).
+size_t sampler_record_bytes(int rows, int vocab);
 cudaError_t launch_sampler(const SamplerArgs& a, cudaStream_t stream);
 cudaError_t launch_init_canvas(int32_t* canvas, int rows, int vocab, uint64_t seed,
                                uint32_t row_offset, cudaStream_t stream);

@@ -7,10 +7,12 @@
 // and output pointers, and latency-critical loops where cudaMalloc's implicit
 // device synchronisation is not acceptable.  dd_sample_renoise needs a
 // caller-provided workspace; this variant instead keeps its scratch (the
-// per-chunk partial records and the device error word) in one file-scope
-// static __device__ array of kStaticScratchBytes, which every GPU that loads
-// the library holds until the process exits.  The caller still passes the
-// logits and every output buffer.
+// device error word, the sampler's ticket counter and row keys, and the
+// per-chunk partial records) in one file-scope static __device__ array of
+// kStaticScratchBytes, which every GPU that loads the library holds until
+// the process exits.  The array starts zeroed, as the counter and the row
+// keys must be, and every call leaves them zero again.  The caller still
+// passes the logits and every output buffer.
 #include <cstdio>
 #include <mutex>
 
@@ -27,7 +29,7 @@ dd_status set_error(dd_status st, const char* msg);
 
 namespace {
 
-constexpr size_t kStaticScratchBytes = 2u << 20;  // 2 MiB per device
+constexpr size_t kStaticScratchBytes = 4u << 20;  // 4 MiB per device
 constexpr int kMaxDevices = 64;
 
 // The scratch itself.  In host code this name is only a host-side handle, not

@@ -4,13 +4,24 @@
 // that are not kept are re-noised to uniformly random vocabulary tokens).
 //
 // Two launches per step:
-//   sample_chunk  streams the logits once (128-bit loads), and for each
-//                 (row, vocabulary chunk) produces a partial record: running
-//                 max, sum of exp, entropy accumulator, and the best Gumbel
-//                 score with its index;
-//   sample_merge  merges a row's records in a fixed order, then draws the
-//                 re-noise decision and the replacement token.
-// HBM traffic is one read of the logits plus a few bytes per row.
+//   sample_scan   one persistent pass over the logits.  Rows are cut into
+//                 chunks of kChunk items (an item = 256 consecutive entries,
+//                 8 per lane of a warp); warps take chunks from a ticket
+//                 counter, so every warp stays busy until the pass ends
+//                 whatever the scheduler's order.  Per chunk the warp writes
+//                 the softmax partials (running max, sum of exp, entropy
+//                 accumulator); the row's best Gumbel score and its index go
+//                 to one 64-bit atomic maximum per row, which all warps also
+//                 read back as the threshold of the exponential-race prune.
+//   sample_merge  merges a row's chunk partials in chunk order (so the sums
+//                 do not depend on which warp took which chunk), reads the
+//                 argmax, draws the re-noise decision and the replacement
+//                 token, and clears the counter and the row maxima for the
+//                 next call.
+// HBM traffic is one read of the logits plus a few bytes per chunk and row.
+#include <algorithm>
+#include <atomic>
+
 #include "dd_device.cuh"
 #include "dd_internal.h"
 
@@ -18,19 +29,16 @@ namespace dd {
 
 namespace {
 
-constexpr int kSampleThreads = 256;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
-// Partial state over a set of vocabulary entries, in log2 units:
-// m = max y, s = sum 2^(y-m), t = sum 2^(y-m) (y-m), with y = logit/tau*log2 e;
-// best = max Gumbel score z - ln(-ln U) (natural units), idx its index.
-struct SampState {
-  float m, s, t, best;
-  int idx;
+// Softmax partials over a set of vocabulary entries, in log2 units:
+// m = max y, s = sum 2^(y-m), t = sum 2^(y-m) (y-m), with y = logit/tau*log2 e.
+struct SumState {
+  float m, s, t;
 };
 
-__device__ __forceinline__ void merge_state(SampState& a, const SampState& b) {
+__device__ __forceinline__ void merge_sums(SumState& a, const SumState& b) {
   const float M = fmaxf(a.m, b.m);
   if (M != -INFINITY) {
     float sa = 0.f, ta = 0.f, sb = 0.f, tb = 0.f;
@@ -48,36 +56,25 @@ __device__ __forceinline__ void merge_state(SampState& a, const SampState& b) {
     a.t = ta + tb;
   }
   a.m = M;
-  if (b.best > a.best || (b.best == a.best && b.idx < a.idx)) {
-    a.best = b.best;
-    a.idx = b.idx;
-  }
-}
-
-__device__ __forceinline__ SampState shfl_state(const SampState& s, int lane_mask) {
-  SampState o;
-  o.m = __shfl_xor_sync(0xffffffffu, s.m, lane_mask);
-  o.s = __shfl_xor_sync(0xffffffffu, s.s, lane_mask);
-  o.t = __shfl_xor_sync(0xffffffffu, s.t, lane_mask);
-  o.best = __shfl_xor_sync(0xffffffffu, s.best, lane_mask);
-  o.idx = __shfl_xor_sync(0xffffffffu, s.idx, lane_mask);
-  return o;
 }
 
 // Butterfly over the warp; every lane ends with the same merged state and
 // the merge tree is fixed, so the result does not depend on scheduling.
-__device__ __forceinline__ void warp_merge(SampState& s) {
+__device__ __forceinline__ void warp_merge_sums(SumState& s) {
+  const int lane = threadIdx.x & 31;
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) {
-    SampState o = shfl_state(s, off);
-    // merge in a lane-order-independent way: always (lower lane) <- (upper)
-    const int lane = threadIdx.x & 31;
+    SumState o;
+    o.m = __shfl_xor_sync(0xffffffffu, s.m, off);
+    o.s = __shfl_xor_sync(0xffffffffu, s.s, off);
+    o.t = __shfl_xor_sync(0xffffffffu, s.t, off);
+    // always (lower lane) <- (upper lane), whichever lane computes it
     if (lane & off) {
-      SampState lo = o;
-      merge_state(lo, s);
+      SumState lo = o;
+      merge_sums(lo, s);
       s = lo;
     } else {
-      merge_state(s, o);
+      merge_sums(s, o);
     }
   }
 }
@@ -99,14 +96,14 @@ __device__ __forceinline__ float warp_max(float v) {
 
 // Logits below -2^15 are treated as -2^15: exp underflows to 0 either way
 // (unless the whole row lies below it), and -inf entries and padding stay
-// out of 0 * inf products.  A power of two keeps x * c2 exact, so a thread
-// that has seen only padding gets d = 0 exactly.
+// out of 0 * inf products.  A power of two keeps x * c2 exact.
 constexpr float kFloorLogit = -32768.0f;
 
-// Per-thread running state.  Softmax sums in log2 units relative to a lazy
-// reference m (raised only when an entry exceeds it by more than 2^8, so the
-// terms stay below 256), kept as packed pairs so two entries update with one
-// f32x2 instruction; best = best Gumbel score (natural units), idx its index.
+// Per-lane running state.  Softmax sums in log2 units relative to a lazy
+// reference m (raised only when an entry exceeds it by more than kLazy, so
+// the terms stay below 2^kLazy), kept as packed pairs so two entries update
+// with one f32x2 instruction; best = the lane's best exact Gumbel score
+// (natural units), idx its index.
 struct Run {
   float m;
   float2 s2, t2;
@@ -127,10 +124,11 @@ __device__ __forceinline__ void raise_ref(Run& st, float ym) {
   st.m = ym;
 }
 
-// Prune threshold factor Kp = (1 + 2^-8) e^(m ln 2 - best_w), clamped; 0 in
-// a warp that holds padding alone (best_w = -inf).
+// Prune threshold factor Kp = (1 + 2^-8) e^(m ln 2 - best_w).  Before any
+// score is known (best_w = -inf) it is 2^126, which makes every entry whose
+// relative weight p is nonzero a candidate.
 __device__ __forceinline__ float prune_factor(float m, float best_w) {
-  return best_w == -INFINITY ? 0.f
+  return best_w == -INFINITY ? 8.507059173023462e37f
                              : fminf(ex2_approx(m - best_w * kLog2e) * 1.00390625f, 1e30f);
 }
 
@@ -147,319 +145,499 @@ __device__ __forceinline__ uint32_t max_bf16x2(uint32_t a, uint32_t b) {
   return r;
 }
 
-__device__ __forceinline__ void unpack8(uint4 raw, float (&x)[8], float& bm) {
-  raw.x = floor_bf16x2(raw.x);
-  raw.y = floor_bf16x2(raw.y);
-  raw.z = floor_bf16x2(raw.z);
-  raw.w = floor_bf16x2(raw.w);
-  const uint32_t mx = max_bf16x2(max_bf16x2(raw.x, raw.y), max_bf16x2(raw.z, raw.w));
-  bm = fmaxf(bf16lo(mx), bf16hi(mx));
-  x[0] = bf16lo(raw.x); x[1] = bf16hi(raw.x);
-  x[2] = bf16lo(raw.y); x[3] = bf16hi(raw.y);
-  x[4] = bf16lo(raw.z); x[5] = bf16hi(raw.z);
-  x[6] = bf16lo(raw.w); x[7] = bf16hi(raw.w);
+// ------------------------------------------------------ row argmax keys
+// The row's best (score, index) as one 64-bit key whose unsigned maximum is
+// the highest score and, among equal scores, the lowest index: the score's
+// bits mapped to an order-preserving unsigned word, then the complemented
+// index.  Key 0 means "no score yet" (it lies below every real score).
+__device__ __forceinline__ uint32_t ord_u32(float f) {
+  const uint32_t b = __float_as_uint(f);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
+__device__ __forceinline__ unsigned long long pack_key(float best, int idx) {
+  return ((unsigned long long)ord_u32(best) << 32) | (unsigned long long)(~(uint32_t)idx);
+}
+__device__ __forceinline__ float key_score(unsigned long long k) {
+  if (k == 0ull) return -INFINITY;
+  const uint32_t u = (uint32_t)(k >> 32);
+  return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
+}
+__device__ __forceinline__ int key_index(unsigned long long k) { return (int)~(uint32_t)k; }
 
-__device__ __forceinline__ void unpack8(float4 a, float4 b, float (&x)[8], float& bm) {
-  x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
-  x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+// Row keys sit 128 bytes apart: every warp reads its row's key often, and
+// keys of different rows then never share a cache line.
+constexpr int kKeyStride = 16;
+
+// ---------------------------------------------------------------- scan pass
+constexpr int kScanThreads = 256;
+constexpr int kScanWarpsPerCta = kScanThreads / 32;
+constexpr int kItem = 256;  // entries per warp-item
+constexpr int kChunk = 8;   // items per chunk (one ticket)
+
+struct ScanParams {
+  PhiloxKey key;      // round keys of the seed (read from the constant bank)
+  int64_t row_stride;
+  uint32_t nchunks;   // rows * nck
+  int rows;
+  int nck;            // chunks per row, ceil(ipr / kChunk)
+  int ipr;            // items per row, ceil(V / 256)
+  int vocab;
+  int jtail;          // index of a row's partial last item, or -1
+  float c2, inv_c2, inv_tau;
+  uint32_t step, row_offset;
+};
+
+// One lane's 8 entries of an item, as loaded.
+template <typename T, bool kVec>
+struct ItemBuf {
+  float v[8];  // scalar path: converted on load, padding as kFloorLogit
+};
+template <>
+struct ItemBuf<__nv_bfloat16, true> {
+  uint4 a;
+};
+template <>
+struct ItemBuf<float, true> {
+  float4 a, b;
+};
+
+// Load entries v0 .. v0+7 of a row (v0 = 256 j + 8 lane).  On the vector
+// path (rows 16-byte aligned, V % 8 == 0) lanes past V re-read the row's
+// last 8 entries instead, which the caller then discards as padding.
+template <typename T, bool kVec>
+__device__ __forceinline__ void load_item(ItemBuf<T, kVec>& b, const T* __restrict__ rowp, int v0,
+                                          int vocab) {
+  if constexpr (kVec) {
+    const int off = min(v0, vocab - 8);
+    if constexpr (sizeof(T) == 2) {
+      b.a = __ldg(reinterpret_cast<const uint4*>(rowp + off));
+    } else {
+      b.a = __ldg(reinterpret_cast<const float4*>(rowp + off));
+      b.b = __ldg(reinterpret_cast<const float4*>(rowp + off) + 1);
+    }
+  } else {
 #pragma unroll
-  for (int i = 0; i < 8; ++i) x[i] = fmaxf(x[i], kFloorLogit);
-  bm = fmaxf(fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3])), fmaxf(fmaxf(x[4], x[5]), fmaxf(x[6], x[7])));
+    for (int i = 0; i < 8; ++i) b.v[i] = (v0 + i < vocab) ? (float)rowp[v0 + i] : kFloorLogit;
+  }
 }
 
-// Reduce the CTA's states and write its chunk record.  Within a warp: the
-// common reference M first, then every lane rescales its sums to M and the
-// sums and the argmax (lowest index on equal scores) reduce by butterflies,
-// a fixed tree, so the result does not depend on scheduling.
-__device__ __forceinline__ SampState warp_reduce(const Run& r) {
-  float M = r.m;
+// Lazy-reference test: does the item hold an entry above the threshold X
+// (X <= (m + kLazy) / c2, the logit at which d = y - m would exceed kLazy)?
+// The bf16 path compares in bf16 with X rounded down to a bf16 value.
+template <typename T, bool kVec>
+struct LazyTest {
+  float x;
+  __device__ __forceinline__ void set(float m, float inv_c2) { x = (m + kLazy) * inv_c2; }
+};
+template <>
+struct LazyTest<__nv_bfloat16, true> {
+  uint32_t x2;  // the threshold as a bf16 pair
+  __device__ __forceinline__ void set(float m, float inv_c2) {
+    const uint32_t f = __float_as_uint((m + kLazy) * inv_c2);
+    uint32_t b = f >> 16;                         // truncation: toward zero
+    if ((f & 0x80000000u) && (f & 0xffffu)) ++b;  // negative: one step further down
+    x2 = b | (b << 16);
+  }
+};
+
+// Unpack one item to floored floats x[8] and test it against the lazy
+// reference threshold.
+template <typename T, bool kVec>
+__device__ __forceinline__ bool unpack_item(const ItemBuf<T, kVec>& b, const LazyTest<T, kVec>& lz,
+                                            float (&x)[8]) {
+  if constexpr (kVec && sizeof(T) == 2) {
+    const uint32_t r0 = floor_bf16x2(b.a.x), r1 = floor_bf16x2(b.a.y);
+    const uint32_t r2 = floor_bf16x2(b.a.z), r3 = floor_bf16x2(b.a.w);
+    const uint32_t mx = max_bf16x2(max_bf16x2(r0, r1), max_bf16x2(r2, r3));
+    x[0] = bf16lo(r0); x[1] = bf16hi(r0);
+    x[2] = bf16lo(r1); x[3] = bf16hi(r1);
+    x[4] = bf16lo(r2); x[5] = bf16hi(r2);
+    x[6] = bf16lo(r3); x[7] = bf16hi(r3);
+    return max_bf16x2(mx, lz.x2) != lz.x2;
+  } else {
+    if constexpr (kVec) {
+      x[0] = b.a.x; x[1] = b.a.y; x[2] = b.a.z; x[3] = b.a.w;
+      x[4] = b.b.x; x[5] = b.b.y; x[6] = b.b.z; x[7] = b.b.w;
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) x[i] = b.v[i];
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) x[i] = fmaxf(x[i], kFloorLogit);
+    const float mx = fmaxf(fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3])),
+                           fmaxf(fmaxf(x[4], x[5]), fmaxf(x[6], x[7])));
+    return mx > lz.x;
+  }
+}
+
+// Exponential-race prune: the score z - ln E (E = -ln U) can beat best_w
+// only if E < e^(z - best_w); since E >= 1 - U, an entry with
+// 1 - U >= e^(z - best_w) (1 + 2^-8) = p Kp is skipped without a logarithm.
+// With U' = 1 + (x >> 9) 2^-23 = U + 1 - 2^-24 an entry stays a candidate
+// when U' > 2 - 2^-23 - p Kp (the constant rounded down to an fp32 value,
+// which only adds candidates).
+constexpr float kPadD = -1000.0f;  // d of padding entries: 2^d flushes to 0
+
+__device__ __forceinline__ float u_prime(uint32_t w) {
+  return __uint_as_float(0x3F800000u | (w >> 9));
+}
+constexpr float kTwoMinus = 1.99999988079071044921875f;  // 2 - 2^-23
+
+__device__ __forceinline__ uint32_t word_of(const uint4& wa, const uint4& wb, int i) {
+  const uint4 wq = i < 4 ? wa : wb;
+  const int i4 = i & 3;
+  return i4 == 0 ? wq.x : i4 == 1 ? wq.y : i4 == 2 ? wq.z : wq.w;
+}
+
+// Per-warp scan state of one chunk.
+struct PartState {
+  Run st;
+  float best_w;  // best Gumbel score of the row known to this warp
+  float Kp;      // prune factor for this lane's reference m
+};
+
+// Exact scores of the item's candidates (rare).  The test is redone entry
+// by entry from re-read logits (L1 hits) exactly as in scan_item, so the
+// same entries qualify; only those get logarithms.  Arguments and results
+// travel by value, so the caller's state stays in registers.
+struct ExactOut {
+  float best;
+  int idx;
+  bool changed;
+};
+
+template <typename T, bool kVec, bool kTail>
+__device__ __noinline__ ExactOut exact_scores(const T* __restrict__ rowp, int v0, uint4 wa,
+                                              uint4 wb, float m, float Kp, float best, int idx,
+                                              float c2, float inv_tau, int vocab) {
+  ItemBuf<T, kVec> rb;
+  load_item<T, kVec>(rb, rowp, v0, vocab);
+  LazyTest<T, kVec> none;
+  none.set(-INFINITY, 1.f);
+  float x[8];
+  (void)unpack_item<T, kVec>(rb, none, x);
+  uint32_t cmask = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    float d = fmaf(x[i], c2, -m);
+    if (kTail && v0 + i >= vocab) d = kPadD;
+    const float pw = ex2_approx(d);
+    if (u_prime(word_of(wa, wb, i)) > fmaf(pw, -Kp, kTwoMinus)) cmask |= 1u << i;
+  }
+  ExactOut o{best, idx, false};
+  while (cmask) {
+    const int i = __ffs(cmask) - 1;
+    cmask &= cmask - 1;
+    const uint32_t v = (uint32_t)(v0 + i);
+    const float xi = fmaxf((float)rowp[v], kFloorLogit);
+    const float sc = gumbel_score(xi * inv_tau, word_of(wa, wb, i));
+    if (sc > o.best || (sc == o.best && (int)v < o.idx)) {
+      o.best = sc;
+      o.idx = (int)v;
+      o.changed = true;
+    }
+  }
+  return o;
+}
+
+// One item, in an order that keeps few values live: the Philox words, the
+// lazy-reference raise (rare, one warp vote), then weights, softmax sums and
+// the candidate test in one sweep, and the exact scores of candidates (rare,
+// one warp vote), whose improvements go to the row key.  `next` (or nullptr)
+// is the lane's address of the item two ahead, loaded into `buf` once this
+// item is unpacked.  kTail: the item reaches past V.
+template <typename T, bool kVec, bool kTail>
+__device__ __forceinline__ void scan_item(PartState& ps, LazyTest<T, kVec>& lz,
+                                          ItemBuf<T, kVec>& buf, const T* next,
+                                          const T* __restrict__ rowp, int v0,
+                                          const ScanParams& p, const PhiloxRow& prow,
+                                          unsigned long long* rkey) {
+  const uint32_t cword = (uint32_t)v0 >> 2;
+  const uint4 wa = philox4x32_10_row(cword, 0u, prow, p.key);
+  const uint4 wb = philox4x32_10_row(cword + 1u, 0u, prow, p.key);
+  float x[8];
+  const bool pend = unpack_item<T, kVec>(buf, lz, x);
+  if (next != nullptr) load_item<T, kVec>(buf, next, 0, 1 << 30);
+  if (__any_sync(0xffffffffu, pend)) {
+    if (pend) {
+      float bm = x[0];
+#pragma unroll
+      for (int i = 1; i < 8; ++i) bm = fmaxf(bm, x[i]);
+      raise_ref(ps.st, fmaxf(bm * p.c2, ps.st.m));
+      ps.Kp = prune_factor(ps.st.m, ps.best_w);
+      lz.set(ps.st.m, p.inv_c2);
+    }
+  }
+  const float2 c22 = make_float2(p.c2, p.c2);
+  const float2 nm = make_float2(-ps.st.m, -ps.st.m);
+  float pmax = 0.f;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    float2 d = __ffma2_rn(make_float2(x[2 * j], x[2 * j + 1]), c22, nm);
+    if constexpr (kTail) {
+      if (v0 + 2 * j >= p.vocab) d.x = kPadD;
+      if (v0 + 2 * j + 1 >= p.vocab) d.y = kPadD;
+    }
+    const float2 pw = make_float2(ex2_approx(d.x), ex2_approx(d.y));
+    ps.st.s2 = __fadd2_rn(ps.st.s2, pw);
+    ps.st.t2 = __ffma2_rn(pw, d, ps.st.t2);
+    pmax = fmaxf(pmax, fmaxf(pw.x, pw.y));
+  }
+  // One test for the lane's 8 entries: an entry i is a candidate only if
+  // U'_i > 2 - 2^-23 - p_i Kp, which implies max U' > 2 - 2^-23 - max p Kp
+  // (fma is monotone in p), so the rare path below runs for every item that
+  // holds a candidate and finds the candidates themselves entry by entry.
+  const uint32_t wmax = __vimax3_u32(__vimax3_u32(wa.x, wa.y, wa.z),
+                                     __vimax3_u32(wa.w, wb.x, wb.y), max(wb.z, wb.w));
+  const bool cand = u_prime(wmax) > fmaf(pmax, -ps.Kp, kTwoMinus);
+  if (__any_sync(0xffffffffu, cand)) {
+    bool changed = false;
+    if (cand) {
+      const ExactOut o = exact_scores<T, kVec, kTail>(rowp, v0, wa, wb, ps.st.m, ps.Kp,
+                                                      ps.st.best, ps.st.idx, p.c2, p.inv_tau,
+                                                      p.vocab);
+      ps.st.best = o.best;
+      ps.st.idx = o.idx;
+      changed = o.changed;
+      if (changed) atomicMax(rkey, pack_key(o.best, o.idx));
+    }
+    if (__any_sync(0xffffffffu, changed)) {
+      ps.best_w = fmaxf(ps.best_w, warp_max(ps.st.best));
+      ps.Kp = prune_factor(ps.st.m, ps.best_w);
+    }
+  }
+}
+
+// Seed of a chunk that finds no score for its row yet: the exact score of
+// each lane's largest entry in the chunk's first item (lowest index among
+// equal values), published to the row key by the warp's best lane.  The
+// reference m is still unset here; the first item always raises it, which
+// recomputes Kp.
+template <typename T, bool kVec>
+__device__ __forceinline__ void seed_chunk(PartState& ps, const ItemBuf<T, kVec>& b, int v0,
+                                           const ScanParams& p, const PhiloxRow& prow,
+                                           unsigned long long* rkey) {
+  LazyTest<T, kVec> none;
+  none.set(-INFINITY, 1.f);
+  float x[8];
+  (void)unpack_item<T, kVec>(b, none, x);
+  float bm = -INFINITY;
+  int jm = -1;
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    if (v0 + i < p.vocab && x[i] > bm) {
+      bm = x[i];
+      jm = i;
+    }
+  if (jm >= 0) {
+    const uint32_t v = (uint32_t)(v0 + jm);
+    const uint4 w = philox4x32_10_row(v >> 2, 0u, prow, p.key);
+    const uint32_t i4 = v & 3u;
+    const uint32_t wj = i4 == 0 ? w.x : i4 == 1 ? w.y : i4 == 2 ? w.z : w.w;
+    ps.st.best = gumbel_score(bm * p.inv_tau, wj);
+    ps.st.idx = (int)v;
+  }
+  ps.best_w = warp_max(ps.st.best);
+  // the lowest lane holding the warp's best has the lowest index among them
+  const unsigned hit = __ballot_sync(0xffffffffu, jm >= 0 && ps.st.best == ps.best_w);
+  if (hit && (int)(threadIdx.x & 31) == __ffs(hit) - 1)
+    atomicMax(rkey, pack_key(ps.st.best, ps.st.idx));
+}
+
+// Adopt the row's best score known grid-wide when it is higher (any score in
+// the row bounds the row's maximum from below, whichever warp found it).
+__device__ __forceinline__ void adopt_key(PartState& ps, unsigned long long k) {
+  const float cb = key_score(k);
+  if (cb > ps.best_w) {
+    ps.best_w = cb;
+    ps.Kp = prune_factor(ps.st.m, cb);
+  }
+}
+
+// Where chunk g lies: row r, items ja .. jb-1, of which ja .. jm-1 are full
+// (jm = jb - 1 when the chunk ends with the row's partial last item).
+template <typename T>
+struct ChunkPos {
+  const T* rowp;
+  uint32_t r;
+  int ja, jm, jb;
+};
+
+// Tickets run over the chunks column by column (chunk 0 of every row, then
+// chunk 1, ...), so the chunks of one row are spread over the whole pass and
+// most of them start with a good threshold from the row key.
+template <typename T>
+__device__ __forceinline__ ChunkPos<T> chunk_pos(const T* __restrict__ logits,
+                                                 const ScanParams& p, uint32_t g) {
+  ChunkPos<T> c;
+  const uint32_t cc = g / (uint32_t)p.rows;
+  c.r = g - cc * (uint32_t)p.rows;
+  c.ja = (int)cc * kChunk;
+  c.jb = min(c.ja + kChunk, p.ipr);
+  c.jm = (c.jb - 1 == p.jtail) ? c.jb - 1 : c.jb;
+  c.rowp = logits + (int64_t)c.r * p.row_stride;
+  return c;
+}
+
+// One chunk: its items with loads issued two items ahead; the partial last
+// item of a row is peeled off and processed with the padding checks.  A and
+// B arrive holding the chunk's first two items when `pre` says so, and
+// `key` its row key.  When `cross`, the last two items' prefetches fetch the
+// first two items of the next chunk `cn` instead, with its row key, which
+// then come back in A, B and `key`; the next chunk starts at item nja of
+// row nr.  Writes the chunk's softmax partials to recs[r * nck + chunk].
+template <typename T, bool kVec>
+__device__ __forceinline__ void scan_chunk(const T* __restrict__ logits, const ScanParams& p,
+                                           uint32_t g, const ChunkPos<T>& c, int lane,
+                                           ItemBuf<T, kVec>& A, ItemBuf<T, kVec>& B, bool pre,
+                                           unsigned long long& key, bool cross, uint32_t nr,
+                                           int nja, float4* __restrict__ recs,
+                                           unsigned long long* __restrict__ row_key) {
+  const int lo8 = lane * 8;
+  const T* rowp = c.rowp;
+  unsigned long long* rkey = row_key + (size_t)c.r * kKeyStride;
+  if (!pre) {
+    if (c.jm > c.ja) load_item<T, kVec>(A, rowp, c.ja * kItem + lo8, p.vocab);
+    if (c.jm > c.ja + 1) load_item<T, kVec>(B, rowp, (c.ja + 1) * kItem + lo8, p.vocab);
+    key = __ldcg(rkey);
+  }
+  const PhiloxRow prow = philox_row(p.row_offset + c.r, p.step, 0u, p.key);
+  PartState ps;
+  ps.st = Run{-INFINITY, make_float2(0.f, 0.f), make_float2(0.f, 0.f), -INFINITY, 0x7fffffff};
+  ps.best_w = key_score(key);
+  ps.Kp = 0.f;
+  LazyTest<T, kVec> lz;
+  lz.set(-INFINITY, p.inv_c2);
+  if constexpr (kVec) {
+    const int ja = c.ja, jm = c.jm;
+    if (jm > ja) {
+      if (ps.best_w == -INFINITY) seed_chunk<T, kVec>(ps, A, ja * kItem + lo8, p, prow, rkey);
+      const T* base = rowp + ja * kItem + lo8;  // this lane's entries of item j
+#pragma unroll 1
+      for (int j = ja; j < jm; j += 2, base += 2 * kItem) {
+        const T* na = base + 2 * kItem;
+        if (j + 2 >= jm) {  // past this chunk: the next chunk's first items
+          na = nullptr;
+          if (cross) {
+            na = logits + (int64_t)nr * p.row_stride + nja * kItem + lo8;
+            key = __ldcg(row_key + (size_t)nr * kKeyStride);
+          }
+        }
+        scan_item<T, kVec, false>(ps, lz, A, na, rowp, j * kItem + lo8, p, prow, rkey);
+        if (j + 1 < jm)
+          scan_item<T, kVec, false>(ps, lz, B, na == nullptr ? nullptr : na + kItem, rowp,
+                                    (j + 1) * kItem + lo8, p, prow, rkey);
+      }
+    }
+    if (jm < c.jb) {
+      ItemBuf<T, kVec> X;
+      load_item<T, kVec>(X, rowp, jm * kItem + lo8, p.vocab);
+      if (ps.best_w == -INFINITY) seed_chunk<T, kVec>(ps, X, jm * kItem + lo8, p, prow, rkey);
+      adopt_key(ps, __ldcg(rkey));
+      scan_item<T, kVec, true>(ps, lz, X, nullptr, rowp, jm * kItem + lo8, p, prow, rkey);
+    }
+  } else {
+#pragma unroll 1
+    for (int j = c.ja; j < c.jb; ++j) {
+      ItemBuf<T, kVec> X;
+      load_item<T, kVec>(X, rowp, j * kItem + lo8, p.vocab);
+      if (ps.best_w == -INFINITY) seed_chunk<T, kVec>(ps, X, j * kItem + lo8, p, prow, rkey);
+      adopt_key(ps, __ldcg(rkey));
+      scan_item<T, kVec, true>(ps, lz, X, nullptr, rowp, j * kItem + lo8, p, prow, rkey);
+    }
+  }
+  // the chunk's softmax partials: common reference first, then the sums by
+  // a fixed butterfly
+  float M = ps.st.m;
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-  float s = r.s2.x + r.s2.y, t = r.t2.x + r.t2.y;
+  float s = ps.st.s2.x + ps.st.s2.y, t = ps.st.t2.x + ps.st.t2.y;
   if (s > 0.f) {
-    const float f = ex2_approx(r.m - M);
-    t = f * fmaf(s, r.m - M, t);
+    const float f = ex2_approx(ps.st.m - M);
+    t = f * fmaf(s, ps.st.m - M, t);
     s *= f;
   } else {
     s = 0.f;
     t = 0.f;
   }
-  float best = r.best;
-  int idx = r.idx;
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) {
     s += __shfl_xor_sync(0xffffffffu, s, off);
     t += __shfl_xor_sync(0xffffffffu, t, off);
-    const float ob = __shfl_xor_sync(0xffffffffu, best, off);
-    const int oi = __shfl_xor_sync(0xffffffffu, idx, off);
-    if (ob > best || (ob == best && oi < idx)) {
-      best = ob;
-      idx = oi;
+  }
+  if (lane == 0) recs[(size_t)c.r * p.nck + (uint32_t)(c.ja / kChunk)] = make_float4(M, s, t, 0.f);
+}
+
+// Persistent: each warp takes chunk tickets until they run out.  Tickets are
+// drawn one chunk ahead, and on the vector path the next chunk's first two
+// items and its row key are in flight while the current chunk ends, so a
+// chunk boundary costs no memory latency.  The hand-over needs an even
+// number of full items in the current chunk (the items alternate between two
+// buffers) and two full items at the start of the next; other chunks (rows
+// whose item count is not a multiple of the chunk, partial last items) load
+// their first items when they start.
+template <typename T, bool kVec>
+__global__ void __launch_bounds__(kScanThreads, 3)
+    sample_scan_kernel(const T* __restrict__ logits, const __grid_constant__ ScanParams p,
+                       float4* __restrict__ recs, unsigned long long* __restrict__ row_key,
+                       uint32_t* __restrict__ ticket) {
+  const int lane = threadIdx.x & 31;
+  uint32_t g = 0, gn_req = 0;
+  if (lane == 0) {
+    g = atomicAdd(ticket, 1u);
+    gn_req = atomicAdd(ticket, 1u);
+  }
+  g = __shfl_sync(0xffffffffu, g, 0);
+  ItemBuf<T, kVec> A, B;
+  unsigned long long key = 0ull;
+  bool pre = false;
+  while (g < p.nchunks) {
+    const uint32_t gn = __shfl_sync(0xffffffffu, gn_req, 0);  // drawn one chunk ago
+    if (lane == 0) gn_req = atomicAdd(ticket, 1u);
+    const ChunkPos<T> c = chunk_pos<T>(logits, p, g);
+    const bool has_next = gn < p.nchunks;
+    bool cross = false;
+    uint32_t nr = 0;
+    int nja = 0;
+    if (kVec && has_next && ((c.jm - c.ja) % 2 == 0) && c.jm == c.jb) {
+      const ChunkPos<T> cn = chunk_pos<T>(logits, p, gn);
+      cross = cn.jm - cn.ja >= 2;
+      nr = cn.r;
+      nja = cn.ja;
     }
-  }
-  return SampState{M, s, t, best, idx};
-}
-
-__device__ __forceinline__ void write_record(const Run& r, ChunkRecord* rec) {
-  const SampState st = warp_reduce(r);
-  __shared__ SampState red[kSampleThreads / 32];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (lane == 0) red[warp] = st;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    SampState a = red[0];
-#pragma unroll
-    for (int w = 1; w < kSampleThreads / 32; ++w) merge_state(a, red[w]);
-    ChunkRecord out;
-    out.m = a.m;
-    out.s = a.s;
-    out.t = a.t;
-    out.best = a.best;
-    out.idx = a.idx;
-    *rec = out;
+    scan_chunk<T, kVec>(logits, p, g, c, lane, A, B, pre, key, cross, nr, nja, recs, row_key);
+    pre = cross;
+    g = gn;
   }
 }
 
-constexpr uint32_t kStageBytes = 32768;  // logits per CTA (one bulk copy)
-
-template <typename T>
-__host__ __device__ constexpr int chunk_elems() { return (int)(kStageBytes / sizeof(T)); }
-
-// Gumbel scores order like floats; as ints for atomicMax on shared memory.
-__device__ __forceinline__ int ord_float(float f) {
-  const int b = __float_as_int(f);
-  return b ^ ((b >> 31) & 0x7fffffff);
-}
-__device__ __forceinline__ float unord_float(int o) {
-  return __int_as_float(o ^ ((o >> 31) & 0x7fffffff));
-}
-
-// One item = 8 consecutive entries x[0..7] (floored, finite) starting at v0,
-// with bm = their max.  `src` points at the item's first entry (in shared
-// memory, or in global memory on the scalar path) and is re-read only on the
-// rare exact path.  best_w is the warp's view of the best Gumbel score so far;
-// cta_best holds the best over the whole CTA (ordered int), which every warp
-// adopts when it is higher than its own.
-template <typename T>
-__device__ __forceinline__ void process_item(Run& st, float& best_w, float& Kp, const float (&x)[8],
-                                             float bm, uint32_t v0, bool seed, const T* src,
-                                             const PhiloxKey& key, const PhiloxRow& prow,
-                                             float c2, float inv_tau, int* cta_best) {
-  const float ym = bm * c2;
-  if (ym > st.m + kLazy) {  // rare after the first item
-    raise_ref(st, ym);
-    Kp = prune_factor(st.m, best_w);
-  }
-  {
-    const float cb = unord_float(*reinterpret_cast<volatile int*>(cta_best));
-    if (cb > best_w) {
-      best_w = cb;
-      Kp = prune_factor(st.m, best_w);
-    }
-  }
-  const float2 c22 = make_float2(c2, c2);
-  const float2 nm = make_float2(-st.m, -st.m);
-  float2 p[4];
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const float2 d = __ffma2_rn(make_float2(x[2 * j], x[2 * j + 1]), c22, nm);
-    p[j] = make_float2(ex2_approx(d.x), ex2_approx(d.y));
-    st.s2 = __fadd2_rn(st.s2, p[j]);
-    st.t2 = __ffma2_rn(p[j], d, st.t2);
-  }
-  // Gumbel words for the 8 entries: two Philox blocks.
-  const uint4 wa = philox4x32_10_row(v0 >> 2, 0u, prow, key);
-  const uint4 wb = philox4x32_10_row((v0 >> 2) + 1u, 0u, prow, key);
-  bool changed = false;
-  if (seed) {
-    // seed the threshold with the exact score of this lane's largest entry
-    if (bm > kFloorLogit) {
-      int j = 7;
-#pragma unroll
-      for (int i = 6; i >= 0; --i) j = (x[i] == bm) ? i : j;
-      const uint4 wq = j < 4 ? wa : wb;
-      const uint32_t i4 = (uint32_t)j & 3u;
-      const uint32_t wj = i4 == 0 ? wq.x : i4 == 1 ? wq.y : i4 == 2 ? wq.z : wq.w;
-      st.best = gumbel_score(bm * inv_tau, wj);
-      st.idx = (int)(v0 + (uint32_t)j);
-    }
-    // the seeded threshold applies to this item's own test below
-    best_w = fmaxf(best_w, warp_max(st.best));
-    if ((threadIdx.x & 31) == 0) atomicMax(cta_best, ord_float(best_w));
-    Kp = prune_factor(st.m, best_w);
-  }
-  // Exponential-race prune: the score z - ln E (E = -ln U) can beat best_w
-  // only if E < e^(z - best_w); since E >= 1 - U, an entry with
-  // 1 - U >= e^(z - best_w) (1 + 2^-8) is skipped without a logarithm.  With
-  // U' = 1 + (x >> 9) 2^-23 = U + 1 - 2^-24 the test reads
-  // U' > 2 - 2^-23 - p Kp.
-  const float2 kk = make_float2(-Kp, -Kp);
-  const float2 cc = make_float2(1.99999988079071044921875f, 1.99999988079071044921875f);
-  const uint32_t w[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
-  float thr[8];
-  bool any = false;
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const float2 t = __ffma2_rn(p[j], kk, cc);
-    thr[2 * j] = t.x;
-    thr[2 * j + 1] = t.y;
-    any |= __uint_as_float(0x3F800000u | (w[2 * j] >> 9)) > t.x;
-    any |= __uint_as_float(0x3F800000u | (w[2 * j + 1] >> 9)) > t.y;
-  }
-  if (any) {
-    // rare exact path: one entry at a time (the logit re-read, its word
-    // selected from the two blocks above), so the code below exists once
-    uint32_t cmask = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-      cmask |= (__uint_as_float(0x3F800000u | (w[i] >> 9)) > thr[i]) ? (1u << i) : 0u;
-    while (cmask) {
-      const int i = __ffs(cmask) - 1;
-      cmask &= cmask - 1;
-      const float xi = fmaxf((float)src[i], kFloorLogit);
-      const uint32_t v = v0 + (uint32_t)i;
-      const uint4 wq = i < 4 ? wa : wb;
-      const int i4 = i & 3;
-      const uint32_t wi = i4 == 0 ? wq.x : i4 == 1 ? wq.y : i4 == 2 ? wq.z : wq.w;
-      const float sc = gumbel_score(xi * inv_tau, wi);
-      if (sc > st.best || (sc == st.best && (int)v < st.idx)) {
-        st.best = sc;
-        st.idx = (int)v;
-        changed = true;
-      }
-    }
-  }
-  if (__any_sync(0xffffffffu, changed)) {
-    best_w = fmaxf(best_w, warp_max(st.best));
-    if ((threadIdx.x & 31) == 0) atomicMax(cta_best, ord_float(best_w));
-    Kp = prune_factor(st.m, best_w);
-  }
-}
-
-// Vector path: rows 16-byte aligned and V % 8 == 0.  Thread 0 fetches the
-// CTA's 32 KB slice of the row with one bulk asynchronous copy into shared
-// memory; all 256 threads then stream it 8 entries at a time.
-template <typename T>
-__global__ void __launch_bounds__(kSampleThreads, 4)
-    sample_chunk_bulk_kernel(const T* __restrict__ logits, int64_t row_stride, int vocab,
-                             int nchunk, float inv_tau, uint64_t seed, uint32_t step,
-                             uint32_t row_offset, ChunkRecord* __restrict__ recs,
-                             uint32_t* __restrict__ err) {
-  constexpr int kElems = chunk_elems<T>();
-  constexpr int kItems = kElems / (kSampleThreads * 8);
-  __shared__ __align__(128) uint8_t buf[kStageBytes];
-  __shared__ uint64_t bar;
-  __shared__ int cta_best;
-  const int row = blockIdx.x / nchunk;
-  const int chunk = blockIdx.x - row * nchunk;
-  const int c0 = chunk * kElems;
-  const int n = min(kElems, vocab - c0);
-  if (threadIdx.x == 0) {
-    mbar_init(&bar, 1);
-    fence_mbar_init();
-    cta_best = ord_float(-INFINITY);
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    mbar_arrive_expect_tx(&bar, (uint32_t)(n * sizeof(T)));
-    bulk_load(buf, logits + (int64_t)row * row_stride + c0, (uint32_t)(n * sizeof(T)), &bar);
-  }
-  const PhiloxKey key = philox_key(seed);
-  const uint32_t grow = row_offset + (uint32_t)row;
-  const PhiloxRow prow = philox_row(grow, step, 0u, key);
-  const float c2 = inv_tau * kLog2e;
-  Run st{-INFINITY, make_float2(0.f, 0.f), make_float2(0.f, 0.f), -INFINITY, 0x7fffffff};
-  float best_w = -INFINITY, Kp = 0.f;
-  if (!mbar_wait_bounded(&bar, 0, nullptr, 1000000000ull)) {
-    // never observed: the copy is plain memory traffic; report and drain
-    if (threadIdx.x == 0) atomicOr(err, kDevErrTimeout);
-    mbar_wait_bounded(&bar, 0, nullptr, 4000000000ull);
-    return;
-  }
-  const T* tb = reinterpret_cast<const T*>(buf);
-#pragma unroll 1
-  for (int k = 0; k < kItems; ++k) {
-    const int e = (k * kSampleThreads + (int)threadIdx.x) * 8;
-    float x[8], bm;
-    if (e < n) {
-      if constexpr (sizeof(T) == 2) {
-        unpack8(*reinterpret_cast<const uint4*>(buf + e * 2), x, bm);
-      } else {
-        const float4* q = reinterpret_cast<const float4*>(buf + e * 4);
-        unpack8(q[0], q[1], x, bm);
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) x[i] = kFloorLogit;
-      bm = kFloorLogit;
-    }
-    process_item<T>(st, best_w, Kp, x, bm, (uint32_t)(c0 + e), k == 0, tb + e, key, prow, c2,
-                    inv_tau, &cta_best);
-  }
-  write_record(st, recs + (int64_t)row * nchunk + chunk);
-}
-
-// Scalar path for unaligned rows or V % 8 != 0: direct loads with bounds
-// checks; entries at or beyond V read as kFloorLogit and never win (their p
-// is 0, so the prune never selects them and they are never re-read).
-template <typename T>
-__global__ void __launch_bounds__(kSampleThreads)
-    sample_chunk_scalar_kernel(const T* __restrict__ logits, int64_t row_stride, int vocab,
-                               int nchunk, float inv_tau, uint64_t seed, uint32_t step,
-                               uint32_t row_offset, ChunkRecord* __restrict__ recs) {
-  constexpr int kElems = chunk_elems<T>();
-  constexpr int kItems = kElems / (kSampleThreads * 8);
-  const int row = blockIdx.x / nchunk;
-  const int chunk = blockIdx.x - row * nchunk;
-  const int c0 = chunk * kElems;
-  const T* rowp = logits + (int64_t)row * row_stride;
-  const PhiloxKey key = philox_key(seed);
-  const uint32_t grow = row_offset + (uint32_t)row;
-  const PhiloxRow prow = philox_row(grow, step, 0u, key);
-  const float c2 = inv_tau * kLog2e;
-  Run st{-INFINITY, make_float2(0.f, 0.f), make_float2(0.f, 0.f), -INFINITY, 0x7fffffff};
-  float best_w = -INFINITY, Kp = 0.f;
-  __shared__ int cta_best;
-  if (threadIdx.x == 0) cta_best = ord_float(-INFINITY);
-  __syncthreads();
-#pragma unroll 1
-  for (int k = 0; k < kItems; ++k) {
-    const int v0 = c0 + (k * kSampleThreads + (int)threadIdx.x) * 8;
-    float x[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-      x[i] = (v0 + i < vocab) ? fmaxf((float)rowp[v0 + i], kFloorLogit) : kFloorLogit;
-    float bm = x[0];
-#pragma unroll
-    for (int i = 1; i < 8; ++i) bm = fmaxf(bm, x[i]);
-    process_item<T>(st, best_w, Kp, x, bm, (uint32_t)v0, k == 0, rowp + v0, key, prow, c2,
-                    inv_tau, &cta_best);
-  }
-  write_record(st, recs + (int64_t)row * nchunk + chunk);
-}
-
+// Merge of a row's chunk partials (in chunk order), the argmax from the row
+// key, then the re-noise draw.  One warp per row.  Clears the ticket counter
+// and the row key for the next call.
 template <typename T>
 __global__ void __launch_bounds__(128)
     sample_merge_kernel(const T* __restrict__ logits, int64_t row_stride, int rows, int vocab,
-                        int nchunk, float inv_tau, float rate, uint64_t seed, uint32_t step,
-                        uint32_t row_offset, const ChunkRecord* __restrict__ recs,
+                        int nck, float inv_tau, float rate, uint64_t seed, uint32_t step,
+                        uint32_t row_offset, const float4* __restrict__ recs,
+                        unsigned long long* __restrict__ row_key, uint32_t* __restrict__ ticket,
                         int32_t* __restrict__ tokens, int32_t* __restrict__ pred,
                         float* __restrict__ conf, float* __restrict__ entropy,
                         uint8_t* __restrict__ renoised) {
+  if (blockIdx.x == 0 && threadIdx.x == 0) *ticket = 0u;
   const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
-  SampState st{-INFINITY, 0.f, 0.f, -INFINITY, 0x7fffffff};
-  for (int c = lane; c < nchunk; c += 32) {
-    const ChunkRecord r = recs[(int64_t)row * nchunk + c];
-    SampState o{r.m, r.s, r.t, r.best, r.idx};
-    merge_state(st, o);
+  SumState st{-INFINITY, 0.f, 0.f};
+  for (int c = lane; c < nck; c += 32) {
+    const float4 r = recs[(int64_t)row * nck + c];
+    merge_sums(st, SumState{r.x, r.y, r.z});
   }
-  warp_merge(st);
+  warp_merge_sums(st);
   if (lane != 0) return;
-  const int p = st.idx;
-  const float x = (float)logits[(int64_t)row * row_stride + p];
+  const unsigned long long key = row_key[(size_t)row * kKeyStride];
+  row_key[(size_t)row * kKeyStride] = 0ull;
+  const int p = key ? key_index(key) : 0;
+  const float x = fmaxf((float)logits[(int64_t)row * row_stride + p], kFloorLogit);
   const float c2 = inv_tau * kLog2e;
   const float cf = ex2_approx(fmaf(x, c2, -st.m)) / st.s;
   const float ent = logf(st.s) - kLn2 * (st.t / st.s);
@@ -483,36 +661,91 @@ __global__ void init_canvas_kernel(int32_t* __restrict__ canvas, int rows, int v
   canvas[r] = (int32_t)(((uint64_t)x * (uint64_t)(uint32_t)vocab) >> 32);
 }
 
-template <typename T>
-cudaError_t launch_sampler_t(const SamplerArgs& a, cudaStream_t stream) {
-  const int nchunk = (a.vocab + chunk_elems<T>() - 1) / chunk_elems<T>();
+// CTAs of the persistent scan grid on the current device (resident CTAs per
+// SM x SMs), cached per device and variant.
+template <typename T, bool kVec>
+int scan_ctas() {
+  constexpr int kMaxDev = 64;
+  static std::atomic<int> cache[kMaxDev];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 1;
+  if (dev < kMaxDev) {
+    const int c = cache[dev].load(std::memory_order_relaxed);
+    if (c > 0) return c;
+  }
+  int sms = 0, occ = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, sample_scan_kernel<T, kVec>,
+                                                    kScanThreads, 0) != cudaSuccess) {
+    cudaGetLastError();
+    sms = 1;
+    occ = 1;
+  }
+  const int n = std::max(1, sms * std::max(occ, 1));
+  if (dev < kMaxDev) cache[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
+
+int chunks_per_row(int vocab) {
+  const int ipr = (vocab + kItem - 1) / kItem;
+  return (ipr + kChunk - 1) / kChunk;
+}
+
+template <typename T, bool kVec>
+cudaError_t launch_sampler_v(const SamplerArgs& a, cudaStream_t stream) {
   const T* lg = static_cast<const T*>(a.logits);
-  const size_t esz = sizeof(T);
-  const bool vec = ((reinterpret_cast<uintptr_t>(lg) & 15u) == 0) &&
-                   (((size_t)a.row_stride * esz) % 16 == 0) && (a.vocab % 8 == 0);
-  const int64_t grid = (int64_t)a.rows * nchunk;
-  if (vec)
-    sample_chunk_bulk_kernel<T><<<(unsigned)grid, kSampleThreads, 0, stream>>>(
-        lg, a.row_stride, a.vocab, nchunk, a.inv_tau, a.seed, a.step, a.row_offset, a.recs,
-        a.err);
-  else
-    sample_chunk_scalar_kernel<T><<<(unsigned)grid, kSampleThreads, 0, stream>>>(
-        lg, a.row_stride, a.vocab, nchunk, a.inv_tau, a.seed, a.step, a.row_offset, a.recs);
+  ScanParams p;
+  p.key = philox_key(a.seed);
+  p.row_stride = a.row_stride;
+  p.vocab = a.vocab;
+  p.ipr = (a.vocab + kItem - 1) / kItem;
+  p.nck = chunks_per_row(a.vocab);
+  p.nchunks = (uint32_t)((uint64_t)a.rows * (uint64_t)p.nck);
+  p.rows = a.rows;
+  p.jtail = (a.vocab % kItem) ? p.ipr - 1 : -1;
+  p.c2 = a.inv_tau * kLog2e;
+  p.inv_c2 = 1.0f / p.c2;
+  p.inv_tau = a.inv_tau;
+  p.step = a.step;
+  p.row_offset = a.row_offset;
+  const SamplerState s = sampler_state(a.state);
+  float4* recs = static_cast<float4*>(a.recs);
+  const int64_t want = ((int64_t)p.nchunks + kScanWarpsPerCta - 1) / kScanWarpsPerCta;
+  const int ctas = (int)std::min<int64_t>(scan_ctas<T, kVec>(), want);
+  sample_scan_kernel<T, kVec><<<ctas, kScanThreads, 0, stream>>>(lg, p, recs, s.row_key, s.ticket);
   note_launch();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   sample_merge_kernel<T><<<(a.rows + 3) / 4, 128, 0, stream>>>(
-      lg, a.row_stride, a.rows, a.vocab, nchunk, a.inv_tau, a.rate, a.seed, a.step,
-      a.row_offset, a.recs, a.tokens, a.pred, a.conf, a.entropy, a.renoised);
+      lg, a.row_stride, a.rows, a.vocab, p.nck, a.inv_tau, a.rate, a.seed, a.step, a.row_offset,
+      recs, s.row_key, s.ticket, a.tokens, a.pred, a.conf, a.entropy, a.renoised);
   note_launch();
   return cudaGetLastError();
 }
 
+template <typename T>
+cudaError_t launch_sampler_t(const SamplerArgs& a, cudaStream_t stream) {
+  const size_t esz = sizeof(T);
+  const bool vec = ((reinterpret_cast<uintptr_t>(a.logits) & 15u) == 0) &&
+                   (((size_t)a.row_stride * esz) % 16 == 0) && (a.vocab % 8 == 0);
+  return vec ? launch_sampler_v<T, true>(a, stream) : launch_sampler_v<T, false>(a, stream);
+}
+
 }  // namespace
 
-int sampler_nchunk(int vocab, bool bf16) {
-  const int ce = bf16 ? chunk_elems<__nv_bfloat16>() : chunk_elems<float>();
-  return (vocab + ce - 1) / ce;
+size_t sampler_state_bytes(int rows) {
+  return 256 + (size_t)rows * kKeyStride * sizeof(unsigned long long);
+}
+
+size_t sampler_record_bytes(int rows, int vocab) {
+  return (size_t)rows * (size_t)chunks_per_row(vocab) * sizeof(float4);
+}
+
+SamplerState sampler_state(void* state) {
+  SamplerState s;
+  s.ticket = static_cast<uint32_t*>(state);
+  s.row_key = reinterpret_cast<unsigned long long*>(static_cast<uint8_t*>(state) + 256);
+  return s;
 }
 
 cudaError_t launch_sampler(const SamplerArgs& a, cudaStream_t stream) {

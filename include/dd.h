@@ -26,8 +26,11 @@
  *     (thread-local).  Nothing aborts or throws across this boundary.
  *   - Device-side faults that kernels detect themselves (a pipeline wait that
  *     exceeded its time limit) are latched in the first 16 bytes of the
- *     workspace and read back by dd_query_device_error.  A workspace must be
- *     cleared once with dd_workspace_init before first use.
+ *     workspace and read back by dd_query_device_error.
+ *   - A workspace must be cleared once with dd_workspace_init before its
+ *     first use.  The sampler keeps a small state in it (a work counter and
+ *     per-row maxima) that every completed call leaves cleared; after a call
+ *     that failed on the device, clear the workspace again.
  *   - There is no CPU fallback: if the CUDA kernels cannot run, calls fail.
  */
 #ifndef DD_H_
@@ -197,10 +200,11 @@ DD_API dd_status dd_denoise_block(const dd_attn_desc* desc, int steps, const voi
  * synchronisation).  The paper has no counterpart: this is a deployment
  * variant of the same sampler step.
  * Arguments and results: exactly as dd_sample_renoise, minus the workspace.
- * Scratch: a static device array of 2 MiB that the library holds on every
+ * Scratch: a static device array of 4 MiB that the library holds on every
  * GPU it is loaded on until the process exits.  A call needs
- * dd_sample_renoise_workspace(rows, vocab, dtype) bytes of it (512 bytes per
- * row at V = 262144 in bf16, so up to 4095 rows); larger calls return
+ * dd_sample_renoise_workspace(rows, vocab, dtype) bytes of it (about 8 bytes
+ * per row plus 16 bytes per 2048 vocabulary entries per row, so up to 2039
+ * rows at V = 262144); larger calls return
  * DD_ERR_UNSUPPORTED before touching the GPU.  The function allocates
  * nothing: no cudaMalloc, cudaFree or allocating library call.
  * The first call on a device looks up the array's device address
@@ -215,7 +219,8 @@ DD_API dd_status dd_sample_renoise_noalloc(const void* logits, dd_dtype dtype, i
                                            float* conf_out, float* entropy_out,
                                            uint8_t* renoised_out, dd_stream_t stream);
 
-/* Clears the error word at the start of a workspace (async on stream). */
+/* Clears a whole workspace: the error word and the sampler's state (async on
+ * stream).  Call once before a workspace's first use. */
 DD_API dd_status dd_workspace_init(void* workspace, size_t workspace_bytes, dd_stream_t stream);
 
 /* Synchronises `stream`, reads the workspace's latched device error and

@@ -128,6 +128,24 @@ def test_deterministic_across_calls():
         assert torch.equal(a[k], b[k]), k
 
 
+def test_workspace_reuse_leaves_state_clear():
+    """The sampler keeps a work counter and per-row maxima in the workspace
+    and clears them at the end of every call: calls that share one workspace
+    (different rows, vocabularies, seeds) give what fresh workspaces give."""
+    a_lg = _gen(256, 262144, 3.0, torch.bfloat16, seed=21, spike=8.0)
+    b_lg = _gen(40, 50000, 2.0, torch.float32, seed=22)
+    ws = dd.new_workspace(max(dd.sample_workspace_bytes(256, 262144),
+                              dd.sample_workspace_bytes(40, 50000)))
+    a1 = _run(a_lg, 1.0, 0.3, 3, 4, workspace=ws)
+    b1 = _run(b_lg, 0.7, 0.5, 4, 5, workspace=ws)
+    a2 = _run(a_lg, 1.0, 0.3, 3, 4, workspace=ws)
+    b_fresh = _run(b_lg, 0.7, 0.5, 4, 5)
+    for k in a1:
+        assert torch.equal(a1[k], a2[k]), k
+        assert torch.equal(b1[k], b_fresh[k]), k
+    check_sampler(b1, oracle.sample_renoise(b_lg.cpu(), 0.7, 0.5, 4, 5))
+
+
 def test_large_seed_and_step():
     lg = _gen(16, 4096, 3.0, torch.bfloat16, seed=9)
     seed, step = 0xDEADBEEFCAFEF00D, 0xFFFFFFF0

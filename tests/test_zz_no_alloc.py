@@ -81,7 +81,7 @@ def test_noalloc_rejects_calls_beyond_its_scratch():
     lib = dd.load()
     prm = dd.SampleParams(1.0, 0.5, 0, 0, 0)
     fake = ctypes.c_void_p(1 << 20)  # never dereferenced: the size check comes first
-    st = lib.dd_sample_renoise_noalloc(fake, dd.DD_BF16, 8192, 262144, 262144, ctypes.byref(prm),
+    st = lib.dd_sample_renoise_noalloc(fake, dd.DD_BF16, 57337, 262144, 262144, ctypes.byref(prm),
                                        fake, None, fake, None, None, None)
     assert st == 2  # DD_ERR_UNSUPPORTED
     assert "static scratch" in dd.last_error()
