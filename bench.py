@@ -271,9 +271,44 @@ def run_ours(args, w, dist, rank, world, local_rank):
         "gpu_launches": int(launches),
         "clocks": clk,
     }
+    if w.steps > 1:
+        res["block"] = run_block(w, dd, dev, dist)
     if rank == 0 and world == 1 and not args.no_cpu:
         res["cpu_baseline"] = cpu_baseline(w, sets[0], frac=args.cpu_sample)
     return res
+
+
+def run_block(w, dd, dev, dist, reps: int = 20):
+    """The whole block loop (dd_denoise_block over the workload's steps, with
+    its rate schedule) on pre-generated per-step inputs: mean device time of
+    one block, max over ranks."""
+    q, kc, vc, lg = workloads.all_steps(w, device=dev)
+    kp, vp, cu = workloads.prefix_kv(w, device=dev)
+    cud = cu.to(dev)
+    desc = dd.attn_desc(q[0], kc[0], w.scale)
+    ws = dd.new_workspace(dd.denoise_block_workspace_bytes(desc, cu.numpy(), w.vocab), dev)
+    attn_out = torch.empty_like(q)
+    canvas = torch.empty(w.rows, dtype=torch.int32, device=dev)
+
+    def block():
+        dd.denoise_block(q, kc, vc, kp, vp, cud, lg, w.rates, w.temperatures, w.seed,
+                         cu_prefix_host=cu.numpy(), scale=w.scale, attn_out=attn_out,
+                         canvas=canvas, keep_history=False, workspace=ws)
+
+    for _ in range(3):
+        block()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        block()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = _max_over_ranks(dist, e0.elapsed_time(e1) / reps)
+    dd.query_device_error(ws)
+    return {"steps": w.steps, "ms_per_block": ms, "blocks_per_s": 1e3 / ms,
+            "timing": f"mean of {reps} eager dd_denoise_block calls, CUDA events"}
 
 
 # The sampler's arithmetic ceiling: per warp-item of 256 logits the scan
