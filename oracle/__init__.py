@@ -82,6 +82,10 @@ def _load():
                                           P, P, P, P, P, P, P, i32]
     lib.oracle_init_canvas.restype = None
     lib.oracle_init_canvas.argtypes = [P, i64, i64, u64, u32]
+    lib.oracle_entropy_accept.argtypes = [P, P, i64, i64, f64, u64, u32, u32, i64, P, P, P, P]
+    lib.oracle_entropy_accept.restype = None
+    lib.oracle_stop_check.argtypes = [P, P, P, i64, i64, f64, P]
+    lib.oracle_stop_check.restype = None
     _lib = lib
     return lib
 
@@ -226,6 +230,51 @@ def init_canvas(rows: int, vocab: int, seed: int, row_offset: int = 0):
     out = np.empty(rows, np.int32)
     lib.oracle_init_canvas(_ptr(out), rows, vocab, seed, row_offset)
     return out
+
+
+# ------------------------------------------------ the pages' sampler policy
+
+def anneal_temperature(s: int, steps: int, t0: float = 0.8, t1: float = 0.4) -> float:
+    """Temperature of step s of a block whose nominal budget is `steps`:
+    annealed linearly from t0 to t1 ("The mechanism", sampler paragraph:
+    tau 0.8 -> 0.4; the pages give the end points only, linear in the step
+    index over the nominal budget is the reading taken), as float32."""
+    if steps <= 1:
+        return float(np.float32(t0))
+    return float(np.float32(t0 + (t1 - t0) * s / (steps - 1)))
+
+
+def entropy_accept(entropy, pred, canvas: int, budget: float, seed: int, step: int, vocab: int,
+                   row_offset: int = 0):
+    """Entropy-budget acceptance (dd_oracle.c: oracle_entropy_accept).
+
+    entropy: float32 [B*C] (rounded to float32 here), pred int32 [B*C].
+    Returns dict(tokens, accepted, n_accepted [B], sum_accepted [B])."""
+    lib = _load()
+    h = np.ascontiguousarray(np.asarray(entropy, dtype=np.float32).reshape(-1))
+    pr = np.ascontiguousarray(np.asarray(pred, dtype=np.int32).reshape(-1))
+    assert h.size == pr.size and h.size % canvas == 0
+    B = h.size // canvas
+    res = {"tokens": np.empty(h.size, np.int32), "accepted": np.empty(h.size, np.uint8),
+           "n_accepted": np.empty(B, np.int32), "sum_accepted": np.empty(B, np.float64)}
+    lib.oracle_entropy_accept(_ptr(h), _ptr(pr), B, canvas, float(budget), int(seed), int(step),
+                              int(row_offset), int(vocab), _ptr(res["tokens"]),
+                              _ptr(res["accepted"]), _ptr(res["n_accepted"]),
+                              _ptr(res["sum_accepted"]))
+    return res
+
+
+def stop_check(entropy, pred, pred_prev, canvas: int, threshold: float = 0.005):
+    """Early-halt test per canvas (dd_oracle.c: oracle_stop_check)."""
+    lib = _load()
+    h = np.ascontiguousarray(np.asarray(entropy, dtype=np.float32).reshape(-1))
+    pr = np.ascontiguousarray(np.asarray(pred, dtype=np.int32).reshape(-1))
+    pp = None if pred_prev is None else np.ascontiguousarray(
+        np.asarray(pred_prev, dtype=np.int32).reshape(-1))
+    B = h.size // canvas
+    done = np.empty(B, np.uint8)
+    lib.oracle_stop_check(_ptr(h), _ptr(pr), _ptr(pp), B, canvas, float(threshold), _ptr(done))
+    return done
 
 
 # --------------------------------------------------------- the block loop

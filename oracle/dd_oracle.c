@@ -17,6 +17,12 @@
  *              per-position entropies from temperature-scaled logits.
  *   [DG-train] same review, section "Training": every canvas token is
  *              corrupted independently with probability t.
+ *   [DG-samp]  same review, section "The mechanism", the paragraph on the
+ *              sampler: temperature annealed 0.8 -> 0.4; positions accepted
+ *              greedily from lowest to highest entropy until a cumulative
+ *              entropy budget (b = 0.1) is exhausted, the rest re-noised to
+ *              uniform random tokens; early halt when the mean canvas entropy
+ *              is below 0.005 and the prediction is stable across two steps.
  *   [Philox]   Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as easy
  *              as 1, 2, 3", SC'11: the Philox-4x32 bijection, 10 rounds.
  *
@@ -29,7 +35,15 @@
  *     3 canvas initialisation (streams 1-3 use counter word 0 = 0, output 0);
  *   - re-noise each position independently when U(stream 1) < rate (fp32);
  *   - replacement token = (x(stream 2) * V) >> 32; canvas init the same with
- *     stream 3 and step 0.
+ *     stream 3 and step 0;
+ *   - entropy-budget acceptance: entropies in increasing order, equal values
+ *     by increasing position; the running sum is float64, summed in that
+ *     order, and a position is accepted while the sum including it stays
+ *     <= b, so the accepted set is a prefix of that order;
+ *   - the early-halt "argmax prediction" is the sampler's prediction (the
+ *     argmax of the Gumbel-perturbed scores); a canvas halts at a step whose
+ *     float64 mean entropy is below the threshold and whose predictions all
+ *     equal the previous step's.
  */
 #include <math.h>
 #include <stdint.h>
@@ -292,5 +306,76 @@ void oracle_init_canvas(int32_t* out, int64_t rows, int64_t vocab, uint64_t seed
   for (int64_t r = 0; r < rows; ++r) {
     const uint32_t x = oracle_word(seed, 3, 0, row_offset + (uint32_t)r, 0);
     out[r] = (int32_t)(((uint64_t)x * (uint64_t)vocab) >> 32);
+  }
+}
+
+/* ------------------------------------------------ the pages' sampler policy */
+
+typedef struct {
+  float h;
+  int64_t pos;
+} ent_pos;
+
+static int cmp_ent_pos(const void* a, const void* b) {
+  const ent_pos* x = (const ent_pos*)a;
+  const ent_pos* y = (const ent_pos*)b;
+  if (x->h < y->h) return -1;
+  if (x->h > y->h) return 1;
+  return x->pos < y->pos ? -1 : (x->pos > y->pos ? 1 : 0);
+}
+
+/* Entropy-budget acceptance [DG-samp].  For each canvas b of C positions
+ * (rows b*C .. b*C+C-1): sort the positions by entropy (ties by position),
+ * accept them in that order while the float64 running sum of accepted
+ * entropies stays <= budget, stop at the first that would exceed it.
+ * Accepted positions keep pred; the others are re-noised to the uniform
+ * replacement token x(stream 2) * V >> 32 of their row (as [DG-mech]).
+ * entropy is float32, the precision the sampler outputs.  n_accepted[b] is
+ * the count and sum_accepted[b] the float64 sum of the accepted entropies. */
+void oracle_entropy_accept(const float* entropy, const int32_t* pred, int64_t B, int64_t C,
+                           double budget, uint64_t seed, uint32_t step, uint32_t row_offset,
+                           int64_t vocab, int32_t* tokens, uint8_t* accepted,
+                           int32_t* n_accepted, double* sum_accepted) {
+  ent_pos* order = (ent_pos*)malloc(sizeof(ent_pos) * (size_t)(C > 0 ? C : 1));
+  for (int64_t b = 0; b < B; ++b) {
+    for (int64_t i = 0; i < C; ++i) {
+      order[i].h = entropy[b * C + i];
+      order[i].pos = i;
+    }
+    qsort(order, (size_t)C, sizeof(ent_pos), cmp_ent_pos);
+    for (int64_t i = 0; i < C; ++i) accepted[b * C + i] = 0;
+    double sum = 0.0;
+    int64_t k = 0;
+    for (; k < C; ++k) {
+      const double next = sum + (double)order[k].h;
+      if (!(next <= budget)) break;
+      sum = next;
+      accepted[b * C + order[k].pos] = 1;
+    }
+    if (n_accepted) n_accepted[b] = (int32_t)k;
+    if (sum_accepted) sum_accepted[b] = sum;
+    for (int64_t i = 0; i < C; ++i) {
+      const int64_t r = b * C + i;
+      const uint32_t x2 = oracle_word(seed, 2, step, row_offset + (uint32_t)r, 0);
+      const int32_t repl = (int32_t)(((uint64_t)x2 * (uint64_t)vocab) >> 32);
+      tokens[r] = accepted[r] ? pred[r] : repl;
+    }
+  }
+  free(order);
+}
+
+/* Early-halt test [DG-samp]: done[b] = 1 when the float64 mean of canvas b's
+ * entropies is below `threshold` and pred equals pred_prev at every position
+ * (pred_prev NULL: no previous step, never done). */
+void oracle_stop_check(const float* entropy, const int32_t* pred, const int32_t* pred_prev,
+                       int64_t B, int64_t C, double threshold, uint8_t* done) {
+  for (int64_t b = 0; b < B; ++b) {
+    double sum = 0.0;
+    int same = pred_prev != NULL;
+    for (int64_t i = 0; i < C; ++i) {
+      sum += (double)entropy[b * C + i];
+      if (pred_prev && pred[b * C + i] != pred_prev[b * C + i]) same = 0;
+    }
+    done[b] = (uint8_t)(same && sum / (double)C < threshold);
   }
 }
