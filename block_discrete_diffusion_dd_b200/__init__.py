@@ -30,6 +30,8 @@ EXPORTS = (
     "dd_sample_renoise", "dd_init_canvas", "dd_denoise_block_workspace", "dd_denoise_block",
     "dd_workspace_init", "dd_query_device_error", "dd_status_string", "dd_last_error",
     "dd_launch_count", "dd_reset_launch_count", "dd_sample_renoise_noalloc",
+    "dd_entropy_accept", "dd_stop_check", "dd_denoise_block_adaptive_workspace",
+    "dd_denoise_block_adaptive",
 )
 
 
@@ -85,6 +87,17 @@ def load() -> ctypes.CDLL:
     lib.dd_denoise_block.restype = i32
     lib.dd_denoise_block.argtypes = [D, i32, P, P, P, P, P, P, P, P, P, i32, P, P, u64, u32, P, P,
                                      P, P, sz, P]
+    f32 = ctypes.c_float
+    lib.dd_entropy_accept.restype = i32
+    lib.dd_entropy_accept.argtypes = [P, P, i32, i32, i32, f32, u64, u32, u32, P, P, P]
+    lib.dd_stop_check.restype = i32
+    lib.dd_stop_check.argtypes = [P, P, P, i32, i32, f32, ctypes.c_int32, P, P, P]
+    lib.dd_denoise_block_adaptive_workspace.restype = sz
+    lib.dd_denoise_block_adaptive_workspace.argtypes = [D, P, i32]
+    lib.dd_denoise_block_adaptive.restype = i32
+    lib.dd_denoise_block_adaptive.argtypes = [D, i32, P, P, P, P, P, P, P, P, P, i32, P, f32, f32,
+                                              u64, u32, P, P, P, ctypes.POINTER(ctypes.c_int),
+                                              P, sz, P]
     lib.dd_workspace_init.restype = i32
     lib.dd_workspace_init.argtypes = [P, sz, P]
     lib.dd_query_device_error.restype = i32
@@ -281,6 +294,69 @@ def denoise_block(q_steps, kc_steps, vc_steps, kp, vp, cu_prefix, logits_steps,
         _ptr(workspace), workspace.numel(), _stream(stream)))
     return {"attn_out": attn_out, "canvas": canvas, "canvas_history": canvas_history,
             "conf_steps": conf_steps}
+
+
+def entropy_accept(entropy: torch.Tensor, pred: torch.Tensor, canvas: int, budget: float,
+                   seed: int, step: int, vocab: int, row_offset: int = 0, tokens=None,
+                   accepted=None, stream=None) -> dict:
+    """dd_entropy_accept: the pages' entropy-budget acceptance per canvas."""
+    R = entropy.numel()
+    if tokens is None:
+        tokens = torch.empty(R, dtype=torch.int32, device=entropy.device)
+    if accepted is None:
+        accepted = torch.empty(R, dtype=torch.uint8, device=entropy.device)
+    _check(load().dd_entropy_accept(_ptr(entropy), _ptr(pred), R // canvas, canvas, vocab,
+                                    float(budget), int(seed), int(step), int(row_offset),
+                                    _ptr(tokens), _ptr(accepted), _stream(stream)))
+    return {"tokens": tokens, "accepted": accepted}
+
+
+def stop_check(entropy: torch.Tensor, pred: torch.Tensor, pred_prev, canvas: int,
+               threshold: float, step: int, done: torch.Tensor, halt_step: torch.Tensor,
+               stream=None):
+    """dd_stop_check: updates done [B] and halt_step [B] in place."""
+    _check(load().dd_stop_check(_ptr(entropy), _ptr(pred), _ptr(pred_prev),
+                                entropy.numel() // canvas, canvas, float(threshold), int(step),
+                                _ptr(done), _ptr(halt_step), _stream(stream)))
+
+
+def denoise_block_adaptive(q_steps, kc_steps, vc_steps, kp, vp, cu_prefix, logits_steps,
+                           temperatures: Sequence[float], budget: float, stop_entropy: float,
+                           seed: int, step0: int = 0, cu_prefix_host=None, scale=None,
+                           attn_out=None, canvas=None, keep_history=True, workspace=None,
+                           stream=None) -> dict:
+    """dd_denoise_block_adaptive: the block loop under the pages' policy.
+
+    Returns dict(canvas, canvas_history [steps_run, R] or None, halt_step [B],
+    steps_run)."""
+    lib = load()
+    S = q_steps.shape[0]
+    desc = attn_desc(q_steps[0], kc_steps[0], scale)
+    cu_h = _host_i32(cu_prefix if cu_prefix_host is None else cu_prefix_host)
+    V = logits_steps.shape[-1]
+    R = desc.batch * desc.canvas
+    dev = q_steps.device
+    if attn_out is None:
+        attn_out = torch.empty_like(q_steps)
+    if canvas is None:
+        canvas = torch.zeros(R, dtype=torch.int32, device=dev)
+    history = torch.empty((S, R), dtype=torch.int32, device=dev) if keep_history else None
+    halt = torch.empty(desc.batch, dtype=torch.int32, device=dev)
+    if workspace is None:
+        workspace = new_workspace(int(lib.dd_denoise_block_adaptive_workspace(
+            ctypes.byref(desc), cu_h.ctypes.data_as(ctypes.c_void_p), V)), dev, stream)
+    temps_h = np.ascontiguousarray(np.asarray(temperatures, dtype=np.float32))
+    assert temps_h.size >= S
+    steps_run = ctypes.c_int(0)
+    _check(lib.dd_denoise_block_adaptive(
+        ctypes.byref(desc), S, _ptr(q_steps), _ptr(kc_steps), _ptr(vc_steps), _ptr(kp), _ptr(vp),
+        _ptr(cu_prefix), cu_h.ctypes.data_as(ctypes.c_void_p), _ptr(attn_out),
+        _ptr(logits_steps), V, temps_h.ctypes.data_as(ctypes.c_void_p), float(budget),
+        float(stop_entropy), int(seed), int(step0), _ptr(canvas), _ptr(history), _ptr(halt),
+        ctypes.byref(steps_run), _ptr(workspace), workspace.numel(), _stream(stream)))
+    n = steps_run.value
+    return {"canvas": canvas, "canvas_history": None if history is None else history[:n],
+            "halt_step": halt, "steps_run": n}
 
 
 def query_device_error(workspace: torch.Tensor, stream=None):

@@ -3,6 +3,8 @@
 // carving, error reporting and the block loop.  All device work happens in
 // the kernels of dd_sampler.cu, dd_attn_tc.cu and dd_attn_simt.cu.
 #include <cmath>
+#include <utility>
+#include <vector>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -342,6 +344,147 @@ dd_status dd_denoise_block(const dd_attn_desc* desc, int steps, const void* q_st
                                       cudaMemcpyDeviceToDevice, s);
       if (e != cudaSuccess) return cuda_fail(e, "canvas copy");
     }
+  }
+  return DD_OK;
+}
+
+dd_status dd_entropy_accept(const float* entropy, const int32_t* pred, int batch, int canvas,
+                            int vocab, float budget, uint64_t seed, uint32_t step,
+                            uint32_t row_offset, int32_t* tokens_out, uint8_t* accepted_out,
+                            dd_stream_t stream) {
+  g_last_error.clear();
+  if (batch < 0 || canvas < 1 || canvas > 1024 || vocab < 1)
+    return fail(DD_ERR_INVALID_ARG, "batch=%d canvas=%d (1..1024) vocab=%d", batch, canvas, vocab);
+  if (std::isnan(budget)) return fail(DD_ERR_INVALID_ARG, "budget is NaN");
+  if ((uint64_t)batch * (uint64_t)canvas + row_offset > (1ull << 32))
+    return fail(DD_ERR_INVALID_ARG, "row_offset + rows exceeds 2^32");
+  if (batch == 0) return DD_OK;
+  if (!entropy || !pred || !tokens_out) return fail(DD_ERR_INVALID_ARG, "NULL required pointer");
+  cudaError_t e = launch_entropy_accept(entropy, pred, batch, canvas, vocab, (double)budget, seed,
+                                        step, row_offset, nullptr, nullptr, 0, tokens_out,
+                                        accepted_out, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "entropy accept");
+  return DD_OK;
+}
+
+dd_status dd_stop_check(const float* entropy, const int32_t* pred, const int32_t* pred_prev,
+                        int batch, int canvas, float threshold, int32_t step, uint8_t* done,
+                        int32_t* halt_step, dd_stream_t stream) {
+  g_last_error.clear();
+  if (batch < 0 || canvas < 1) return fail(DD_ERR_INVALID_ARG, "batch=%d canvas=%d", batch, canvas);
+  if (batch == 0) return DD_OK;
+  if (!entropy || !pred || !done || !halt_step)
+    return fail(DD_ERR_INVALID_ARG, "NULL required pointer");
+  cudaError_t e = launch_stop_check(entropy, pred, pred_prev, batch, canvas, (double)threshold,
+                                    step, done, halt_step, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "stop check");
+  return DD_OK;
+}
+
+namespace {
+// Adaptive-loop workspace: the block-loop layout, then two prediction
+// buffers, the entropies and the per-canvas halt flags.
+size_t adaptive_ws_layout(const dd_attn_desc* desc, int64_t total, const int32_t* cu_prefix_host,
+                          int vocab, size_t* state_off, size_t* conf_off, size_t* extra_off) {
+  const size_t base = block_ws_layout(desc, total, cu_prefix_host, vocab, state_off, conf_off);
+  const size_t rows = (size_t)desc->batch * desc->canvas;
+  if (extra_off) *extra_off = base;
+  return base + 2 * align256(rows * 4) + align256(rows * 4) + align256((size_t)desc->batch);
+}
+}  // namespace
+
+size_t dd_denoise_block_adaptive_workspace(const dd_attn_desc* desc,
+                                           const int32_t* cu_prefix_host, int vocab) {
+  int64_t total = 0;
+  if (vocab < 1 || check_attn_desc(desc, cu_prefix_host, &total) != DD_OK) return 0;
+  return adaptive_ws_layout(desc, total, cu_prefix_host, vocab, nullptr, nullptr, nullptr);
+}
+
+dd_status dd_denoise_block_adaptive(const dd_attn_desc* desc, int max_steps, const void* q_steps,
+                                    const void* kc_steps, const void* vc_steps,
+                                    const void* k_prefix, const void* v_prefix,
+                                    const int32_t* cu_prefix, const int32_t* cu_prefix_host,
+                                    void* attn_out, const void* logits_steps, int vocab,
+                                    const float* temperature_host, float budget,
+                                    float stop_entropy, uint64_t seed, uint32_t step0,
+                                    int32_t* canvas, int32_t* canvas_history,
+                                    int32_t* halt_step, int* steps_run, void* workspace,
+                                    size_t workspace_bytes, dd_stream_t stream) {
+  g_last_error.clear();
+  int64_t total = 0;
+  dd_status st = check_attn_desc(desc, cu_prefix_host, &total);
+  if (st != DD_OK) return st;
+  if (max_steps < 0) return fail(DD_ERR_INVALID_ARG, "max_steps < 0");
+  if (max_steps > 0 && !temperature_host) return fail(DD_ERR_INVALID_ARG, "temperature_host is NULL");
+  if (!canvas || !halt_step || !steps_run) return fail(DD_ERR_INVALID_ARG, "NULL required pointer");
+  if (desc->canvas > 1024) return fail(DD_ERR_UNSUPPORTED, "canvas > 1024");
+  if (std::isnan(budget) || std::isnan(stop_entropy))
+    return fail(DD_ERR_INVALID_ARG, "budget / stop_entropy is NaN");
+  if ((uint64_t)step0 + (uint64_t)max_steps > (1ull << 32))
+    return fail(DD_ERR_INVALID_ARG, "step0 + max_steps exceeds 2^32");
+  if (vocab < 1) return fail(DD_ERR_INVALID_ARG, "vocab=%d", vocab);
+  const int B = desc->batch, C = desc->canvas, Hq = desc->heads_q, Hkv = desc->heads_kv;
+  const int D = desc->head_dim;
+  const int rows = B * C;
+  const size_t es = elem_size(desc->dtype);
+  const size_t q_step = (size_t)rows * Hq * D * es;
+  const size_t kv_step = (size_t)rows * Hkv * D * es;
+  const size_t lg_step = (size_t)rows * (size_t)vocab * es;
+  size_t state_off = 0, conf_off = 0, extra_off = 0;
+  const size_t need = adaptive_ws_layout(desc, total, cu_prefix_host, vocab, &state_off,
+                                         &conf_off, &extra_off);
+  if (!workspace) return fail(DD_ERR_WORKSPACE, "workspace is NULL");
+  if (workspace_bytes < need)
+    return fail(DD_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", workspace_bytes, need);
+  *steps_run = 0;
+  if (B == 0) return DD_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* const ws = static_cast<uint8_t*>(workspace);
+  int32_t* pred_a = reinterpret_cast<int32_t*>(ws + extra_off);
+  int32_t* pred_b = reinterpret_cast<int32_t*>(ws + extra_off + align256((size_t)rows * 4));
+  float* ent = reinterpret_cast<float*>(ws + extra_off + 2 * align256((size_t)rows * 4));
+  uint8_t* done = ws + extra_off + 3 * align256((size_t)rows * 4);
+  float* conf = reinterpret_cast<float*>(ws + conf_off);
+  cudaError_t e = cudaMemsetAsync(done, 0, (size_t)B, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(halt_step, 0xff, (size_t)B * sizeof(int32_t), s);
+  if (e != cudaSuccess) return cuda_fail(e, "adaptive loop init");
+  std::vector<uint8_t> done_h((size_t)B);
+  int32_t* cur = pred_a;
+  int32_t* prev = pred_b;
+  for (int i = 0; i < max_steps; ++i) {
+    st = run_attn(desc, static_cast<const uint8_t*>(q_steps) + i * q_step,
+                  static_cast<const uint8_t*>(kc_steps) + i * kv_step,
+                  static_cast<const uint8_t*>(vc_steps) + i * kv_step, k_prefix, v_prefix,
+                  cu_prefix, cu_prefix_host, static_cast<uint8_t*>(attn_out) + i * q_step,
+                  nullptr, workspace, state_off, s);
+    if (st != DD_OK) return st;
+    dd_sample_params sp;
+    sp.temperature = temperature_host[i];
+    sp.renoise_rate = 0.f;  // the acceptance rule below decides the re-noise
+    sp.seed = seed;
+    sp.step = step0 + (uint32_t)i;
+    sp.row_offset = 0;
+    st = run_sampler(static_cast<const uint8_t*>(logits_steps) + i * lg_step, desc->dtype, rows,
+                     vocab, vocab, &sp, cur, nullptr, conf, ent, nullptr, workspace, state_off, s,
+                     ws + state_off);
+    if (st != DD_OK) return st;
+    e = launch_stop_check(ent, cur, i > 0 ? prev : nullptr, B, C, (double)stop_entropy, i, done,
+                          halt_step, s);
+    if (e == cudaSuccess)
+      e = launch_entropy_accept(ent, cur, B, C, vocab, (double)budget, seed, step0 + (uint32_t)i, 0,
+                                done, halt_step, i, canvas, nullptr, s);
+    if (e == cudaSuccess && canvas_history)
+      e = cudaMemcpyAsync(canvas_history + (size_t)i * rows, canvas, (size_t)rows * sizeof(int32_t),
+                          cudaMemcpyDeviceToDevice, s);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(done_h.data(), done, (size_t)B, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e, "adaptive step");
+    *steps_run = i + 1;
+    bool all = true;
+    for (int b = 0; b < B; ++b) all = all && done_h[(size_t)b] != 0;
+    if (all) break;
+    std::swap(cur, prev);
   }
   return DD_OK;
 }

@@ -38,6 +38,16 @@ size_t sampler_state_bytes(int rows);
 // Per-chunk partial records (16 bytes per chunk of 2048 entries).
 size_t sampler_record_bytes(int rows, int vocab);
 cudaError_t launch_sampler(const SamplerArgs& a, cudaStream_t stream);
+
+// The pages' acceptance rule and early-halt test (dd_policy.cu); C <= 1024.
+cudaError_t launch_entropy_accept(const float* entropy, const int32_t* pred, int B, int C,
+                                  int vocab, double budget, uint64_t seed, uint32_t step,
+                                  uint32_t row_offset, const uint8_t* done,
+                                  const int32_t* halt_step, int32_t cur, int32_t* tokens,
+                                  uint8_t* accepted, cudaStream_t stream);
+cudaError_t launch_stop_check(const float* entropy, const int32_t* pred, const int32_t* pred_prev,
+                              int B, int C, double threshold, int32_t cur, uint8_t* done,
+                              int32_t* halt_step, cudaStream_t stream);
 cudaError_t launch_init_canvas(int32_t* canvas, int rows, int vocab, uint64_t seed,
                                uint32_t row_offset, cudaStream_t stream);
 

@@ -219,6 +219,73 @@ DD_API dd_status dd_sample_renoise_noalloc(const void* logits, dd_dtype dtype, i
                                            float* conf_out, float* entropy_out,
                                            uint8_t* renoised_out, dd_stream_t stream);
 
+/* ---- The pages' own sampler policy ("DiffusionGemma Technical Report",
+ * "The mechanism", sampler paragraph): temperature annealed 0.8 -> 0.4,
+ * positions accepted greedily from lowest to highest entropy until a
+ * cumulative entropy budget (b = 0.1) is exhausted and the rest re-noised to
+ * uniform random tokens, early halt when the mean canvas entropy is below
+ * 0.005 and the prediction is stable across two steps.  The benchmark spec's
+ * scheduled-rate loop (dd_denoise_block) stays the default; these calls are
+ * the pages' alternative. */
+
+/* Entropy-budget acceptance for `batch` canvases of `canvas` positions
+ * (rows b*canvas .. b*canvas+canvas-1): positions are taken in increasing
+ * entropy (equal entropies: lower position first) and accepted while the
+ * float64 running sum of accepted entropies stays <= budget; the first that
+ * would exceed it ends the acceptance.  tokens_out = pred at accepted
+ * positions, elsewhere the uniform replacement token of the row as in
+ * dd_sample_renoise: (x(2, 0) * V) >> 32 under key seed, counter
+ * (0, row_offset + row, step, 2).
+ *   entropy      fp32 [rows] (as dd_sample_renoise outputs it)
+ *   pred         int32 [rows]
+ *   tokens_out   int32 [rows]
+ *   accepted_out uint8 [rows] or NULL
+ * canvas must be 1..1024. */
+DD_API dd_status dd_entropy_accept(const float* entropy, const int32_t* pred, int batch, int canvas,
+                                   int vocab, float budget, uint64_t seed, uint32_t step,
+                                   uint32_t row_offset, int32_t* tokens_out, uint8_t* accepted_out,
+                                   dd_stream_t stream);
+
+/* Early-halt test, per canvas: a canvas not yet done halts at this step when
+ * the float64 mean of its entropies (summed in position order) is below
+ * `threshold` and pred equals pred_prev at every position (pred_prev NULL:
+ * no previous step, no halt).  Halting sets done[b] = 1 and halt_step[b] =
+ * step; canvases already done are left alone.
+ *   entropy fp32 [rows]; pred, pred_prev int32 [rows]
+ *   done uint8 [batch] (in/out); halt_step int32 [batch] (out) */
+DD_API dd_status dd_stop_check(const float* entropy, const int32_t* pred, const int32_t* pred_prev,
+                               int batch, int canvas, float threshold, int32_t step, uint8_t* done,
+                               int32_t* halt_step, dd_stream_t stream);
+
+/* Workspace bytes for dd_denoise_block_adaptive. */
+DD_API size_t dd_denoise_block_adaptive_workspace(const dd_attn_desc* desc,
+                                                  const int32_t* cu_prefix_host, int vocab);
+
+/* The block loop under the pages' policy: up to max_steps steps; step s runs
+ * dd_canvas_attn and the sampler (temperature_host[s], Philox step
+ * step0 + s, no scheduled re-noise), then dd_stop_check against step s - 1's
+ * predictions, then dd_entropy_accept into `canvas`.  A canvas that halts at
+ * step s takes its whole prediction as its final canvas and is left
+ * unchanged by later steps; the loop ends when every canvas has halted or
+ * after max_steps.  Unlike every other call here, it synchronises `stream`
+ * once per step to read the halt flags (that is what lets it stop early).
+ * Arguments as dd_denoise_block, plus:
+ *   temperature_host  host fp32 [max_steps] (the pages anneal 0.8 -> 0.4)
+ *   budget, stop_entropy  the pages' b = 0.1 and 0.005
+ *   canvas            int32 [R], in/out (its initial content is only the
+ *                     model's input, which is synthetic here)
+ *   canvas_history    int32 [max_steps, R] or NULL: the canvas after each
+ *                     step run
+ *   halt_step         device int32 [B]: the step each canvas halted at, or -1
+ *   steps_run         host int: steps run */
+DD_API dd_status dd_denoise_block_adaptive(
+    const dd_attn_desc* desc, int max_steps, const void* q_steps, const void* kc_steps,
+    const void* vc_steps, const void* k_prefix, const void* v_prefix, const int32_t* cu_prefix,
+    const int32_t* cu_prefix_host, void* attn_out, const void* logits_steps, int vocab,
+    const float* temperature_host, float budget, float stop_entropy, uint64_t seed,
+    uint32_t step0, int32_t* canvas, int32_t* canvas_history, int32_t* halt_step, int* steps_run,
+    void* workspace, size_t workspace_bytes, dd_stream_t stream);
+
 /* Clears a whole workspace: the error word and the sampler's state (async on
  * stream).  Call once before a workspace's first use. */
 DD_API dd_status dd_workspace_init(void* workspace, size_t workspace_bytes, dd_stream_t stream);

@@ -146,3 +146,44 @@ def test_init_canvas_rejects_bad_arguments(lib):
     assert lib.dd_init_canvas(None, 4, 10, 0, 0, None) == 1
     assert lib.dd_init_canvas(FAKE, 4, 0, 0, 0, None) == 1
     assert lib.dd_init_canvas(None, 0, 10, 0, 0, None) == 0
+
+
+def test_policy_entries_reject_bad_arguments(lib):
+    acc = lib.dd_entropy_accept
+    assert acc(FAKE, FAKE, 2, 2000, 16, 0.1, 0, 0, 0, FAKE, None, None) == 1      # canvas > 1024
+    assert acc(FAKE, FAKE, 2, 0, 16, 0.1, 0, 0, 0, FAKE, None, None) == 1
+    assert acc(FAKE, FAKE, 2, 8, 0, 0.1, 0, 0, 0, FAKE, None, None) == 1          # vocab
+    assert acc(FAKE, FAKE, 2, 8, 16, float("nan"), 0, 0, 0, FAKE, None, None) == 1
+    assert acc(None, FAKE, 2, 8, 16, 0.1, 0, 0, 0, FAKE, None, None) == 1
+    assert acc(FAKE, FAKE, 2, 8, 16, 0.1, 0, 0, 0, None, None, None) == 1
+    assert acc(FAKE, FAKE, 1, 8, 16, 0.1, 0, 0, 0xFFFFFFFC, FAKE, None, None) == 1  # row_offset
+    assert acc(None, None, 0, 8, 16, 0.1, 0, 0, 0, None, None, None) == 0         # empty: no-op
+    stop = lib.dd_stop_check
+    assert stop(FAKE, FAKE, None, 2, 8, 0.005, 0, None, FAKE, None) == 1
+    assert stop(FAKE, FAKE, None, 2, 8, 0.005, 0, FAKE, None, None) == 1
+    assert stop(FAKE, FAKE, None, -1, 8, 0.005, 0, FAKE, FAKE, None) == 1
+    assert stop(None, None, None, 0, 8, 0.005, 0, None, None, None) == 0
+    d = _desc()
+    cu = _cu([16])
+    wa = lib.dd_denoise_block_adaptive_workspace(ctypes.byref(d),
+                                                cu.ctypes.data_as(ctypes.c_void_p), 1024)
+    wb = lib.dd_denoise_block_workspace(ctypes.byref(d), cu.ctypes.data_as(ctypes.c_void_p), 1024)
+    assert wa > wb > 0
+    t = np.full(4, 0.8, np.float32)
+    n = ctypes.c_int(-5)
+    args = [ctypes.byref(d), 4, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+            cu.ctypes.data_as(ctypes.c_void_p), FAKE, FAKE, 1024,
+            t.ctypes.data_as(ctypes.c_void_p), 0.1, 0.005, 0, 0, FAKE, None, FAKE,
+            ctypes.byref(n), FAKE, 16, None]
+    ad = lib.dd_denoise_block_adaptive
+    assert ad(*args) == 3                                         # workspace too small
+    for i, v in [(1, -1), (12, None), (17, None), (19, None), (20, None), (13, float("nan"))]:
+        bad = list(args)
+        bad[i] = v
+        assert ad(*bad) == 1, i
+    big = _desc(C=2048)
+    bad = list(args)
+    bad[0] = ctypes.byref(big)
+    bad[21] = FAKE
+    bad[22] = 1 << 40
+    assert ad(*bad) == 2                                          # canvas > 1024
