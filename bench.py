@@ -18,6 +18,7 @@ previous step's inputs from L2.
 from __future__ import annotations
 
 import argparse
+import ctypes
 import json
 import os
 import statistics
@@ -508,6 +509,94 @@ def run_reference(args, w, dist, rank, world):
             "gpu_launches": 0}
 
 
+def run_policy(w, reps: int = 10, max_steps: int = 12, budget: float = 0.1,
+               stop_entropy: float = 0.005):
+    """The pages' adaptive block (dd_denoise_block_adaptive) on the 12-step
+    geometry (B=1, prefix 8192, V = 262144) with synthetic logits that sharpen
+    step by step (N(0, 1.5^2) plus a spike of 3 + 4 s at one token per row),
+    so the canvas halts early; temperatures annealed 0.8 -> 0.4 over a
+    nominal 48 steps.  Also times dd_entropy_accept alone on 8 canvases."""
+    import block_discrete_diffusion_dd_b200 as dd
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    g = torch.Generator(device=dev).manual_seed(w.seed)
+    R, V = w.rows, w.vocab
+    qs, ks, vs, ls = [], [], [], []
+    hot = torch.randint(0, V, (R,), generator=g, device=dev)
+    for s in range(max_steps):
+        q, kc, vc = workloads.canvas_qkv(w, s, device=dev)
+        lg = torch.randn((R, V), generator=g, device=dev) * 1.5
+        lg[torch.arange(R, device=dev), hot] += 3.0 + 4.0 * s
+        qs.append(q), ks.append(kc), vs.append(vc), ls.append(lg.to(torch.bfloat16))
+        del lg
+    q, kc, vc, lg = torch.stack(qs), torch.stack(ks), torch.stack(vs), torch.stack(ls)
+    del qs, ks, vs, ls
+    kp, vp, cu = workloads.prefix_kv(w, device=dev)
+    cud = cu.to(dev)
+    temps = [float(np.float32(0.8 - 0.4 * s / 47)) for s in range(max_steps)]
+    desc = dd.attn_desc(q[0], kc[0], w.scale)
+    ws = dd.new_workspace(int(dd.load().dd_denoise_block_adaptive_workspace(
+        ctypes.byref(desc), cu.numpy().ctypes.data_as(ctypes.c_void_p), V)), dev)
+    attn_out = torch.empty_like(q)
+
+    def block():
+        canvas = torch.zeros(R, dtype=torch.int32, device=dev)
+        return dd.denoise_block_adaptive(q, kc, vc, kp, vp, cud, lg, temps, budget, stop_entropy,
+                                         w.seed, cu_prefix_host=cu, scale=w.scale,
+                                         attn_out=attn_out, canvas=canvas, keep_history=False,
+                                         workspace=ws)
+
+    for _ in range(2):
+        res = block()
+    torch.cuda.synchronize()
+    wall, dev_ms = [], []
+    for _ in range(reps):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        t0 = time.perf_counter()
+        e0.record()
+        res = block()
+        e1.record()
+        torch.cuda.synchronize()
+        wall.append((time.perf_counter() - t0) * 1e3)
+        dev_ms.append(e0.elapsed_time(e1))
+    n = res["steps_run"]
+    # the acceptance kernel alone, 8 canvases of 256
+    h = torch.rand(8 * 256, device=dev) * 0.01
+    pr = torch.randint(0, V, (8 * 256,), dtype=torch.int32, device=dev)
+    out = {"tokens": torch.empty(8 * 256, dtype=torch.int32, device=dev),
+           "accepted": torch.empty(8 * 256, dtype=torch.uint8, device=dev)}
+    for _ in range(5):
+        dd.entropy_accept(h, pr, 256, budget, 0, 0, V, tokens=out["tokens"],
+                          accepted=out["accepted"])
+    side = torch.cuda.Stream(device=dev)
+    side.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()      # 100 back-to-back calls, no host in the way
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(graph, stream=side):
+            for _ in range(100):
+                dd.entropy_accept(h, pr, 256, budget, 0, 0, V, tokens=out["tokens"],
+                                  accepted=out["accepted"], stream=side)
+    torch.cuda.current_stream().wait_stream(side)
+    graph.replay()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    graph.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    return {"metric": "adaptive block (the pages' policy): ms per block", "unit": "ms",
+            "value": statistics.median(wall), "device_ms": statistics.median(dev_ms),
+            "steps_run": n, "max_steps": max_steps, "ms_per_step": statistics.median(wall) / n,
+            "halt_step": res["halt_step"].cpu().tolist(),
+            "entropy_accept_us_8_canvases": e0.elapsed_time(e1) * 10.0,
+            "config": {"workload": w.name + " geometry, sharpening synthetic logits",
+                       "budget": budget, "stop_entropy": stop_entropy,
+                       "temperature": "0.8 -> 0.4 over 48 nominal steps"},
+            "timing": "median of %d calls; wall clock includes the per-step halt-flag reads" % reps}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -520,6 +609,8 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-sample", type=float, default=0.125)
     ap.add_argument("--ref-sample", type=float, default=1.0 / 32)
+    ap.add_argument("--policy", action="store_true",
+                    help="time the pages' adaptive block loop instead (one JSON line)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     w = workloads.WORKLOADS[args.workload]
@@ -533,6 +624,9 @@ def main():
     from block_discrete_diffusion_dd_b200 import build as libbuild
     if not os.path.exists(libbuild.LIB):
         libbuild.build()
+    if args.policy:
+        print(json.dumps(run_policy(workloads.WORKLOADS["block12_L8192"])), flush=True)
+        return
     dist, rank, world, local_rank = _dist()
     if world != args.gpus and rank == 0:
         print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)

@@ -183,6 +183,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   Barriers* bars = reinterpret_cast<Barriers*>(smem + kOffBar);
+  pdl_wait();
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   volatile int* abort_flag = &bars->abort;
 
@@ -509,6 +511,8 @@ template <typename TOut>
 __global__ void __launch_bounds__(256)
     attn_combine_kernel(const TcParams p, int total_units, TOut* __restrict__ out,
                         float* __restrict__ lse_out) {
+  pdl_wait();
+  pdl_trigger();
   const int nc = cdiv(p.C, BN);
   constexpr int kBlocksPerTile = BM / kCombineRowsPerCta;
   int q = blockIdx.x / kBlocksPerTile;  // (b, g, t) group
@@ -728,14 +732,15 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t stream) {
   tp.part_lse = reinterpret_cast<float*>(scratch + (size_t)pl.slots * BM * HD * sizeof(float));
   tp.err = a.err;
 
-  attn_tc_kernel<<<pl.units, kThreads, kSmemBytes, stream>>>(mQ, mKp, mVp, mKc, mVc, tp);
+  cudaError_t e = launch_pdl(attn_tc_kernel, dim3(pl.units), dim3(kThreads), kSmemBytes, stream,
+                             mQ, mKp, mVp, mKc, mVc, tp);
   note_launch();
-  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  attn_combine_kernel<__nv_bfloat16><<<pl.groups * (BM / kCombineRowsPerCta), 256, 0, stream>>>(
-      tp, pl.slots, static_cast<__nv_bfloat16*>(a.out), a.lse);
+  e = launch_pdl(attn_combine_kernel<__nv_bfloat16>,
+                 dim3(pl.groups * (BM / kCombineRowsPerCta)), dim3(256), 0, stream, tp,
+                 (int)pl.slots, static_cast<__nv_bfloat16*>(a.out), a.lse);
   note_launch();
-  return cudaGetLastError();
+  return e;
 }
 
 }  // namespace dd

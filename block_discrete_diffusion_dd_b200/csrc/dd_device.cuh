@@ -103,6 +103,17 @@ __device__ __forceinline__ float uniform24(uint32_t x) {
   return __uint2float_rn((x >> 9) * 2u + 1u) * 5.9604644775390625e-08f;
 }
 
+// ------------------------------------------- programmatic dependent launch
+// The step's kernels are launched with programmatic stream serialisation:
+// a kernel may be scheduled while the previous one on the stream is still
+// running, and waits here, before its first global memory access, until
+// that grid has completed and its writes are visible.  pdl_trigger lets the
+// next kernel on the stream be scheduled as early.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- bf16 bits
 __device__ __forceinline__ float bf16lo(uint32_t w) {
   uint32_t r;  // bytes (b1 b0 0 0): the low bf16 as the top half of a float

@@ -21,6 +21,9 @@ __device__ __forceinline__ uint32_t ord_u32(float f) {
   const uint32_t b = __float_as_uint(f);
   return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
+__device__ __forceinline__ float unord_u32(uint32_t u) {
+  return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
+}
 
 // Entropy-budget acceptance for canvas blockIdx.x.  Keys (entropy order,
 // then position) are sorted by a bitonic network in shared memory; thread 0
@@ -60,15 +63,14 @@ __global__ void __launch_bounds__(kMaxCanvas)
         __syncthreads();
       }
     }
-    if (i == 0) {
+    if (i == 0) {  // the sorted keys carry the entropies' bits
       double sum = 0.0;
-      const float* h = entropy + (int64_t)b * C;
       for (int k = 0; k < C; ++k) {
-        const int pos = (int)(uint32_t)key[k];
-        const double next = sum + (double)h[pos];
+        const unsigned long long kv = key[k];
+        const double next = sum + (double)unord_u32((uint32_t)(kv >> 32));
         if (!(next <= budget)) break;
         sum = next;
-        acc[pos] = 1;
+        acc[(uint32_t)kv] = 1;
       }
     }
     __syncthreads();
@@ -91,16 +93,18 @@ __global__ void __launch_bounds__(256)
     stop_check_kernel(const float* __restrict__ entropy, const int32_t* __restrict__ pred,
                       const int32_t* __restrict__ pred_prev, int C, double threshold,
                       int32_t cur, uint8_t* __restrict__ done, int32_t* __restrict__ halt_step) {
+  __shared__ float h[kMaxCanvas];
   const int b = blockIdx.x;
   if (done[b]) return;
   bool same = pred_prev != nullptr;
-  if (same)
-    for (int i = threadIdx.x; i < C; i += blockDim.x)
-      same &= pred[(int64_t)b * C + i] == pred_prev[(int64_t)b * C + i];
+  for (int i = threadIdx.x; i < C; i += blockDim.x) {
+    h[i] = entropy[(int64_t)b * C + i];
+    if (pred_prev) same &= pred[(int64_t)b * C + i] == pred_prev[(int64_t)b * C + i];
+  }
   same = __syncthreads_and(same) != 0;
   if (threadIdx.x == 0 && same) {
     double sum = 0.0;
-    for (int i = 0; i < C; ++i) sum += (double)entropy[(int64_t)b * C + i];
+    for (int i = 0; i < C; ++i) sum += (double)h[i];
     if (sum / (double)C < threshold) {
       done[b] = 1;
       halt_step[b] = cur;

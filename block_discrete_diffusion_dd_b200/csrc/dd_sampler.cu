@@ -581,6 +581,8 @@ __global__ void __launch_bounds__(kScanThreads, 3)
     sample_scan_kernel(const T* __restrict__ logits, const __grid_constant__ ScanParams p,
                        float4* __restrict__ recs, unsigned long long* __restrict__ row_key,
                        uint32_t* __restrict__ ticket) {
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   uint32_t g = 0, gn_req = 0;
   if (lane == 0) {
@@ -623,6 +625,8 @@ __global__ void __launch_bounds__(128)
                         int32_t* __restrict__ tokens, int32_t* __restrict__ pred,
                         float* __restrict__ conf, float* __restrict__ entropy,
                         uint8_t* __restrict__ renoised) {
+  pdl_wait();
+  pdl_trigger();
   if (blockIdx.x == 0 && threadIdx.x == 0) *ticket = 0u;
   const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -712,15 +716,16 @@ cudaError_t launch_sampler_v(const SamplerArgs& a, cudaStream_t stream) {
   float4* recs = static_cast<float4*>(a.recs);
   const int64_t want = ((int64_t)p.nchunks + kScanWarpsPerCta - 1) / kScanWarpsPerCta;
   const int ctas = (int)std::min<int64_t>(scan_ctas<T, kVec>(), want);
-  sample_scan_kernel<T, kVec><<<ctas, kScanThreads, 0, stream>>>(lg, p, recs, s.row_key, s.ticket);
+  cudaError_t e = launch_pdl(sample_scan_kernel<T, kVec>, dim3(ctas), dim3(kScanThreads), 0,
+                             stream, lg, p, recs, s.row_key, s.ticket);
   note_launch();
-  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  sample_merge_kernel<T><<<(a.rows + 3) / 4, 128, 0, stream>>>(
-      lg, a.row_stride, a.rows, a.vocab, p.nck, a.inv_tau, a.rate, a.seed, a.step, a.row_offset,
-      recs, s.row_key, s.ticket, a.tokens, a.pred, a.conf, a.entropy, a.renoised);
+  e = launch_pdl(sample_merge_kernel<T>, dim3((a.rows + 3) / 4), dim3(128), 0, stream, lg,
+                 a.row_stride, a.rows, a.vocab, p.nck, a.inv_tau, a.rate, a.seed, a.step,
+                 a.row_offset, (const float4*)recs, s.row_key, s.ticket, a.tokens, a.pred,
+                 a.conf, a.entropy, a.renoised);
   note_launch();
-  return cudaGetLastError();
+  return e;
 }
 
 template <typename T>
