@@ -507,6 +507,28 @@ __global__ void __launch_bounds__(kThreads, 1)
 // 16 CTAs per 128-row tile); lane s holds split s's weight.
 constexpr int kCombineRowsPerCta = 8;
 
+// Final row of the combine: O = acc / wsum (4 columns per lane) and the
+// natural-log LSE.
+template <typename TOut>
+__device__ __forceinline__ void combine_store(const TcParams& p, TOut* __restrict__ out,
+                                              float* __restrict__ lse_out, int b, int g, int pr,
+                                              int lane, float4 acc, float mx, float wsum) {
+  const float inv = 1.f / wsum;
+  const int i = pr / p.group, h = g * p.group + (pr - i * p.group);
+  TOut* orow = out + (((size_t)b * p.C + i) * p.Hq + h) * HD + lane * 4;
+  if constexpr (sizeof(TOut) == 2) {
+    uint2 v;
+    v.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+    v.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+    *reinterpret_cast<uint2*>(orow) = v;
+  } else {
+    *reinterpret_cast<float4*>(orow) =
+        make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+  }
+  if (lse_out && lane == 0)
+    lse_out[((size_t)b * p.Hq + h) * p.C + i] = (mx + __log2f(wsum)) * 0.6931471805599453f;
+}
+
 template <typename TOut>
 __global__ void __launch_bounds__(256)
     attn_combine_kernel(const TcParams p, int total_units, TOut* __restrict__ out,
@@ -541,6 +563,35 @@ __global__ void __launch_bounds__(256)
   const int r = rbase + warp;
   const int pr = t * BM + r;
   if (pr >= p.C * p.group) return;
+  if (nsplit <= 16) {
+    // common case: every split's row and LSE requested at once (one L2
+    // round trip), then the weights and the sum
+    const float lse_l = lane < nsplit ? p.part_lse[(size_t)(u0 + lane) * BM + r] : -INFINITY;
+    float4 o[16];
+#pragma unroll
+    for (int u = 0; u < 16; ++u)
+      o[u] = u < nsplit ? *reinterpret_cast<const float4*>(
+                              p.part_o + ((size_t)(u0 + u) * BM + r) * HD + lane * 4)
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
+    float mx = lse_l;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    const float wl = lane < nsplit ? exp2f(lse_l - mx) : 0.f;
+    float wsum = wl;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, off);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      const float w = __shfl_sync(0xffffffffu, wl, u);  // 0 past nsplit
+      acc.x = fmaf(w, o[u].x, acc.x);
+      acc.y = fmaf(w, o[u].y, acc.y);
+      acc.z = fmaf(w, o[u].z, acc.z);
+      acc.w = fmaf(w, o[u].w, acc.w);
+    }
+    combine_store<TOut>(p, out, lse_out, b, g, pr, lane, acc, mx, wsum);
+    return;
+  }
   // split weights, 32 splits per pass
   float mx = -INFINITY;
   for (int s0 = 0; s0 < nsplit; s0 += 32) {
@@ -559,30 +610,26 @@ __global__ void __launch_bounds__(256)
     for (int off = 16; off > 0; off >>= 1) ws += __shfl_xor_sync(0xffffffffu, ws, off);
     wsum += ws;
     const int n = min(32, nsplit - s0);
-    for (int j = 0; j < n; ++j) {
-      const float w = __shfl_sync(0xffffffffu, wl, j);
-      const float4 o = *reinterpret_cast<const float4*>(
-          p.part_o + ((size_t)(u0 + s0 + j) * BM + r) * HD + lane * 4);
-      acc.x = fmaf(w, o.x, acc.x);
-      acc.y = fmaf(w, o.y, acc.y);
-      acc.z = fmaf(w, o.z, acc.z);
-      acc.w = fmaf(w, o.w, acc.w);
+    // eight splits' rows in flight at a time (L2 latency, not bandwidth, is
+    // what a one-row-at-a-time loop waits on)
+    for (int j0 = 0; j0 < n; j0 += 8) {
+      float4 o[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        o[u] = j0 + u < n ? *reinterpret_cast<const float4*>(
+                                p.part_o + ((size_t)(u0 + s0 + j0 + u) * BM + r) * HD + lane * 4)
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const float w = __shfl_sync(0xffffffffu, wl, j0 + u);  // 0 past nsplit
+        acc.x = fmaf(w, o[u].x, acc.x);
+        acc.y = fmaf(w, o[u].y, acc.y);
+        acc.z = fmaf(w, o[u].z, acc.z);
+        acc.w = fmaf(w, o[u].w, acc.w);
+      }
     }
   }
-  const float inv = 1.f / wsum;
-  const int i = pr / p.group, h = g * p.group + (pr - i * p.group);
-  TOut* orow = out + (((size_t)b * p.C + i) * p.Hq + h) * HD + lane * 4;
-  if constexpr (sizeof(TOut) == 2) {
-    uint2 v;
-    v.x = pack_bf16x2(acc.x * inv, acc.y * inv);
-    v.y = pack_bf16x2(acc.z * inv, acc.w * inv);
-    *reinterpret_cast<uint2*>(orow) = v;
-  } else {
-    *reinterpret_cast<float4*>(orow) =
-        make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-  }
-  if (lse_out && lane == 0)
-    lse_out[((size_t)b * p.Hq + h) * p.C + i] = (mx + __log2f(wsum)) * 0.6931471805599453f;
+  combine_store<TOut>(p, out, lse_out, b, g, pr, lane, acc, mx, wsum);
 }
 
 // ----------------------------------------------------------------- host
