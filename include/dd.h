@@ -202,9 +202,9 @@ DD_API dd_status dd_denoise_block(const dd_attn_desc* desc, int steps, const voi
  * Arguments and results: exactly as dd_sample_renoise, minus the workspace.
  * Scratch: a static device array of 4 MiB that the library holds on every
  * GPU it is loaded on until the process exits.  A call needs
- * dd_sample_renoise_workspace(rows, vocab, dtype) bytes of it (about 8 bytes
- * per row plus 16 bytes per 2048 vocabulary entries per row, so up to 2039
- * rows at V = 262144); larger calls return
+ * dd_sample_renoise_workspace(rows, vocab, dtype) bytes of it (about 512
+ * bytes, plus 128 bytes per row, plus 16 bytes per 2048 vocabulary entries
+ * per row: up to 1927 rows at V = 262144); larger calls return
  * DD_ERR_UNSUPPORTED before touching the GPU.  The function allocates
  * nothing: no cudaMalloc, cudaFree or allocating library call.
  * The first call on a device looks up the array's device address
