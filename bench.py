@@ -102,11 +102,15 @@ class ClockSampler:
 
 
 def _dist():
+    """One process per GPU (NCCL; gloo when no GPU is visible, which the CPU
+    tests of the multi-rank plumbing use).  Replicas only: the process group
+    carries the barrier and the max-over-ranks timing, no data."""
     n = int(os.environ.get("WORLD_SIZE", "1"))
     if n > 1:
         import datetime
         import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
         return dist, dist.get_rank(), n, int(os.environ.get("LOCAL_RANK", "0"))
     return None, 0, 1, 0
 
@@ -114,7 +118,8 @@ def _dist():
 def _max_over_ranks(dist, x: float) -> float:
     if dist is None:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -122,7 +127,8 @@ def _max_over_ranks(dist, x: float) -> float:
 def _barrier(dist):
     if dist is not None:
         dist.barrier()
-    torch.cuda.synchronize()
+    if torch.cuda.is_available():
+        torch.cuda.synchronize()
 
 
 def make_inputs(w, rank: int, dev):
