@@ -20,6 +20,11 @@ Parity status per function (what pins it; tests/test_oracle_*.py):
   canvas_attn               -- float64 torch SDPA, pure-Python brute force,
                                closed forms, permutation/zero-prefix/GQA
                                invariants.
+  e4m3_value / E4M3 inputs  -- closed-form codes of the OCP E4M3 encoding,
+                               torch's float8_e4m3fn decoding of all 256
+                               codes; E4M3 attention with power-of-two
+                               per-tensor factors equals the float32 path on
+                               the exactly scaled values.
   sample_renoise            -- chi-square of Gumbel-max vs softmax, scipy
                                log-softmax/entropy, spike and constant-logit
                                closed forms, binomial re-noise rate,
@@ -43,6 +48,7 @@ _LIB = os.path.join(_HERE, "liboracle.so")
 
 BF16 = 0
 F32 = 1
+E4M3 = 2
 
 _lib = None
 
@@ -75,8 +81,10 @@ def _load():
     lib.oracle_philox_blocks.restype = None
     lib.oracle_philox_blocks.argtypes = [P, P, i64, P]
     lib.oracle_canvas_attn.restype = i32
-    lib.oracle_canvas_attn.argtypes = [i32, i32, i32, i32, i32, f64, i32, P, P, P, P, P, P, P, i32,
-                                       P, P, i32]
+    lib.oracle_canvas_attn.argtypes = [i32, i32, i32, i32, i32, f64, i32, P, P, P, P, P, P, P, P,
+                                       i32, P, P, i32]
+    lib.oracle_e4m3_value.restype = f64
+    lib.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
     lib.oracle_sample_renoise.restype = i32
     lib.oracle_sample_renoise.argtypes = [P, i32, i64, i64, i64, P, i64, f64, f32, u64, u32, u32,
                                           P, P, P, P, P, P, P, i32]
@@ -97,8 +105,8 @@ def _ptr(a):
 def _raw(x):
     """(numpy array, dtype code) from a torch tensor or numpy array.
 
-    bf16 tensors are passed as their raw 16-bit patterns; the C side upcasts
-    them exactly.  Anything else must already be float32.
+    bf16 and E4M3 tensors are passed as their raw 16- and 8-bit patterns; the
+    C side decodes them exactly.  Anything else must already be float32.
     """
     try:
         import torch
@@ -106,6 +114,8 @@ def _raw(x):
             x = x.detach().cpu().contiguous()
             if x.dtype == torch.bfloat16:
                 return np.ascontiguousarray(x.view(torch.int16).numpy().view(np.uint16)), BF16
+            if x.dtype == torch.float8_e4m3fn:
+                return np.ascontiguousarray(x.view(torch.uint8).numpy()), E4M3
             if x.dtype == torch.float32:
                 return np.ascontiguousarray(x.numpy()), F32
             raise TypeError(f"oracle: unsupported tensor dtype {x.dtype}")
@@ -149,12 +159,20 @@ def uniform(x: int) -> float:
 
 # ------------------------------------------------------- canvas attention
 
-def canvas_attn(q, kc, vc, kp, vp, cu_prefix, scale=None, positions=None, threads=0):
+def e4m3_value(code: int) -> float:
+    """The value of one E4M3 byte (OCP OFP8 E4M3 encoding)."""
+    return _load().oracle_e4m3_value(int(code) & 0xFF)
+
+
+def canvas_attn(q, kc, vc, kp, vp, cu_prefix, scale=None, positions=None, threads=0,
+                qkv_scale=None):
     """float64 attention over [prefix_b || canvas_b] for every (b, i, h).
 
     Shapes: q [B,C,Hq,D]; kc, vc [B,C,Hkv,D]; kp, vp [sum L_b, Hkv, D];
     cu_prefix [B+1] int.  positions: optional list of canvas positions to
-    compute (others are NaN).  Returns (out [B,C,Hq,D], lse [B,Hq,C]).
+    compute (others are NaN).  qkv_scale: optional per-tensor factors
+    (q, k, v) multiplying the stored values (8-bit inputs with per-tensor
+    scales).  Returns (out [B,C,Hq,D], lse [B,Hq,C]).
     """
     lib = _load()
     qa, dt = _raw(q)
@@ -176,7 +194,10 @@ def canvas_attn(q, kc, vc, kp, vp, cu_prefix, scale=None, positions=None, thread
     else:
         pos = np.ascontiguousarray(np.asarray(positions, dtype=np.int32))
         npos = pos.size
-    rc = lib.oracle_canvas_attn(B, C, Hq, Hkv, D, float(scale), dt, _ptr(qa), _ptr(kca),
+    sc = None if qkv_scale is None else np.ascontiguousarray(np.asarray(qkv_scale, np.float64))
+    if sc is not None and sc.shape != (3,):
+        raise ValueError("oracle: qkv_scale must hold three factors")
+    rc = lib.oracle_canvas_attn(B, C, Hq, Hkv, D, float(scale), dt, _ptr(sc), _ptr(qa), _ptr(kca),
                                 _ptr(vca), _ptr(kpa), _ptr(vpa), _ptr(cu), _ptr(pos), npos,
                                 _ptr(out), _ptr(lse), int(threads))
     if rc != 0:

@@ -55,6 +55,7 @@
 
 #define ORACLE_BF16 0
 #define ORACLE_F32 1
+#define ORACLE_E4M3 2
 
 /* ---------------------------------------------------------------- Philox */
 
@@ -114,7 +115,26 @@ void oracle_philox_blocks(const uint32_t* ctrs, const uint32_t* keys, int64_t n,
 
 /* ------------------------------------------------------------ input upcast */
 
-/* bf16 -> float64 is exact: the bf16 bits are the top half of a float32. */
+/*
+ * The 8-bit E4M3 floating-point format (OCP "8-bit Floating Point
+ * Specification (OFP8)", rev. 1.0, the E4M3 encoding): one sign bit, four
+ * exponent bits with bias 7, three mantissa bits.  An exponent field of 0
+ * encodes the subnormals m * 2^-9; S.1111.111 is NaN; there are no
+ * infinities, so the largest finite magnitude is 1.75 * 2^8 = 448.
+ */
+double oracle_e4m3_value(uint8_t x) {
+  const int sign = x >> 7, e = (x >> 3) & 15, m = x & 7;
+  double v;
+  if (e == 15 && m == 7) return NAN;
+  if (e == 0)
+    v = ldexp((double)m, -9);
+  else
+    v = ldexp(1.0 + (double)m / 8.0, e - 7);
+  return sign ? -v : v;
+}
+
+/* bf16 -> float64 is exact: the bf16 bits are the top half of a float32.
+ * E4M3 -> float64 is exact too (four significant bits). */
 static double load_elem(const void* base, int dtype, int64_t idx) {
   if (dtype == ORACLE_BF16) {
     const uint16_t h = ((const uint16_t*)base)[idx];
@@ -123,6 +143,7 @@ static double load_elem(const void* base, int dtype, int64_t idx) {
     memcpy(&f, &bits, 4);
     return (double)f;
   }
+  if (dtype == ORACLE_E4M3) return oracle_e4m3_value(((const uint8_t*)base)[idx]);
   return (double)((const float*)base)[idx];
 }
 
@@ -147,9 +168,13 @@ static void set_threads(int n_threads) {
  * with cu_prefix[B+1]; out [B,C,Hq,D]; lse [B,Hq,C] (may be NULL).
  * pos_sel (n_pos entries) restricts the canvas positions computed; rows not
  * selected are left untouched.  n_pos < 0 means every position.
+ * qkv_scale (NULL = all 1) holds per-tensor factors (q, k, v): the value of
+ * an element is its stored value times its tensor's factor (the per-tensor
+ * scaling of 8-bit inputs); K's factor covers Kp and Kc, V's Vp and Vc.
  * Returns 0, or -1 on bad arguments.
  */
 int oracle_canvas_attn(int B, int C, int Hq, int Hkv, int D, double scale, int dtype,
+                       const double* qkv_scale,
                        const void* q, const void* kc, const void* vc, const void* kp,
                        const void* vp, const int32_t* cu_prefix, const int32_t* pos_sel,
                        int n_pos, double* out, double* lse, int n_threads) {
@@ -157,6 +182,9 @@ int oracle_canvas_attn(int B, int C, int Hq, int Hkv, int D, double scale, int d
   for (int b = 0; b < B; ++b)
     if (cu_prefix[b + 1] < cu_prefix[b] || cu_prefix[0] != 0) return -1;
   const int group = Hq / Hkv;
+  const double sq = qkv_scale ? qkv_scale[0] : 1.0;
+  const double sk = qkv_scale ? qkv_scale[1] : 1.0;
+  const double sv = qkv_scale ? qkv_scale[2] : 1.0;
   const int npos = n_pos < 0 ? C : n_pos;
   const int64_t n_rows = (int64_t)B * npos * Hq;
   set_threads(n_threads);
@@ -183,7 +211,7 @@ int oracle_canvas_attn(int B, int C, int Hq, int Hkv, int D, double scale, int d
       const int nk = L + C;
 
       for (int d = 0; d < D; ++d)
-        qv[d] = load_elem(q, dtype, (((int64_t)b * C + i) * Hq + h) * D + d);
+        qv[d] = sq * load_elem(q, dtype, (((int64_t)b * C + i) * Hq + h) * D + d);
 
       /* scores over [prefix || canvas] */
       for (int j = 0; j < nk; ++j) {
@@ -192,7 +220,8 @@ int oracle_canvas_attn(int B, int C, int Hq, int Hkv, int D, double scale, int d
         if (j < L) { kb = kp; krow = (int64_t)cu_prefix[b] + j; }
         else       { kb = kc; krow = (int64_t)b * C + (j - L); }
         double dot = 0.0;
-        for (int d = 0; d < D; ++d) dot += qv[d] * load_elem(kb, dtype, (krow * Hkv + g) * D + d);
+        for (int d = 0; d < D; ++d)
+          dot += qv[d] * (sk * load_elem(kb, dtype, (krow * Hkv + g) * D + d));
         s[j] = scale * dot;
       }
       double m = -INFINITY;
@@ -207,7 +236,8 @@ int oracle_canvas_attn(int B, int C, int Hq, int Hkv, int D, double scale, int d
         int64_t vrow;
         if (j < L) { vb = vp; vrow = (int64_t)cu_prefix[b] + j; }
         else       { vb = vc; vrow = (int64_t)b * C + (j - L); }
-        for (int d = 0; d < D; ++d) acc[d] += p * load_elem(vb, dtype, (vrow * Hkv + g) * D + d);
+        for (int d = 0; d < D; ++d)
+          acc[d] += p * (sv * load_elem(vb, dtype, (vrow * Hkv + g) * D + d));
       }
       double* o = out + (((int64_t)b * C + i) * Hq + h) * D;
       for (int d = 0; d < D; ++d) o[d] = acc[d];

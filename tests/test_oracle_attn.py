@@ -164,3 +164,75 @@ def test_position_subset_matches_full(oracle_mod):
     np.testing.assert_array_equal(out_s[:, pos], out[:, pos])
     np.testing.assert_array_equal(lse_s[:, :, pos], lse[:, :, pos])
     assert np.isnan(out_s[:, 1]).all()
+
+
+# ------------------------------------------------------------ 8-bit inputs
+# E4M3 bytes (OCP "8-bit Floating Point Specification (OFP8)", E4M3 encoding:
+# bias 7, three mantissa bits, subnormals m * 2^-9, S.1111.111 = NaN, no
+# infinities) with one scale factor per tensor.
+
+@pytest.mark.parametrize("code,value", [
+    (0x00, 0.0), (0x01, 2.0 ** -9), (0x07, 7 * 2.0 ** -9), (0x08, 2.0 ** -6),
+    (0x38, 1.0), (0x3C, 1.5), (0x3F, 1.875), (0x40, 2.0), (0x7E, 448.0),
+    (0xB8, -1.0), (0xFE, -448.0), (0x81, -(2.0 ** -9)),
+])
+def test_e4m3_closed_forms(oracle_mod, code, value):
+    assert oracle_mod.e4m3_value(code) == value
+
+
+def test_e4m3_nan_codes_and_negative_zero(oracle_mod):
+    assert math.isnan(oracle_mod.e4m3_value(0x7F)) and math.isnan(oracle_mod.e4m3_value(0xFF))
+    z = oracle_mod.e4m3_value(0x80)
+    assert z == 0.0 and math.copysign(1.0, z) < 0
+
+
+def test_e4m3_all_codes_match_torch(oracle_mod):
+    """Every code against torch's float8_e4m3fn decoding (a library routine)."""
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = np.array([oracle_mod.e4m3_value(c) for c in range(256)])
+    np.testing.assert_array_equal(np.isnan(got), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    np.testing.assert_array_equal(got[ok], ref[ok])
+
+
+def _e4m3_problem(B, C, Hq, Hkv, D, lens, seed, gains=(40.0, 50.0, 30.0)):
+    g = torch.Generator().manual_seed(seed)
+
+    def r(*shape, gain):
+        return (torch.randn(shape, generator=g) * gain).clamp(-448, 448).to(torch.float8_e4m3fn)
+
+    n = int(sum(lens))
+    q = r(B, C, Hq, D, gain=gains[0])
+    kc, vc = r(B, C, Hkv, D, gain=gains[1]), r(B, C, Hkv, D, gain=gains[2])
+    kp, vp = r(n, Hkv, D, gain=gains[1]), r(n, Hkv, D, gain=gains[2])
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    return q, kc, vc, kp, vp, cu
+
+
+@pytest.mark.parametrize("B,C,Hq,Hkv,D,lens", [(2, 24, 4, 2, 32, (0, 45)),
+                                               (1, 40, 8, 2, 16, (70,))])
+def test_e4m3_scaled_matches_float64_sdpa(oracle_mod, B, C, Hq, Hkv, D, lens):
+    """E4M3 inputs with distinct per-tensor factors against float64 SDPA on
+    the decoded, scaled values (decoded by torch)."""
+    q, kc, vc, kp, vp, cu = _e4m3_problem(B, C, Hq, Hkv, D, lens, seed=B + D)
+    sq, sk, sv = 2.0 ** -5, 0.75 * 2.0 ** -6, 3.0 * 2.0 ** -7
+    scale = 1.0 / math.sqrt(D)
+    out, lse = oracle_mod.canvas_attn(q, kc, vc, kp, vp, cu, scale, qkv_scale=(sq, sk, sv))
+    dec = [t.to(torch.float64) * f for t, f in ((q, sq), (kc, sk), (vc, sv), (kp, sk), (vp, sv))]
+    ref, ref_lse = _sdpa(*dec, cu, scale)
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, ref_lse, rtol=0, atol=1e-12)
+
+
+def test_e4m3_power_of_two_factors_equal_float32_path(oracle_mod):
+    """Power-of-two factors scale exactly: the E4M3 path must equal the
+    float32 path on the scaled values bit for bit."""
+    q, kc, vc, kp, vp, cu = _e4m3_problem(2, 16, 4, 1, 8, (9, 20), seed=11)
+    f = (2.0 ** -4, 2.0 ** -7, 2.0 ** -3)
+    out, lse = oracle_mod.canvas_attn(q, kc, vc, kp, vp, cu, 0.3, qkv_scale=f)
+    ts = [t.to(torch.float32) * s for t, s in ((q, f[0]), (kc, f[1]), (vc, f[2]), (kp, f[1]),
+                                               (vp, f[2]))]
+    out32, lse32 = oracle_mod.canvas_attn(*ts, cu, 0.3)
+    np.testing.assert_array_equal(out, out32)
+    np.testing.assert_array_equal(lse, lse32)
