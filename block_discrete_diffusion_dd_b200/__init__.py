@@ -20,7 +20,7 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libdd.so")
 
-DD_BF16, DD_F32 = 0, 1
+DD_BF16, DD_F32, DD_E4M3 = 0, 1, 2
 STATUS = {0: "DD_OK", 1: "DD_ERR_INVALID_ARG", 2: "DD_ERR_UNSUPPORTED", 3: "DD_ERR_WORKSPACE",
           4: "DD_ERR_CUDA", 5: "DD_ERR_DEVICE_TIMEOUT", 6: "DD_ERR_DEVICE_BOUNDS"}
 
@@ -31,7 +31,7 @@ EXPORTS = (
     "dd_workspace_init", "dd_query_device_error", "dd_status_string", "dd_last_error",
     "dd_launch_count", "dd_reset_launch_count", "dd_sample_renoise_noalloc",
     "dd_entropy_accept", "dd_stop_check", "dd_denoise_block_adaptive_workspace",
-    "dd_denoise_block_adaptive",
+    "dd_denoise_block_adaptive", "dd_canvas_attn_fp8",
 )
 
 
@@ -45,6 +45,10 @@ class AttnDesc(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int), ("canvas", ctypes.c_int), ("heads_q", ctypes.c_int),
                 ("heads_kv", ctypes.c_int), ("head_dim", ctypes.c_int), ("scale", ctypes.c_float),
                 ("dtype", ctypes.c_int)]
+
+
+class Fp8Scales(ctypes.Structure):
+    _fields_ = [("q", ctypes.c_float), ("k", ctypes.c_float), ("v", ctypes.c_float)]
 
 
 class SampleParams(ctypes.Structure):
@@ -72,6 +76,9 @@ def load() -> ctypes.CDLL:
     lib.dd_canvas_attn_workspace.argtypes = [D, P]
     lib.dd_canvas_attn.restype = i32
     lib.dd_canvas_attn.argtypes = [D, P, P, P, P, P, P, P, P, P, P, sz, P]
+    lib.dd_canvas_attn_fp8.restype = i32
+    lib.dd_canvas_attn_fp8.argtypes = [D, P, P, P, P, P, P, P, ctypes.POINTER(Fp8Scales), P, P, P,
+                                       sz, P]
     lib.dd_sample_renoise_workspace.restype = sz
     lib.dd_sample_renoise_workspace.argtypes = [i32, i32, i32]
     lib.dd_sample_renoise.restype = i32
@@ -133,7 +140,9 @@ def _dtype_code(t: torch.Tensor) -> int:
         return DD_BF16
     if t.dtype == torch.float32:
         return DD_F32
-    raise TypeError(f"unsupported dtype {t.dtype} (bf16 or fp32)")
+    if t.dtype == torch.float8_e4m3fn:
+        return DD_E4M3
+    raise TypeError(f"unsupported dtype {t.dtype} (bf16, fp32 or float8_e4m3fn)")
 
 
 def _host_i32(x) -> np.ndarray:
@@ -181,6 +190,29 @@ def canvas_attn(q, kc, vc, kp, vp, cu_prefix, cu_prefix_host=None, scale=None, o
     _check(lib.dd_canvas_attn(ctypes.byref(desc), _ptr(q), _ptr(kc), _ptr(vc), _ptr(kp), _ptr(vp),
                               _ptr(cu_prefix), cu_h.ctypes.data_as(ctypes.c_void_p), _ptr(out),
                               _ptr(lse), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return out, lse
+
+
+def canvas_attn_fp8(q, kc, vc, kp, vp, cu_prefix, scales, cu_prefix_host=None, scale=None,
+                    out=None, lse=None, want_lse=False, workspace=None, stream=None):
+    """dd_canvas_attn_fp8: float8_e4m3fn q [B,C,Hq,D], kc/vc [B,C,Hkv,D],
+    kp/vp [sumL,Hkv,D]; scales = (f_q, f_k, f_v) per-tensor factors.
+    Returns (out bf16 [B,C,Hq,D], lse or None)."""
+    lib = load()
+    desc = attn_desc(q, kc, scale)
+    cu_h = _host_i32(cu_prefix if cu_prefix_host is None else cu_prefix_host)
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
+    if want_lse and lse is None:
+        lse = torch.empty((desc.batch, desc.heads_q, desc.canvas), dtype=torch.float32,
+                          device=q.device)
+    if workspace is None:
+        workspace = new_workspace(canvas_attn_workspace_bytes(desc, cu_h), q.device, stream)
+    f = Fp8Scales(*(float(x) for x in scales))
+    _check(lib.dd_canvas_attn_fp8(ctypes.byref(desc), _ptr(q), _ptr(kc), _ptr(vc), _ptr(kp),
+                                  _ptr(vp), _ptr(cu_prefix), cu_h.ctypes.data_as(ctypes.c_void_p),
+                                  ctypes.byref(f), _ptr(out), _ptr(lse), _ptr(workspace),
+                                  workspace.numel(), _stream(stream)))
     return out, lse
 
 

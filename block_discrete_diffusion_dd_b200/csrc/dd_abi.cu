@@ -38,10 +38,12 @@ dd_status cuda_fail(cudaError_t e, const char* what) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-size_t elem_size(dd_dtype t) { return t == DD_BF16 ? 2 : 4; }
+size_t elem_size(dd_dtype t) { return t == DD_BF16 ? 2 : t == DD_E4M3 ? 1 : 4; }
 
 // Validates the geometry and the host prefix offsets; fills total prefix.
-dd_status check_attn_desc(const dd_attn_desc* d, const int32_t* cu_host, int64_t* total) {
+// DD_E4M3 is accepted only where the caller can take it (allow_e4m3).
+dd_status check_attn_desc(const dd_attn_desc* d, const int32_t* cu_host, int64_t* total,
+                          bool allow_e4m3 = false) {
   if (!d) return fail(DD_ERR_INVALID_ARG, "desc is NULL");
   if (d->batch < 0 || d->canvas < 1 || d->heads_q < 1 || d->heads_kv < 1)
     return fail(DD_ERR_INVALID_ARG, "bad geometry B=%d C=%d Hq=%d Hkv=%d", d->batch, d->canvas,
@@ -49,7 +51,10 @@ dd_status check_attn_desc(const dd_attn_desc* d, const int32_t* cu_host, int64_t
   if (d->heads_q % d->heads_kv != 0)
     return fail(DD_ERR_INVALID_ARG, "heads_q (%d) is not a multiple of heads_kv (%d)",
                 d->heads_q, d->heads_kv);
-  if (d->dtype != DD_BF16 && d->dtype != DD_F32)
+  if (d->dtype == DD_E4M3 && !allow_e4m3)
+    return fail(DD_ERR_INVALID_ARG,
+                "DD_E4M3 inputs need per-tensor factors: use dd_canvas_attn_fp8");
+  if (d->dtype != DD_BF16 && d->dtype != DD_F32 && d->dtype != DD_E4M3)
     return fail(DD_ERR_INVALID_ARG, "unknown dtype %d", (int)d->dtype);
   if (d->head_dim != 64 && d->head_dim != 128)
     return fail(DD_ERR_UNSUPPORTED, "head_dim %d (supported: 64, 128)", d->head_dim);
@@ -80,6 +85,8 @@ AttnArgs make_attn_args(const dd_attn_desc* d, int64_t total, const int32_t* cu_
   a.D = d->head_dim;
   a.scale = d->scale;
   a.bf16 = d->dtype == DD_BF16;
+  a.e4m3 = d->dtype == DD_E4M3;
+  a.q_scale = a.k_scale = a.v_scale = 1.0f;
   a.total_prefix = total;
   return a;
 }
@@ -119,11 +126,13 @@ size_t block_ws_layout(const dd_attn_desc* desc, int64_t total, const int32_t* c
   return cf + align256((size_t)rows * sizeof(float));
 }
 
+// `f8` (NULL unless d->dtype is DD_E4M3): the per-tensor factors.
 dd_status run_attn(const dd_attn_desc* d, const void* q, const void* kc, const void* vc,
                    const void* kp, const void* vp, const int32_t* cu, const int32_t* cu_host,
-                   void* out, float* lse, void* ws, size_t ws_bytes, cudaStream_t stream) {
+                   void* out, float* lse, void* ws, size_t ws_bytes, cudaStream_t stream,
+                   const dd_fp8_scales* f8 = nullptr) {
   int64_t total = 0;
-  dd_status st = check_attn_desc(d, cu_host, &total);
+  dd_status st = check_attn_desc(d, cu_host, &total, f8 != nullptr);
   if (st != DD_OK) return st;
   if (d->batch == 0) return DD_OK;
   if (!q || !kc || !vc || !out || !cu) return fail(DD_ERR_INVALID_ARG, "NULL tensor pointer");
@@ -134,6 +143,11 @@ dd_status run_attn(const dd_attn_desc* d, const void* q, const void* kc, const v
   if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u))
     return fail(DD_ERR_WORKSPACE, "workspace must be non-NULL and 256-byte aligned");
   AttnArgs a = make_attn_args(d, total, cu_host);
+  if (a.e4m3) {
+    a.q_scale = f8->q;
+    a.k_scale = f8->k;
+    a.v_scale = f8->v;
+  }
   a.q = q;
   a.kc = kc;
   a.vc = vc;
@@ -146,6 +160,9 @@ dd_status run_attn(const dd_attn_desc* d, const void* q, const void* kc, const v
   a.err = static_cast<uint32_t*>(ws);
   a.scratch = static_cast<uint8_t*>(ws) + kHeaderBytes;
   const bool tc = attn_tc_supported(a);
+  if (a.e4m3 && !tc)
+    return fail(DD_ERR_UNSUPPORTED,
+                "E4M3 attention needs head_dim 128 and (heads_q / heads_kv) dividing 128");
   const size_t need = kHeaderBytes + (tc ? attn_tc_scratch_bytes(a) : attn_simt_scratch_bytes(a));
   if (ws_bytes < need)
     return fail(DD_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", ws_bytes, need);
@@ -237,7 +254,7 @@ extern "C" {
 
 size_t dd_canvas_attn_workspace(const dd_attn_desc* desc, const int32_t* cu_prefix_host) {
   int64_t total = 0;
-  if (check_attn_desc(desc, cu_prefix_host, &total) != DD_OK) return 0;
+  if (check_attn_desc(desc, cu_prefix_host, &total, true) != DD_OK) return 0;
   return attn_ws_bytes(make_attn_args(desc, total, cu_prefix_host));
 }
 
@@ -248,6 +265,28 @@ dd_status dd_canvas_attn(const dd_attn_desc* desc, const void* q, const void* k_
   g_last_error.clear();
   return run_attn(desc, q, k_canvas, v_canvas, k_prefix, v_prefix, cu_prefix, cu_prefix_host, out,
                   lse, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+dd_status dd_canvas_attn_fp8(const dd_attn_desc* desc, const void* q, const void* k_canvas,
+                             const void* v_canvas, const void* k_prefix, const void* v_prefix,
+                             const int32_t* cu_prefix, const int32_t* cu_prefix_host,
+                             const dd_fp8_scales* scales, void* out, float* lse, void* workspace,
+                             size_t workspace_bytes, dd_stream_t stream) {
+  g_last_error.clear();
+  if (!desc) return fail(DD_ERR_INVALID_ARG, "desc is NULL");
+  if (desc->dtype != DD_E4M3)
+    return fail(DD_ERR_INVALID_ARG, "dd_canvas_attn_fp8 takes DD_E4M3 inputs");
+  if (!scales) return fail(DD_ERR_INVALID_ARG, "scales is NULL");
+  if (!(std::isfinite(scales->q) && scales->q > 0.f && std::isfinite(scales->k) &&
+        scales->k > 0.f && std::isfinite(scales->v) && scales->v > 0.f))
+    return fail(DD_ERR_INVALID_ARG, "scale factors must be finite and > 0");
+  if (!std::isfinite((double)desc->scale * 1.4426950408889634 * (double)scales->q *
+                     (double)scales->k) ||
+      (double)desc->scale * 1.4426950408889634 * (double)scales->q * (double)scales->k >
+          3.0e38)
+    return fail(DD_ERR_INVALID_ARG, "scale * q factor * k factor overflows float32");
+  return run_attn(desc, q, k_canvas, v_canvas, k_prefix, v_prefix, cu_prefix, cu_prefix_host, out,
+                  lse, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream), scales);
 }
 
 size_t dd_sample_renoise_workspace(int rows, int vocab, dd_dtype dtype) {

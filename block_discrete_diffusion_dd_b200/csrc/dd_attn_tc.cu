@@ -51,23 +51,15 @@ constexpr int BM = 128;  // query rows per tile
 constexpr int BN = 128;  // keys per tile
 constexpr int HD = 128;  // head dim
 constexpr int kQT = 2;   // query tiles per CTA
-constexpr int kStages = 2;
+constexpr int kMaxStages = 4;
 constexpr int kSoftmaxWarps = 8 * kQT;  // two warps per 32 query rows
 constexpr int kWarpTMA = kSoftmaxWarps, kWarpMMA = kSoftmaxWarps + 1;
 constexpr int kThreads = (kSoftmaxWarps + 2) * 32;
-constexpr uint32_t kHalf = 128 * 64 * 2;  // 128 rows x 128 bytes
-constexpr uint32_t kTile = 2 * kHalf;     // 128 x 128 bf16
-constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffK = kOffQ + kQT * kTile;
-constexpr uint32_t kOffV = kOffK + kStages * kTile;
-constexpr uint32_t kOffX = kOffV + kStages * kTile;  // row-max exchange [q][slot][half][row]
-constexpr uint32_t kOffBar = kOffX + kQT * 2 * 2 * BM * 4;
+constexpr uint32_t kHalf = 128 * 64 * 2;  // bf16: 128 rows x 64 elements (128 bytes)
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemO = kQT * BN;     // O columns start after the S/P regions
 constexpr int kStageStride = HD + 4;       // padded fp32 row of the O staging area
-static_assert(kQT * BM * kStageStride * 4 <= kOffX, "O staging fits the operand buffers");
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per wait
-constexpr float kLazyRescale = 8.0f;              // log2 units
 #ifndef DD_POLY_PAIRS
 #define DD_POLY_PAIRS 0
 #endif
@@ -77,7 +69,7 @@ constexpr int kPolyPairs = DD_POLY_PAIRS;
 
 struct Barriers {
   uint64_t q_full;
-  uint64_t k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
+  uint64_t k_full[kMaxStages], k_empty[kMaxStages], v_full[kMaxStages], v_empty[kMaxStages];
   uint64_t s_full[kQT], p_full[kQT], o_done[kQT];
   uint64_t xch[kQT][4];  // per (query tile, 32-row group): the two column halves meet
   uint64_t staged[kQT];  // per query tile: all 8 warps have staged their O rows
@@ -87,12 +79,38 @@ struct Barriers {
   int unit_b, unit_g, unit_tp, unit_s, unit_valid, unit_nsplit, unit_slot0;
 };
 
-constexpr uint32_t kSmemBytes = kOffBar + sizeof(Barriers) + 1024;
-static_assert(kSmemBytes <= 232448, "shared memory budget");
+// Operand layout per input type.  A query or key row of HD elements is one
+// 128-byte swizzle atom wide for E4M3 and two (the halves d < 64, d >= 64,
+// kHalf apart) for bf16.  The E4M3 tiles are half the size, so they get a
+// deeper K/V ring, which also leaves room for the O staging area.
+//
+// P = 2^(x - m_ref) with x the log2-domain score.  O is rescaled only when
+// the row max exceeds m_ref + kLazy + kBias, and m_ref is set kBias below
+// the row max, so every P lies in (0, 2^8].  For E4M3 P (largest finite
+// value 448) the bias keeps P in the normal range down to 2^-12 of the row
+// maximum (E4M3 subnormals start at 2^-6).
+template <bool kF8>
+struct Lay {
+  static constexpr uint32_t kRow = kF8 ? HD : 2 * HD;  // bytes per row
+  static constexpr uint32_t kTile = BM * kRow;
+  static constexpr int kStages = kF8 ? 4 : 2;
+  static constexpr uint32_t kOffQ = 0;
+  static constexpr uint32_t kOffK = kOffQ + kQT * kTile;
+  static constexpr uint32_t kOffV = kOffK + kStages * kTile;
+  static constexpr uint32_t kOffX = kOffV + kStages * kTile;  // row-max exchange [q][slot][half][row]
+  static constexpr uint32_t kOffBar = kOffX + kQT * 2 * 2 * BM * 4;
+  static constexpr uint32_t kSmemBytes = kOffBar + sizeof(Barriers) + 1024;
+  static constexpr float kBias = kF8 ? 6.0f : 0.0f;  // log2 units
+  static constexpr float kLazy = kF8 ? 2.0f : 8.0f;  // log2 units
+  static_assert(kStages <= kMaxStages, "barrier arrays");
+  static_assert(kQT * BM * kStageStride * 4 <= kOffX, "O staging fits the operand buffers");
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+};
 
 struct TcParams {
   int B, C, Hq, Hkv, group, T, chunk;
-  float scale_log2;
+  float scale_log2;  // softmax scale * log2(e), times the Q and K factors
+  float out_scale;   // the V factor (1 for bf16)
   const int32_t* cu_prefix;
   float* part_o;    // [slots][BM][HD], slot = (b, g, t, split)
   float* part_lse;  // [slots][BM]   log2 units
@@ -141,48 +159,92 @@ __device__ __forceinline__ uint64_t desc_at(uint64_t base, uint32_t off) {
   return base + (uint64_t)(off >> 4);
 }
 
-// S_q = Q_q K^T into the S/P region of query tile q (K-major operands).
+// S_q = Q_q K^T into the S/P region of query tile q (K-major operands):
+// K = 16 elements (32 bytes) per bf16 MMA, 32 elements (32 bytes) per E4M3
+// MMA, stepping through the 128-byte swizzle rows.
+template <bool kF8>
 __device__ __forceinline__ void issue_s(uint32_t tmem, uint64_t dQ, uint64_t dK, int q, int st) {
-  constexpr uint32_t idS = idesc_bf16_f32(BM, BN, 0, 0);
+  using G = Lay<kF8>;
   const uint32_t dS = tmem + (uint32_t)(q * BN);
-  const uint64_t aq = desc_at(dQ, q * kTile), bk = desc_at(dK, st * kTile);
+  const uint64_t aq = desc_at(dQ, q * G::kTile), bk = desc_at(dK, st * G::kTile);
+  if constexpr (kF8) {
+    constexpr uint32_t idS = idesc_e4m3_f32(BM, BN, 0, 0);
 #pragma unroll
-  for (int kk = 0; kk < HD / 16; ++kk) {
-    const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-    tc_mma_ss(dS, desc_at(aq, off), desc_at(bk, off), idS, kk > 0);
+    for (int kk = 0; kk < HD / 32; ++kk)
+      tc_mma_ss_f8(dS, desc_at(aq, kk * 32), desc_at(bk, kk * 32), idS, kk > 0);
+  } else {
+    constexpr uint32_t idS = idesc_bf16_f32(BM, BN, 0, 0);
+#pragma unroll
+    for (int kk = 0; kk < HD / 16; ++kk) {
+      const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
+      tc_mma_ss(dS, desc_at(aq, off), desc_at(bk, off), idS, kk > 0);
+    }
   }
 }
 
+// O_q (+)= P_q V for one 128-key tile: P from tensor memory (aP), V from the
+// ring stage at descriptor bv (MN-major).  The two column halves of P sit
+// BN/2 columns apart: keys 0-63 from column 0, keys 64-127 from column 64,
+// 2 keys per column for bf16 and 4 for E4M3.
+template <bool kF8>
+__device__ __forceinline__ void issue_pv(uint32_t dO, uint32_t aP, uint64_t bv, bool acc0) {
+  if constexpr (kF8) {
+    constexpr uint32_t idPV = idesc_e4m3_f32(BM, HD, 0, 1);
+#pragma unroll
+    for (int kk = 0; kk < BN / 32; ++kk)  // 32 keys = 8 columns of P, 4 KB of V
+      tc_mma_ts_f8(dO, aP + (uint32_t)((kk >> 1) * (BN / 2) + (kk & 1) * 8),
+                   desc_at(bv, kk * 32 * HD), idPV, (acc0 || kk > 0) ? 1u : 0u);
+  } else {
+    constexpr uint32_t idPV = idesc_bf16_f32(BM, HD, 0, 1);
+#pragma unroll
+    for (int kk = 0; kk < BN / 16; ++kk)  // 16 keys = 8 columns of P, 2 KB of each half of V
+      tc_mma_ts(dO, aP + (uint32_t)((kk >> 2) * (BN / 2) + (kk & 3) * 8),
+                desc_at(bv, kk * 16 * 128), idPV, (acc0 || kk > 0) ? 1u : 0u);
+  }
+}
+
+// One tile of 128 rows (HD elements each) of a [rows, heads, HD] tensor:
+// one copy for E4M3 (128-byte rows), two 64-element halves for bf16.
+template <bool kF8>
+__device__ __forceinline__ void load_rows(uint8_t* dst, const CUtensorMap* map, uint64_t* bar,
+                                          int head, int row0) {
+  tma_load_3d(dst, map, bar, 0, head, row0);
+  if constexpr (!kF8) tma_load_3d(dst + kHalf, map, bar, 64, head, row0);
+}
+
 // One 128-key tile of K (v = 0) or V (v = 1) into ring stage j % kStages.
+template <bool kF8>
 __device__ __forceinline__ bool load_kv(Barriers* bars, uint8_t* smem, int j, int v, int k_begin,
                                         int np, int p0, int b, int C, int g,
                                         const CUtensorMap* tmKp, const CUtensorMap* tmVp,
                                         const CUtensorMap* tmKc, const CUtensorMap* tmVc,
                                         volatile int* abort_flag) {
-  const int st = j % kStages, rd = j / kStages;
+  using G = Lay<kF8>;
+  const int st = j % G::kStages, rd = j / G::kStages;
   uint64_t* empty = v ? &bars->v_empty[st] : &bars->k_empty[st];
   uint64_t* full = v ? &bars->v_full[st] : &bars->k_full[st];
   if (rd > 0 && !mbar_wait_bounded(empty, (rd - 1) & 1, abort_flag, kWaitLimitNs)) return false;
   const int k = k_begin + j;
   const CUtensorMap* map = k < np ? (v ? tmVp : tmKp) : (v ? tmVc : tmKc);
   const int row0 = k < np ? p0 + k * BN : b * C + (k - np) * BN;
-  uint8_t* dst = smem + (v ? kOffV : kOffK) + st * kTile;
-  mbar_arrive_expect_tx(full, kTile);
-  tma_load_3d(dst, map, full, 0, g, row0);
-  tma_load_3d(dst + kHalf, map, full, 64, g, row0);
+  uint8_t* dst = smem + (v ? G::kOffV : G::kOffK) + st * G::kTile;
+  mbar_arrive_expect_tx(full, G::kTile);
+  load_rows<kF8>(dst, map, full, g, row0);
   return true;
 }
 
+template <bool kF8>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                    const __grid_constant__ CUtensorMap tmKp,
                    const __grid_constant__ CUtensorMap tmVp,
                    const __grid_constant__ CUtensorMap tmKc,
                    const __grid_constant__ CUtensorMap tmVc, const TcParams p) {
+  using G = Lay<kF8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  Barriers* bars = reinterpret_cast<Barriers*>(smem + kOffBar);
+  Barriers* bars = reinterpret_cast<Barriers*>(smem + G::kOffBar);
   pdl_wait();
   pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -190,7 +252,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
-    for (int i = 0; i < kStages; ++i) {
+    for (int i = 0; i < G::kStages; ++i) {
       mbar_init(&bars->k_full[i], 1);
       mbar_init(&bars->k_empty[i], 1);
       mbar_init(&bars->v_full[i], 1);
@@ -235,25 +297,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tensormap(&tmKc);
       prefetch_tensormap(&tmVp);
       prefetch_tensormap(&tmVc);
-      mbar_arrive_expect_tx(&bars->q_full, nq * kTile);
+      mbar_arrive_expect_tx(&bars->q_full, nq * G::kTile);
       for (int q = 0; q < nq; ++q) {
         const int qpos = b * p.C + (tp * kQT + q) * (BM / p.group);
-        uint8_t* dst = smem + kOffQ + q * kTile;
-        tma_load_3d(dst, &tmQ, &bars->q_full, 0, g * p.group, qpos);
-        tma_load_3d(dst + kHalf, &tmQ, &bars->q_full, 64, g * p.group, qpos);
+        load_rows<kF8>(smem + G::kOffQ + q * G::kTile, &tmQ, &bars->q_full, g * p.group, qpos);
       }
       // in the order the MMAs consume them: K0, then V_j, K_{j+1}
       int kiss = 0, viss = 0;
-      if (load_kv(bars, smem, 0, 0, k_begin, np, p0, b, p.C, g, &tmKp, &tmVp, &tmKc, &tmVc,
+      if (load_kv<kF8>(bars, smem, 0, 0, k_begin, np, p0, b, p.C, g, &tmKp, &tmVp, &tmKc, &tmVc,
                   abort_flag)) {
         kiss = 1;
         for (int j = 0; j < n; ++j) {
-          if (!load_kv(bars, smem, j, 1, k_begin, np, p0, b, p.C, g, &tmKp, &tmVp, &tmKc, &tmVc,
+          if (!load_kv<kF8>(bars, smem, j, 1, k_begin, np, p0, b, p.C, g, &tmKp, &tmVp, &tmKc, &tmVc,
                        abort_flag))
             break;
           viss = j + 1;
           if (j + 1 < n) {
-            if (!load_kv(bars, smem, j + 1, 0, k_begin, np, p0, b, p.C, g, &tmKp, &tmVp, &tmKc,
+            if (!load_kv<kF8>(bars, smem, j + 1, 0, k_begin, np, p0, b, p.C, g, &tmKp, &tmVp, &tmKc,
                          &tmVc, abort_flag))
               break;
             kiss = j + 2;
@@ -261,34 +321,39 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       // drain: loads still in flight must land before the CTA exits
-      for (int j = max(0, kiss - kStages); j < kiss; ++j)
-        mbar_wait_bounded(&bars->k_full[j % kStages], (j / kStages) & 1, nullptr, kWaitLimitNs);
-      for (int j = max(0, viss - kStages); j < viss; ++j)
-        mbar_wait_bounded(&bars->v_full[j % kStages], (j / kStages) & 1, nullptr, kWaitLimitNs);
+      for (int j = max(0, kiss - G::kStages); j < kiss; ++j)
+        mbar_wait_bounded(&bars->k_full[j % G::kStages], (j / G::kStages) & 1, nullptr,
+                          kWaitLimitNs);
+      for (int j = max(0, viss - G::kStages); j < viss; ++j)
+        mbar_wait_bounded(&bars->v_full[j % G::kStages], (j / G::kStages) & 1, nullptr,
+                          kWaitLimitNs);
       mbar_wait_bounded(&bars->q_full, 0, nullptr, kWaitLimitNs);
     }
     __syncwarp();
   } else if (warp == kWarpMMA) {
     if (lane == 0 && n > 0) {
-      constexpr uint32_t idPV = idesc_bf16_f32(BM, HD, 0, 1);
-      const uint64_t dQ = smem_desc_sw128(smem_u32(smem + kOffQ), 16, 1024);
-      const uint64_t dK = smem_desc_sw128(smem_u32(smem + kOffK), 16, 1024);
-      const uint64_t dV = smem_desc_sw128(smem_u32(smem + kOffV), kHalf, 1024);
+      // K-major Q and K (the leading offset is unused with 128-byte
+      // swizzling); MN-major V: 8-key groups 1024 bytes apart along K,
+      // 128-byte atoms along d kHalf apart (bf16; E4M3 rows are one atom)
+      const uint64_t dQ = smem_desc_sw128(smem_u32(smem + G::kOffQ), 16, 1024);
+      const uint64_t dK = smem_desc_sw128(smem_u32(smem + G::kOffK), 16, 1024);
+      const uint64_t dV = smem_desc_sw128(smem_u32(smem + G::kOffV), kF8 ? G::kTile : kHalf, 1024);
       bool ok = mbar_wait_bounded(&bars->q_full, 0, abort_flag, kWaitLimitNs) &&
                 mbar_wait_bounded(&bars->k_full[0], 0, abort_flag, kWaitLimitNs);
       tc_fence_after();
       if (ok) {
         for (int q = 0; q < nq; ++q) {
-          issue_s(tmem, dQ, dK, q, 0);
+          issue_s<kF8>(tmem, dQ, dK, q, 0);
           tc_commit(&bars->s_full[q]);
         }
         tc_commit(&bars->k_empty[0]);
       }
       for (int j = 0; ok && j < n; ++j) {
-        const int vst = j % kStages;
+        const int vst = j % G::kStages;
         const bool more = j + 1 < n;
-        const int kst = (j + 1) % kStages;
-        if (!mbar_wait_bounded(&bars->v_full[vst], (j / kStages) & 1, abort_flag, kWaitLimitNs)) {
+        const int kst = (j + 1) % G::kStages;
+        if (!mbar_wait_bounded(&bars->v_full[vst], (j / G::kStages) & 1, abort_flag,
+                               kWaitLimitNs)) {
           ok = false;
           break;
         }
@@ -298,23 +363,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after();
-          // O_q += P_q(j) V_j, P_q from TMEM (8 columns per 16 keys)
-          const uint32_t dO = tmem + kTmemO + (uint32_t)(q * HD);
-          const uint32_t aP = tmem + (uint32_t)(q * BN);
-          const uint64_t bv = desc_at(dV, vst * kTile);
-          // keys 0-63 are packed in columns 0-31, keys 64-127 in 64-95
-#pragma unroll
-          for (int kk = 0; kk < BN / 16; ++kk)
-            tc_mma_ts(dO, aP + (uint32_t)((kk >> 2) * (BN / 2) + (kk & 3) * 8),
-                      desc_at(bv, kk * 16 * 128), idPV, (j > 0 || kk > 0) ? 1u : 0u);
+          // O_q += P_q(j) V_j, P_q from TMEM
+          issue_pv<kF8>(tmem + kTmemO + (uint32_t)(q * HD), tmem + (uint32_t)(q * BN),
+                        desc_at(dV, vst * G::kTile), j > 0);
           if (more) {
-            if (q == 0 && !mbar_wait_bounded(&bars->k_full[kst], ((j + 1) / kStages) & 1,
+            if (q == 0 && !mbar_wait_bounded(&bars->k_full[kst], ((j + 1) / G::kStages) & 1,
                                              abort_flag, kWaitLimitNs)) {
               ok = false;
               break;
             }
             tc_fence_after();
-            issue_s(tmem, dQ, dK, q, kst);
+            issue_s<kF8>(tmem, dQ, dK, q, kst);
             tc_commit(&bars->s_full[q]);
           }
         }
@@ -336,7 +395,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_base = (uint32_t)(wl * 32) << 16;  // TMEM lane field
     const uint32_t tS = tmem + lane_base + (uint32_t)(q * BN);
     const uint32_t tO = tmem + lane_base + kTmemO + (uint32_t)(q * HD + h * (HD / 2));
-    float* xch = reinterpret_cast<float*>(smem + kOffX) + q * (2 * 2 * BM);
+    float* xch = reinterpret_cast<float*>(smem + G::kOffX) + q * (2 * 2 * BM);
     uint64_t* xbar = &bars->xch[q][wl];
     const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
     float m_ref = -INFINITY, l = 0.f;
@@ -355,26 +414,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       return xch[(ph & 1) * (2 * BM) + (h ^ 1) * BM + r];
     };
-    // P = 2^(s * scale_log2 - mref) as bf16 pairs into packed columns
-    // [h*64, h*64 + 32) of the S/P region: inside this half's own S columns,
-    // so it never overwrites S the other half has yet to read; returns the
-    // partial row sum
+    // P = 2^(s * scale_log2 - mref), packed (bf16 pairs or E4M3 quads)
+    // into columns from h*64 of the S/P region: inside this half's own S
+    // columns, so it never overwrites S the other half has yet to read;
+    // returns the partial row sum (of the unrounded P)
     auto emit_p = [&](const float (&sv)[BN / 2], float mref) -> float {
       const float2 nm = make_float2(-mref, -mref);
       float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                        make_float2(0.f, 0.f)};
+      constexpr int kKeysPerStore = kF8 ? 32 : 16;  // 8 packed columns per store
 #pragma unroll
-      for (int hh = 0; hh < BN / 32; ++hh) {  // 16 keys -> 8 packed columns per store
+      for (int hh = 0; hh < (BN / 2) / kKeysPerStore; ++hh) {
         uint32_t w[8];
+        float2 prev = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int c = hh * 16 + 2 * e;
+        for (int e = 0; e < kKeysPerStore / 2; ++e) {
+          const int c = hh * kKeysPerStore + 2 * e;
           const float2 d = __ffma2_rn(make_float2(sv[c], sv[c + 1]), sl2, nm);
           // kPolyPairs of every 8 pairs take the FMA-pipe exponential
-          const float2 pp = e < kPolyPairs ? exp2_poly2(d)
-                                           : make_float2(ex2_approx(d.x), ex2_approx(d.y));
+          const float2 pp = (e & 7) < kPolyPairs
+                                ? exp2_poly2(d)
+                                : make_float2(ex2_approx(d.x), ex2_approx(d.y));
           acc[e & 3] = __fadd2_rn(acc[e & 3], pp);
-          w[e] = pack_bf16x2(pp.x, pp.y);
+          if constexpr (kF8) {
+            if (e & 1) w[e >> 1] = pack_e4m3x4(prev, pp);
+            prev = pp;
+          } else {
+            w[e] = pack_bf16x2(pp.x, pp.y);
+          }
         }
         tmem_st8(tS + (uint32_t)(h * (BN / 2) + hh * 8), w);
       }
@@ -416,23 +483,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       post(mh, j);
       float lt;
       if (j == 0) {
-        // first tile: the reference is the row max itself
+        // first tile: the reference is the row max (less the bias)
         const float mx = fmaxf(mh, take(j)) * p.scale_log2;
         if (!ok) break;
-        m_ref = mx;
+        m_ref = mx - G::kBias;
         lt = emit_p(sv, m_ref);
       } else {
         // later tiles: P with the current reference first; the row max
         // (the partner's post has usually arrived by then) decides, rarely,
-        // that the reference must rise by more than 2^8 and P be redone
+        // that P would exceed 2^8, so the reference rises and P is redone
         lt = emit_p(sv, m_ref);
         const float mx = fmaxf(mh, take(j)) * p.scale_log2;
         if (!ok) break;
         // lazy rescale (warp-uniform decision so tcgen05.ld/st stay
         // converged; both halves see the same row maxima, so they decide
         // alike); PV_q(j-1) is complete because S_q(j) is
-        if (__any_sync(0xffffffffu, mx > m_ref + kLazyRescale)) {
-          const float m_new = fmaxf(m_ref, mx);
+        if (__any_sync(0xffffffffu, mx > m_ref + (G::kLazy + G::kBias))) {
+          const float m_new = fmaxf(m_ref, mx - G::kBias);
           const float alpha = ex2_approx(m_ref - m_new);
           l *= alpha;
 #pragma unroll 1
@@ -467,7 +534,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // O / l staged row-wise in shared memory (free now: every MMA has
       // completed), then copied out in whole 512-byte rows
       tc_fence_after();
-      const float inv = 1.f / lrow;
+      const float inv = p.out_scale / lrow;
       float* stage = reinterpret_cast<float*>(smem) + q * (BM * kStageStride);
       float* srow = stage + r * kStageStride + h * (HD / 2);
 #pragma unroll
@@ -652,20 +719,22 @@ EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-// 3-D map over a [rows, heads, 128] bf16 tensor, box (64, box_heads, box_rows),
-// 128-byte swizzle; rows outside [0, rows) read as zero.
+// 3-D map over a [rows, heads, 128] tensor of bf16 (f8 = false) or 8-bit
+// elements (f8 = true, copied as bytes), box (128 bytes of a row, box_heads,
+// box_rows), 128-byte swizzle; rows outside [0, rows) read as zero.
 bool encode_map(CUtensorMap* m, const void* base, int64_t rows, int heads, int box_heads,
-                int box_rows) {
+                int box_rows, bool f8) {
   EncodeTiledFn fn = get_encode_fn();
   if (!fn) return false;
+  const cuuint64_t esz = f8 ? 1 : 2;
   const cuuint64_t dims[3] = {(cuuint64_t)HD, (cuuint64_t)heads, (cuuint64_t)rows};
-  const cuuint64_t strides[2] = {(cuuint64_t)HD * 2, (cuuint64_t)heads * HD * 2};
-  const cuuint32_t box[3] = {64, (cuuint32_t)box_heads, (cuuint32_t)box_rows};
+  const cuuint64_t strides[2] = {(cuuint64_t)HD * esz, (cuuint64_t)heads * HD * esz};
+  const cuuint32_t box[3] = {(cuuint32_t)(128 / esz), (cuuint32_t)box_heads, (cuuint32_t)box_rows};
   const cuuint32_t estr[3] = {1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
-         CUDA_SUCCESS;
+  return fn(m, f8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+            const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 int num_sms() {
@@ -723,7 +792,7 @@ Plan make_plan(const AttnArgs& a) {
 }  // namespace
 
 bool attn_tc_supported(const AttnArgs& a) {
-  if (!a.bf16 || a.D != HD) return false;
+  if (!(a.bf16 || a.e4m3) || a.D != HD) return false;
   const int group = a.Hq / a.Hkv;
   if (group < 1 || BM % group != 0) return false;
   // TMA: 16-byte aligned bases (rows of 256 bytes are always aligned)
@@ -740,24 +809,31 @@ size_t attn_tc_scratch_bytes(const AttnArgs& a) {
   return (size_t)pl.slots * BM * (HD + 1) * sizeof(float) + 256;
 }
 
-cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t stream) {
-  static std::once_flag attr_once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(attr_once, [] {
-    attr_err = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    (int)kSmemBytes);
+template <bool kF8>
+cudaError_t set_smem_attr() {
+  static std::once_flag once;
+  static cudaError_t err = cudaSuccess;
+  std::call_once(once, [] {
+    err = cudaFuncSetAttribute(attn_tc_kernel<kF8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)Lay<kF8>::kSmemBytes);
   });
+  return err;
+}
+
+cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t stream) {
+  const bool f8 = a.e4m3;
+  cudaError_t attr_err = f8 ? set_smem_attr<true>() : set_smem_attr<false>();
   if (attr_err != cudaSuccess) return attr_err;
 
   const Plan pl = make_plan(a);
   const int group = a.Hq / a.Hkv;
   CUtensorMap mQ, mKp, mVp, mKc, mVc;
-  bool ok = encode_map(&mQ, a.q, (int64_t)a.B * a.C, a.Hq, group, BM / group) &&
-            encode_map(&mKc, a.kc, (int64_t)a.B * a.C, a.Hkv, 1, BN) &&
-            encode_map(&mVc, a.vc, (int64_t)a.B * a.C, a.Hkv, 1, BN);
+  bool ok = encode_map(&mQ, a.q, (int64_t)a.B * a.C, a.Hq, group, BM / group, f8) &&
+            encode_map(&mKc, a.kc, (int64_t)a.B * a.C, a.Hkv, 1, BN, f8) &&
+            encode_map(&mVc, a.vc, (int64_t)a.B * a.C, a.Hkv, 1, BN, f8);
   if (a.total_prefix > 0) {
-    ok = ok && encode_map(&mKp, a.kp, a.total_prefix, a.Hkv, 1, BN) &&
-         encode_map(&mVp, a.vp, a.total_prefix, a.Hkv, 1, BN);
+    ok = ok && encode_map(&mKp, a.kp, a.total_prefix, a.Hkv, 1, BN, f8) &&
+         encode_map(&mVp, a.vp, a.total_prefix, a.Hkv, 1, BN, f8);
   } else {  // no prefix rows anywhere: the prefix maps are never read
     mKp = mKc;
     mVp = mVc;
@@ -772,15 +848,21 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t stream) {
   tp.group = group;
   tp.T = pl.T;
   tp.chunk = pl.chunk;
-  tp.scale_log2 = a.scale * 1.4426950408889634f;
+  tp.scale_log2 = f8 ? (float)((double)a.scale * 1.4426950408889634 * (double)a.q_scale *
+                               (double)a.k_scale)
+                     : a.scale * 1.4426950408889634f;
+  tp.out_scale = f8 ? a.v_scale : 1.0f;
   tp.cu_prefix = a.cu_prefix;
   uint8_t* scratch = static_cast<uint8_t*>(a.scratch);
   tp.part_o = reinterpret_cast<float*>(scratch);
   tp.part_lse = reinterpret_cast<float*>(scratch + (size_t)pl.slots * BM * HD * sizeof(float));
   tp.err = a.err;
 
-  cudaError_t e = launch_pdl(attn_tc_kernel, dim3(pl.units), dim3(kThreads), kSmemBytes, stream,
-                             mQ, mKp, mVp, mKc, mVc, tp);
+  cudaError_t e =
+      f8 ? launch_pdl(attn_tc_kernel<true>, dim3(pl.units), dim3(kThreads), Lay<true>::kSmemBytes,
+                      stream, mQ, mKp, mVp, mKc, mVc, tp)
+         : launch_pdl(attn_tc_kernel<false>, dim3(pl.units), dim3(kThreads),
+                      Lay<false>::kSmemBytes, stream, mQ, mKp, mVp, mKc, mVc, tp);
   note_launch();
   if (e != cudaSuccess) return e;
   e = launch_pdl(attn_combine_kernel<__nv_bfloat16>,

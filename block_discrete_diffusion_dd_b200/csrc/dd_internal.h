@@ -77,6 +77,8 @@ struct AttnArgs {
   int B, C, Hq, Hkv, D;
   float scale;
   bool bf16;
+  bool e4m3;                         // 8-bit E4M3 inputs, bf16 output
+  float q_scale, k_scale, v_scale;   // E4M3 per-tensor factors
   const void *q, *kc, *vc, *kp, *vp;
   const int32_t* cu_prefix;       // device [B+1]
   const int32_t* cu_prefix_host;  // host [B+1]
@@ -89,7 +91,7 @@ struct AttnArgs {
   size_t scratch_bytes;
 };
 
-// Tensor-core (tcgen05) path: bf16, D = 128, (Hq/Hkv) divides 128.
+// Tensor-core (tcgen05) path: bf16 or E4M3, D = 128, (Hq/Hkv) divides 128.
 bool attn_tc_supported(const AttnArgs& a);
 size_t attn_tc_scratch_bytes(const AttnArgs& a);
 cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t stream);

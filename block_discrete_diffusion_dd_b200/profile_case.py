@@ -1,10 +1,11 @@
 """Run a few calls of the denoise-step kernels on one workload, for profilers.
 
-    python -m block_discrete_diffusion_dd_b200.profile_case [workload] [calls]
+    python -m block_discrete_diffusion_dd_b200.profile_case [workload] [calls] [e4m3]
 
-Each call is one dd_canvas_attn and one dd_sample_renoise on the workload's
-step-0 inputs (generated on the GPU), so a profiler that skips the first call
-of each kernel sees warm code and a cold-cache second call.
+Each call is one dd_canvas_attn (dd_canvas_attn_fp8 on the workload's E4M3
+inputs with `e4m3`) and one dd_sample_renoise on the workload's step-0
+inputs (generated on the GPU), so a profiler that skips the first call of
+each kernel sees warm code and a cold-cache second call.
 """
 from __future__ import annotations
 
@@ -24,16 +25,23 @@ import workloads  # noqa: E402
 def main(argv):
     name = argv[1] if len(argv) > 1 else "b1_L4096"
     calls = int(argv[2]) if len(argv) > 2 else 2
+    e4m3 = len(argv) > 3 and argv[3] == "e4m3"
     w = workloads.WORKLOADS[name]
-    q, kc, vc = workloads.canvas_qkv(w, 0, device="cuda")
-    kp, vp, cu = workloads.prefix_kv(w, device="cuda")
+    if e4m3:
+        q, kc, vc, kp, vp, cu, f = workloads.e4m3_attn_inputs(w, 0, device="cuda")
+    else:
+        q, kc, vc = workloads.canvas_qkv(w, 0, device="cuda")
+        kp, vp, cu = workloads.prefix_kv(w, device="cuda")
     lg = workloads.logits(w, 0, device="cuda")
     cud = cu.cuda()
     for i in range(calls):
-        dd.canvas_attn(q, kc, vc, kp, vp, cud, cu, scale=w.scale)
+        if e4m3:
+            dd.canvas_attn_fp8(q, kc, vc, kp, vp, cud, f, cu, scale=w.scale)
+        else:
+            dd.canvas_attn(q, kc, vc, kp, vp, cud, cu, scale=w.scale)
         dd.sample_renoise(lg, w.temperatures[0], w.rates[0], w.seed, i)
     torch.cuda.synchronize()
-    print(f"{name}: {calls} calls ok")
+    print(f"{name}{' e4m3' if e4m3 else ''}: {calls} calls ok")
 
 
 if __name__ == "__main__":

@@ -61,7 +61,10 @@ typedef enum {
   DD_ERR_DEVICE_BOUNDS = 6
 } dd_status;
 
-typedef enum { DD_BF16 = 0, DD_F32 = 1 } dd_dtype;
+/* Element types.  DD_E4M3 (8-bit floating point, OCP OFP8 E4M3 encoding:
+ * bias 7, 3 mantissa bits, largest finite value 448) is taken only by
+ * dd_canvas_attn_fp8, with one scale factor per tensor. */
+typedef enum { DD_BF16 = 0, DD_F32 = 1, DD_E4M3 = 2 } dd_dtype;
 
 /* Geometry of one canvas-attention call.
  *   batch     B >= 1 canvases (batch rows)
@@ -71,15 +74,17 @@ typedef enum { DD_BF16 = 0, DD_F32 = 1 } dd_dtype;
  *             the pages do not state the head mapping, this is the usual one).
  *   head_dim  D in {64, 128}
  *   scale     softmax scale (1/sqrt(D) in every workload here)
- *   dtype     DD_BF16 (tensor cores, fp32 accumulation) or DD_F32 (fp32 FMA) */
+ *   dtype     DD_BF16 (tensor cores, fp32 accumulation), DD_F32 (fp32 FMA)
+ *             or DD_E4M3 (tensor cores, fp32 accumulation; dd_canvas_attn_fp8) */
 typedef struct {
   int batch, canvas, heads_q, heads_kv, head_dim;
   float scale;
   dd_dtype dtype;
 } dd_attn_desc;
 
-/* Workspace bytes that dd_canvas_attn needs for this geometry and these
- * prefix lengths (cu_prefix_host: [B+1] host array, see dd_canvas_attn).
+/* Workspace bytes that dd_canvas_attn (or dd_canvas_attn_fp8, for a
+ * DD_E4M3 desc) needs for this geometry and these prefix lengths
+ * (cu_prefix_host: [B+1] host array, see dd_canvas_attn).
  * Returns 0 if the arguments are invalid. */
 DD_API size_t dd_canvas_attn_workspace(const dd_attn_desc* desc, const int32_t* cu_prefix_host);
 
@@ -101,11 +106,42 @@ DD_API size_t dd_canvas_attn_workspace(const dd_attn_desc* desc, const int32_t* 
  *                the two must agree, which is not checked on the device)
  *   out          [B, C, Hq, D], element type = desc->dtype
  *   lse          optional fp32 [B, Hq, C]: natural-log sum of exp of scores
- *   workspace    >= dd_canvas_attn_workspace(...) bytes, 256-byte aligned */
+ *   workspace    >= dd_canvas_attn_workspace(...) bytes, 256-byte aligned
+ * desc->dtype DD_E4M3 is rejected here (DD_ERR_INVALID_ARG): the 8-bit path
+ * is dd_canvas_attn_fp8. */
 DD_API dd_status dd_canvas_attn(const dd_attn_desc* desc, const void* q, const void* k_canvas,
                          const void* v_canvas, const void* k_prefix, const void* v_prefix,
                          const int32_t* cu_prefix, const int32_t* cu_prefix_host, void* out,
                          float* lse, void* workspace, size_t workspace_bytes, dd_stream_t stream);
+
+/* Per-tensor scale factors of 8-bit attention inputs: the value of an
+ * element is its E4M3 value times its tensor's factor.  `k` covers both
+ * k_prefix and k_canvas, `v` both v_prefix and v_canvas.  Finite and > 0. */
+typedef struct {
+  float q, k, v;
+} dd_fp8_scales;
+
+/* dd_canvas_attn on 8-bit inputs: the same definition and layouts, with
+ * desc->dtype = DD_E4M3, q / k_* / v_* holding E4M3 bytes (one byte per
+ * element) and `scales` their factors:
+ *   O[b,i,h,:] = f_v * sum_j softmax_j(scale * f_q * f_k * <q, k_j>) v_j
+ * The pages quote their step times for 8-bit inference ("DiffusionGemma
+ * Technical Report", "The numbers, honestly"); this is the attention of
+ * that step on the tensor cores' 8-bit path (kind::f8f6f4, fp32
+ * accumulation).  The softmax probabilities are rounded to E4M3 for the
+ * P.V product (relative rounding error <= 2^-4 per probability); the
+ * row sums and the output use the unrounded fp32 values.
+ *   out   [B, C, Hq, D] bf16
+ *   lse   optional fp32 [B, Hq, C]
+ * Requires head_dim 128 and (heads_q / heads_kv) dividing 128, else
+ * DD_ERR_UNSUPPORTED.  Same workspace as dd_canvas_attn
+ * (dd_canvas_attn_workspace with the DD_E4M3 desc). */
+DD_API dd_status dd_canvas_attn_fp8(const dd_attn_desc* desc, const void* q,
+                                    const void* k_canvas, const void* v_canvas,
+                                    const void* k_prefix, const void* v_prefix,
+                                    const int32_t* cu_prefix, const int32_t* cu_prefix_host,
+                                    const dd_fp8_scales* scales, void* out, float* lse,
+                                    void* workspace, size_t workspace_bytes, dd_stream_t stream);
 
 /* Sampler parameters for one step.
  *   temperature   tau > 0; logits are divided by it (the method anneals it

@@ -6,6 +6,17 @@ Tolerances:
                            inputs the outputs are ~0.02 in size, so the
                            absolute bound alone would be weak)
   attention, fp32 inputs : max |err| <= 1e-5
+  attention, E4M3 inputs : the kernel rounds each softmax probability P to
+                           E4M3 for the P.V product (relative error <= 2^-4
+                           in E4M3's normal range; P >= 2^-6 * max P is
+                           normal, smaller P err by <= 2^-10 absolute with
+                           max P >= 2^6).  With independent rounding errors
+                           the output's relative RMS error is about
+                           2^-4 / sqrt(3) * E[1/m^2]^(1/2) ~ 0.026 (m the
+                           mantissa in [1, 2)), at most 2^-4 / sqrt(3) =
+                           0.036: gate 5e-2.  Max |err| <= max|V| (2^-4 +
+                           n_keys 2^-16) + 2^-8 max|O| (the bf16 output)
+                           bounds it rigorously.
   confidence             : relative error <= 1e-5
   entropy                : |err| <= 1e-5 * max(1, |H|)
   token ids              : bit-exact, except a sampled id at a position that
@@ -60,6 +71,14 @@ def check_sampler(got: dict, ref: dict, rows=None, conf_rtol=1e-5, ent_tol=1e-5)
     return {"rows": int(tokens.size), "near_ties": int(near.sum()),
             "near_tie_mismatches": int(mism.sum()), "kept_exact": int(keep_ok.sum()),
             "conf_max_rel": float(rel.max()) if rel.size else 0.0}
+
+
+FP8_REL_RMS = 5e-2
+
+
+def fp8_max_abs(v_max: float, n_keys: int, o_max: float) -> float:
+    """The E4M3 path's rigorous max |err| bound (see the module docstring)."""
+    return v_max * (2.0 ** -4 + n_keys * 2.0 ** -16) + 2.0 ** -8 * o_max
 
 
 def check_attn(got, ref, dtype, positions=None, max_abs=None, rel_rms=1e-2) -> dict:

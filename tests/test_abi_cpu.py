@@ -122,6 +122,30 @@ def test_attention_rejects_null_and_misaligned(lib):
     assert _attn(lib, _desc(B=0), cu[:1]) == 0                   # empty batch: no-op
 
 
+def _attn_fp8(lib, desc, cu, scales=(1.0, 1.0, 1.0), ptr=FAKE, ws=FAKE, ws_bytes=1 << 30):
+    f = None if scales is None else ctypes.byref(dd.Fp8Scales(*scales))
+    return lib.dd_canvas_attn_fp8(ctypes.byref(desc), ptr, ptr, ptr, ptr, ptr, FAKE,
+                                  cu.ctypes.data_as(ctypes.c_void_p), f, ptr, None, ws, ws_bytes,
+                                  None)
+
+
+def test_fp8_attention_rejects_bad_arguments(lib):
+    cu = _cu([16])
+    e4 = _desc(dtype=dd.DD_E4M3)
+    assert _attn(lib, e4, cu) == 1                                  # needs the fp8 entry
+    assert "dd_canvas_attn_fp8" in dd.last_error()
+    assert _attn_fp8(lib, _desc(), cu) == 1                         # bf16 desc
+    assert _attn_fp8(lib, e4, cu, scales=None) == 1
+    for bad in ((0.0, 1.0, 1.0), (1.0, -1.0, 1.0), (1.0, 1.0, float("inf")),
+                (1.0, float("nan"), 1.0), (1e30, 1e30, 1.0)):
+        assert _attn_fp8(lib, e4, cu, scales=bad) == 1, bad
+    assert _attn_fp8(lib, _desc(D=64, dtype=dd.DD_E4M3), cu) == 2   # no kernel for D = 64
+    assert _attn_fp8(lib, _desc(Hq=12, Hkv=4, dtype=dd.DD_E4M3), cu) == 2  # group 3 !| 128
+    assert _attn_fp8(lib, e4, cu, ptr=ctypes.c_void_p((1 << 20) + 4)) == 1
+    assert _attn_fp8(lib, e4, cu, ws_bytes=300) == 3
+    assert dd.canvas_attn_workspace_bytes(e4, cu) > 0
+
+
 def test_block_rejects_bad_arguments(lib):
     d = _desc()
     cu = _cu([16])

@@ -23,13 +23,16 @@ in "The numbers, honestly"; ~12 passes per block in "The mechanism"):
 
 Every tensor is drawn in float32 from a torch.Generator seeded with a hash
 of (seed, workload, tensor name, step), then rounded to bf16 (round to
-nearest even) where the workload is bf16.  The generator's device is the
+nearest even) where the workload is bf16.  The 8-bit attention inputs are
+the same float32 draws rounded to E4M3 under a power-of-two per-tensor
+factor (e4m3_attn_inputs).  The generator's device is the
 caller's choice; the same device always gives the same bits.
 """
 from __future__ import annotations
 
 import dataclasses
 import hashlib
+import math
 from typing import List, Optional
 
 import numpy as np
@@ -140,6 +143,32 @@ def prefix_kv(w: Workload, device="cpu"):
     kp = _normal(w, "kp", 0, (n, w.heads_kv, w.head_dim), 1.0, device)
     vp = _normal(w, "vp", 0, (n, w.heads_kv, w.head_dim), 1.0, device)
     return kp, vp, torch.from_numpy(w.cu_prefix)
+
+
+def to_e4m3(xs):
+    """Round float32 tensors that share one scale factor to E4M3.
+
+    The factor is the power of two f = 2^ceil(log2(amax / 448)) over all of
+    them (448 = the largest finite E4M3 value), so x / f is exact in float32
+    and never overflows; torch rounds x / f to the nearest E4M3 value (ties
+    to even).  Returns (list of float8_e4m3fn tensors, f)."""
+    amax = max(float(x.abs().max()) for x in xs if x.numel()) if any(x.numel() for x in xs) else 0.0
+    f = 2.0 ** math.ceil(math.log2(amax / 448.0)) if amax > 0 else 1.0
+    return [(x / f).to(torch.float8_e4m3fn) for x in xs], f
+
+
+def e4m3_attn_inputs(w: Workload, step: int = 0, device="cpu", q_gain: float = 1.0):
+    """The attention inputs of `w` drawn as for bf16 (same seeds, float32
+    normals), then rounded to E4M3 with one factor for Q, one shared by Kp and
+    Kc, one shared by Vp and Vc.  Returns q, kc, vc, kp, vp (float8_e4m3fn),
+    cu_prefix and the factors (f_q, f_k, f_v)."""
+    f32 = dataclasses.replace(w, dtype="f32")
+    q, kc, vc = canvas_qkv(f32, step, device, q_gain)
+    kp, vp, cu = prefix_kv(f32, device)
+    (q8,), fq = to_e4m3([q])
+    (kc8, kp8), fk = to_e4m3([kc, kp])
+    (vc8, vp8), fv = to_e4m3([vc, vp])
+    return q8, kc8, vc8, kp8, vp8, cu, (fq, fk, fv)
 
 
 def logits(w: Workload, step: int = 0, device="cpu", rows: Optional[int] = None):
