@@ -24,15 +24,17 @@
 //              memory to agree on the row max.  Each half reads its 64 S
 //              columns (fp32) from TMEM, runs the online softmax in fp32
 //              (log2 domain; O is rescaled only when the running max grows
-//              by more than 2^8) and writes its half of P back as bf16 into
-//              its own half of the same TMEM region (columns 0-31 and
-//              64-95), where the P.V MMA reads it directly;
-//   warp 16    TMA producer: Q, then K and V tiles (2-stage rings of 128
-//              keys) in the order the MMAs consume them;
+//              past a margin) and writes its half of P back (bf16 pairs in
+//              columns 0-31 / 64-95, E4M3 quads in 0-15 / 64-79) into its
+//              own half of the same TMEM region, where the P.V MMA reads it;
+//   warp 16    TMA producer: Q, then K and V tiles (rings of 128 keys, 2
+//              stages for bf16, 4 for E4M3) in the order the MMAs consume
+//              them;
 //   warp 17    allocates all 512 TMEM columns (per query tile: S/P 128, O
-//              128) and issues every MMA from one thread, in the order
-//              PV_0(j), S_0(j+1), PV_1(j), S_1(j+1): each softmax warpgroup
-//              works while the tensor core runs the other tile's MMAs.
+//              128) and issues every MMA from one elected lane of the
+//              converged warp, in the order PV_0(j), S_0(j+1), PV_1(j),
+//              S_1(j+1): each softmax warpgroup works while the tensor core
+//              runs the other tile's MMAs.
 // The tensor core executes one thread's MMAs in issue order, so:
 //   - S_q(j+1) overwrites P_q(j) only after PV_q(j) has read it;
 //   - when S_q(j) is complete, PV_q(j-1) is complete too, so the softmax
@@ -331,60 +333,77 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else if (warp == kWarpMMA) {
-    if (lane == 0 && n > 0) {
+    if (n > 0) {
+      // The whole warp runs this loop, so every MMA operand is warp-uniform
+      // (computed once per warp rather than moved out of one lane's
+      // registers before each MMA); one elected lane issues the MMAs and
+      // their commits (a commit tracks the MMAs of the thread issuing it).
+      const bool leader = elect_one_sync();
       // K-major Q and K (the leading offset is unused with 128-byte
       // swizzling); MN-major V: 8-key groups 1024 bytes apart along K,
       // 128-byte atoms along d kHalf apart (bf16; E4M3 rows are one atom)
       const uint64_t dQ = smem_desc_sw128(smem_u32(smem + G::kOffQ), 16, 1024);
       const uint64_t dK = smem_desc_sw128(smem_u32(smem + G::kOffK), 16, 1024);
       const uint64_t dV = smem_desc_sw128(smem_u32(smem + G::kOffV), kF8 ? G::kTile : kHalf, 1024);
-      bool ok = mbar_wait_bounded(&bars->q_full, 0, abort_flag, kWaitLimitNs) &&
-                mbar_wait_bounded(&bars->k_full[0], 0, abort_flag, kWaitLimitNs);
+      auto wait = [&](uint64_t* bar, uint32_t parity) {
+        return __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity, abort_flag, kWaitLimitNs));
+      };
+      auto commit = [&](uint64_t* bar) {
+        if (leader) tc_commit(bar);
+        __syncwarp();
+      };
+      bool ok = wait(&bars->q_full, 0) && wait(&bars->k_full[0], 0);
       tc_fence_after();
       if (ok) {
         for (int q = 0; q < nq; ++q) {
-          issue_s<kF8>(tmem, dQ, dK, q, 0);
-          tc_commit(&bars->s_full[q]);
+          if (leader) {
+            issue_s<kF8>(tmem, dQ, dK, q, 0);
+            tc_commit(&bars->s_full[q]);
+          }
+          __syncwarp();
         }
-        tc_commit(&bars->k_empty[0]);
+        commit(&bars->k_empty[0]);
       }
       for (int j = 0; ok && j < n; ++j) {
         const int vst = j % G::kStages;
         const bool more = j + 1 < n;
         const int kst = (j + 1) % G::kStages;
-        if (!mbar_wait_bounded(&bars->v_full[vst], (j / G::kStages) & 1, abort_flag,
-                               kWaitLimitNs)) {
+        if (!wait(&bars->v_full[vst], (j / G::kStages) & 1)) {
           ok = false;
           break;
         }
         for (int q = 0; q < nq; ++q) {
-          if (!mbar_wait_bounded(&bars->p_full[q], j & 1, abort_flag, kWaitLimitNs)) {
+          if (!wait(&bars->p_full[q], j & 1)) {
             ok = false;
             break;
           }
           tc_fence_after();
           // O_q += P_q(j) V_j, P_q from TMEM
-          issue_pv<kF8>(tmem + kTmemO + (uint32_t)(q * HD), tmem + (uint32_t)(q * BN),
-                        desc_at(dV, vst * G::kTile), j > 0);
+          const uint32_t dO = tmem + kTmemO + (uint32_t)(q * HD), aP = tmem + (uint32_t)(q * BN);
+          const uint64_t bv = desc_at(dV, vst * G::kTile);
+          if (leader) issue_pv<kF8>(dO, aP, bv, j > 0);
+          __syncwarp();
           if (more) {
-            if (q == 0 && !mbar_wait_bounded(&bars->k_full[kst], ((j + 1) / G::kStages) & 1,
-                                             abort_flag, kWaitLimitNs)) {
+            if (q == 0 && !wait(&bars->k_full[kst], ((j + 1) / G::kStages) & 1)) {
               ok = false;
               break;
             }
             tc_fence_after();
-            issue_s<kF8>(tmem, dQ, dK, q, kst);
-            tc_commit(&bars->s_full[q]);
+            if (leader) {
+              issue_s<kF8>(tmem, dQ, dK, q, kst);
+              tc_commit(&bars->s_full[q]);
+            }
+            __syncwarp();
           }
         }
         if (!ok) break;
-        tc_commit(&bars->v_empty[vst]);
-        if (more) tc_commit(&bars->k_empty[kst]);
+        commit(&bars->v_empty[vst]);
+        if (more) commit(&bars->k_empty[kst]);
       }
       if (ok)
-        for (int q = 0; q < nq; ++q) tc_commit(&bars->o_done[q]);
+        for (int q = 0; q < nq; ++q) commit(&bars->o_done[q]);
       // every MMA issued above has completed before TMEM is released
-      tc_commit(&bars->mma_final);
+      commit(&bars->mma_final);
       mbar_wait_bounded(&bars->mma_final, 0, nullptr, kWaitLimitNs);
     }
     __syncwarp();
