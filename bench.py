@@ -318,6 +318,74 @@ def run_block(w, dd, dev, dist, reps: int = 20):
             "timing": f"mean of {reps} eager dd_denoise_block calls, CUDA events"}
 
 
+def run_attn_e4m3(w, reps: int = 50):
+    """Canvas attention on E4M3 inputs (dd_canvas_attn_fp8) beside the bf16
+    kernel on the same workload: device time of one call (attention + split
+    combine), CUDA events around the call only, L2 flushed before every
+    call (a 256 MB write), median of `reps`."""
+    import block_discrete_diffusion_dd_b200 as dd
+    dev = torch.device("cuda", torch.cuda.current_device())
+    q8, kc8, vc8, kp8, vp8, cu, f = workloads.e4m3_attn_inputs(w, 0, device=dev)
+    q, kc, vc = workloads.canvas_qkv(w, 0, device=dev)
+    kp, vp, _ = workloads.prefix_kv(w, device=dev)
+    cud = cu.to(dev)
+    d8, d16 = dd.attn_desc(q8, kc8, w.scale), dd.attn_desc(q, kc, w.scale)
+    ws8 = dd.new_workspace(dd.canvas_attn_workspace_bytes(d8, cu), dev)
+    ws16 = dd.new_workspace(dd.canvas_attn_workspace_bytes(d16, cu), dev)
+    o8 = torch.empty(q8.shape, dtype=torch.bfloat16, device=dev)
+    o16 = torch.empty_like(q)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    calls = {
+        "e4m3": lambda: dd.canvas_attn_fp8(q8, kc8, vc8, kp8, vp8, cud, f, cu, scale=w.scale,
+                                           out=o8, workspace=ws8),
+        "bf16": lambda: dd.canvas_attn(q, kc, vc, kp, vp, cud, cu, scale=w.scale, out=o16,
+                                       workspace=ws16),
+    }
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    time.sleep(0.3)
+    t_wall0 = time.time()
+    ms = {}
+    for name, fn in calls.items():
+        for _ in range(5):
+            fn()
+        ts = []
+        for _ in range(reps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        ms[name] = statistics.median(ts)
+    t_wall1 = time.time()
+    time.sleep(0.2)
+    clocks.stop()
+    dd.query_device_error(ws8)
+    dd.query_device_error(ws16)
+    hbm, tf_burst, tf_sus, src = _peaks()
+    flops = w.attn_flops()
+    tf8, tf16 = flops / ms["e4m3"] / 1e9, flops / ms["bf16"] / 1e9
+    return {
+        "metric": "canvas attention throughput, E4M3 inputs", "value": tf8, "unit": "TFLOP/s",
+        "higher_is_better": True, "dtype": "e4m3", "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "canvas": w.canvas,
+                   "heads_q": w.heads_q, "heads_kv": w.heads_kv, "head_dim": w.head_dim,
+                   "prefix": list(w.prefix_lens), "factors": list(f),
+                   "l2": "flushed (256 MB write) before every call"},
+        "ms": ms["e4m3"],
+        "roofline": {"bound": "tensor", "achieved": tf8, "peak": 2 * tf_burst, "unit": "TFLOP/s",
+                     "frac": tf8 / (2 * tf_burst), "flops": flops,
+                     "traffic": (_profile_traffic().get("attention_e4m3")
+                                 if w.name == "b1_L4096" else None),
+                     "peak_source": f"{src} bf16 burst x 2 (nominal E4M3 / bf16 ratio)"},
+        "bf16_same_workload": {"ms": ms["bf16"], "TFLOP/s": tf16, "frac": tf16 / tf_burst},
+        "timing": f"median of {reps} calls, CUDA events around each call",
+        "clocks": clocks.summary(t_wall0, t_wall1),
+    }
+
+
 # The sampler's arithmetic ceiling: per warp-item of 256 logits the scan
 # issues 2 Philox4x32-10 blocks x 18 IMAD.WIDE (two of the 20 products per
 # block are row-invariant and hoisted) plus 16 packed fp32 ops, all on the
@@ -617,6 +685,8 @@ def main():
     ap.add_argument("--ref-sample", type=float, default=1.0 / 32)
     ap.add_argument("--policy", action="store_true",
                     help="time the pages' adaptive block loop instead (one JSON line)")
+    ap.add_argument("--attn-e4m3", action="store_true",
+                    help="time canvas attention on E4M3 inputs beside bf16 (one JSON line)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     w = workloads.WORKLOADS[args.workload]
@@ -632,6 +702,9 @@ def main():
         libbuild.build()
     if args.policy:
         print(json.dumps(run_policy(workloads.WORKLOADS["block12_L8192"])), flush=True)
+        return
+    if args.attn_e4m3:
+        print(json.dumps(run_attn_e4m3(w)), flush=True)
         return
     dist, rank, world, local_rank = _dist()
     if world != args.gpus and rank == 0:
