@@ -314,8 +314,25 @@ def run_block(w, dd, dev, dist, reps: int = 20):
     torch.cuda.synchronize()
     ms = _max_over_ranks(dist, e0.elapsed_time(e1) / reps)
     dd.query_device_error(ws)
+    # the same loop captured once (dd_denoise_block_graph) and replayed
+    g = dd.denoise_block_graph(q, kc, vc, kp, vp, cud, lg, w.rates, w.temperatures, w.seed,
+                               cu_prefix_host=cu.numpy(), scale=w.scale, attn_out=attn_out,
+                               canvas=canvas, keep_history=False, workspace=ws)
+    for _ in range(3):
+        g.launch()
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(reps):
+        g.launch()
+    e1.record()
+    torch.cuda.synchronize()
+    ms_g = _max_over_ranks(dist, e0.elapsed_time(e1) / reps)
+    g.destroy()
+    dd.query_device_error(ws)
     return {"steps": w.steps, "ms_per_block": ms, "blocks_per_s": 1e3 / ms,
-            "timing": f"mean of {reps} eager dd_denoise_block calls, CUDA events"}
+            "ms_per_block_graph": ms_g, "blocks_per_s_graph": 1e3 / ms_g,
+            "timing": f"mean of {reps} eager dd_denoise_block calls, and of {reps} replays of "
+                      "the same loop captured once (dd_denoise_block_graph), CUDA events"}
 
 
 def run_attn_e4m3(w, reps: int = 50):

@@ -31,7 +31,8 @@ EXPORTS = (
     "dd_workspace_init", "dd_query_device_error", "dd_status_string", "dd_last_error",
     "dd_launch_count", "dd_reset_launch_count", "dd_sample_renoise_noalloc",
     "dd_entropy_accept", "dd_stop_check", "dd_denoise_block_adaptive_workspace",
-    "dd_denoise_block_adaptive", "dd_canvas_attn_fp8",
+    "dd_denoise_block_adaptive", "dd_canvas_attn_fp8", "dd_denoise_block_graph_create",
+    "dd_denoise_block_graph_launch", "dd_denoise_block_graph_destroy",
 )
 
 
@@ -94,6 +95,13 @@ def load() -> ctypes.CDLL:
     lib.dd_denoise_block.restype = i32
     lib.dd_denoise_block.argtypes = [D, i32, P, P, P, P, P, P, P, P, P, i32, P, P, u64, u32, P, P,
                                      P, P, sz, P]
+    lib.dd_denoise_block_graph_create.restype = i32
+    lib.dd_denoise_block_graph_create.argtypes = [ctypes.POINTER(P), D, i32, P, P, P, P, P, P, P,
+                                                  P, P, i32, P, P, u64, u32, P, P, P, P, sz]
+    lib.dd_denoise_block_graph_launch.restype = i32
+    lib.dd_denoise_block_graph_launch.argtypes = [P, P]
+    lib.dd_denoise_block_graph_destroy.restype = i32
+    lib.dd_denoise_block_graph_destroy.argtypes = [P]
     f32 = ctypes.c_float
     lib.dd_entropy_accept.restype = i32
     lib.dd_entropy_accept.argtypes = [P, P, i32, i32, i32, f32, u64, u32, u32, P, P, P]
@@ -326,6 +334,75 @@ def denoise_block(q_steps, kc_steps, vc_steps, kp, vp, cu_prefix, logits_steps,
         _ptr(workspace), workspace.numel(), _stream(stream)))
     return {"attn_out": attn_out, "canvas": canvas, "canvas_history": canvas_history,
             "conf_steps": conf_steps}
+
+
+class BlockGraph:
+    """dd_denoise_block captured once (dd_denoise_block_graph_create) and
+    replayed with one launch (launch()).  Holds every captured tensor, so the
+    buffers outlive the graph; new inputs enter by writing into them
+    (`tensors` maps the argument names to those tensors)."""
+
+    def __init__(self, handle, tensors: dict, keep: tuple):
+        self._h = handle
+        self.tensors = tensors
+        self._keep = keep
+
+    def launch(self, stream=None):
+        if self._h is None:
+            raise RuntimeError("BlockGraph: destroyed")
+        _check(load().dd_denoise_block_graph_launch(self._h, _stream(stream)))
+        return self.tensors
+
+    def destroy(self):
+        if self._h is not None:
+            h, self._h = self._h, None
+            _check(load().dd_denoise_block_graph_destroy(h))
+
+    def __del__(self):
+        try:
+            self.destroy()
+        except Exception:
+            pass
+
+
+def denoise_block_graph(q_steps, kc_steps, vc_steps, kp, vp, cu_prefix, logits_steps,
+                        rates: Sequence[float], temperatures: Sequence[float], seed: int,
+                        step0: int = 0, cu_prefix_host=None, scale=None, attn_out=None,
+                        canvas=None, canvas_history=None, conf_steps=None, keep_history=True,
+                        workspace=None) -> BlockGraph:
+    """dd_denoise_block_graph_create with the arguments of denoise_block."""
+    lib = load()
+    S = q_steps.shape[0]
+    desc = attn_desc(q_steps[0], kc_steps[0], scale)
+    cu_h = _host_i32(cu_prefix if cu_prefix_host is None else cu_prefix_host)
+    V = logits_steps.shape[-1]
+    R = desc.batch * desc.canvas
+    dev = q_steps.device
+    if attn_out is None:
+        attn_out = torch.empty_like(q_steps)
+    if canvas is None:
+        canvas = torch.empty(R, dtype=torch.int32, device=dev)
+    if keep_history and canvas_history is None:
+        canvas_history = torch.empty((S, R), dtype=torch.int32, device=dev)
+    if keep_history and conf_steps is None:
+        conf_steps = torch.empty((S, R), dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = new_workspace(denoise_block_workspace_bytes(desc, cu_h, V), dev)
+    rates_h = np.ascontiguousarray(np.asarray(rates, dtype=np.float32))
+    temps_h = np.ascontiguousarray(np.asarray(temperatures, dtype=np.float32))
+    assert rates_h.size >= S and temps_h.size >= S
+    h = ctypes.c_void_p()
+    _check(lib.dd_denoise_block_graph_create(
+        ctypes.byref(h), ctypes.byref(desc), S, _ptr(q_steps), _ptr(kc_steps), _ptr(vc_steps),
+        _ptr(kp), _ptr(vp), _ptr(cu_prefix), cu_h.ctypes.data_as(ctypes.c_void_p),
+        _ptr(attn_out), _ptr(logits_steps), V, rates_h.ctypes.data_as(ctypes.c_void_p),
+        temps_h.ctypes.data_as(ctypes.c_void_p), int(seed), int(step0), _ptr(canvas),
+        _ptr(canvas_history), _ptr(conf_steps), _ptr(workspace), workspace.numel()))
+    tensors = {"q_steps": q_steps, "kc_steps": kc_steps, "vc_steps": vc_steps, "kp": kp, "vp": vp,
+               "cu_prefix": cu_prefix, "logits_steps": logits_steps, "attn_out": attn_out,
+               "canvas": canvas, "canvas_history": canvas_history, "conf_steps": conf_steps,
+               "workspace": workspace}
+    return BlockGraph(h, tensors, (cu_h, rates_h, temps_h))
 
 
 def entropy_accept(entropy: torch.Tensor, pred: torch.Tensor, canvas: int, budget: float,

@@ -432,6 +432,80 @@ size_t adaptive_ws_layout(const dd_attn_desc* desc, int64_t total, const int32_t
 }
 }  // namespace
 
+// A captured block loop: one instantiated CUDA graph and the number of
+// library kernels one replay launches.
+struct dd_block_graph_st {
+  cudaGraphExec_t exec;
+  uint64_t launches;
+};
+
+dd_status dd_denoise_block_graph_create(
+    dd_block_graph* out, const dd_attn_desc* desc, int steps, const void* q_steps,
+    const void* kc_steps, const void* vc_steps, const void* k_prefix, const void* v_prefix,
+    const int32_t* cu_prefix, const int32_t* cu_prefix_host, void* attn_out,
+    const void* logits_steps, int vocab, const float* rate_host, const float* temperature_host,
+    uint64_t seed, uint32_t step0, int32_t* canvas, int32_t* canvas_history, float* conf_steps,
+    void* workspace, size_t workspace_bytes) {
+  g_last_error.clear();
+  if (!out) return fail(DD_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  cudaStream_t s = nullptr;
+  cudaError_t e = cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking);
+  if (e != cudaSuccess) return cuda_fail(e, "capture stream");
+  // relaxed mode: the first call of a kernel sets its attributes and
+  // queries its occupancy, which are not stream work
+  e = cudaStreamBeginCapture(s, cudaStreamCaptureModeRelaxed);
+  if (e != cudaSuccess) {
+    cudaStreamDestroy(s);
+    return cuda_fail(e, "begin capture");
+  }
+  const uint64_t l0 = g_launches;
+  dd_status st = dd_denoise_block(desc, steps, q_steps, kc_steps, vc_steps, k_prefix, v_prefix,
+                                  cu_prefix, cu_prefix_host, attn_out, logits_steps, vocab,
+                                  rate_host, temperature_host, seed, step0, canvas, canvas_history,
+                                  conf_steps, workspace, workspace_bytes,
+                                  reinterpret_cast<dd_stream_t>(s));
+  const uint64_t launches = g_launches - l0;
+  g_launches = l0;  // captured, not launched
+  const std::string detail = g_last_error;
+  cudaGraph_t graph = nullptr;
+  e = cudaStreamEndCapture(s, &graph);
+  cudaStreamDestroy(s);
+  if (st != DD_OK) {
+    if (graph) cudaGraphDestroy(graph);
+    g_last_error = detail;
+    return st;
+  }
+  if (e != cudaSuccess) {
+    if (graph) cudaGraphDestroy(graph);
+    return cuda_fail(e, "end capture");
+  }
+  cudaGraphExec_t exec = nullptr;
+  e = cudaGraphInstantiate(&exec, graph, 0);
+  cudaGraphDestroy(graph);
+  if (e != cudaSuccess) return cuda_fail(e, "instantiate block graph");
+  *out = new dd_block_graph_st{exec, launches};
+  return DD_OK;
+}
+
+dd_status dd_denoise_block_graph_launch(dd_block_graph g, dd_stream_t stream) {
+  g_last_error.clear();
+  if (!g) return fail(DD_ERR_INVALID_ARG, "graph is NULL");
+  cudaError_t e = cudaGraphLaunch(g->exec, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "launch block graph");
+  g_launches += g->launches;
+  return DD_OK;
+}
+
+dd_status dd_denoise_block_graph_destroy(dd_block_graph g) {
+  g_last_error.clear();
+  if (!g) return DD_OK;
+  cudaError_t e = cudaGraphExecDestroy(g->exec);
+  delete g;
+  if (e != cudaSuccess) return cuda_fail(e, "destroy block graph");
+  return DD_OK;
+}
+
 size_t dd_denoise_block_adaptive_workspace(const dd_attn_desc* desc,
                                            const int32_t* cu_prefix_host, int vocab) {
   int64_t total = 0;

@@ -229,6 +229,34 @@ DD_API dd_status dd_denoise_block(const dd_attn_desc* desc, int steps, const voi
                            int32_t* canvas, int32_t* canvas_history, float* conf_steps,
                            void* workspace, size_t workspace_bytes, dd_stream_t stream);
 
+/* A block loop captured once and replayed with a single launch.  The loop
+ * takes 4 kernels per step (attention, split combine, sampler pass, row
+ * merge).  At about 0.1 ms per step, launching them one by one from the
+ * host shows up in the block time, and a graph removes that cost.
+ *   dd_denoise_block_graph_create captures one dd_denoise_block call with
+ *     exactly these arguments (the same as dd_denoise_block, without the
+ *     stream) into a CUDA graph and instantiates it.  It validates the
+ *     arguments like dd_denoise_block, launches nothing, and on success
+ *     stores a handle in *out (NULL on failure).  The handle is a small host
+ *     object; no device memory is allocated.
+ *   dd_denoise_block_graph_launch replays the captured call on `stream`:
+ *     the same pointers, sizes, rates, temperatures, seed and step0.  New
+ *     inputs enter by overwriting the contents of the captured buffers.
+ *     Every buffer must stay allocated while the handle exists.  Replays
+ *     that may overlap in time must not share a workspace.
+ *   dd_denoise_block_graph_destroy frees the handle (NULL is accepted).
+ * A replay gives results identical to the eager call. */
+typedef struct dd_block_graph_st* dd_block_graph;
+DD_API dd_status dd_denoise_block_graph_create(
+    dd_block_graph* out, const dd_attn_desc* desc, int steps, const void* q_steps,
+    const void* kc_steps, const void* vc_steps, const void* k_prefix, const void* v_prefix,
+    const int32_t* cu_prefix, const int32_t* cu_prefix_host, void* attn_out,
+    const void* logits_steps, int vocab, const float* rate_host, const float* temperature_host,
+    uint64_t seed, uint32_t step0, int32_t* canvas, int32_t* canvas_history, float* conf_steps,
+    void* workspace, size_t workspace_bytes);
+DD_API dd_status dd_denoise_block_graph_launch(dd_block_graph graph, dd_stream_t stream);
+DD_API dd_status dd_denoise_block_graph_destroy(dd_block_graph graph);
+
 /* dd_sample_renoise without a workspace, for callers that may not allocate
  * device memory (code inside another framework's memory pool or fixed
  * budget, plugin or callback code handed only its input and output

@@ -146,6 +146,19 @@ def test_fp8_attention_rejects_bad_arguments(lib):
     assert dd.canvas_attn_workspace_bytes(e4, cu) > 0
 
 
+def test_block_graph_rejects_bad_handles(lib):
+    d = _desc()
+    cu = _cu([16])
+    r = np.zeros(1, np.float32)
+    args = [ctypes.byref(d), 1, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+            cu.ctypes.data_as(ctypes.c_void_p), FAKE, FAKE, 1024,
+            r.ctypes.data_as(ctypes.c_void_p), r.ctypes.data_as(ctypes.c_void_p), 0, 0, FAKE,
+            None, None, FAKE, 16]
+    assert lib.dd_denoise_block_graph_create(None, *args) == 1       # no handle slot
+    assert lib.dd_denoise_block_graph_launch(None, None) == 1
+    assert lib.dd_denoise_block_graph_destroy(None) == 0
+
+
 def test_block_rejects_bad_arguments(lib):
     d = _desc()
     cu = _cu([16])

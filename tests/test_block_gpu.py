@@ -73,3 +73,37 @@ def test_block_without_history_buffers():
     tok = out["canvas"].cpu().numpy()
     bad = (tok != ref["tokens"]) & (ref["gap"] >= 1e-5)
     assert not bad.any()
+
+
+def test_block_graph_replays_the_eager_loop(block12):
+    """dd_denoise_block_graph: one capture, replays identical to the eager
+    loop, including after new inputs are written into the captured buffers,
+    and with the launch count of the eager loop."""
+    w, qs, kcs, vcs, ls, kp, vp, cu = block12
+    eager = dd.denoise_block(qs, kcs, vcs, kp, vp, cu.to(DEV), ls, w.rates, w.temperatures,
+                             seed=w.seed, cu_prefix_host=cu)
+    torch.cuda.synchronize()
+    qb, lb = qs.clone(), ls.clone()
+    g = dd.denoise_block_graph(qb, kcs, vcs, kp, vp, cu.to(DEV), lb, w.rates, w.temperatures,
+                               seed=w.seed, cu_prefix_host=cu)
+    torch.cuda.synchronize()
+    dd.reset_launch_count()
+    for _ in range(2):
+        out = g.launch()
+        torch.cuda.synchronize()
+        assert torch.equal(out["canvas_history"], eager["canvas_history"])
+        assert torch.equal(out["conf_steps"], eager["conf_steps"])
+        assert torch.equal(out["attn_out"], eager["attn_out"])
+    assert dd.launch_count() == 2 * 4 * w.steps
+    # new inputs through the captured buffers: the step-order reversed
+    qb.copy_(qs.flip(0))
+    lb.copy_(ls.flip(0))
+    ref = dd.denoise_block(qs.flip(0).contiguous(), kcs, vcs, kp, vp, cu.to(DEV),
+                           ls.flip(0).contiguous(), w.rates, w.temperatures, seed=w.seed,
+                           cu_prefix_host=cu)
+    out = g.launch()
+    torch.cuda.synchronize()
+    assert torch.equal(out["canvas_history"], ref["canvas_history"])
+    assert torch.equal(out["attn_out"], ref["attn_out"])
+    g.destroy()
+    dd.query_device_error(g.tensors["workspace"])
