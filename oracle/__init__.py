@@ -33,6 +33,10 @@ Parity status per function (what pins it; tests/test_oracle_*.py):
                                rule pinned above.
   denoise_block             -- a loop of the two pinned functions (plain
                                Python), checked for step0-restart identity.
+  soft_embed                -- pure-Python brute force, closed forms
+                               (constant logits -> mean embedding, one
+                               dominant logit -> its embedding row),
+                               temperature scaling, linearity in E.
 """
 from __future__ import annotations
 
@@ -296,6 +300,46 @@ def stop_check(entropy, pred, pred_prev, canvas: int, threshold: float = 0.005):
     done = np.empty(B, np.uint8)
     lib.oracle_stop_check(_ptr(h), _ptr(pr), _ptr(pp), B, canvas, float(threshold), _ptr(done))
     return done
+
+
+# ---------------------------------------- self-conditioning soft embedding
+
+def _f64(x) -> np.ndarray:
+    """float64 copy of a bf16 or float32 tensor / array (exact decoding)."""
+    a, dt = _raw(x)
+    if dt == BF16:
+        return (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return a.astype(np.float64)
+
+
+def soft_embed(logits, tau: float, emb, rows=None, cols=None, v_chunk: int = 16384):
+    """The self-conditioning signal before its MLP ("DiffusionGemma Technical
+    Report" (paperfeed review), "The mechanism", self-conditioning
+    paragraph): the step's predicted token distribution of each position,
+    p0 = softmax(logits / tau) (the distribution the sampler draws from),
+    pushed through the embedding matrix E:
+        out[r, :] = sum_v p0[r, v] E[v, :].
+    Plain float64: logits [R, V] and E [V, d] (bf16 or float32, decoded
+    exactly); the softmax with its row maximum subtracted; the sum over v in
+    chunks of v_chunk (a plain matrix product per chunk).  rows / cols
+    restrict the output rows / embedding columns computed."""
+    lg = _f64(logits)
+    if rows is not None:
+        lg = lg[np.asarray(rows)]
+    z = lg / float(tau)
+    z -= z.max(axis=1, keepdims=True)
+    p = np.exp(z)
+    p /= p.sum(axis=1, keepdims=True)
+    e_raw, e_dt = _raw(emb)
+    if cols is not None:
+        e_raw = e_raw[:, np.asarray(cols)]
+    out = np.zeros((p.shape[0], e_raw.shape[1]), np.float64)
+    for v0 in range(0, p.shape[1], v_chunk):
+        blk = e_raw[v0:v0 + v_chunk]
+        e = ((blk.astype(np.uint32) << 16).view(np.float32).astype(np.float64) if e_dt == BF16
+             else blk.astype(np.float64))
+        out += p[:, v0:v0 + v_chunk] @ e
+    return out
 
 
 # --------------------------------------------------------- the block loop

@@ -184,6 +184,14 @@ def logits(w: Workload, step: int = 0, device="cpu", rows: Optional[int] = None)
     return x.to(w.torch_dtype)
 
 
+def embedding(w: Workload, d: Optional[int] = None, device="cpu"):
+    """A synthetic embedding matrix E [V, d], i.i.d. N(0, 1), in the
+    workload's dtype.  d defaults to Hq * D, the model width the attention
+    geometry implies (the pages do not state it)."""
+    d = w.heads_q * w.head_dim if d is None else d
+    return _normal(w, "embedding", 0, (w.vocab, d), 1.0, device)
+
+
 def all_steps(w: Workload, device="cpu"):
     """Per-step canvas Q/K/V and logits for every step of the workload."""
     qs, kcs, vcs, ls = [], [], [], []
