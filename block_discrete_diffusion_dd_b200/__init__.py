@@ -33,6 +33,7 @@ EXPORTS = (
     "dd_entropy_accept", "dd_stop_check", "dd_denoise_block_adaptive_workspace",
     "dd_denoise_block_adaptive", "dd_canvas_attn_fp8", "dd_denoise_block_graph_create",
     "dd_denoise_block_graph_launch", "dd_denoise_block_graph_destroy",
+    "dd_soft_embed_workspace", "dd_soft_embed",
 )
 
 
@@ -102,6 +103,10 @@ def load() -> ctypes.CDLL:
     lib.dd_denoise_block_graph_launch.argtypes = [P, P]
     lib.dd_denoise_block_graph_destroy.restype = i32
     lib.dd_denoise_block_graph_destroy.argtypes = [P]
+    lib.dd_soft_embed_workspace.restype = sz
+    lib.dd_soft_embed_workspace.argtypes = [i32, i32, i32]
+    lib.dd_soft_embed.restype = i32
+    lib.dd_soft_embed.argtypes = [P, i32, i32, i32, i64, ctypes.c_float, P, i32, P, P, sz, P]
     f32 = ctypes.c_float
     lib.dd_entropy_accept.restype = i32
     lib.dd_entropy_accept.argtypes = [P, P, i32, i32, i32, f32, u64, u32, u32, P, P, P]
@@ -334,6 +339,29 @@ def denoise_block(q_steps, kc_steps, vc_steps, kp, vp, cu_prefix, logits_steps,
         _ptr(workspace), workspace.numel(), _stream(stream)))
     return {"attn_out": attn_out, "canvas": canvas, "canvas_history": canvas_history,
             "conf_steps": conf_steps}
+
+
+def soft_embed_workspace_bytes(rows: int, vocab: int, d: int) -> int:
+    return int(load().dd_soft_embed_workspace(rows, vocab, d))
+
+
+def soft_embed(logits: torch.Tensor, temperature: float, emb: torch.Tensor, out=None,
+               rows: Optional[int] = None, vocab: Optional[int] = None,
+               row_stride: Optional[int] = None, workspace=None, stream=None) -> torch.Tensor:
+    """dd_soft_embed: softmax(logits / temperature) @ emb, bf16 [rows, d]."""
+    lib = load()
+    R = logits.shape[0] if rows is None else rows
+    V = logits.shape[-1] if vocab is None else vocab
+    stride = logits.stride(0) if row_stride is None else row_stride
+    d = emb.shape[-1]
+    if out is None:
+        out = torch.empty((R, d), dtype=torch.bfloat16, device=logits.device)
+    if workspace is None:
+        workspace = new_workspace(soft_embed_workspace_bytes(R, V, d), logits.device, stream)
+    _check(lib.dd_soft_embed(_ptr(logits), _dtype_code(logits), R, V, stride, float(temperature),
+                             _ptr(emb), d, _ptr(out), _ptr(workspace), workspace.numel(),
+                             _stream(stream)))
+    return out
 
 
 class BlockGraph:

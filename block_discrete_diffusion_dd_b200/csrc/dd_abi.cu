@@ -432,6 +432,51 @@ size_t adaptive_ws_layout(const dd_attn_desc* desc, int64_t total, const int32_t
 }
 }  // namespace
 
+size_t dd_soft_embed_workspace(int rows, int vocab, int d) {
+  if (rows < 0 || vocab < 1 || d < 64 || d % 64 != 0) return 0;
+  return kHeaderBytes + soft_embed_scratch_bytes(rows, vocab, d);
+}
+
+dd_status dd_soft_embed(const void* logits, dd_dtype dtype, int rows, int vocab,
+                        int64_t row_stride, float temperature, const void* emb, int d, void* out,
+                        void* workspace, size_t workspace_bytes, dd_stream_t stream) {
+  g_last_error.clear();
+  if (dtype != DD_BF16 && dtype != DD_F32 && dtype != DD_E4M3)
+    return fail(DD_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+  if (dtype != DD_BF16) return fail(DD_ERR_UNSUPPORTED, "soft embedding takes bf16 logits and E");
+  if (rows < 0 || vocab < 1) return fail(DD_ERR_INVALID_ARG, "rows=%d vocab=%d", rows, vocab);
+  if (d < 64 || d % 64 != 0) return fail(DD_ERR_UNSUPPORTED, "d=%d (a multiple of 64)", d);
+  if (row_stride < vocab || row_stride % 8 != 0)
+    return fail(DD_ERR_INVALID_ARG, "row_stride (%lld) must be >= vocab and a multiple of 8",
+                (long long)row_stride);
+  if (!std::isfinite(temperature) || temperature < 1e-3f)
+    return fail(DD_ERR_INVALID_ARG, "temperature must be finite and >= 1e-3");
+  if (rows == 0) return DD_OK;
+  if (rows > 65535 * 256) return fail(DD_ERR_UNSUPPORTED, "rows=%d", rows);
+  if (!logits || !emb || !out) return fail(DD_ERR_INVALID_ARG, "NULL tensor pointer");
+  if (!aligned16(logits) || !aligned16(emb) || !aligned16(out))
+    return fail(DD_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return fail(DD_ERR_WORKSPACE, "workspace must be non-NULL and 256-byte aligned");
+  const size_t need = kHeaderBytes + soft_embed_scratch_bytes(rows, vocab, d);
+  if (workspace_bytes < need)
+    return fail(DD_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", workspace_bytes, need);
+  SoftEmbedArgs a{};
+  a.logits = logits;
+  a.rows = rows;
+  a.vocab = vocab;
+  a.row_stride = row_stride;
+  a.temperature = temperature;
+  a.emb = emb;
+  a.d = d;
+  a.out = out;
+  a.err = static_cast<uint32_t*>(workspace);
+  a.scratch = static_cast<uint8_t*>(workspace) + kHeaderBytes;
+  cudaError_t e = launch_soft_embed(a, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "soft embedding");
+  return DD_OK;
+}
+
 // A captured block loop: one instantiated CUDA graph and the number of
 // library kernels one replay launches.
 struct dd_block_graph_st {

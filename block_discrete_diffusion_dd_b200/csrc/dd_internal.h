@@ -100,6 +100,27 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t stream);
 size_t attn_simt_scratch_bytes(const AttnArgs& a);
 cudaError_t launch_attn_simt(const AttnArgs& a, cudaStream_t stream);
 
+// Self-conditioning soft embedding (dd_soft_embed.cu): bf16 logits [rows, V]
+// (row stride a multiple of 8), bf16 E [V, d] (d a multiple of 64), bf16 out
+// [rows, d]; 16-byte aligned pointers, validated by the ABI layer.
+struct SoftEmbedArgs {
+  const void* logits;
+  int rows, vocab;
+  int64_t row_stride;
+  float temperature;
+  const void* emb;
+  int d;
+  void* out;
+  uint32_t* err;
+  void* scratch;  // soft_embed_scratch_bytes
+};
+struct SoftEmbedPlan {
+  int ksteps, ksteps_per_split, splits, grid_x, grid_z;
+};
+SoftEmbedPlan soft_embed_plan(int rows, int vocab, int d);
+size_t soft_embed_scratch_bytes(int rows, int vocab, int d);
+cudaError_t launch_soft_embed(const SoftEmbedArgs& a, cudaStream_t stream);
+
 // Launch accounting (per host thread).
 void note_launch();
 

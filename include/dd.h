@@ -257,6 +257,34 @@ DD_API dd_status dd_denoise_block_graph_create(
 DD_API dd_status dd_denoise_block_graph_launch(dd_block_graph graph, dd_stream_t stream);
 DD_API dd_status dd_denoise_block_graph_destroy(dd_block_graph graph);
 
+/* Self-conditioning soft embedding ("DiffusionGemma Technical Report",
+ * "The mechanism", self-conditioning paragraph: the previous step's
+ * predicted token distribution, pushed through the embedding matrix E, is
+ * the input of a small MLP that conditions the next step).  This computes
+ * the contraction; the MLP (7.8M parameters, weights not public) is not
+ * part of the library:
+ *   out[r, :] = sum_v softmax(logits[r, :] / temperature)_v * E[v, :]
+ * Arguments:
+ *   logits       bf16 [rows, vocab] with row_stride elements between rows
+ *                (row_stride >= vocab, a multiple of 8)
+ *   dtype        DD_BF16 (the only type taken; others DD_ERR_UNSUPPORTED)
+ *   temperature  tau >= 1e-3 (the distribution the sampler draws from)
+ *   emb          E, bf16 [vocab, d], row-major; d a multiple of 64
+ *                (else DD_ERR_UNSUPPORTED)
+ *   out          bf16 [rows, d]
+ *   workspace    >= dd_soft_embed_workspace(rows, vocab, d) bytes, 256-byte
+ *                aligned (row log-sum-exps and fp32 partial sums)
+ * The probabilities are rounded to bf16 for the tensor-core product
+ * (relative error <= 2^-8 each); accumulation is fp32; the partial sums
+ * of the vocabulary splits are added in a fixed order (the result does not
+ * depend on scheduling).  Returns 0 from the workspace query on invalid
+ * arguments. */
+DD_API size_t dd_soft_embed_workspace(int rows, int vocab, int d);
+DD_API dd_status dd_soft_embed(const void* logits, dd_dtype dtype, int rows, int vocab,
+                               int64_t row_stride, float temperature, const void* emb, int d,
+                               void* out, void* workspace, size_t workspace_bytes,
+                               dd_stream_t stream);
+
 /* dd_sample_renoise without a workspace, for callers that may not allocate
  * device memory (code inside another framework's memory pool or fixed
  * budget, plugin or callback code handed only its input and output

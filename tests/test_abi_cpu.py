@@ -146,6 +146,30 @@ def test_fp8_attention_rejects_bad_arguments(lib):
     assert dd.canvas_attn_workspace_bytes(e4, cu) > 0
 
 
+def _soft(lib, rows=4, vocab=100, stride=104, temp=1.0, d=128, dtype=0, ptr=FAKE, ws=FAKE,
+          ws_bytes=1 << 30):
+    return lib.dd_soft_embed(ptr, dtype, rows, vocab, stride, temp, ptr, d, ptr, ws, ws_bytes,
+                             None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dtype=1), 2), (dict(dtype=9), 1), (dict(d=96), 2), (dict(d=0), 2), (dict(stride=99), 1),
+    (dict(stride=101), 1), (dict(temp=0.0), 1), (dict(temp=float("inf")), 1), (dict(vocab=0), 1),
+    (dict(rows=-1), 1), (dict(ptr=None), 1), (dict(ptr=ctypes.c_void_p((1 << 20) + 8)), 1),
+    (dict(ws=None), 3), (dict(ws_bytes=512), 3),
+])
+def test_soft_embed_rejects_bad_arguments(lib, kw, code):
+    assert _soft(lib, **kw) == code
+    assert dd.last_error()
+
+
+def test_soft_embed_workspace_and_empty_call(lib):
+    assert _soft(lib, rows=0, ptr=None, ws=None) == 0
+    assert lib.dd_soft_embed_workspace(256, 262144, 100) == 0
+    n = lib.dd_soft_embed_workspace(256, 262144, 2048)
+    assert n >= 256 + 256 * 4 + 256 * 2048 * 4   # at least one split of fp32 partials
+
+
 def test_block_graph_rejects_bad_handles(lib):
     d = _desc()
     cu = _cu([16])
