@@ -403,6 +403,59 @@ def run_attn_e4m3(w, reps: int = 50):
     }
 
 
+def run_soft_embed(w, reps: int = 30):
+    """The self-conditioning soft embedding softmax(logits / tau) E on the
+    workload's logits and a synthetic E [V, Hq * D] (dd_soft_embed: row
+    log-sum-exp, split-K tensor-core product, fixed-order split reduction):
+    device time of one call, CUDA events around the call only, L2 flushed
+    before every call, median of `reps`."""
+    import block_discrete_diffusion_dd_b200 as dd
+    dev = torch.device("cuda", torch.cuda.current_device())
+    lg = workloads.logits(w, 0, device=dev)
+    E = workloads.embedding(w, device=dev)
+    d = E.shape[1]
+    ws = dd.new_workspace(dd.soft_embed_workspace_bytes(w.rows, w.vocab, d), dev)
+    out = torch.empty((w.rows, d), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    time.sleep(0.3)
+    t_wall0 = time.time()
+    for _ in range(3):
+        dd.soft_embed(lg, w.temperatures[0], E, out=out, workspace=ws)
+    ts = []
+    for _ in range(reps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        dd.soft_embed(lg, w.temperatures[0], E, out=out, workspace=ws)
+        e1.record()
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    t_wall1 = time.time()
+    time.sleep(0.2)
+    clocks.stop()
+    dd.query_device_error(ws)
+    ms = statistics.median(ts)
+    hbm, tf_burst, tf_sus, src = _peaks()
+    flops = 2 * w.rows * w.vocab * d
+    nbytes = (w.vocab * d + w.rows * w.vocab + w.rows * d) * 2
+    gbs, tfs = nbytes / ms / 1e6, flops / ms / 1e9
+    return {
+        "metric": "self-conditioning soft embedding softmax(logits / tau) E", "value": ms * 1e3,
+        "unit": "us per call", "higher_is_better": False, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "rows": w.rows, "vocab": w.vocab, "d": d,
+                   "temperature": w.temperatures[0],
+                   "l2": "flushed (256 MB write) before every call"},
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
+                     "frac": gbs / hbm, "bytes": nbytes, "peak_source": src},
+        "tensor": {"achieved": tfs, "peak": tf_burst, "unit": "TFLOP/s", "frac": tfs / tf_burst,
+                   "flops": flops},
+        "timing": f"median of {reps} calls, CUDA events around each call",
+        "clocks": clocks.summary(t_wall0, t_wall1),
+    }
+
+
 # The sampler's arithmetic ceiling: per warp-item of 256 logits the scan
 # issues 2 Philox4x32-10 blocks x 18 IMAD.WIDE (two of the 20 products per
 # block are row-invariant and hoisted) plus 16 packed fp32 ops, all on the
@@ -704,6 +757,8 @@ def main():
                     help="time the pages' adaptive block loop instead (one JSON line)")
     ap.add_argument("--attn-e4m3", action="store_true",
                     help="time canvas attention on E4M3 inputs beside bf16 (one JSON line)")
+    ap.add_argument("--soft-embed", action="store_true",
+                    help="time the self-conditioning soft embedding (one JSON line)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     w = workloads.WORKLOADS[args.workload]
@@ -722,6 +777,9 @@ def main():
         return
     if args.attn_e4m3:
         print(json.dumps(run_attn_e4m3(w)), flush=True)
+        return
+    if args.soft_embed:
+        print(json.dumps(run_soft_embed(w)), flush=True)
         return
     dist, rank, world, local_rank = _dist()
     if world != args.gpus and rank == 0:

@@ -85,42 +85,66 @@ __device__ __forceinline__ void lse_merge(float& m, float& s, float m2, float s2
   m = mn;
 }
 
-// lse2[r] = log2 sum_v 2^(z_v c), c = log2(e) / tau: one pass over the row
-// with 16-byte loads; each thread keeps a running maximum m and the sum of
-// 2^(t - m), rescaled when m grows; the pairs are merged across the CTA.
-__global__ void __launch_bounds__(256)
+// lse2[r] = log2 sum_v 2^(z_v c), c = log2(e) / tau: one pass over the row.
+// Each thread loads four 16-byte vectors at a time (32 entries, all four
+// requests in flight before the arithmetic), keeps a running maximum m and
+// the sum of 2^(t - m), rescaled once per 32 entries when m grows; the
+// pairs are merged across the CTA.
+constexpr int LSE_THREADS = 512;
+__device__ __forceinline__ void lse_vec8(uint4 w, float c, float (&t)[8]) {
+  const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    t[2 * k] = bf16lo(ww[k]) * c;
+    t[2 * k + 1] = bf16hi(ww[k]) * c;
+  }
+}
+
+template <int U>
+__device__ __forceinline__ void lse_block(const uint4 (&w)[U], float c, float& m, float& s) {
+  float t[U][8];
+  float mx = -INFINITY;
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    lse_vec8(w[u], c, t[u]);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) mx = fmaxf(mx, t[u][k]);
+  }
+  const float mn = fmaxf(m, mx);
+  if (mn == -INFINITY) return;
+  float acc = (m == mn) ? s : s * ex2_approx(m - mn);
+#pragma unroll
+  for (int u = 0; u < U; ++u)
+#pragma unroll
+    for (int k = 0; k < 8; ++k) acc += ex2_approx(t[u][k] - mn);
+  s = acc;
+  m = mn;
+}
+
+__global__ void __launch_bounds__(LSE_THREADS)
     row_lse_kernel(const __nv_bfloat16* __restrict__ logits, int64_t row_stride, int vocab,
                    float c, float* __restrict__ lse2) {
   pdl_wait();
   pdl_trigger();
-  __shared__ float red_m[8], red_s[8];
+  __shared__ float red_m[LSE_THREADS / 32], red_s[LSE_THREADS / 32];
   const int r = blockIdx.x;
   const __nv_bfloat16* row = logits + (int64_t)r * row_stride;
   const uint4* rv = reinterpret_cast<const uint4*>(row);
   const int nvec = vocab / 8;
+  constexpr int U = 4;
   float m = -INFINITY, s = 0.f;
-#pragma unroll 4
-  for (int i = threadIdx.x; i < nvec; i += blockDim.x) {
-    const uint4 w = __ldcs(rv + i);
-    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-    float t[8];
+  int i = threadIdx.x;
+  for (; i + (U - 1) * LSE_THREADS < nvec; i += U * LSE_THREADS) {
+    uint4 w[U];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      t[2 * k] = bf16lo(ww[k]) * c;
-      t[2 * k + 1] = bf16hi(ww[k]) * c;
-    }
-    float mx = fmaxf(fmaxf(fmaxf(t[0], t[1]), fmaxf(t[2], t[3])),
-                     fmaxf(fmaxf(t[4], t[5]), fmaxf(t[6], t[7])));
-    const float mn = fmaxf(m, mx);
-    if (mn != -INFINITY) {
-      float acc = (m == mn) ? s : s * ex2_approx(m - mn);
-#pragma unroll
-      for (int k = 0; k < 8; ++k) acc += ex2_approx(t[k] - mn);
-      s = acc;
-      m = mn;
-    }
+    for (int u = 0; u < U; ++u) w[u] = __ldcs(rv + i + u * LSE_THREADS);
+    lse_block<U>(w, c, m, s);
   }
-  for (int v = nvec * 8 + threadIdx.x; v < vocab; v += blockDim.x)
+  for (; i < nvec; i += LSE_THREADS) {
+    const uint4 w[1] = {__ldcs(rv + i)};
+    lse_block<1>(w, c, m, s);
+  }
+  for (int v = nvec * 8 + threadIdx.x; v < vocab; v += LSE_THREADS)
     lse_merge(m, s, __bfloat162float(row[v]) * c, 1.f);
   for (int o = 16; o > 0; o >>= 1) {
     const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
@@ -135,7 +159,7 @@ __global__ void __launch_bounds__(256)
   __syncthreads();
   if (threadIdx.x == 0) {
     float mm = red_m[0], ss = red_s[0];
-    for (int i = 1; i < 8; ++i) lse_merge(mm, ss, red_m[i], red_s[i]);
+    for (int k = 1; k < LSE_THREADS / 32; ++k) lse_merge(mm, ss, red_m[k], red_s[k]);
     lse2[r] = mm + __log2f(ss);
   }
 }
@@ -457,7 +481,7 @@ cudaError_t launch_soft_embed(const SoftEmbedArgs& a, cudaStream_t stream) {
       scratch + (((size_t)a.rows * sizeof(float) + 255) & ~static_cast<size_t>(255)));
   const float c = (float)(1.4426950408889634 / (double)a.temperature);
 
-  cudaError_t e = launch_pdl(row_lse_kernel, dim3(a.rows), dim3(256), 0, stream,
+  cudaError_t e = launch_pdl(row_lse_kernel, dim3(a.rows), dim3(LSE_THREADS), 0, stream,
                              static_cast<const __nv_bfloat16*>(a.logits), a.row_stride, a.vocab,
                              c, lse2);
   note_launch();
