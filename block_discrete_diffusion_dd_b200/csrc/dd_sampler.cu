@@ -614,17 +614,21 @@ __global__ void __launch_bounds__(kScanThreads, 3)
 }
 
 // Merge of a row's chunk partials (in chunk order), the argmax from the row
-// key, then the re-noise draw.  One warp per row.  Clears the ticket counter
-// and the row key for the next call.
+// key, then the re-noise draw.  One warp per row.  Clears the ticket counter,
+// the row key and the row's chunk records for the next call: a completed
+// call leaves every byte of state and records it used at zero, so calls of
+// other shapes that share the workspace (and lay these out differently)
+// start from a clear state.  An argmax index outside the row (a state the
+// caller did not clear) is replaced by 0 and latched as a bounds error.
 template <typename T>
 __global__ void __launch_bounds__(128)
     sample_merge_kernel(const T* __restrict__ logits, int64_t row_stride, int rows, int vocab,
                         int nck, float inv_tau, float rate, uint64_t seed, uint32_t step,
-                        uint32_t row_offset, const float4* __restrict__ recs,
+                        uint32_t row_offset, float4* __restrict__ recs,
                         unsigned long long* __restrict__ row_key, uint32_t* __restrict__ ticket,
                         int32_t* __restrict__ tokens, int32_t* __restrict__ pred,
                         float* __restrict__ conf, float* __restrict__ entropy,
-                        uint8_t* __restrict__ renoised) {
+                        uint8_t* __restrict__ renoised, uint32_t* __restrict__ err) {
   pdl_wait();
   pdl_trigger();
   if (blockIdx.x == 0 && threadIdx.x == 0) *ticket = 0u;
@@ -633,14 +637,20 @@ __global__ void __launch_bounds__(128)
   if (row >= rows) return;
   SumState st{-INFINITY, 0.f, 0.f};
   for (int c = lane; c < nck; c += 32) {
-    const float4 r = recs[(int64_t)row * nck + c];
+    float4* rc = recs + (int64_t)row * nck + c;
+    const float4 r = *rc;
+    *rc = make_float4(0.f, 0.f, 0.f, 0.f);
     merge_sums(st, SumState{r.x, r.y, r.z});
   }
   warp_merge_sums(st);
   if (lane != 0) return;
   const unsigned long long key = row_key[(size_t)row * kKeyStride];
   row_key[(size_t)row * kKeyStride] = 0ull;
-  const int p = key ? key_index(key) : 0;
+  int p = key ? key_index(key) : 0;
+  if ((unsigned)p >= (unsigned)vocab) {
+    p = 0;
+    atomicOr(err, kDevErrBounds);
+  }
   const float x = fmaxf((float)logits[(int64_t)row * row_stride + p], kFloorLogit);
   const float c2 = inv_tau * kLog2e;
   const float cf = ex2_approx(fmaf(x, c2, -st.m)) / st.s;
@@ -722,8 +732,8 @@ cudaError_t launch_sampler_v(const SamplerArgs& a, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   e = launch_pdl(sample_merge_kernel<T>, dim3((a.rows + 3) / 4), dim3(128), 0, stream, lg,
                  a.row_stride, a.rows, a.vocab, p.nck, a.inv_tau, a.rate, a.seed, a.step,
-                 a.row_offset, (const float4*)recs, s.row_key, s.ticket, a.tokens, a.pred,
-                 a.conf, a.entropy, a.renoised);
+                 a.row_offset, recs, s.row_key, s.ticket, a.tokens, a.pred, a.conf, a.entropy,
+                 a.renoised, a.err);
   note_launch();
   return e;
 }

@@ -29,8 +29,9 @@
  *     workspace and read back by dd_query_device_error.
  *   - A workspace must be cleared once with dd_workspace_init before its
  *     first use.  The sampler keeps a small state in it (a work counter and
- *     per-row maxima) that every completed call leaves cleared; after a call
- *     that failed on the device, clear the workspace again.
+ *     per-row maxima) and per-chunk records, all of which every completed
+ *     call leaves cleared, so calls of any shape may share a workspace;
+ *     after a call that failed on the device, clear the workspace again.
  *   - There is no CPU fallback: if the CUDA kernels cannot run, calls fail.
  */
 #ifndef DD_H_

@@ -146,6 +146,24 @@ def test_workspace_reuse_leaves_state_clear():
     check_sampler(b1, oracle.sample_renoise(b_lg.cpu(), 0.7, 0.5, 4, 5))
 
 
+def test_workspace_shared_across_row_counts_with_negative_logits():
+    """A call with fewer rows lays its chunk records over the row maxima of
+    a call with more rows; the records are cleared at the end of every call,
+    so a later call whose best scores are all far below zero still starts
+    from a clear state (a leftover value would outrank every real score)."""
+    few = _gen(40, 50000, 2.0, torch.float32, seed=31)
+    neg = (_gen(256, 8192, 1.0, torch.float32, seed=32) - 40.0).contiguous()
+    ws = dd.new_workspace(max(dd.sample_workspace_bytes(40, 50000, torch.float32),
+                              dd.sample_workspace_bytes(256, 8192, torch.float32)))
+    _run(few, 1.0, 0.5, 1, 2, workspace=ws)
+    got = _run(neg, 1.0, 0.0, 3, 4, workspace=ws)
+    dd.query_device_error(ws)
+    fresh = _run(neg, 1.0, 0.0, 3, 4)
+    for k in got:
+        assert torch.equal(got[k], fresh[k]), k
+    check_sampler(got, oracle.sample_renoise(neg.cpu(), 1.0, 0.0, 3, 4))
+
+
 def test_large_seed_and_step():
     lg = _gen(16, 4096, 3.0, torch.bfloat16, seed=9)
     seed, step = 0xDEADBEEFCAFEF00D, 0xFFFFFFF0
