@@ -30,8 +30,12 @@
  *   - A workspace must be cleared once with dd_workspace_init before its
  *     first use.  The sampler keeps a small state in it (a work counter and
  *     per-row maxima) and per-chunk records, all of which every completed
- *     call leaves cleared, so calls of any shape may share a workspace;
- *     after a call that failed on the device, clear the workspace again.
+ *     call leaves cleared, so sampler calls of any shape may share a
+ *     workspace.  A dd_denoise_block or dd_denoise_block_adaptive workspace
+ *     also holds attention scratch that calls do not clear: it serves one
+ *     geometry (batch, canvas, heads, prefix lengths, vocabulary); clear it
+ *     with dd_workspace_init before using it for another.  After a call
+ *     that failed on the device, clear the workspace again.
  *   - There is no CPU fallback: if the CUDA kernels cannot run, calls fail.
  */
 #ifndef DD_H_
