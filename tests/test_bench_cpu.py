@@ -1,0 +1,47 @@
+"""Host-side pieces of bench.py that need no GPU: the sampler's arithmetic
+ceiling (the denominator beside the HBM fraction) and the reading of the
+committed per-launch DRAM traffic, which must go to None for a kernel whose
+source changed after the counters were taken."""
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+
+
+def test_sampler_alu_ceiling_arithmetic():
+    # 148 SMs x 4 sub-partitions; per warp-item of 256 bf16 logits (512 B)
+    # 36 IMAD.WIDE x 4 + 16 packed fp32 x 2 = 176 heavy-pipe cycles
+    c = bench._sampler_alu_ceiling(1000.0, 1965.0)
+    expect = 592 * 1965e6 / 176 * 512 / 1e9
+    assert c["heavy_cycles_per_256_logits"] == 176
+    assert c["peak"] == pytest.approx(expect, rel=1e-12)
+    assert c["frac"] == pytest.approx(1000.0 / expect, rel=1e-12)
+    assert bench._sampler_alu_ceiling(1000.0, None) is None
+
+
+def test_profile_traffic_tracks_the_source(tmp_path, monkeypatch):
+    src = tmp_path / "block_discrete_diffusion_dd_b200" / "csrc"
+    src.mkdir(parents=True)
+    (src / "k.cu").write_text("kernel source\n")
+    (tmp_path / "profiles").mkdir()
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    sha = bench._source_sha("k.cu")
+    (tmp_path / "profiles" / "traffic.txt").write_text(
+        "# comment line\n"
+        f"good 123456 k.cu {sha}\n"
+        "stale 999 k.cu 0000000000000000\n")
+    t = bench._profile_traffic()
+    assert t["good"] == 123456.0
+    assert t["stale"] is None
+
+
+def test_committed_traffic_entries_parse():
+    t = bench._profile_traffic()
+    for k in ("sampler", "attention", "attention_e4m3", "soft_embed"):
+        assert k in t
