@@ -13,14 +13,15 @@
 //   soft_embed_kernel   split-K tcgen05 GEMM.  A CTA owns 256 rows (two
 //                       128-row MMA tiles), 256 embedding columns and a range
 //                       of the vocabulary.  Per 32-entry vocabulary step, TMA
-//                       brings the logits tile and the E tile; eight warps
-//                       turn the logits into probabilities
-//                       2^(z log2(e)/tau - lse) and write them as bf16
-//                       straight into the swizzled A-operand layout; one
-//                       elected lane of the MMA warp multiplies them with E
-//                       (B operand, MN-major) into fp32 accumulators in
-//                       tensor memory (2 x 256 columns).  The same warps
-//                       write the CTA's fp32 partial at the end;
+//                       brings the logits tile and the E tile (a 4-deep
+//                       ring); sixteen warps (two threads per row) turn the
+//                       logits into probabilities 2^(z log2(e)/tau - lse)
+//                       and write them as bf16 straight into the swizzled
+//                       A-operand layout; one elected lane of the MMA warp
+//                       multiplies them with E (B operand, MN-major) into
+//                       fp32 accumulators in tensor memory (2 x 256
+//                       columns).  Eight of those warps write the CTA's fp32
+//                       partial at the end;
 //   soft_embed_reduce   sums the partials of the vocabulary splits in a
 //                       fixed order and rounds to bf16.
 // Every mbarrier wait is bounded; on expiry the CTA latches an error word,
