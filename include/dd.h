@@ -321,9 +321,9 @@ DD_API dd_status dd_sample_renoise_noalloc(const void* logits, dd_dtype dtype, i
  * positions accepted greedily from lowest to highest entropy until a
  * cumulative entropy budget (b = 0.1) is exhausted and the rest re-noised to
  * uniform random tokens, early halt when the mean canvas entropy is below
- * 0.005 and the prediction is stable across two steps.  The benchmark spec's
- * scheduled-rate loop (dd_denoise_block) stays the default; these calls are
- * the pages' alternative. */
+ * 0.005 and the prediction is stable across two steps.  The scheduled-rate
+ * loop (dd_denoise_block) stays the default; these calls are the pages'
+ * alternative. */
 
 /* Entropy-budget acceptance for `batch` canvases of `canvas` positions
  * (rows b*canvas .. b*canvas+canvas-1): positions are taken in increasing
