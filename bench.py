@@ -329,10 +329,34 @@ def run_block(w, dd, dev, dist, reps: int = 20):
     ms_g = _max_over_ranks(dist, e0.elapsed_time(e1) / reps)
     g.destroy()
     dd.query_device_error(ws)
-    return {"steps": w.steps, "ms_per_block": ms, "blocks_per_s": 1e3 / ms,
-            "ms_per_block_graph": ms_g, "blocks_per_s_graph": 1e3 / ms_g,
-            "timing": f"mean of {reps} eager dd_denoise_block calls, and of {reps} replays of "
-                      "the same loop captured once (dd_denoise_block_graph), CUDA events"}
+    res = {"steps": w.steps, "ms_per_block": ms, "blocks_per_s": 1e3 / ms,
+           "ms_per_block_graph": ms_g, "blocks_per_s_graph": 1e3 / ms_g,
+           "timing": f"mean of {reps} eager dd_denoise_block calls, and of {reps} replays of "
+                     "the same loop captured once (dd_denoise_block_graph), CUDA events"}
+    if w.dtype == "bf16" and w.head_dim == 128:
+        # the same block with 8-bit attention inputs (dd_denoise_block_fp8)
+        q8, kc8, vc8, kp8, vp8, _, f8 = workloads.e4m3_block_inputs(w, device=dev)
+
+        def block8():
+            dd.denoise_block_fp8(q8, kc8, vc8, kp8, vp8, cud, f8, lg, w.rates, w.temperatures,
+                                 w.seed, cu_prefix_host=cu.numpy(), scale=w.scale,
+                                 attn_out=attn_out, canvas=canvas, keep_history=False,
+                                 workspace=ws)
+
+        for _ in range(3):
+            block8()
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(reps):
+            block8()
+        e1.record()
+        torch.cuda.synchronize()
+        ms8 = _max_over_ranks(dist, e0.elapsed_time(e1) / reps)
+        dd.query_device_error(ws)
+        res.update({"ms_per_block_e4m3": ms8, "blocks_per_s_e4m3": 1e3 / ms8,
+                    "timing_e4m3": f"mean of {reps} eager dd_denoise_block_fp8 calls on the "
+                                   "same block, E4M3 attention inputs, bf16 logits"})
+    return res
 
 
 def run_attn_e4m3(w, reps: int = 50):

@@ -33,7 +33,7 @@ EXPORTS = (
     "dd_entropy_accept", "dd_stop_check", "dd_denoise_block_adaptive_workspace",
     "dd_denoise_block_adaptive", "dd_canvas_attn_fp8", "dd_denoise_block_graph_create",
     "dd_denoise_block_graph_launch", "dd_denoise_block_graph_destroy",
-    "dd_soft_embed_workspace", "dd_soft_embed",
+    "dd_soft_embed_workspace", "dd_soft_embed", "dd_denoise_block_fp8",
 )
 
 
@@ -96,6 +96,9 @@ def load() -> ctypes.CDLL:
     lib.dd_denoise_block.restype = i32
     lib.dd_denoise_block.argtypes = [D, i32, P, P, P, P, P, P, P, P, P, i32, P, P, u64, u32, P, P,
                                      P, P, sz, P]
+    lib.dd_denoise_block_fp8.restype = i32
+    lib.dd_denoise_block_fp8.argtypes = [D, i32, P, P, P, P, P, P, P, P, P, P, i32, P, P, u64, u32,
+                                         P, P, P, P, sz, P]
     lib.dd_denoise_block_graph_create.restype = i32
     lib.dd_denoise_block_graph_create.argtypes = [ctypes.POINTER(P), D, i32, P, P, P, P, P, P, P,
                                                   P, P, i32, P, P, u64, u32, P, P, P, P, sz]
@@ -311,6 +314,27 @@ def denoise_block(q_steps, kc_steps, vc_steps, kp, vp, cu_prefix, logits_steps,
 
     q_steps [S,B,C,Hq,D], kc/vc_steps [S,B,C,Hkv,D], logits_steps [S,B*C,V].
     Returns dict(attn_out, canvas, canvas_history, conf_steps)."""
+    return _block_loop(None, q_steps, kc_steps, vc_steps, kp, vp, cu_prefix, logits_steps, rates,
+                       temperatures, seed, step0, cu_prefix_host, scale, attn_out, canvas,
+                       canvas_history, conf_steps, keep_history, workspace, stream)
+
+
+def denoise_block_fp8(q_steps, kc_steps, vc_steps, kp, vp, cu_prefix, scales_steps,
+                      logits_steps, rates: Sequence[float], temperatures: Sequence[float],
+                      seed: int, step0: int = 0, cu_prefix_host=None, scale=None, attn_out=None,
+                      canvas=None, canvas_history=None, conf_steps=None, keep_history=True,
+                      workspace=None, stream=None) -> dict:
+    """dd_denoise_block_fp8: as denoise_block with float8_e4m3fn attention
+    inputs, scales_steps = one (f_q, f_k, f_v) per step, bf16 logits; the
+    attention output is bf16."""
+    return _block_loop(scales_steps, q_steps, kc_steps, vc_steps, kp, vp, cu_prefix, logits_steps,
+                       rates, temperatures, seed, step0, cu_prefix_host, scale, attn_out, canvas,
+                       canvas_history, conf_steps, keep_history, workspace, stream)
+
+
+def _block_loop(scales_steps, q_steps, kc_steps, vc_steps, kp, vp, cu_prefix, logits_steps, rates,
+                temperatures, seed, step0, cu_prefix_host, scale, attn_out, canvas,
+                canvas_history, conf_steps, keep_history, workspace, stream) -> dict:
     lib = load()
     S = q_steps.shape[0]
     desc = attn_desc(q_steps[0], kc_steps[0], scale)
@@ -319,7 +343,8 @@ def denoise_block(q_steps, kc_steps, vc_steps, kp, vp, cu_prefix, logits_steps,
     R = desc.batch * desc.canvas
     dev = q_steps.device
     if attn_out is None:
-        attn_out = torch.empty_like(q_steps)
+        attn_out = torch.empty(q_steps.shape, device=dev, dtype=(
+            q_steps.dtype if scales_steps is None else torch.bfloat16))
     if canvas is None:
         canvas = torch.empty(R, dtype=torch.int32, device=dev)
     if keep_history and canvas_history is None:
@@ -331,12 +356,19 @@ def denoise_block(q_steps, kc_steps, vc_steps, kp, vp, cu_prefix, logits_steps,
     rates_h = np.ascontiguousarray(np.asarray(rates, dtype=np.float32))
     temps_h = np.ascontiguousarray(np.asarray(temperatures, dtype=np.float32))
     assert rates_h.size >= S and temps_h.size >= S
-    _check(lib.dd_denoise_block(
-        ctypes.byref(desc), S, _ptr(q_steps), _ptr(kc_steps), _ptr(vc_steps), _ptr(kp), _ptr(vp),
-        _ptr(cu_prefix), cu_h.ctypes.data_as(ctypes.c_void_p), _ptr(attn_out), _ptr(logits_steps),
-        V, rates_h.ctypes.data_as(ctypes.c_void_p), temps_h.ctypes.data_as(ctypes.c_void_p),
-        int(seed), int(step0), _ptr(canvas), _ptr(canvas_history), _ptr(conf_steps),
-        _ptr(workspace), workspace.numel(), _stream(stream)))
+    head = (ctypes.byref(desc), S, _ptr(q_steps), _ptr(kc_steps), _ptr(vc_steps), _ptr(kp),
+            _ptr(vp), _ptr(cu_prefix), cu_h.ctypes.data_as(ctypes.c_void_p))
+    tail = (_ptr(attn_out), _ptr(logits_steps), V, rates_h.ctypes.data_as(ctypes.c_void_p),
+            temps_h.ctypes.data_as(ctypes.c_void_p), int(seed), int(step0), _ptr(canvas),
+            _ptr(canvas_history), _ptr(conf_steps), _ptr(workspace), workspace.numel(),
+            _stream(stream))
+    if scales_steps is None:
+        _check(lib.dd_denoise_block(*head, *tail))
+    else:
+        assert len(scales_steps) >= S
+        f = (Fp8Scales * max(S, 1))(*(Fp8Scales(*(float(x) for x in scales_steps[i]))
+                                      for i in range(S)))
+        _check(lib.dd_denoise_block_fp8(*head, ctypes.cast(f, ctypes.c_void_p), *tail))
     return {"attn_out": attn_out, "canvas": canvas, "canvas_history": canvas_history,
             "conf_steps": conf_steps}
 

@@ -267,6 +267,21 @@ dd_status dd_canvas_attn(const dd_attn_desc* desc, const void* q, const void* k_
                   lse, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
+// The per-tensor factors of one E4M3 attention call (`step` >= 0 names the
+// block-loop step in the message).
+static dd_status check_fp8_scales(const dd_attn_desc* desc, const dd_fp8_scales* f, int step) {
+  char where[32] = "";
+  if (step >= 0) snprintf(where, sizeof where, "step %d: ", step);
+  if (!(std::isfinite(f->q) && f->q > 0.f && std::isfinite(f->k) && f->k > 0.f &&
+        std::isfinite(f->v) && f->v > 0.f))
+    return fail(DD_ERR_INVALID_ARG, "%sscale factors must be finite and > 0", where);
+  const double logit_gain =
+      (double)desc->scale * 1.4426950408889634 * (double)f->q * (double)f->k;
+  if (!std::isfinite(logit_gain) || logit_gain > 3.0e38)
+    return fail(DD_ERR_INVALID_ARG, "%sscale * q factor * k factor overflows float32", where);
+  return DD_OK;
+}
+
 dd_status dd_canvas_attn_fp8(const dd_attn_desc* desc, const void* q, const void* k_canvas,
                              const void* v_canvas, const void* k_prefix, const void* v_prefix,
                              const int32_t* cu_prefix, const int32_t* cu_prefix_host,
@@ -277,14 +292,8 @@ dd_status dd_canvas_attn_fp8(const dd_attn_desc* desc, const void* q, const void
   if (desc->dtype != DD_E4M3)
     return fail(DD_ERR_INVALID_ARG, "dd_canvas_attn_fp8 takes DD_E4M3 inputs");
   if (!scales) return fail(DD_ERR_INVALID_ARG, "scales is NULL");
-  if (!(std::isfinite(scales->q) && scales->q > 0.f && std::isfinite(scales->k) &&
-        scales->k > 0.f && std::isfinite(scales->v) && scales->v > 0.f))
-    return fail(DD_ERR_INVALID_ARG, "scale factors must be finite and > 0");
-  if (!std::isfinite((double)desc->scale * 1.4426950408889634 * (double)scales->q *
-                     (double)scales->k) ||
-      (double)desc->scale * 1.4426950408889634 * (double)scales->q * (double)scales->k >
-          3.0e38)
-    return fail(DD_ERR_INVALID_ARG, "scale * q factor * k factor overflows float32");
+  dd_status st = check_fp8_scales(desc, scales, -1);
+  if (st != DD_OK) return st;
   return run_attn(desc, q, k_canvas, v_canvas, k_prefix, v_prefix, cu_prefix, cu_prefix_host, out,
                   lse, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream), scales);
 }
@@ -322,21 +331,29 @@ dd_status dd_init_canvas(int32_t* canvas, int rows, int vocab, uint64_t seed, ui
 size_t dd_denoise_block_workspace(const dd_attn_desc* desc, const int32_t* cu_prefix_host,
                                   int vocab) {
   int64_t total = 0;
-  if (vocab < 1 || check_attn_desc(desc, cu_prefix_host, &total) != DD_OK) return 0;
+  if (vocab < 1 || check_attn_desc(desc, cu_prefix_host, &total, true) != DD_OK) return 0;
   return block_ws_layout(desc, total, cu_prefix_host, vocab, nullptr, nullptr);
 }
 
-dd_status dd_denoise_block(const dd_attn_desc* desc, int steps, const void* q_steps,
-                           const void* kc_steps, const void* vc_steps, const void* k_prefix,
-                           const void* v_prefix, const int32_t* cu_prefix,
-                           const int32_t* cu_prefix_host, void* attn_out,
-                           const void* logits_steps, int vocab, const float* rate_host,
-                           const float* temperature_host, uint64_t seed, uint32_t step0,
-                           int32_t* canvas, int32_t* canvas_history, float* conf_steps,
-                           void* workspace, size_t workspace_bytes, dd_stream_t stream) {
-  g_last_error.clear();
+// The block loop behind dd_denoise_block and dd_denoise_block_fp8.  With
+// E4M3 attention inputs (scales_host: one set of factors per step) the
+// attention output is bf16 and the logits are bf16; otherwise both have the
+// attention inputs' type.
+static dd_status block_loop(const dd_attn_desc* desc, int steps, const void* q_steps,
+                            const void* kc_steps, const void* vc_steps, const void* k_prefix,
+                            const void* v_prefix, const int32_t* cu_prefix,
+                            const int32_t* cu_prefix_host, const dd_fp8_scales* scales_host,
+                            void* attn_out, const void* logits_steps, int vocab,
+                            const float* rate_host, const float* temperature_host, uint64_t seed,
+                            uint32_t step0, int32_t* canvas, int32_t* canvas_history,
+                            float* conf_steps, void* workspace, size_t workspace_bytes,
+                            dd_stream_t stream) {
+  const bool f8 = scales_host != nullptr;
+  if (!f8 && desc && desc->dtype == DD_E4M3)
+    return fail(DD_ERR_INVALID_ARG,
+                "DD_E4M3 inputs need per-step factors: use dd_denoise_block_fp8");
   int64_t total = 0;
-  dd_status st = check_attn_desc(desc, cu_prefix_host, &total);
+  dd_status st = check_attn_desc(desc, cu_prefix_host, &total, f8);
   if (st != DD_OK) return st;
   if (steps < 0) return fail(DD_ERR_INVALID_ARG, "steps < 0");
   if (steps > 0 && (!rate_host || !temperature_host))
@@ -347,10 +364,12 @@ dd_status dd_denoise_block(const dd_attn_desc* desc, int steps, const void* q_st
   const int B = desc->batch, C = desc->canvas, Hq = desc->heads_q, Hkv = desc->heads_kv;
   const int D = desc->head_dim;
   const int rows = B * C;
-  const size_t es = elem_size(desc->dtype);
+  const dd_dtype out_t = f8 ? DD_BF16 : desc->dtype;  // attention output and logits
+  const size_t es = elem_size(desc->dtype), os = elem_size(out_t);
   const size_t q_step = (size_t)rows * Hq * D * es;
   const size_t kv_step = (size_t)rows * Hkv * D * es;
-  const size_t lg_step = (size_t)rows * (size_t)vocab * es;
+  const size_t o_step = (size_t)rows * Hq * D * os;
+  const size_t lg_step = (size_t)rows * (size_t)vocab * os;
   if (vocab < 1) return fail(DD_ERR_INVALID_ARG, "vocab=%d", vocab);
   size_t state_off = 0, conf_off = 0;
   const size_t need = block_ws_layout(desc, total, cu_prefix_host, vocab, &state_off, &conf_off);
@@ -362,8 +381,8 @@ dd_status dd_denoise_block(const dd_attn_desc* desc, int steps, const void* q_st
     st = run_attn(desc, static_cast<const uint8_t*>(q_steps) + i * q_step,
                   static_cast<const uint8_t*>(kc_steps) + i * kv_step,
                   static_cast<const uint8_t*>(vc_steps) + i * kv_step, k_prefix, v_prefix,
-                  cu_prefix, cu_prefix_host, static_cast<uint8_t*>(attn_out) + i * q_step,
-                  nullptr, workspace, state_off, s);
+                  cu_prefix, cu_prefix_host, static_cast<uint8_t*>(attn_out) + i * o_step,
+                  nullptr, workspace, state_off, s, f8 ? scales_host + i : nullptr);
     if (st != DD_OK) return st;
     dd_sample_params sp;
     sp.temperature = temperature_host[i];
@@ -374,9 +393,9 @@ dd_status dd_denoise_block(const dd_attn_desc* desc, int steps, const void* q_st
     int32_t* tok = canvas_history ? canvas_history + (size_t)i * rows : canvas;
     float* conf = conf_steps ? conf_steps + (size_t)i * rows
                              : reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + conf_off);
-    st = run_sampler(static_cast<const uint8_t*>(logits_steps) + i * lg_step, desc->dtype, rows,
-                     vocab, vocab, &sp, tok, nullptr, conf, nullptr, nullptr, workspace,
-                     state_off, s, static_cast<uint8_t*>(workspace) + state_off);
+    st = run_sampler(static_cast<const uint8_t*>(logits_steps) + i * lg_step, out_t, rows, vocab,
+                     vocab, &sp, tok, nullptr, conf, nullptr, nullptr, workspace, state_off, s,
+                     static_cast<uint8_t*>(workspace) + state_off);
     if (st != DD_OK) return st;
     if (canvas_history && i == steps - 1) {
       cudaError_t e = cudaMemcpyAsync(canvas, tok, (size_t)rows * sizeof(int32_t),
@@ -385,6 +404,46 @@ dd_status dd_denoise_block(const dd_attn_desc* desc, int steps, const void* q_st
     }
   }
   return DD_OK;
+}
+
+dd_status dd_denoise_block(const dd_attn_desc* desc, int steps, const void* q_steps,
+                           const void* kc_steps, const void* vc_steps, const void* k_prefix,
+                           const void* v_prefix, const int32_t* cu_prefix,
+                           const int32_t* cu_prefix_host, void* attn_out,
+                           const void* logits_steps, int vocab, const float* rate_host,
+                           const float* temperature_host, uint64_t seed, uint32_t step0,
+                           int32_t* canvas, int32_t* canvas_history, float* conf_steps,
+                           void* workspace, size_t workspace_bytes, dd_stream_t stream) {
+  g_last_error.clear();
+  return block_loop(desc, steps, q_steps, kc_steps, vc_steps, k_prefix, v_prefix, cu_prefix,
+                    cu_prefix_host, nullptr, attn_out, logits_steps, vocab, rate_host,
+                    temperature_host, seed, step0, canvas, canvas_history, conf_steps, workspace,
+                    workspace_bytes, stream);
+}
+
+dd_status dd_denoise_block_fp8(const dd_attn_desc* desc, int steps, const void* q_steps,
+                               const void* kc_steps, const void* vc_steps, const void* k_prefix,
+                               const void* v_prefix, const int32_t* cu_prefix,
+                               const int32_t* cu_prefix_host, const dd_fp8_scales* scales_host,
+                               void* attn_out, const void* logits_steps, int vocab,
+                               const float* rate_host, const float* temperature_host,
+                               uint64_t seed, uint32_t step0, int32_t* canvas,
+                               int32_t* canvas_history, float* conf_steps, void* workspace,
+                               size_t workspace_bytes, dd_stream_t stream) {
+  g_last_error.clear();
+  if (!desc) return fail(DD_ERR_INVALID_ARG, "desc is NULL");
+  if (desc->dtype != DD_E4M3)
+    return fail(DD_ERR_INVALID_ARG, "dd_denoise_block_fp8 takes DD_E4M3 inputs");
+  if (steps > 0 && !scales_host) return fail(DD_ERR_INVALID_ARG, "scales_host is NULL");
+  for (int i = 0; i < steps; ++i) {
+    dd_status st = check_fp8_scales(desc, scales_host + i, i);
+    if (st != DD_OK) return st;
+  }
+  static const dd_fp8_scales kNone = {1.f, 1.f, 1.f};
+  return block_loop(desc, steps, q_steps, kc_steps, vc_steps, k_prefix, v_prefix, cu_prefix,
+                    cu_prefix_host, steps > 0 ? scales_host : &kNone, attn_out, logits_steps,
+                    vocab, rate_host, temperature_host, seed, step0, canvas, canvas_history,
+                    conf_steps, workspace, workspace_bytes, stream);
 }
 
 dd_status dd_entropy_accept(const float* entropy, const int32_t* pred, int batch, int canvas,

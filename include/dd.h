@@ -203,7 +203,8 @@ DD_API dd_status dd_sample_renoise(const void* logits, dd_dtype dtype, int rows,
 DD_API dd_status dd_init_canvas(int32_t* canvas, int rows, int vocab, uint64_t seed, uint32_t row_offset,
                          dd_stream_t stream);
 
-/* Workspace bytes for dd_denoise_block (the larger of the two steps' needs). */
+/* Workspace bytes for dd_denoise_block, or for dd_denoise_block_fp8 when
+ * desc->dtype is DD_E4M3 (the larger of the two steps' needs). */
 DD_API size_t dd_denoise_block_workspace(const dd_attn_desc* desc, const int32_t* cu_prefix_host,
                                   int vocab);
 
@@ -233,6 +234,25 @@ DD_API dd_status dd_denoise_block(const dd_attn_desc* desc, int steps, const voi
                            const float* temperature_host, uint64_t seed, uint32_t step0,
                            int32_t* canvas, int32_t* canvas_history, float* conf_steps,
                            void* workspace, size_t workspace_bytes, dd_stream_t stream);
+
+/* dd_denoise_block with 8-bit attention inputs: step s runs
+ * dd_canvas_attn_fp8 with the factors scales_host[s], then
+ * dd_sample_renoise on bf16 logits.  desc->dtype must be DD_E4M3; q_steps,
+ * kc_steps, vc_steps, k_prefix and v_prefix are E4M3 with the shapes of
+ * dd_denoise_block; attn_out is bf16 [S, B, C, Hq, D]; logits_steps is bf16
+ * [S, R, V].  scales_host: host array of `steps` factor sets, each
+ * validated like dd_canvas_attn_fp8's (DD_ERR_INVALID_ARG names the step).
+ * Every other argument, the workspace query and the results' meaning are
+ * those of dd_denoise_block. */
+DD_API dd_status dd_denoise_block_fp8(const dd_attn_desc* desc, int steps, const void* q_steps,
+                               const void* kc_steps, const void* vc_steps, const void* k_prefix,
+                               const void* v_prefix, const int32_t* cu_prefix,
+                               const int32_t* cu_prefix_host, const dd_fp8_scales* scales_host,
+                               void* attn_out, const void* logits_steps, int vocab,
+                               const float* rate_host, const float* temperature_host,
+                               uint64_t seed, uint32_t step0, int32_t* canvas,
+                               int32_t* canvas_history, float* conf_steps, void* workspace,
+                               size_t workspace_bytes, dd_stream_t stream);
 
 /* A block loop captured once and replayed with a single launch.  The loop
  * takes 4 kernels per step (attention, split combine, sampler pass, row

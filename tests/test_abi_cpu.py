@@ -203,6 +203,36 @@ def test_block_rejects_bad_arguments(lib):
     assert lib.dd_denoise_block(*bad) == 1
 
 
+def test_block_fp8_rejects_bad_arguments(lib):
+    e4 = _desc(dtype=dd.DD_E4M3)
+    cu = _cu([16])
+    cuh = cu.ctypes.data_as(ctypes.c_void_p)
+    r = np.zeros(2, np.float32)
+    rp = r.ctypes.data_as(ctypes.c_void_p)
+    good = (dd.Fp8Scales * 2)(dd.Fp8Scales(1.0, 1.0, 1.0), dd.Fp8Scales(0.5, 2.0, 1.0))
+    ws = lib.dd_denoise_block_workspace(ctypes.byref(e4), cuh, 1024)
+    assert ws > 0                                               # E4M3 geometry is queried
+
+    def call(desc=e4, scales=ctypes.cast(good, ctypes.c_void_p), ws_bytes=ws, steps=2):
+        return lib.dd_denoise_block_fp8(ctypes.byref(desc), steps, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                        FAKE, cuh, scales, FAKE, FAKE, 1024, rp, rp, 0, 0, FAKE,
+                                        None, None, FAKE, ws_bytes, None)
+
+    assert call(ws_bytes=16) == 3                                # workspace too small
+    assert call(desc=_desc()) == 1                               # bf16 desc
+    assert "DD_E4M3" in dd.last_error()
+    assert call(scales=None) == 1
+    for bad in ((0.0, 1.0, 1.0), (1.0, float("nan"), 1.0), (1e30, 1e30, 1.0)):
+        sc = (dd.Fp8Scales * 2)(dd.Fp8Scales(1.0, 1.0, 1.0), dd.Fp8Scales(*bad))
+        assert call(scales=ctypes.cast(sc, ctypes.c_void_p)) == 1, bad
+        assert "step 1" in dd.last_error()
+    assert call(scales=None, steps=0, ws_bytes=16) == 3          # steps 0: factors unused
+    args = [ctypes.byref(e4), 1, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, cuh, FAKE, FAKE, 1024, rp,
+            rp, 0, 0, FAKE, None, None, FAKE, ws, None]
+    assert lib.dd_denoise_block(*args) == 1                      # E4M3 needs the fp8 entry
+    assert "dd_denoise_block_fp8" in dd.last_error()
+
+
 def test_init_canvas_rejects_bad_arguments(lib):
     assert lib.dd_init_canvas(None, 4, 10, 0, 0, None) == 1
     assert lib.dd_init_canvas(FAKE, 4, 0, 0, 0, None) == 1

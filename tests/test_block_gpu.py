@@ -111,3 +111,37 @@ def test_block_graph_replays_the_eager_loop(block12):
     assert torch.equal(out["attn_out"], ref["attn_out"])
     g.destroy()
     dd.query_device_error(g.tensors["workspace"])
+
+
+def test_block_fp8_matches_the_step_calls_and_the_oracle():
+    """dd_denoise_block_fp8: every step identical to dd_canvas_attn_fp8 +
+    dd_sample_renoise called one by one; attention within the E4M3 bound of
+    the oracle, tokens equal to the oracle's away from near-ties."""
+    from test_attn_fp8_gpu import _check
+    w = workloads.scaled(workloads.WORKLOADS["block12_L8192"], prefix_lens=(700,), vocab=20000,
+                         steps=3, rates=(0.9, 0.4, 0.0), temperatures=(1.0, 0.8, 0.7),
+                         name="block3_e4m3")
+    qs, kcs, vcs, kp, vp, cu, f = workloads.e4m3_block_inputs(w, device=DEV)
+    ls = torch.stack([workloads.logits(w, s, device=DEV) for s in range(w.steps)])
+    assert ls.dtype == torch.bfloat16
+    out = dd.denoise_block_fp8(qs, kcs, vcs, kp, vp, cu.to(DEV), f, ls, w.rates, w.temperatures,
+                               seed=5, cu_prefix_host=cu, scale=w.scale)
+    torch.cuda.synchronize()
+    assert out["attn_out"].dtype == torch.bfloat16
+    assert torch.equal(out["canvas"], out["canvas_history"][-1])
+    for s in range(w.steps):
+        o, _ = dd.canvas_attn_fp8(qs[s], kcs[s], vcs[s], kp, vp, cu.to(DEV), f[s], cu,
+                                  scale=w.scale)
+        r = dd.sample_renoise(ls[s], w.temperatures[s], w.rates[s], 5, s)
+        torch.cuda.synchronize()
+        assert torch.equal(out["attn_out"][s], o)
+        assert torch.equal(out["canvas_history"][s], r["tokens"])
+        assert torch.equal(out["conf_steps"][s], r["conf"])
+        ref = oracle.sample_renoise(ls[s].cpu(), w.temperatures[s], w.rates[s], 5, s)
+        check_sampler({"tokens": out["canvas_history"][s], "conf": out["conf_steps"][s]}, ref)
+    pos = np.array([0, 77, 255], np.int32)
+    for s in (0, 2):
+        ref_o, _ = oracle.canvas_attn(qs[s].cpu(), kcs[s].cpu(), vcs[s].cpu(), kp.cpu(), vp.cpu(),
+                                      cu.numpy(), w.scale, positions=pos, qkv_scale=f[s])
+        _check(out["attn_out"][s], ref_o, vcs[s].cpu(), vp.cpu(), f[s][2], 700 + 256,
+               positions=pos)

@@ -25,7 +25,8 @@ Every tensor is drawn in float32 from a torch.Generator seeded with a hash
 of (seed, workload, tensor name, step), then rounded to bf16 (round to
 nearest even) where the workload is bf16.  The 8-bit attention inputs are
 the same float32 draws rounded to E4M3 under a power-of-two per-tensor
-factor (e4m3_attn_inputs).  The generator's device is the
+factor (e4m3_attn_inputs; e4m3_block_inputs for a block of steps).  The
+generator's device is the
 caller's choice; the same device always gives the same bits.
 """
 from __future__ import annotations
@@ -169,6 +170,29 @@ def e4m3_attn_inputs(w: Workload, step: int = 0, device="cpu", q_gain: float = 1
     (kc8, kp8), fk = to_e4m3([kc, kp])
     (vc8, vp8), fv = to_e4m3([vc, vp])
     return q8, kc8, vc8, kp8, vp8, cu, (fq, fk, fv)
+
+
+def e4m3_block_inputs(w: Workload, device="cpu"):
+    """The attention inputs of every step of `w` in E4M3, for the block loop.
+
+    The prefix cache is fixed across steps while one K factor (and one V
+    factor) covers the prefix and the step's canvas keys in a call, so the K
+    factor is taken over Kp and every step's Kc together (likewise V); Q
+    gets its own factor per step.  Returns q_steps [S,B,C,Hq,D], kc_steps,
+    vc_steps [S,B,C,Hkv,D] (float8_e4m3fn), kp, vp, cu_prefix and the list
+    of per-step factors (f_q[s], f_k, f_v)."""
+    f32 = dataclasses.replace(w, dtype="f32")
+    steps = [canvas_qkv(f32, s, device) for s in range(w.steps)]
+    kp, vp, cu = prefix_kv(f32, device)
+    (kp8, *kcs), fk = to_e4m3([kp] + [x[1] for x in steps])
+    (vp8, *vcs), fv = to_e4m3([vp] + [x[2] for x in steps])
+    qs, fq = zip(*(to_e4m3([x[0]]) for x in steps))
+
+    def stack(ts):
+        return torch.stack([t.view(torch.uint8) for t in ts]).view(torch.float8_e4m3fn)
+
+    return (stack([q[0] for q in qs]), stack(kcs), stack(vcs), kp8, vp8, cu,
+            [(f, fk, fv) for f in fq])
 
 
 def logits(w: Workload, step: int = 0, device="cpu", rows: Optional[int] = None):
