@@ -44,7 +44,7 @@ def _rank_main(rank, world, port, out):
 
 def test_rank_plumbing_on_two_gloo_ranks():
     world, port = 2, _free_port()
-    with mp.Manager() as mgr:
+    with mp.get_context("spawn").Manager() as mgr:  # no fork of a threaded process
         out = mgr.dict()
         mp.start_processes(_rank_main, args=(world, port, out), nprocs=world, start_method="spawn")
         res = dict(out)
