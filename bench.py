@@ -729,6 +729,30 @@ def run_policy(w, reps: int = 10, max_steps: int = 12, budget: float = 0.1,
         wall.append((time.perf_counter() - t0) * 1e3)
         dev_ms.append(e0.elapsed_time(e1))
     n = res["steps_run"]
+    # the same loop kept on the device (dd_denoise_block_adaptive_graph):
+    # one graph launch per block, no per-step host read
+    ag = dd.denoise_block_adaptive_graph(q, kc, vc, kp, vp, cud, lg, temps, budget, stop_entropy,
+                                         w.seed, cu_prefix_host=cu, scale=w.scale,
+                                         attn_out=attn_out, keep_history=False)
+    for _ in range(2):
+        t = ag.launch()
+    torch.cuda.synchronize()
+    g_wall, g_dev = [], []
+    for _ in range(reps):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        t0 = time.perf_counter()
+        e0.record()
+        t = ag.launch()
+        e1.record()
+        torch.cuda.synchronize()
+        g_wall.append((time.perf_counter() - t0) * 1e3)
+        g_dev.append(e0.elapsed_time(e1))
+    g_steps = int(t["steps_run"].item())
+    same = bool(torch.equal(t["canvas"], res["canvas"]) and
+                torch.equal(t["halt_step"], res["halt_step"]))
+    dd.query_device_error(t["workspace"])
+    ag.destroy()
     # the acceptance kernel alone, 8 canvases of 256
     h = torch.rand(8 * 256, device=dev) * 0.01
     pr = torch.randint(0, V, (8 * 256,), dtype=torch.int32, device=dev)
@@ -759,6 +783,11 @@ def run_policy(w, reps: int = 10, max_steps: int = 12, budget: float = 0.1,
             "steps_run": n, "max_steps": max_steps, "ms_per_step": statistics.median(wall) / n,
             "halt_step": res["halt_step"].cpu().tolist(),
             "entropy_accept_us_8_canvases": e0.elapsed_time(e1) * 10.0,
+            "device_loop": {"ms_per_block": statistics.median(g_dev),
+                            "wall_ms_per_block": statistics.median(g_wall),
+                            "steps_run": g_steps, "same_result_as_eager": same,
+                            "timing": "median of %d replays of dd_denoise_block_adaptive_graph "
+                                      "(one IF node per step), CUDA events" % reps},
             "config": {"workload": w.name + " geometry, sharpening synthetic logits",
                        "budget": budget, "stop_entropy": stop_entropy,
                        "temperature": "0.8 -> 0.4 over 48 nominal steps"},

@@ -34,6 +34,8 @@ EXPORTS = (
     "dd_denoise_block_adaptive", "dd_canvas_attn_fp8", "dd_denoise_block_graph_create",
     "dd_denoise_block_graph_launch", "dd_denoise_block_graph_destroy",
     "dd_soft_embed_workspace", "dd_soft_embed", "dd_denoise_block_fp8",
+    "dd_denoise_block_adaptive_graph_create", "dd_denoise_block_adaptive_graph_launch",
+    "dd_denoise_block_adaptive_graph_destroy",
 )
 
 
@@ -73,6 +75,7 @@ def load() -> ctypes.CDLL:
     lib = ctypes.CDLL(LIB_PATH)
     P, i32, i64, u32, u64, sz = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_uint32,
                                  ctypes.c_uint64, ctypes.c_size_t)
+    f32 = ctypes.c_float
     D = ctypes.POINTER(AttnDesc)
     lib.dd_canvas_attn_workspace.restype = sz
     lib.dd_canvas_attn_workspace.argtypes = [D, P]
@@ -106,11 +109,18 @@ def load() -> ctypes.CDLL:
     lib.dd_denoise_block_graph_launch.argtypes = [P, P]
     lib.dd_denoise_block_graph_destroy.restype = i32
     lib.dd_denoise_block_graph_destroy.argtypes = [P]
+    lib.dd_denoise_block_adaptive_graph_create.restype = i32
+    lib.dd_denoise_block_adaptive_graph_create.argtypes = [ctypes.POINTER(P), D, i32, P, P, P, P,
+                                                           P, P, P, P, P, i32, P, f32, f32, u64,
+                                                           u32, P, P, P, P, P, sz]
+    lib.dd_denoise_block_adaptive_graph_launch.restype = i32
+    lib.dd_denoise_block_adaptive_graph_launch.argtypes = [P, P]
+    lib.dd_denoise_block_adaptive_graph_destroy.restype = i32
+    lib.dd_denoise_block_adaptive_graph_destroy.argtypes = [P]
     lib.dd_soft_embed_workspace.restype = sz
     lib.dd_soft_embed_workspace.argtypes = [i32, i32, i32]
     lib.dd_soft_embed.restype = i32
     lib.dd_soft_embed.argtypes = [P, i32, i32, i32, i64, ctypes.c_float, P, i32, P, P, sz, P]
-    f32 = ctypes.c_float
     lib.dd_entropy_accept.restype = i32
     lib.dd_entropy_accept.argtypes = [P, P, i32, i32, i32, f32, u64, u32, u32, P, P, P]
     lib.dd_stop_check.restype = i32
@@ -402,6 +412,8 @@ class BlockGraph:
     buffers outlive the graph; new inputs enter by writing into them
     (`tensors` maps the argument names to those tensors)."""
 
+    _prefix = "dd_denoise_block_graph"
+
     def __init__(self, handle, tensors: dict, keep: tuple):
         self._h = handle
         self.tensors = tensors
@@ -409,14 +421,14 @@ class BlockGraph:
 
     def launch(self, stream=None):
         if self._h is None:
-            raise RuntimeError("BlockGraph: destroyed")
-        _check(load().dd_denoise_block_graph_launch(self._h, _stream(stream)))
+            raise RuntimeError(f"{type(self).__name__}: destroyed")
+        _check(getattr(load(), self._prefix + "_launch")(self._h, _stream(stream)))
         return self.tensors
 
     def destroy(self):
         if self._h is not None:
             h, self._h = self._h, None
-            _check(load().dd_denoise_block_graph_destroy(h))
+            _check(getattr(load(), self._prefix + "_destroy")(h))
 
     def __del__(self):
         try:
@@ -526,6 +538,53 @@ def denoise_block_adaptive(q_steps, kc_steps, vc_steps, kp, vp, cu_prefix, logit
     n = steps_run.value
     return {"canvas": canvas, "canvas_history": None if history is None else history[:n],
             "halt_step": halt, "steps_run": n}
+
+
+class AdaptiveGraph(BlockGraph):
+    """dd_denoise_block_adaptive captured once with the loop on the device
+    (dd_denoise_block_adaptive_graph_create); launch() replays it without
+    any host synchronisation.  tensors["steps_run"] is a device int32 [1]."""
+    _prefix = "dd_denoise_block_adaptive_graph"
+
+
+def denoise_block_adaptive_graph(q_steps, kc_steps, vc_steps, kp, vp, cu_prefix, logits_steps,
+                                 temperatures: Sequence[float], budget: float,
+                                 stop_entropy: float, seed: int, step0: int = 0,
+                                 cu_prefix_host=None, scale=None, attn_out=None, canvas=None,
+                                 keep_history=True, workspace=None) -> AdaptiveGraph:
+    """dd_denoise_block_adaptive_graph_create with the arguments of
+    denoise_block_adaptive."""
+    lib = load()
+    S = q_steps.shape[0]
+    desc = attn_desc(q_steps[0], kc_steps[0], scale)
+    cu_h = _host_i32(cu_prefix if cu_prefix_host is None else cu_prefix_host)
+    V = logits_steps.shape[-1]
+    R = desc.batch * desc.canvas
+    dev = q_steps.device
+    if attn_out is None:
+        attn_out = torch.empty_like(q_steps)
+    if canvas is None:
+        canvas = torch.zeros(R, dtype=torch.int32, device=dev)
+    history = torch.empty((S, R), dtype=torch.int32, device=dev) if keep_history else None
+    halt = torch.empty(desc.batch, dtype=torch.int32, device=dev)
+    steps_run = torch.zeros(1, dtype=torch.int32, device=dev)
+    if workspace is None:
+        workspace = new_workspace(int(lib.dd_denoise_block_adaptive_workspace(
+            ctypes.byref(desc), cu_h.ctypes.data_as(ctypes.c_void_p), V)), dev)
+    temps_h = np.ascontiguousarray(np.asarray(temperatures, dtype=np.float32))
+    assert temps_h.size >= S
+    h = ctypes.c_void_p()
+    _check(lib.dd_denoise_block_adaptive_graph_create(
+        ctypes.byref(h), ctypes.byref(desc), S, _ptr(q_steps), _ptr(kc_steps), _ptr(vc_steps),
+        _ptr(kp), _ptr(vp), _ptr(cu_prefix), cu_h.ctypes.data_as(ctypes.c_void_p),
+        _ptr(attn_out), _ptr(logits_steps), V, temps_h.ctypes.data_as(ctypes.c_void_p),
+        float(budget), float(stop_entropy), int(seed), int(step0), _ptr(canvas), _ptr(history),
+        _ptr(halt), _ptr(steps_run), _ptr(workspace), workspace.numel()))
+    tensors = {"q_steps": q_steps, "kc_steps": kc_steps, "vc_steps": vc_steps, "kp": kp, "vp": vp,
+               "cu_prefix": cu_prefix, "logits_steps": logits_steps, "attn_out": attn_out,
+               "canvas": canvas, "canvas_history": history, "halt_step": halt,
+               "steps_run": steps_run, "workspace": workspace}
+    return AdaptiveGraph(h, tensors, (cu_h, temps_h))
 
 
 def query_device_error(workspace: torch.Tensor, stream=None):

@@ -230,6 +230,9 @@ dd_status run_sampler(const void* logits, dd_dtype dtype, int rows, int vocab, i
 
 void note_launch() { ++g_launches; }
 
+thread_local bool g_pdl_off = false;
+bool pdl_enabled() { return !g_pdl_off; }
+
 // Entry for callers that bring their own scratch region (dd_noalloc.cu):
 // the same validation and kernels as dd_sample_renoise.
 dd_status sample_with_scratch(const void* logits, dd_dtype dtype, int rows, int vocab,
@@ -617,6 +620,123 @@ size_t dd_denoise_block_adaptive_workspace(const dd_attn_desc* desc,
   return adaptive_ws_layout(desc, total, cu_prefix_host, vocab, nullptr, nullptr, nullptr);
 }
 
+// Validated arguments and workspace regions of one adaptive block loop.
+struct AdaptiveLoop {
+  const dd_attn_desc* desc;
+  const uint8_t *q, *kc, *vc, *logits;
+  const void *kp, *vp;
+  const int32_t *cu, *cu_host;
+  uint8_t* attn_out;
+  int vocab, B, C, rows;
+  const float* temps;
+  float budget, stop_entropy;
+  uint64_t seed;
+  uint32_t step0;
+  int32_t *canvas, *history, *halt_step;
+  void* ws;
+  size_t state_off, q_step, kv_step, lg_step;
+  int32_t* pred[2];  // step i writes pred[i % 2] and compares with pred[(i + 1) % 2]
+  float *ent, *conf;
+  uint8_t* done;
+};
+
+static dd_status adaptive_prepare(AdaptiveLoop* L, const dd_attn_desc* desc, int max_steps,
+                                  const void* q_steps, const void* kc_steps, const void* vc_steps,
+                                  const void* k_prefix, const void* v_prefix,
+                                  const int32_t* cu_prefix, const int32_t* cu_prefix_host,
+                                  void* attn_out, const void* logits_steps, int vocab,
+                                  const float* temperature_host, float budget, float stop_entropy,
+                                  uint64_t seed, uint32_t step0, int32_t* canvas,
+                                  int32_t* canvas_history, int32_t* halt_step, void* workspace,
+                                  size_t workspace_bytes) {
+  int64_t total = 0;
+  dd_status st = check_attn_desc(desc, cu_prefix_host, &total);
+  if (st != DD_OK) return st;
+  if (max_steps < 0) return fail(DD_ERR_INVALID_ARG, "max_steps < 0");
+  if (max_steps > 0 && !temperature_host) return fail(DD_ERR_INVALID_ARG, "temperature_host is NULL");
+  if (!canvas || !halt_step) return fail(DD_ERR_INVALID_ARG, "NULL required pointer");
+  if (desc->canvas > 1024) return fail(DD_ERR_UNSUPPORTED, "canvas > 1024");
+  if (std::isnan(budget) || std::isnan(stop_entropy))
+    return fail(DD_ERR_INVALID_ARG, "budget / stop_entropy is NaN");
+  if ((uint64_t)step0 + (uint64_t)max_steps > (1ull << 32))
+    return fail(DD_ERR_INVALID_ARG, "step0 + max_steps exceeds 2^32");
+  if (vocab < 1) return fail(DD_ERR_INVALID_ARG, "vocab=%d", vocab);
+  L->desc = desc;
+  L->B = desc->batch;
+  L->C = desc->canvas;
+  L->rows = L->B * L->C;
+  const size_t es = elem_size(desc->dtype);
+  L->q_step = (size_t)L->rows * desc->heads_q * desc->head_dim * es;
+  L->kv_step = (size_t)L->rows * desc->heads_kv * desc->head_dim * es;
+  L->lg_step = (size_t)L->rows * (size_t)vocab * es;
+  size_t conf_off = 0, extra_off = 0;
+  const size_t need = adaptive_ws_layout(desc, total, cu_prefix_host, vocab, &L->state_off,
+                                         &conf_off, &extra_off);
+  if (!workspace) return fail(DD_ERR_WORKSPACE, "workspace is NULL");
+  if (workspace_bytes < need)
+    return fail(DD_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", workspace_bytes, need);
+  uint8_t* const ws = static_cast<uint8_t*>(workspace);
+  const size_t pred_bytes = align256((size_t)L->rows * 4);
+  L->pred[0] = reinterpret_cast<int32_t*>(ws + extra_off);
+  L->pred[1] = reinterpret_cast<int32_t*>(ws + extra_off + pred_bytes);
+  L->ent = reinterpret_cast<float*>(ws + extra_off + 2 * pred_bytes);
+  L->done = ws + extra_off + 3 * pred_bytes;
+  L->conf = reinterpret_cast<float*>(ws + conf_off);
+  L->q = static_cast<const uint8_t*>(q_steps);
+  L->kc = static_cast<const uint8_t*>(kc_steps);
+  L->vc = static_cast<const uint8_t*>(vc_steps);
+  L->logits = static_cast<const uint8_t*>(logits_steps);
+  L->kp = k_prefix;
+  L->vp = v_prefix;
+  L->cu = cu_prefix;
+  L->cu_host = cu_prefix_host;
+  L->attn_out = static_cast<uint8_t*>(attn_out);
+  L->vocab = vocab;
+  L->temps = temperature_host;
+  L->budget = budget;
+  L->stop_entropy = stop_entropy;
+  L->seed = seed;
+  L->step0 = step0;
+  L->canvas = canvas;
+  L->history = canvas_history;
+  L->halt_step = halt_step;
+  L->ws = workspace;
+  return DD_OK;
+}
+
+// The work of step i on stream s: attention, the sampler (no scheduled
+// re-noise: the acceptance rule decides it), the halt test against step
+// i - 1's predictions, the acceptance into the canvas, the history copy.
+static dd_status adaptive_step(const AdaptiveLoop& L, int i, cudaStream_t s) {
+  dd_status st = run_attn(L.desc, L.q + i * L.q_step, L.kc + i * L.kv_step, L.vc + i * L.kv_step,
+                          L.kp, L.vp, L.cu, L.cu_host, L.attn_out + i * L.q_step, nullptr, L.ws,
+                          L.state_off, s);
+  if (st != DD_OK) return st;
+  dd_sample_params sp;
+  sp.temperature = L.temps[i];
+  sp.renoise_rate = 0.f;
+  sp.seed = L.seed;
+  sp.step = L.step0 + (uint32_t)i;
+  sp.row_offset = 0;
+  int32_t* cur = L.pred[i % 2];
+  int32_t* prev = i > 0 ? L.pred[(i + 1) % 2] : nullptr;
+  st = run_sampler(L.logits + i * L.lg_step, L.desc->dtype, L.rows, L.vocab, L.vocab, &sp, cur,
+                   nullptr, L.conf, L.ent, nullptr, L.ws, L.state_off, s,
+                   static_cast<uint8_t*>(L.ws) + L.state_off);
+  if (st != DD_OK) return st;
+  cudaError_t e = launch_stop_check(L.ent, cur, prev, L.B, L.C, (double)L.stop_entropy, i,
+                                    L.done, L.halt_step, s);
+  if (e == cudaSuccess)
+    e = launch_entropy_accept(L.ent, cur, L.B, L.C, L.vocab, (double)L.budget, L.seed,
+                              L.step0 + (uint32_t)i, 0, L.done, L.halt_step, i, L.canvas, nullptr,
+                              s);
+  if (e == cudaSuccess && L.history)
+    e = cudaMemcpyAsync(L.history + (size_t)i * L.rows, L.canvas, (size_t)L.rows * sizeof(int32_t),
+                        cudaMemcpyDeviceToDevice, s);
+  if (e != cudaSuccess) return cuda_fail(e, "adaptive step");
+  return DD_OK;
+}
+
 dd_status dd_denoise_block_adaptive(const dd_attn_desc* desc, int max_steps, const void* q_steps,
                                     const void* kc_steps, const void* vc_steps,
                                     const void* k_prefix, const void* v_prefix,
@@ -628,81 +748,182 @@ dd_status dd_denoise_block_adaptive(const dd_attn_desc* desc, int max_steps, con
                                     int32_t* halt_step, int* steps_run, void* workspace,
                                     size_t workspace_bytes, dd_stream_t stream) {
   g_last_error.clear();
-  int64_t total = 0;
-  dd_status st = check_attn_desc(desc, cu_prefix_host, &total);
+  if (!steps_run) return fail(DD_ERR_INVALID_ARG, "NULL required pointer");
+  AdaptiveLoop L;
+  dd_status st = adaptive_prepare(&L, desc, max_steps, q_steps, kc_steps, vc_steps, k_prefix,
+                                  v_prefix, cu_prefix, cu_prefix_host, attn_out, logits_steps,
+                                  vocab, temperature_host, budget, stop_entropy, seed, step0,
+                                  canvas, canvas_history, halt_step, workspace, workspace_bytes);
   if (st != DD_OK) return st;
-  if (max_steps < 0) return fail(DD_ERR_INVALID_ARG, "max_steps < 0");
-  if (max_steps > 0 && !temperature_host) return fail(DD_ERR_INVALID_ARG, "temperature_host is NULL");
-  if (!canvas || !halt_step || !steps_run) return fail(DD_ERR_INVALID_ARG, "NULL required pointer");
-  if (desc->canvas > 1024) return fail(DD_ERR_UNSUPPORTED, "canvas > 1024");
-  if (std::isnan(budget) || std::isnan(stop_entropy))
-    return fail(DD_ERR_INVALID_ARG, "budget / stop_entropy is NaN");
-  if ((uint64_t)step0 + (uint64_t)max_steps > (1ull << 32))
-    return fail(DD_ERR_INVALID_ARG, "step0 + max_steps exceeds 2^32");
-  if (vocab < 1) return fail(DD_ERR_INVALID_ARG, "vocab=%d", vocab);
-  const int B = desc->batch, C = desc->canvas, Hq = desc->heads_q, Hkv = desc->heads_kv;
-  const int D = desc->head_dim;
-  const int rows = B * C;
-  const size_t es = elem_size(desc->dtype);
-  const size_t q_step = (size_t)rows * Hq * D * es;
-  const size_t kv_step = (size_t)rows * Hkv * D * es;
-  const size_t lg_step = (size_t)rows * (size_t)vocab * es;
-  size_t state_off = 0, conf_off = 0, extra_off = 0;
-  const size_t need = adaptive_ws_layout(desc, total, cu_prefix_host, vocab, &state_off,
-                                         &conf_off, &extra_off);
-  if (!workspace) return fail(DD_ERR_WORKSPACE, "workspace is NULL");
-  if (workspace_bytes < need)
-    return fail(DD_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", workspace_bytes, need);
   *steps_run = 0;
-  if (B == 0) return DD_OK;
+  if (L.B == 0) return DD_OK;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  uint8_t* const ws = static_cast<uint8_t*>(workspace);
-  int32_t* pred_a = reinterpret_cast<int32_t*>(ws + extra_off);
-  int32_t* pred_b = reinterpret_cast<int32_t*>(ws + extra_off + align256((size_t)rows * 4));
-  float* ent = reinterpret_cast<float*>(ws + extra_off + 2 * align256((size_t)rows * 4));
-  uint8_t* done = ws + extra_off + 3 * align256((size_t)rows * 4);
-  float* conf = reinterpret_cast<float*>(ws + conf_off);
-  cudaError_t e = cudaMemsetAsync(done, 0, (size_t)B, s);
-  if (e == cudaSuccess) e = cudaMemsetAsync(halt_step, 0xff, (size_t)B * sizeof(int32_t), s);
+  cudaError_t e = cudaMemsetAsync(L.done, 0, (size_t)L.B, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(halt_step, 0xff, (size_t)L.B * sizeof(int32_t), s);
   if (e != cudaSuccess) return cuda_fail(e, "adaptive loop init");
-  std::vector<uint8_t> done_h((size_t)B);
-  int32_t* cur = pred_a;
-  int32_t* prev = pred_b;
+  std::vector<uint8_t> done_h((size_t)L.B);
   for (int i = 0; i < max_steps; ++i) {
-    st = run_attn(desc, static_cast<const uint8_t*>(q_steps) + i * q_step,
-                  static_cast<const uint8_t*>(kc_steps) + i * kv_step,
-                  static_cast<const uint8_t*>(vc_steps) + i * kv_step, k_prefix, v_prefix,
-                  cu_prefix, cu_prefix_host, static_cast<uint8_t*>(attn_out) + i * q_step,
-                  nullptr, workspace, state_off, s);
+    st = adaptive_step(L, i, s);
     if (st != DD_OK) return st;
-    dd_sample_params sp;
-    sp.temperature = temperature_host[i];
-    sp.renoise_rate = 0.f;  // the acceptance rule below decides the re-noise
-    sp.seed = seed;
-    sp.step = step0 + (uint32_t)i;
-    sp.row_offset = 0;
-    st = run_sampler(static_cast<const uint8_t*>(logits_steps) + i * lg_step, desc->dtype, rows,
-                     vocab, vocab, &sp, cur, nullptr, conf, ent, nullptr, workspace, state_off, s,
-                     ws + state_off);
-    if (st != DD_OK) return st;
-    e = launch_stop_check(ent, cur, i > 0 ? prev : nullptr, B, C, (double)stop_entropy, i, done,
-                          halt_step, s);
-    if (e == cudaSuccess)
-      e = launch_entropy_accept(ent, cur, B, C, vocab, (double)budget, seed, step0 + (uint32_t)i, 0,
-                                done, halt_step, i, canvas, nullptr, s);
-    if (e == cudaSuccess && canvas_history)
-      e = cudaMemcpyAsync(canvas_history + (size_t)i * rows, canvas, (size_t)rows * sizeof(int32_t),
-                          cudaMemcpyDeviceToDevice, s);
-    if (e == cudaSuccess)
-      e = cudaMemcpyAsync(done_h.data(), done, (size_t)B, cudaMemcpyDeviceToHost, s);
+    e = cudaMemcpyAsync(done_h.data(), L.done, (size_t)L.B, cudaMemcpyDeviceToHost, s);
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
     if (e != cudaSuccess) return cuda_fail(e, "adaptive step");
     *steps_run = i + 1;
     bool all = true;
-    for (int b = 0; b < B; ++b) all = all && done_h[(size_t)b] != 0;
+    for (int b = 0; b < L.B; ++b) all = all && done_h[(size_t)b] != 0;
     if (all) break;
-    std::swap(cur, prev);
   }
+  return DD_OK;
+}
+
+struct dd_adaptive_graph_st {
+  cudaGraphExec_t exec;
+  uint64_t launches;  // kernels of every step body (an upper bound per replay)
+};
+
+// Builds and instantiates the adaptive loop's graph: memset nodes that reset
+// the loop state, then one IF node per step on a handle whose default is 1.
+// A failed CUDA call returns DD_ERR_CUDA with the call's name.
+static dd_status build_adaptive_graph(const AdaptiveLoop& L, int max_steps, int32_t* steps_run,
+                                      cudaGraphExec_t* exec_out, uint64_t* launches_out) {
+  dd_status st = DD_OK;
+  const char* what = nullptr;  // the CUDA call that failed
+  cudaError_t e = cudaSuccess;
+  auto ok = [&](cudaError_t r, const char* call) {
+    if (r != cudaSuccess && e == cudaSuccess) {
+      e = r;
+      what = call;
+    }
+    return e == cudaSuccess;
+  };
+  cudaGraph_t graph = nullptr;
+  cudaStream_t s = nullptr;
+  if (!ok(cudaGraphCreate(&graph, 0), "cudaGraphCreate")) return cuda_fail(e, "cudaGraphCreate");
+  // the loop's state is reset by the graph itself on every replay
+  std::vector<cudaGraphNode_t> deps;
+  auto add_memset = [&](void* dst, unsigned value, unsigned elem, size_t n) {
+    cudaMemsetParams mp = {};
+    mp.dst = dst;
+    mp.pitch = n * elem;
+    mp.value = value;
+    mp.elementSize = elem;
+    mp.width = n;
+    mp.height = 1;
+    cudaGraphNode_t node = nullptr;
+    if (ok(cudaGraphAddMemsetNode(&node, graph, nullptr, 0, &mp), "cudaGraphAddMemsetNode"))
+      deps.push_back(node);
+  };
+  add_memset(steps_run, 0u, 4, 1);
+  if (L.B > 0) add_memset(L.done, 0u, 1, (size_t)L.B);
+  if (L.B > 0) add_memset(L.halt_step, 0xffffffffu, 4, (size_t)L.B);
+  // one handle per IF node (a handle serves a single conditional node): step
+  // 0's defaults to 1 at every launch, the others to 0; step i's gate sets
+  // step i + 1's, so once every canvas has halted no later body runs
+  std::vector<cudaGraphConditionalHandle> handles(L.B > 0 ? (size_t)max_steps : 0);
+  for (size_t i = 0; i < handles.size(); ++i)
+    ok(cudaGraphConditionalHandleCreate(&handles[i], graph, i == 0 ? 1u : 0u,
+                                        cudaGraphCondAssignDefault),
+       "cudaGraphConditionalHandleCreate");
+  if (L.B > 0) ok(cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking), "cudaStreamCreateWithFlags");
+  const uint64_t l0 = g_launches;
+  for (int i = 0; e == cudaSuccess && st == DD_OK && L.B > 0 && i < max_steps; ++i) {
+    cudaGraphNodeParams np = {};
+    np.type = cudaGraphNodeTypeConditional;
+    np.conditional.handle = handles[(size_t)i];
+    np.conditional.type = cudaGraphCondTypeIf;
+    np.conditional.size = 1;
+    cudaGraphNode_t node = nullptr;
+    if (!ok(cudaGraphAddNode(&node, graph, deps.data(), deps.size(), &np), "cudaGraphAddNode"))
+      break;
+    cudaGraph_t body = np.conditional.phGraph_out[0];
+    if (!ok(cudaStreamBeginCaptureToGraph(s, body, nullptr, nullptr, 0,
+                                          cudaStreamCaptureModeRelaxed),
+            "cudaStreamBeginCaptureToGraph"))
+      break;
+    st = adaptive_step(L, i, s);
+    cudaError_t eg = cudaSuccess;
+    if (st == DD_OK) {
+      const bool has_next = i + 1 < max_steps;
+      eg = launch_adaptive_gate(L.done, L.B, i, steps_run,
+                                has_next ? handles[(size_t)i + 1] : handles[(size_t)i], has_next,
+                                s);
+    }
+    cudaGraph_t captured = nullptr;
+    const std::string detail = g_last_error;
+    ok(cudaStreamEndCapture(s, &captured), "cudaStreamEndCapture");
+    if (st != DD_OK) g_last_error = detail;
+    ok(eg, "gate kernel launch");
+    deps.assign(1, node);
+  }
+  *launches_out = g_launches - l0;
+  g_launches = l0;  // captured, not launched
+  if (s) cudaStreamDestroy(s);
+  if (st == DD_OK && e == cudaSuccess)
+    ok(cudaGraphInstantiate(exec_out, graph, 0), "cudaGraphInstantiate");
+  const std::string detail = g_last_error;
+  cudaGraphDestroy(graph);
+  g_last_error = detail;
+  if (st != DD_OK) return st;
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return cuda_fail(e, what);
+  }
+  return DD_OK;
+}
+
+dd_status dd_denoise_block_adaptive_graph_create(
+    dd_adaptive_graph* out, const dd_attn_desc* desc, int max_steps, const void* q_steps,
+    const void* kc_steps, const void* vc_steps, const void* k_prefix, const void* v_prefix,
+    const int32_t* cu_prefix, const int32_t* cu_prefix_host, void* attn_out,
+    const void* logits_steps, int vocab, const float* temperature_host, float budget,
+    float stop_entropy, uint64_t seed, uint32_t step0, int32_t* canvas, int32_t* canvas_history,
+    int32_t* halt_step, int32_t* steps_run, void* workspace, size_t workspace_bytes) {
+  g_last_error.clear();
+  if (!out) return fail(DD_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  if (!steps_run) return fail(DD_ERR_INVALID_ARG, "NULL required pointer");
+  AdaptiveLoop L;
+  dd_status st = adaptive_prepare(&L, desc, max_steps, q_steps, kc_steps, vc_steps, k_prefix,
+                                  v_prefix, cu_prefix, cu_prefix_host, attn_out, logits_steps,
+                                  vocab, temperature_host, budget, stop_entropy, seed, step0,
+                                  canvas, canvas_history, halt_step, workspace, workspace_bytes);
+  if (st != DD_OK) return st;
+  cudaGraphExec_t exec = nullptr;
+  uint64_t launches = 0;
+  st = build_adaptive_graph(L, max_steps, steps_run, &exec, &launches);
+  if (st == DD_ERR_CUDA) {
+    // programmatic dependencies inside conditional bodies are not accepted
+    // everywhere: build again with plain launches
+    const std::string first = g_last_error;
+    g_pdl_off = true;
+    st = build_adaptive_graph(L, max_steps, steps_run, &exec, &launches);
+    g_pdl_off = false;
+    if (st != DD_OK) {
+      const std::string second = g_last_error;
+      return fail(st, "with programmatic launches: %s; with plain launches: %s", first.c_str(),
+                  second.c_str());
+    }
+  }
+  if (st != DD_OK) return st;
+  *out = new dd_adaptive_graph_st{exec, launches};
+  return DD_OK;
+}
+
+dd_status dd_denoise_block_adaptive_graph_launch(dd_adaptive_graph g, dd_stream_t stream) {
+  g_last_error.clear();
+  if (!g) return fail(DD_ERR_INVALID_ARG, "graph is NULL");
+  cudaError_t e = cudaGraphLaunch(g->exec, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "launch adaptive graph");
+  g_launches += g->launches;
+  return DD_OK;
+}
+
+dd_status dd_denoise_block_adaptive_graph_destroy(dd_adaptive_graph g) {
+  g_last_error.clear();
+  if (!g) return DD_OK;
+  cudaError_t e = cudaGraphExecDestroy(g->exec);
+  delete g;
+  if (e != cudaSuccess) return cuda_fail(e, "destroy adaptive graph");
   return DD_OK;
 }
 

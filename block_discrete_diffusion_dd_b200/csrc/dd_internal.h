@@ -10,9 +10,14 @@
 
 namespace dd {
 
+// False on this host thread while work is captured where programmatic
+// dependencies are not accepted (launch_pdl then launches plainly).
+bool pdl_enabled();
+
 // Launch with programmatic stream serialisation (the kernel calls pdl_wait
 // before touching global memory): its launch overlaps the tail of the
 // previous kernel on the stream, in eager launches and in captured graphs.
+// (pdl_wait and launch_dependents are no-ops in a plain launch.)
 template <typename... KArgs, typename... Args>
 cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
                        cudaStream_t stream, Args&&... args) {
@@ -25,7 +30,7 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
@@ -69,6 +74,12 @@ cudaError_t launch_entropy_accept(const float* entropy, const int32_t* pred, int
 cudaError_t launch_stop_check(const float* entropy, const int32_t* pred, const int32_t* pred_prev,
                               int B, int C, double threshold, int32_t cur, uint8_t* done,
                               int32_t* halt_step, cudaStream_t stream);
+// Writes steps_run = step + 1 and (has_next) sets the next step's IF-node
+// condition of the on-device adaptive loop: 1 while a canvas is running, 0
+// once all have halted.
+cudaError_t launch_adaptive_gate(const uint8_t* done, int B, int32_t step, int32_t* steps_run,
+                                 cudaGraphConditionalHandle next, bool has_next,
+                                 cudaStream_t stream);
 cudaError_t launch_init_canvas(int32_t* canvas, int rows, int vocab, uint64_t seed,
                                uint32_t row_offset, cudaStream_t stream);
 

@@ -112,6 +112,24 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// Gate between two steps of the on-device adaptive loop: one warp reads
+// every canvas's halt flag, records that `step` has run, and (has_next) sets
+// the condition of the next step's IF node to 1 while some canvas is still
+// running and to 0 once all have halted.  A step whose body is skipped sets
+// nothing, so every later condition keeps its default 0.
+__global__ void __launch_bounds__(32)
+    adaptive_gate_kernel(const uint8_t* __restrict__ done, int B, int32_t step,
+                         int32_t* __restrict__ steps_run, cudaGraphConditionalHandle next,
+                         int has_next) {
+  bool all = true;
+  for (int b = threadIdx.x; b < B; b += 32) all = all && done[b] != 0;
+  all = __all_sync(0xffffffffu, all);
+  if (threadIdx.x == 0) {
+    *steps_run = step + 1;
+    if (has_next) cudaGraphSetConditional(next, all ? 0u : 1u);
+  }
+}
+
 int pow2_at_least(int c) {
   int n = 32;
   while (n < c) n <<= 1;
@@ -137,6 +155,14 @@ cudaError_t launch_stop_check(const float* entropy, const int32_t* pred, const i
                               int32_t* halt_step, cudaStream_t stream) {
   stop_check_kernel<<<B, 256, 0, stream>>>(entropy, pred, pred_prev, C, threshold, cur, done,
                                            halt_step);
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_adaptive_gate(const uint8_t* done, int B, int32_t step, int32_t* steps_run,
+                                 cudaGraphConditionalHandle next, bool has_next,
+                                 cudaStream_t stream) {
+  adaptive_gate_kernel<<<1, 32, 0, stream>>>(done, B, step, steps_run, next, has_next ? 1 : 0);
   note_launch();
   return cudaGetLastError();
 }

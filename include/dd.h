@@ -403,6 +403,38 @@ DD_API dd_status dd_denoise_block_adaptive(
     uint32_t step0, int32_t* canvas, int32_t* canvas_history, int32_t* halt_step, int* steps_run,
     void* workspace, size_t workspace_bytes, dd_stream_t stream);
 
+/* dd_denoise_block_adaptive with the loop kept on the device.  The steps
+ * are captured once into a CUDA graph: memset nodes that reset the loop
+ * state, then one conditional (IF) node per step, run in order.  A small
+ * kernel at the end of each step's body reads the halt flags and sets the
+ * next step's condition, to 0 once every canvas has halted, so the
+ * remaining steps' bodies are skipped on the device.  No step waits for the
+ * host.
+ *   dd_denoise_block_adaptive_graph_create captures the loop with exactly
+ *     these arguments (those of dd_denoise_block_adaptive, without the
+ *     stream, with steps_run a DEVICE int32 written by the graph) and
+ *     instantiates it.  It validates like dd_denoise_block_adaptive,
+ *     launches nothing and stores a handle in *out (NULL on failure).
+ *   dd_denoise_block_adaptive_graph_launch replays it on `stream`.  The
+ *     results (canvas, canvas_history rows 0 .. steps_run - 1, halt_step,
+ *     *steps_run) equal those of the eager call with the same arguments.
+ *     dd_launch_count counts every kernel of every step body per replay,
+ *     an upper bound, as the bodies skipped on the device are not known to
+ *     the host.  Buffers must stay allocated while the handle exists, and
+ *     replays that may overlap in time must not share a workspace.
+ *   dd_denoise_block_adaptive_graph_destroy frees it (NULL is accepted). */
+typedef struct dd_adaptive_graph_st* dd_adaptive_graph;
+DD_API dd_status dd_denoise_block_adaptive_graph_create(
+    dd_adaptive_graph* out, const dd_attn_desc* desc, int max_steps, const void* q_steps,
+    const void* kc_steps, const void* vc_steps, const void* k_prefix, const void* v_prefix,
+    const int32_t* cu_prefix, const int32_t* cu_prefix_host, void* attn_out,
+    const void* logits_steps, int vocab, const float* temperature_host, float budget,
+    float stop_entropy, uint64_t seed, uint32_t step0, int32_t* canvas, int32_t* canvas_history,
+    int32_t* halt_step, int32_t* steps_run, void* workspace, size_t workspace_bytes);
+DD_API dd_status dd_denoise_block_adaptive_graph_launch(dd_adaptive_graph graph,
+                                                        dd_stream_t stream);
+DD_API dd_status dd_denoise_block_adaptive_graph_destroy(dd_adaptive_graph graph);
+
 /* Clears a whole workspace: the error word and the sampler's state (async on
  * stream).  Call once before a workspace's first use. */
 DD_API dd_status dd_workspace_init(void* workspace, size_t workspace_bytes, dd_stream_t stream);

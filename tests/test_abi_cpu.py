@@ -233,6 +233,28 @@ def test_block_fp8_rejects_bad_arguments(lib):
     assert "dd_denoise_block_fp8" in dd.last_error()
 
 
+def test_adaptive_graph_rejects_bad_arguments(lib):
+    d = _desc()
+    cu = _cu([16])
+    t = np.full(2, 0.8, np.float32)
+    h = ctypes.c_void_p(123)
+
+    def create(out=ctypes.byref(h), steps_run=FAKE, ws_bytes=16, canvas=FAKE, temps=True):
+        return lib.dd_denoise_block_adaptive_graph_create(
+            out, ctypes.byref(d), 2, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+            cu.ctypes.data_as(ctypes.c_void_p), FAKE, FAKE, 1024,
+            t.ctypes.data_as(ctypes.c_void_p) if temps else None, 0.1, 0.005, 0, 0, canvas,
+            None, FAKE, steps_run, FAKE, ws_bytes)
+
+    assert create(out=None) == 1
+    assert create() == 3 and h.value is None                 # workspace too small; no handle
+    assert create(steps_run=None) == 1
+    assert create(canvas=None) == 1
+    assert create(temps=False) == 1
+    assert lib.dd_denoise_block_adaptive_graph_launch(None, None) == 1
+    assert lib.dd_denoise_block_adaptive_graph_destroy(None) == 0
+
+
 def test_init_canvas_rejects_bad_arguments(lib):
     assert lib.dd_init_canvas(None, 4, 10, 0, 0, None) == 1
     assert lib.dd_init_canvas(FAKE, 4, 0, 0, 0, None) == 1

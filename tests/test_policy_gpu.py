@@ -128,3 +128,59 @@ def test_adaptive_loop_equals_its_pieces_and_the_oracle_rule():
     np.testing.assert_array_equal(res["canvas"].cpu().numpy(), canvas.cpu().numpy())
     # the logits sharpen fast enough that every canvas halts before the last step
     assert (res["halt_step"].cpu().numpy() >= 1).all() and n < S
+
+
+def test_adaptive_graph_replays_the_eager_loop():
+    """dd_denoise_block_adaptive_graph: the loop on the device (one IF node
+    per step, cleared once every canvas has halted) gives the eager loop's
+    canvas, history, halt steps and step count, replay after replay, and
+    again after new inputs are written into the captured buffers."""
+    w, q, kc, vc, lg, kp, vp, cu = _adaptive_inputs()
+    S = q.shape[0]
+    temps = [oracle.anneal_temperature(s, 48) for s in range(S)]
+    budget, thr, seed = 0.1, 0.005, 21
+    cud = cu.to(DEV)
+    eager = dd.denoise_block_adaptive(q, kc, vc, kp, vp, cud, lg, temps, budget, thr, seed,
+                                      cu_prefix_host=cu, scale=w.scale)
+    n = eager["steps_run"]
+    assert n < S                                   # halts early: later bodies are skipped
+    lb = lg.clone()
+    g = dd.denoise_block_adaptive_graph(q, kc, vc, kp, vp, cud, lb, temps, budget, thr, seed,
+                                        cu_prefix_host=cu, scale=w.scale)
+    for _ in range(2):
+        t = g.launch()
+        torch.cuda.synchronize()
+        assert int(t["steps_run"].item()) == n
+        assert torch.equal(t["canvas"], eager["canvas"])
+        assert torch.equal(t["halt_step"], eager["halt_step"])
+        assert torch.equal(t["canvas_history"][:n], eager["canvas_history"])
+    # flatter logits for the first steps: the loop runs longer
+    lb[:2].copy_((lg[:2].float() * 0.25).to(torch.bfloat16))
+    ref = dd.denoise_block_adaptive(q, kc, vc, kp, vp, cud, lb.clone(), temps, budget, thr, seed,
+                                    cu_prefix_host=cu, scale=w.scale)
+    t = g.launch()
+    torch.cuda.synchronize()
+    m = ref["steps_run"]
+    assert int(t["steps_run"].item()) == m
+    assert torch.equal(t["canvas"], ref["canvas"])
+    assert torch.equal(t["halt_step"], ref["halt_step"])
+    assert torch.equal(t["canvas_history"][:m], ref["canvas_history"])
+    g.destroy()
+    dd.query_device_error(t["workspace"])
+
+
+def test_adaptive_graph_with_no_halt_runs_every_step():
+    """A threshold no canvas meets: every body runs; steps_run = max_steps."""
+    w, q, kc, vc, lg, kp, vp, cu = _adaptive_inputs(B=1, S=3)
+    temps = [0.8, 0.7, 0.6]
+    eager = dd.denoise_block_adaptive(q, kc, vc, kp, vp, cu.to(DEV), lg, temps, 0.1, -1.0, 4,
+                                      cu_prefix_host=cu, scale=w.scale)
+    assert eager["steps_run"] == 3
+    g = dd.denoise_block_adaptive_graph(q, kc, vc, kp, vp, cu.to(DEV), lg, temps, 0.1, -1.0, 4,
+                                        cu_prefix_host=cu, scale=w.scale)
+    t = g.launch()
+    torch.cuda.synchronize()
+    assert int(t["steps_run"].item()) == 3
+    assert torch.equal(t["canvas_history"], eager["canvas_history"])
+    assert t["halt_step"].tolist() == [-1]
+    g.destroy()
