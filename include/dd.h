@@ -18,7 +18,9 @@
  *   - Tensors are dense row-major ("C order"), last dimension fastest, with
  *     the shapes given below.  Device pointers must be 16-byte aligned.
  *   - Every call is asynchronous on `stream` (0 = the legacy default stream)
- *     and makes no host synchronisation, except dd_query_device_error.
+ *     and makes no host synchronisation, except dd_query_device_error and
+ *     dd_denoise_block_adaptive (which reads the halt flags after every
+ *     step; dd_denoise_block_adaptive_graph_* keep that loop on the device).
  *   - Errors: arguments are validated on the host BEFORE any launch.  Invalid
  *     shapes/pointers return DD_ERR_INVALID_ARG, shapes without a kernel
  *     return DD_ERR_UNSUPPORTED, a too-small workspace DD_ERR_WORKSPACE, a
