@@ -8,6 +8,11 @@ pass + row merge): every step of the hot path, through the C ABI
 8 kv heads, head_dim 128, prefix 4096, canvas 256, vocabulary 262144, bf16.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+  python bench.py --workload block12_L8192   # + the 12-step block loop: eager,
+                                             #   replayed graph, E4M3 inputs
+  python bench.py --policy       # the pages' adaptive block, eager and on-device loop
+  python bench.py --attn-e4m3 [--workload W]  # attention on 8-bit inputs beside bf16
+  python bench.py --soft-embed   # the self-conditioning soft embedding
 
 Prints ONE JSON line (rank 0).  `value` is canvas-steps/s over all ranks
 (each rank runs its own independent canvases: no collective on the data
