@@ -37,6 +37,11 @@ Parity status per function (what pins it; tests/test_oracle_*.py):
                                (constant logits -> mean embedding, one
                                dominant logit -> its embedding row),
                                temperature scaling, linearity in E.
+
+Regression fixtures: tests/golden/*.json, written from this package alone by
+tests/golden/make_golden.py (the pages print no worked example), freeze its
+outputs on small inputs; tests/test_golden_cpu.py checks that they still
+hold.
 """
 from __future__ import annotations
 
