@@ -145,3 +145,22 @@ def test_block_fp8_matches_the_step_calls_and_the_oracle():
                                       cu.numpy(), w.scale, positions=pos, qkv_scale=f[s])
         _check(out["attn_out"][s], ref_o, vcs[s].cpu(), vp.cpu(), f[s][2], 700 + 256,
                positions=pos)
+
+
+def test_block_fp8_ragged_batch_without_history():
+    """dd_denoise_block_fp8 on two canvases with prefixes 0 and 700 and no
+    history buffers: the final canvas equals the last step's one-by-one
+    calls (tokens of a rate-0 step are the sampled ids)."""
+    w = workloads.scaled(workloads.WORKLOADS["block12_L8192"], batch=2, prefix_lens=(0, 700),
+                         vocab=3000, steps=2, rates=(0.6, 0.0), temperatures=(1.0, 0.9),
+                         name="block2_e4m3_ragged")
+    qs, kcs, vcs, kp, vp, cu, f = workloads.e4m3_block_inputs(w, device=DEV)
+    ls = torch.stack([workloads.logits(w, s, device=DEV) for s in range(w.steps)])
+    out = dd.denoise_block_fp8(qs, kcs, vcs, kp, vp, cu.to(DEV), f, ls, w.rates, w.temperatures,
+                               seed=9, cu_prefix_host=cu, scale=w.scale, keep_history=False)
+    o, _ = dd.canvas_attn_fp8(qs[1], kcs[1], vcs[1], kp, vp, cu.to(DEV), f[1], cu, scale=w.scale)
+    r = dd.sample_renoise(ls[1], w.temperatures[1], w.rates[1], 9, 1)
+    torch.cuda.synchronize()
+    assert out["canvas_history"] is None and out["conf_steps"] is None
+    assert torch.equal(out["attn_out"][1], o)
+    assert torch.equal(out["canvas"], r["tokens"])
