@@ -4,8 +4,11 @@
 A step = canvas attention over [prefix KV || canvas KV] (tcgen05 kernel +
 split merge) followed by the vocabulary-wide sampler and re-noise (chunk
 pass + row merge): every step of the hot path, through the C ABI
-(dd_canvas_attn, dd_sample_renoise).  Default workload: batch 1, 16 query /
-8 kv heads, head_dim 128, prefix 4096, canvas 256, vocabulary 262144, bf16.
+(dd_canvas_attn, dd_sample_renoise).  Default workload (`ragged_b8`, the
+largest single-GPU configuration): a ragged batch of 8 canvases, 16 query /
+8 kv heads, head_dim 128, prefix lengths drawn from [512, 16384], canvas
+256, vocabulary 262144 (2048 x 262144 bf16 logits per step), bf16.  The
+batch-1 step is `--workload b1_L4096`.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
   python bench.py --workload block12_L8192   # + the 12-step block loop: eager,
@@ -17,8 +20,9 @@ pass + row merge): every step of the hot path, through the C ABI
 Prints ONE JSON line (rank 0).  `value` is canvas-steps/s over all ranks
 (each rank runs its own independent canvases: no collective on the data
 path), from CUDA events on the launch stream, max over ranks.  Inputs are
-rotated among 3 sets of ~152 MB each (> 126 MB L2) so no step reads the
-previous step's inputs from L2.
+rotated among 3 sets, each larger than the 126 MB L2 (1.35 GB for
+ragged_b8, 152 MB for b1_L4096), so no step reads the previous step's
+inputs from L2.
 """
 from __future__ import annotations
 
@@ -286,7 +290,7 @@ def run_ours(args, w, dist, rank, world, local_rank):
     if w.steps > 1:
         res["block"] = run_block(w, dd, dev, dist)
     if rank == 0 and world == 1 and not args.no_cpu:
-        res["cpu_baseline"] = cpu_baseline(w, sets[0], frac=args.cpu_sample)
+        res["cpu_baseline"] = cpu_baseline(w, sets[0])
     return res
 
 
@@ -588,95 +592,133 @@ def _profile_traffic() -> dict:
     return out
 
 
-def cpu_baseline(w, s, frac: float, budget_s: float = 10.0):
-    """The oracle, as it stands, on this host's cores, on a bounded sample of
-    the workload: slices of `frac` of the canvas positions (attention, all
-    heads) and of the rows (sampler), repeated over different positions and
-    rows for about `budget_s` seconds, scaled to whole steps."""
+def _cpu_model() -> str:
+    """The host CPU's model name (lscpu), for the baseline's record."""
+    try:
+        out = subprocess.run(["lscpu"], capture_output=True, text=True, timeout=10).stdout
+        for line in out.splitlines():
+            if line.startswith("Model name:"):
+                return line.split(":", 1)[1].strip()
+    except Exception:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def _host_cores() -> int:
+    if "OMP_NUM_THREADS" in os.environ:
+        return int(os.environ["OMP_NUM_THREADS"])
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def oracle_sample_plan(w, cores: int):
+    """The bounded sample of one step that both CPU legs (the `cpu_baseline`
+    of our line and the `--impl reference` arm) time: `npos` canvas positions
+    of every batch row and head for the attention, and `nrows` sampler rows,
+    at least two units of work per core (and 16 rows) so every core is busy.
+    The step time is extrapolated from it: attention x C / npos, sampler x
+    R / nrows."""
+    npos = min(w.canvas, max(8, -(-2 * cores // (w.batch * w.heads_q))))
+    nrows = min(w.rows, max(16, 2 * cores))
+    return npos, nrows
+
+
+def _oracle_sample(w, s, lg, npos, nrows, rep, threads=0):
+    """One timed sample of the oracle step: (attention s, sampler s), over
+    positions and rows spread evenly and rotated by `rep`."""
+    import oracle
+    off = (rep * 37) % w.canvas
+    pos = ((np.arange(npos) * (w.canvas // npos) + off) % w.canvas).astype(np.int32)
+    sel = ((np.arange(nrows) * (w.rows // nrows) + off) % w.rows).astype(np.int64)
+    t0 = time.perf_counter()
+    oracle.canvas_attn(s["q"], s["kc"], s["vc"], s["kp"], s["vp"], s["cu_host"], w.scale,
+                       positions=pos, threads=threads)
+    t1 = time.perf_counter()
+    oracle.sample_renoise(lg, w.temperatures[0], w.rates[0], w.seed, rep, rows=sel,
+                          threads=threads)
+    t2 = time.perf_counter()
+    return t1 - t0, t2 - t1
+
+
+def _extrapolate(w, t_attn, t_samp, npos, nrows):
+    return t_attn * (w.canvas / npos) + t_samp * (w.rows / nrows)
+
+
+def cpu_baseline(w, s, budget_s: float = 10.0):
+    """The oracle, as it stands, on this host's cores, on the bounded sample
+    of oracle_sample_plan, repeated for about `budget_s` seconds and
+    extrapolated to whole steps; plus one sample on a single thread."""
     import oracle
     oracle.build()
-    npos = max(1, int(round(w.canvas * frac)))
-    rows = max(1, int(round(w.rows * frac)))
+    cores = _host_cores()
+    npos, nrows = oracle_sample_plan(w, cores)
     q, kc, vc, kp, vp = (s[k].cpu() for k in ("q", "kc", "vc", "kp", "vp"))
+    host = {"q": q, "kc": kc, "vc": vc, "kp": kp, "vp": vp, "cu_host": s["cu_host"]}
     lg = s["logits"].cpu()
-    t_attn = t_samp = 0.0
+    ta = ts = 0.0
     reps = 0
     t_start = time.perf_counter()
     while reps == 0 or time.perf_counter() - t_start < budget_s:
-        off = (reps * 37) % w.canvas
-        pos = ((np.arange(npos) * (w.canvas // npos) + off) % w.canvas).astype(np.int32)
-        sel = ((np.arange(rows) * (w.rows // rows) + off) % w.rows).astype(np.int64)
-        t0 = time.perf_counter()
-        oracle.canvas_attn(q, kc, vc, kp, vp, s["cu_host"], w.scale, positions=pos)
-        t1 = time.perf_counter()
-        oracle.sample_renoise(lg, w.temperatures[0], w.rates[0], w.seed, reps, rows=sel)
-        t2 = time.perf_counter()
-        t_attn += t1 - t0
-        t_samp += t2 - t1
-        reps += 1
-    step_s = (t_attn * (w.canvas / npos) + t_samp * (w.rows / rows)) / reps
-    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+        a, b = _oracle_sample(w, host, lg, npos, nrows, reps)
+        ta, ts, reps = ta + a, ts + b, reps + 1
+    step_s = _extrapolate(w, ta / reps, ts / reps, npos, nrows)
+    a1, b1 = _oracle_sample(w, host, lg, npos, nrows, reps, threads=1)
+    step1_s = _extrapolate(w, a1, b1, npos, nrows)
     return {"value": w.batch / step_s, "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": f"{reps} x ({npos}/{w.canvas} canvas positions, all heads, for attention "
-                      f"+ {rows}/{w.rows} sampler rows), float64, {t_attn + t_samp:.1f} s of "
-                      "wall time on all host cores, scaled to whole steps",
-            "seconds": t_attn + t_samp}
+            "extrapolated": True,
+            "sample": f"{reps} x ({npos}/{w.canvas} canvas positions of every batch row and "
+                      f"head for attention + {nrows}/{w.rows} sampler rows), float64, "
+                      f"{ta + ts:.1f} s on {cores} host cores; extrapolated to whole steps",
+            "per_step_s": {"attention": ta / reps * (w.canvas / npos),
+                           "sampler": ts / reps * (w.rows / nrows)},
+            "one_thread": {"value": w.batch / step1_s, "unit": UNIT,
+                           "per_step_s": {"attention": a1 * (w.canvas / npos),
+                                          "sampler": b1 * (w.rows / nrows)}},
+            "cpu_model": _cpu_model(), "seconds": ta + ts}
 
 
 def run_reference(args, w, dist, rank, world):
-    """The reference arm: the oracle timed on host cores, each step a bounded
-    sample of the workload scaled to a whole step."""
+    """The reference arm: the oracle timed on host cores, each step the
+    bounded sample of oracle_sample_plan (the same sample as our line's
+    cpu_baseline), extrapolated to a whole step."""
     if rank != 0:
         return None
     import oracle
     oracle.build()
-    frac = args.ref_sample
-    s = {}
+    cores = _host_cores()
+    npos, nrows = oracle_sample_plan(w, cores)
     ws0 = workloads.scaled(w)
+    s = {}
     s["q"], s["kc"], s["vc"] = workloads.canvas_qkv(ws0, 0)
     s["kp"], s["vp"], cu = workloads.prefix_kv(ws0)
     s["cu_host"] = cu.numpy()
     lg = workloads.logits(ws0, 0)
-    # size the per-step sample so the whole run stays within ~2 minutes
-    budget = 120.0 / (args.warmup + args.steps)
-    t0 = time.perf_counter()
-    oracle.canvas_attn(s["q"], s["kc"], s["vc"], s["kp"], s["vp"], s["cu_host"], w.scale,
-                       positions=np.arange(max(1, int(w.canvas * frac)), dtype=np.int32))
-    oracle.sample_renoise(lg, w.temperatures[0], w.rates[0], w.seed, 0,
-                          rows=np.arange(max(1, int(w.rows * frac))))
-    probe = time.perf_counter() - t0
-    if probe > budget:
-        frac = max(frac * budget / probe, 1.0 / w.canvas)
-    npos = max(1, int(round(w.canvas * frac)))
-    rows = max(1, int(round(w.rows * frac)))
-    times = []
+    ta, ts = [], []
     for i in range(args.warmup + args.steps):
-        off = (i * 7) % w.canvas
-        pos = ((np.arange(npos) * (w.canvas // npos) + off) % w.canvas).astype(np.int32)
-        sel = ((np.arange(rows) * (w.rows // rows) + off) % w.rows).astype(np.int64)
-        t0 = time.perf_counter()
-        oracle.canvas_attn(s["q"], s["kc"], s["vc"], s["kp"], s["vp"], s["cu_host"], w.scale,
-                           positions=pos)
-        t1 = time.perf_counter()
-        oracle.sample_renoise(lg, w.temperatures[0], w.rates[0], w.seed, i, rows=sel)
-        t2 = time.perf_counter()
+        a, b = _oracle_sample(w, s, lg, npos, nrows, i)
         if i >= args.warmup:
-            times.append((t1 - t0) * (w.canvas / npos) + (t2 - t1) * (w.rows / rows))
-    step_s = statistics.mean(times)
-    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+            ta.append(a)
+            ts.append(b)
+    t_attn, t_samp = statistics.mean(ta), statistics.mean(ts)
+    step_s = _extrapolate(w, t_attn, t_samp, npos, nrows)
     value = w.batch / step_s
-    sample = (f"{npos}/{w.canvas} canvas positions (all heads) and {rows}/{w.rows} sampler rows "
-              "per step, float64 oracle, scaled to a whole step")
+    sample = (f"{npos}/{w.canvas} canvas positions of every batch row and head (attention) and "
+              f"{nrows}/{w.rows} sampler rows per step, float64 oracle on {cores} host cores; "
+              "extrapolated to a whole step")
     return {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "impl": "reference",
+            "impl": "reference", "extrapolated": True,
+            "timed_ms_per_step": (t_attn + t_samp) * 1e3,
             "config": {"workload": w.name, "batch_per_gpu": w.batch, "canvas": w.canvas,
                        "heads_q": w.heads_q, "heads_kv": w.heads_kv, "head_dim": w.head_dim,
                        "prefix": list(w.prefix_lens), "vocab": w.vocab,
                        "parallelism": "host cores (rank 0 only)"},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                             "sample": sample},
+                             "sample": sample, "cpu_model": _cpu_model()},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0},
             "gpu_launches": 0}
@@ -805,12 +847,10 @@ def main():
     ap.add_argument("--steps", type=int, default=20000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="b1_L4096", choices=list(workloads.WORKLOADS))
+    ap.add_argument("--workload", default="ragged_b8", choices=list(workloads.WORKLOADS))
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--no-cpu", action="store_true")
-    ap.add_argument("--cpu-sample", type=float, default=0.125)
-    ap.add_argument("--ref-sample", type=float, default=1.0 / 32)
     ap.add_argument("--policy", action="store_true",
                     help="time the pages' adaptive block loop instead (one JSON line)")
     ap.add_argument("--attn-e4m3", action="store_true",

@@ -174,10 +174,13 @@ dd_status run_attn(const dd_attn_desc* d, const void* q, const void* kc, const v
 
 // `state` is the sampler's persistent state, or nullptr for the standalone
 // layout (state after the header, records after the state).
-dd_status run_sampler(const void* logits, dd_dtype dtype, int rows, int vocab, int64_t row_stride,
-                      const dd_sample_params* p, int32_t* tokens, int32_t* pred, float* conf,
-                      float* entropy, uint8_t* renoised, void* ws, size_t ws_bytes,
-                      cudaStream_t stream, void* state = nullptr) {
+}  // namespace
+
+// The argument checks of a sampler call that need neither a device nor a
+// workspace; a call with rows == 0 passes them and then does nothing.
+dd_status check_sampler_call(const void* logits, dd_dtype dtype, int rows, int vocab,
+                             int64_t row_stride, const dd_sample_params* p,
+                             const int32_t* tokens, const float* conf) {
   if (!p) return fail(DD_ERR_INVALID_ARG, "params is NULL");
   if (dtype != DD_BF16 && dtype != DD_F32)
     return fail(DD_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
@@ -191,8 +194,20 @@ dd_status run_sampler(const void* logits, dd_dtype dtype, int rows, int vocab, i
     return fail(DD_ERR_INVALID_ARG, "renoise_rate must lie in [0, 1]");
   if ((uint64_t)rows + p->row_offset > (1ull << 32))
     return fail(DD_ERR_INVALID_ARG, "row_offset + rows exceeds 2^32");
+  if (rows > 0 && (!logits || !tokens || !conf))
+    return fail(DD_ERR_INVALID_ARG, "NULL required pointer");
+  return DD_OK;
+}
+
+namespace {
+
+dd_status run_sampler(const void* logits, dd_dtype dtype, int rows, int vocab, int64_t row_stride,
+                      const dd_sample_params* p, int32_t* tokens, int32_t* pred, float* conf,
+                      float* entropy, uint8_t* renoised, void* ws, size_t ws_bytes,
+                      cudaStream_t stream, void* state = nullptr) {
+  dd_status st = check_sampler_call(logits, dtype, rows, vocab, row_stride, p, tokens, conf);
+  if (st != DD_OK) return st;
   if (rows == 0) return DD_OK;
-  if (!logits || !tokens || !conf) return fail(DD_ERR_INVALID_ARG, "NULL required pointer");
   if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u))
     return fail(DD_ERR_WORKSPACE, "workspace must be non-NULL and 256-byte aligned");
   const size_t need = state ? kHeaderBytes + sampler_record_bytes(rows, vocab)
@@ -234,12 +249,23 @@ thread_local bool g_pdl_off = false;
 bool pdl_enabled() { return !g_pdl_off; }
 
 // Entry for callers that bring their own scratch region (dd_noalloc.cu):
-// the same validation and kernels as dd_sample_renoise.
+// the same validation and kernels as dd_sample_renoise.  After the checks,
+// and before the kernels, the part of the scratch the call reads before
+// writing (the error word, the work counter and this call's row maxima) is
+// cleared on the stream, so a call that failed on the device earlier, and
+// left that state dirty, cannot affect this one.
 dd_status sample_with_scratch(const void* logits, dd_dtype dtype, int rows, int vocab,
                               int64_t row_stride, const dd_sample_params* p, int32_t* tokens,
                               int32_t* pred, float* conf, float* entropy, uint8_t* renoised,
                               void* scratch, size_t scratch_bytes, cudaStream_t stream) {
   g_last_error.clear();
+  dd_status st = check_sampler_call(logits, dtype, rows, vocab, row_stride, p, tokens, conf);
+  if (st != DD_OK || rows == 0) return st;
+  const size_t clear = kHeaderBytes + align256(sampler_state_bytes(rows));
+  if (!scratch || scratch_bytes < clear)
+    return fail(DD_ERR_WORKSPACE, "scratch too small: %zu < %zu bytes", scratch_bytes, clear);
+  cudaError_t e = cudaMemsetAsync(scratch, 0, clear, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "clearing the sampler state");
   return run_sampler(logits, dtype, rows, vocab, row_stride, p, tokens, pred, conf, entropy,
                      renoised, scratch, scratch_bytes, stream);
 }

@@ -10,9 +10,12 @@
 // device error word, the sampler's ticket counter and row keys, and the
 // per-chunk partial records) in one file-scope static __device__ array of
 // kStaticScratchBytes, which every GPU that loads the library holds until
-// the process exits.  The array starts zeroed, as the counter and the row
-// keys must be, and every call leaves them zero again.  The caller still
-// passes the logits and every output buffer.
+// the process exits.  Every call clears the part of it that it reads before
+// writing (error word, counter, its rows' maxima) on the stream before its
+// kernels run, so a call that failed on the device cannot leave a later one
+// wrong.  The caller still passes the logits and every output buffer.
+#include <cuda.h>
+
 #include <cstdio>
 #include <mutex>
 
@@ -25,6 +28,9 @@ dd_status sample_with_scratch(const void* logits, dd_dtype dtype, int rows, int 
                               int64_t row_stride, const dd_sample_params* p, int32_t* tokens,
                               int32_t* pred, float* conf, float* entropy, uint8_t* renoised,
                               void* scratch, size_t scratch_bytes, cudaStream_t stream);
+dd_status check_sampler_call(const void* logits, dd_dtype dtype, int rows, int vocab,
+                             int64_t row_stride, const dd_sample_params* p,
+                             const int32_t* tokens, const float* conf);
 dd_status set_error(dd_status st, const char* msg);
 
 namespace {
@@ -37,10 +43,49 @@ constexpr int kMaxDevices = 64;
 static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
 
 std::mutex g_setup_mu;
-void* g_scratch_addr[kMaxDevices] = {};
 
-// Once per device, with that device current: resolve the array's device
-// address.  Returns nullptr (and sets the error text) on failure.
+// The array's device address is looked up once per CUDA context: a device
+// reset (or any teardown of the context) reloads the module, and the array
+// may then sit at another address.  The context is identified by its
+// driver-assigned id, which is never reused within a process.
+struct ScratchAddr {
+  unsigned long long ctx_id;
+  void* ptr;
+};
+ScratchAddr g_scratch_addr[kMaxDevices] = {};
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+// Id of the current context, or 0 if the driver cannot tell (the address is
+// then looked up again on every call).
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(f);
+    f = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(f);
+    cudaGetLastError();
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current && get_id && get_current(&ctx) == CUDA_SUCCESS && ctx != nullptr &&
+      get_id(ctx, &id) == CUDA_SUCCESS)
+    return id;
+  return 0;
+}
+
+// With the device current: the array's device address in the current
+// context, looked up (cudaGetSymbolAddress) the first time a context is
+// seen.  Returns nullptr (and sets the error text) on failure.
 void* scratch_for_current_device(dd_status* st) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
@@ -48,8 +93,12 @@ void* scratch_for_current_device(dd_status* st) {
     *st = set_error(DD_ERR_CUDA, "dd_sample_renoise_noalloc: no usable current CUDA device");
     return nullptr;
   }
+  // cudaGetSymbolAddress below also makes the device's primary context
+  // current if none is, so the id is read after it on a first call
   std::lock_guard<std::mutex> lock(g_setup_mu);
-  if (g_scratch_addr[dev] == nullptr) {
+  ScratchAddr& slot = g_scratch_addr[dev];
+  const unsigned long long id = current_context_id();
+  if (slot.ptr == nullptr || id == 0 || slot.ctx_id != id) {
     void* ptr = nullptr;
     e = cudaGetSymbolAddress(&ptr, g_static_scratch);
     if (e != cudaSuccess || ptr == nullptr) {
@@ -59,9 +108,10 @@ void* scratch_for_current_device(dd_status* st) {
       *st = set_error(DD_ERR_CUDA, msg);
       return nullptr;
     }
-    g_scratch_addr[dev] = ptr;
+    slot.ptr = ptr;
+    slot.ctx_id = current_context_id();
   }
-  return g_scratch_addr[dev];
+  return slot.ptr;
 }
 
 }  // namespace
@@ -75,7 +125,11 @@ extern "C" dd_status dd_sample_renoise_noalloc(const void* logits, dd_dtype dtyp
                                                int32_t* tokens_out, int32_t* pred_out,
                                                float* conf_out, float* entropy_out,
                                                uint8_t* renoised_out, dd_stream_t stream) {
-  // size check first: it needs no device
+  // every check that needs no device comes first: a rejected call queues no
+  // GPU work (and leaves nothing in a graph being captured)
+  dd_status st = check_sampler_call(logits, dtype, rows, vocab, row_stride, params, tokens_out,
+                                    conf_out);
+  if (st != DD_OK) return st;
   const size_t need = dd_sample_renoise_workspace(rows, vocab, dtype);
   if (need == 0)
     return set_error(DD_ERR_INVALID_ARG, "dd_sample_renoise_noalloc: invalid rows/vocab/dtype");
@@ -89,14 +143,10 @@ extern "C" dd_status dd_sample_renoise_noalloc(const void* logits, dd_dtype dtyp
     return set_error(DD_ERR_UNSUPPORTED, msg);
   }
   if (rows == 0) return DD_OK;
-  dd_status st = DD_OK;
   void* scratch = scratch_for_current_device(&st);
   if (scratch == nullptr) return st;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  // the error word is OR-accumulated by the kernels: it starts every call at
-  // zero (the partial records need no clearing: each is written before read)
-  cudaError_t e = cudaMemsetAsync(scratch, 0, 16, s);
-  if (e != cudaSuccess) return set_error(DD_ERR_CUDA, "dd_sample_renoise_noalloc: memset failed");
+  // clears the state this call reads, then runs the kernels
   return sample_with_scratch(logits, dtype, rows, vocab, row_stride, params, tokens_out, pred_out,
-                             conf_out, entropy_out, renoised_out, scratch, kStaticScratchBytes, s);
+                             conf_out, entropy_out, renoised_out, scratch, kStaticScratchBytes,
+                             reinterpret_cast<cudaStream_t>(stream));
 }

@@ -326,12 +326,20 @@ DD_API dd_status dd_soft_embed(const void* logits, dd_dtype dtype, int rows, int
  * per row: up to 1927 rows at V = 262144); larger calls return
  * DD_ERR_UNSUPPORTED before touching the GPU.  The function allocates
  * nothing: no cudaMalloc, cudaFree or allocating library call.
- * The first call on a device looks up the array's device address
- * (cudaGetSymbolAddress), so make that first call before any stream capture.
+ * Arguments are checked before any GPU work is queued (a rejected call
+ * queues nothing); rows == 0 returns DD_OK after the same checks as
+ * dd_sample_renoise.  Each call clears, on the stream and before its
+ * kernels, the part of the array it reads before writing (an error word, a
+ * work counter and its rows' maxima, about 512 + 128 * rows bytes), so a
+ * call that failed on the device does not affect later calls.
+ * The first call in each CUDA context (on each device, and again after a
+ * device reset) looks up the array's device address with
+ * cudaGetSymbolAddress, so make that call before any stream capture.
  * Every call shares the array: calls that overlap on the GPU (two streams,
- * or two host threads) race and may return wrong results.  Device-side
- * timeouts are latched in the array but not reported by this entry point;
- * use dd_sample_renoise and dd_query_device_error to observe them. */
+ * or two host threads) race and may return wrong results.  A bounds error
+ * that the merge kernel detects is cleared by the next call and is not
+ * reported by this entry point (dd_sample_renoise with
+ * dd_query_device_error reports it). */
 DD_API dd_status dd_sample_renoise_noalloc(const void* logits, dd_dtype dtype, int rows, int vocab,
                                            int64_t row_stride, const dd_sample_params* params,
                                            int32_t* tokens_out, int32_t* pred_out,

@@ -33,6 +33,14 @@ Parity status per function (what pins it; tests/test_oracle_*.py):
                                rule pinned above.
   denoise_block             -- a loop of the two pinned functions (plain
                                Python), checked for step0-restart identity.
+  entropy_accept / stop_check -- greedy budgeted-prefix properties, closed
+                               forms, ties, the strict threshold.
+  denoise_block_adaptive    -- a loop of the pinned sampler, halt test and
+                               acceptance (plain Python); closed cases built
+                               so every step's outcome is known: a halt at
+                               a chosen step, two canvases halting at
+                               different steps with the first frozen, no
+                               halt within max_steps.
   soft_embed                -- pure-Python brute force, closed forms
                                (constant logits -> mean embedding, one
                                dominant logit -> its embedding row),
@@ -305,6 +313,100 @@ def stop_check(entropy, pred, pred_prev, canvas: int, threshold: float = 0.005):
     done = np.empty(B, np.uint8)
     lib.oracle_stop_check(_ptr(h), _ptr(pr), _ptr(pp), B, canvas, float(threshold), _ptr(done))
     return done
+
+
+def _acceptance_margin(h32: np.ndarray, budget: float) -> float:
+    """How far one canvas's acceptance is from flipping: the distance of the
+    budget to the float64 running sum on either side of the cut, and the gap
+    between the last accepted and the first rejected entropy (a smaller
+    perturbation of the entropies cannot change the accepted set)."""
+    order = np.lexsort((np.arange(h32.size), h32))     # entropy, then position
+    hs = [float(x) for x in h32[order]]
+    total, k = 0.0, 0
+    while k < len(hs) and total + hs[k] <= budget:     # the acceptance walk
+        total += hs[k]
+        k += 1
+    m = np.inf
+    if k > 0:
+        m = min(m, budget - total)
+    if k < len(hs):
+        m = min(m, total + hs[k] - budget)
+        if k > 0:
+            m = min(m, hs[k] - hs[k - 1])
+    return float(m)
+
+
+def denoise_block_adaptive(logits_steps, temperatures, budget: float, stop_entropy: float,
+                           seed: int, canvas: int, max_steps=None, step0: int = 0,
+                           init_canvas=None, threads: int = 0):
+    """The pages' adaptive block loop ("DiffusionGemma Technical Report"
+    (paperfeed review), "The mechanism", sampler paragraph): per step, the
+    sampler at that step's temperature with no scheduled re-noise, the halt
+    test (low mean entropy and the same prediction as the previous step),
+    then the entropy-budget acceptance.  Readings: a canvas that halts at
+    step s takes its step-s prediction everywhere and later steps leave it
+    alone; the loop ends once every canvas has halted, or after max_steps.
+
+    The sampler's entropies are rounded to float32 (the precision the step
+    outputs them in) before the halt test and the acceptance, which sum
+    them in float64.  Composed in plain Python from sample_renoise,
+    stop_check and entropy_accept, each pinned on its own.
+
+    logits_steps: [S, B*canvas, V] (bf16 or float32).  Returns a dict:
+      canvas [B*C], history [steps_run, B*C], halt_step [B] (-1 = never),
+      steps_run, and per step (lists of [B] arrays) the margins of its
+      decisions, for telling a genuine mismatch from a near-boundary one:
+      min_gap (smallest top-two Gumbel score gap in the canvas),
+      stop_margin (|mean entropy - stop_entropy|), accept_margin
+      (_acceptance_margin), plus pred and entropy (float32) per step.
+    """
+    S = len(logits_steps) if max_steps is None else int(max_steps)
+    R = int(logits_steps[0].shape[0])
+    assert R % canvas == 0
+    B = R // canvas
+    cur = (np.zeros(R, np.int32) if init_canvas is None
+           else np.asarray(init_canvas, np.int32).copy())
+    done = np.zeros(B, bool)
+    halt = np.full(B, -1, np.int32)
+    prev = None
+    out = {"history": [], "min_gap": [], "stop_margin": [], "accept_margin": [], "pred": [],
+           "entropy": []}
+    steps_run = 0
+    for s in range(S):
+        r = sample_renoise(logits_steps[s], temperatures[s], 0.0, seed, step0 + s,
+                           threads=threads)
+        pred = r["pred"]
+        h32 = r["entropy"].astype(np.float32)
+        now = stop_check(h32, pred, prev, canvas, stop_entropy).astype(bool) & ~done
+        acc = entropy_accept(h32, pred, canvas, budget, seed, step0 + s, int(
+            logits_steps[s].shape[-1]))
+        gap, stop_m, acc_m = (np.empty(B) for _ in range(3))
+        for b in range(B):
+            sl = slice(b * canvas, (b + 1) * canvas)
+            gap[b] = r["gap"][sl].min()
+            stop_m[b] = abs(h32[sl].astype(np.float64).sum() / canvas - stop_entropy)
+            acc_m[b] = _acceptance_margin(h32[sl], budget)
+            if done[b]:
+                continue                        # halted at an earlier step: frozen
+            if now[b]:
+                cur[sl] = pred[sl]              # halts now: its whole prediction
+                halt[b] = s
+            else:
+                cur[sl] = acc["tokens"][sl]
+        done |= now
+        out["history"].append(cur.copy())
+        out["min_gap"].append(gap)
+        out["stop_margin"].append(stop_m)
+        out["accept_margin"].append(acc_m)
+        out["pred"].append(pred)
+        out["entropy"].append(h32)
+        prev = pred
+        steps_run = s + 1
+        if done.all():
+            break
+    out.update(canvas=cur, halt_step=halt, steps_run=steps_run,
+               history=np.stack(out["history"]) if out["history"] else np.zeros((0, R), np.int32))
+    return out
 
 
 # ---------------------------------------- self-conditioning soft embedding

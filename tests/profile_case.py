@@ -1,7 +1,7 @@
 """Run a few calls of the denoise-step kernels on one workload, for profilers.
 
-    python -m block_discrete_diffusion_dd_b200.profile_case [workload] [calls] [e4m3]
-    python -m block_discrete_diffusion_dd_b200.profile_case [workload] [calls] soft_embed [vocab]
+    python tests/profile_case.py [workload] [calls] [e4m3]
+    python tests/profile_case.py [workload] [calls] soft_embed [vocab]
 
 Each call is one dd_canvas_attn (dd_canvas_attn_fp8 on the workload's E4M3
 inputs with `e4m3`) and one dd_sample_renoise on the workload's step-0

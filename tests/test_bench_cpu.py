@@ -45,3 +45,30 @@ def test_committed_traffic_entries_parse():
     t = bench._profile_traffic()
     for k in ("sampler", "attention", "attention_e4m3", "soft_embed"):
         assert k in t
+
+
+def test_oracle_sample_plan_keeps_every_core_busy():
+    import workloads
+    for name, w in workloads.WORKLOADS.items():
+        for cores in (1, 8, 16, 64):
+            npos, nrows = bench.oracle_sample_plan(w, cores)
+            assert 1 <= npos <= w.canvas and 1 <= nrows <= w.rows
+            assert nrows == w.rows or nrows >= max(16, 2 * cores)
+            assert npos == w.canvas or npos * w.batch * w.heads_q >= 2 * cores
+
+
+def test_reference_arm_runs_the_oracle_on_the_shared_sample():
+    """The --impl reference arm on the small fp32 workload: the oracle on the
+    host cores, on the same sample plan as our line's cpu_baseline."""
+    import types
+    import workloads
+    w = workloads.WORKLOADS["tiny_fp32"]
+    args = types.SimpleNamespace(steps=2, warmup=1)
+    r = bench.run_reference(args, w, None, 0, 1)
+    assert r["impl"] == "reference" and r["extrapolated"] is True
+    assert r["value"] > 0 and r["unit"] == bench.UNIT and r["gpu_launches"] == 0
+    npos, nrows = bench.oracle_sample_plan(w, r["cpu_baseline"]["cores"])
+    assert f"{npos}/{w.canvas}" in r["cpu_baseline"]["sample"]
+    assert f"{nrows}/{w.rows}" in r["cpu_baseline"]["sample"]
+    assert r["e2e"]["value"] == r["value"]
+    assert bench.run_reference(args, w, None, 1, 2) is None      # other ranks: no work

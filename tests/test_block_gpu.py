@@ -21,7 +21,15 @@ def block12():
     return w, qs, kcs, vcs, ls, kp, vp, cu
 
 
-def test_block12_every_step_matches_oracle(block12):
+@pytest.fixture(scope="module")
+def block12_ref(block12):
+    """The oracle's sampler of every step of the 12-step block."""
+    w, qs, kcs, vcs, ls, kp, vp, cu = block12
+    return [oracle.sample_renoise(ls[s].cpu(), w.temperatures[s], w.rates[s], w.seed, s)
+            for s in range(w.steps)]
+
+
+def test_block12_every_step_matches_oracle(block12, block12_ref):
     w, qs, kcs, vcs, ls, kp, vp, cu = block12
     init = dd.init_canvas(w.rows, w.vocab, w.seed)
     np.testing.assert_array_equal(init.cpu().numpy(), oracle.init_canvas(w.rows, w.vocab, w.seed))
@@ -32,7 +40,7 @@ def test_block12_every_step_matches_oracle(block12):
     assert torch.equal(out["canvas"], hist[-1])
     ties = 0
     for s in range(w.steps):
-        ref = oracle.sample_renoise(ls[s].cpu(), w.temperatures[s], w.rates[s], w.seed, s)
+        ref = block12_ref[s]
         got = {"tokens": hist[s], "conf": out["conf_steps"][s]}
         st = check_sampler(got, ref)
         ties += st["near_tie_mismatches"]
@@ -75,10 +83,11 @@ def test_block_without_history_buffers():
     assert not bad.any()
 
 
-def test_block_graph_replays_the_eager_loop(block12):
-    """dd_denoise_block_graph: one capture, replays identical to the eager
-    loop, including after new inputs are written into the captured buffers,
-    and with the launch count of the eager loop."""
+def test_block_graph_replays_the_eager_loop(block12, block12_ref):
+    """dd_denoise_block_graph: one capture, every replay's steps against the
+    oracle, replays identical to the eager loop, including after new inputs
+    are written into the captured buffers, and with the launch count of the
+    eager loop."""
     w, qs, kcs, vcs, ls, kp, vp, cu = block12
     eager = dd.denoise_block(qs, kcs, vcs, kp, vp, cu.to(DEV), ls, w.rates, w.temperatures,
                              seed=w.seed, cu_prefix_host=cu)
@@ -95,6 +104,9 @@ def test_block_graph_replays_the_eager_loop(block12):
     for _ in range(2):
         out = g.launch()
         torch.cuda.synchronize()
+        for s in range(w.steps):
+            check_sampler({"tokens": out["canvas_history"][s], "conf": out["conf_steps"][s]},
+                          block12_ref[s])
         assert torch.equal(out["canvas_history"], eager["canvas_history"])
         assert torch.equal(out["conf_steps"], eager["conf_steps"])
         assert torch.equal(out["attn_out"], eager["attn_out"])

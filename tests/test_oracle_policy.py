@@ -112,3 +112,108 @@ def test_anneal_schedule():
     assert all(a > b for a, b in zip(t, t[1:]))                      # strictly decreasing
     assert np.allclose(np.diff(t), -0.4 / 47, atol=1e-7)            # linear
     assert oracle.anneal_temperature(0, 1) == pytest.approx(0.8)
+
+
+# ------------------------------------------------ the adaptive block loop
+# Closed cases for oracle.denoise_block_adaptive, built so that the outcome
+# of every step is known without running the loop: a "flat" row (all logits
+# equal) has entropy ln V > budget, so it is never accepted and is re-noised
+# to its replacement token; a "peaked" row (one logit 60 above the rest) has
+# an entropy below 1e-20 and a prediction fixed at its hot token (the Gumbel
+# noise lies in [-2.8, 16.7], far below the 60 / tau lead).
+
+V_LOOP, C_LOOP = 64, 8
+
+
+def _loop_logits(peaked, hot):
+    """peaked: bool [S, R]; hot: int [R] -> float32 logits [S, R, V]."""
+    S, R = peaked.shape
+    lg = np.zeros((S, R, V_LOOP), np.float32)
+    for s in range(S):
+        for r in range(R):
+            if peaked[s, r]:
+                lg[s, r, hot[r]] = 60.0
+    return lg
+
+
+def _replacements(lg_s, seed, step):
+    # rate 1: every position takes its uniform replacement token (pinned in
+    # test_oracle_sampler.py)
+    return oracle.sample_renoise(lg_s, 1.0, 1.0, seed, step)["tokens"]
+
+
+def test_adaptive_loop_halts_at_the_second_stable_low_entropy_step():
+    S, k, seed = 6, 3, 17
+    hot = np.arange(C_LOOP, dtype=np.int32) * 7 % V_LOOP
+    peaked = np.zeros((S, C_LOOP), bool)
+    peaked[k - 1:] = True                     # stable from step k-1: halts at step k
+    lg = _loop_logits(peaked, hot)
+    temps = [oracle.anneal_temperature(s, 48) for s in range(S)]
+    r = oracle.denoise_block_adaptive(lg, temps, 0.1, 0.005, seed, C_LOOP)
+    assert r["steps_run"] == k + 1 and list(r["halt_step"]) == [k]
+    for s in range(k - 1):                    # flat steps: nothing fits the budget
+        np.testing.assert_array_equal(r["history"][s], _replacements(lg[s], seed, s))
+    np.testing.assert_array_equal(r["history"][k - 1], hot)   # all accepted (entropy ~ 0)
+    np.testing.assert_array_equal(r["history"][k], hot)       # halts: its prediction
+    np.testing.assert_array_equal(r["canvas"], hot)
+
+
+def test_adaptive_loop_freezes_a_halted_canvas_and_waits_for_the_others():
+    """Canvas 0 halts at step 2, canvas 1 at step 4; canvas 0's logits turn
+    flat again after it halted, which must not change it."""
+    S, seed = 7, 5
+    R = 2 * C_LOOP
+    hot = (np.arange(R, dtype=np.int32) * 11 + 3) % V_LOOP
+    peaked = np.zeros((S, R), bool)
+    peaked[1:3, :C_LOOP] = True               # canvas 0: stable at steps 1, 2 -> halts at 2
+    peaked[3:, C_LOOP:] = True                # canvas 1: stable from step 3 -> halts at 4
+    lg = _loop_logits(peaked, hot)
+    temps = [0.8] * S
+    r = oracle.denoise_block_adaptive(lg, temps, 0.1, 0.005, seed, C_LOOP)
+    assert r["steps_run"] == 5 and list(r["halt_step"]) == [2, 4]
+    c0, c1 = slice(0, C_LOOP), slice(C_LOOP, R)
+    np.testing.assert_array_equal(r["history"][0][c0], _replacements(lg[0], seed, 0)[c0])
+    for s in range(1, 5):
+        np.testing.assert_array_equal(r["history"][s][c0], hot[c0])     # accepted, then frozen
+    for s in range(3):
+        np.testing.assert_array_equal(r["history"][s][c1], _replacements(lg[s], seed, s)[c1])
+    for s in (3, 4):
+        np.testing.assert_array_equal(r["history"][s][c1], hot[c1])
+    np.testing.assert_array_equal(r["canvas"], hot)
+
+
+def test_adaptive_loop_without_a_halt_runs_every_step():
+    S, seed = 4, 2
+    hot = np.arange(C_LOOP, dtype=np.int32) + 40
+    peaked = np.ones((S, C_LOOP), bool)
+    peaked[:, 5] = False                      # one flat position: mean entropy ln(64) / 8
+    lg = _loop_logits(peaked, hot)
+    r = oracle.denoise_block_adaptive(lg, [0.8] * S, 0.1, 0.005, seed, C_LOOP)
+    assert r["steps_run"] == S and list(r["halt_step"]) == [-1]
+    for s in range(S):                        # the 7 peaked positions fit the budget
+        want = hot.copy()
+        want[5] = _replacements(lg[s], seed, s)[5]
+        np.testing.assert_array_equal(r["history"][s], want)
+    # a threshold no canvas can meet, on logits that would halt at step 1
+    r2 = oracle.denoise_block_adaptive(_loop_logits(np.ones((S, C_LOOP), bool), hot), [0.8] * S,
+                                       0.1, -1.0, seed, C_LOOP)
+    assert r2["steps_run"] == S and list(r2["halt_step"]) == [-1]
+    assert (r2["history"] == hot).all()
+
+
+def test_adaptive_loop_margins():
+    """The margins the GPU tests use to tell near-boundary decisions apart:
+    the stop margin is |mean entropy - threshold|; the acceptance margin is
+    the distance of the budget to the cut, or the entropy gap at the cut."""
+    h = np.array([0.03, 0.01, 0.05, 0.02], np.float32)      # sorted: .01 .02 .03 .05
+    # sums .01 .03 .06 | .11 > 0.1: margin = min(0.1 - 0.06, 0.11 - 0.1, 0.05 - 0.03)
+    m = oracle._acceptance_margin(h, 0.1)
+    want = min(0.1 - (0.01 + 0.02 + 0.03), (0.01 + 0.02 + 0.03 + 0.05) - 0.1, 0.05 - 0.03)
+    assert m == pytest.approx(want, abs=1e-7)
+    assert oracle._acceptance_margin(np.zeros(4, np.float32), 0.1) == pytest.approx(0.1)
+    assert oracle._acceptance_margin(np.full(3, 5.0, np.float32), 0.1) == pytest.approx(4.9)
+    S = 2
+    hot = np.arange(C_LOOP, dtype=np.int32)
+    lg = _loop_logits(np.zeros((S, C_LOOP), bool), hot)
+    r = oracle.denoise_block_adaptive(lg, [1.0] * S, 0.1, 0.005, 1, C_LOOP)
+    assert r["stop_margin"][0][0] == pytest.approx(np.log(V_LOOP) - 0.005, rel=1e-6)

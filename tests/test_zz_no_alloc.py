@@ -8,8 +8,11 @@ Checked through the C ABI against dd_sample_renoise (same kernels, so the
 outputs must agree to the tolerances of the other sampler tests: token ids
 exactly, confidences and entropies within 1e-5), on two calls in a row with
 different shapes, so the second call runs on the scratch the first one
-left behind.  Collected last on purpose (file name), so that a failure here
-cannot hide another test's result.
+left behind; that a call allocates no device memory (the free memory the
+driver reports is the same before and after it); the size limit at its
+edge (1927 rows of 262144 entries pass, 1928 are rejected); and correct
+results after calls that were rejected.  Collected last on purpose (file
+name), so that a failure here cannot hide another test's result.
 """
 import ctypes
 
@@ -33,11 +36,11 @@ def _outputs(R):
             "renoised": torch.full((R,), 7, dtype=torch.uint8, device=DEV)}
 
 
-def _noalloc_abi(logits, tau, rate, seed, step, row_offset=0):
+def _noalloc_abi(logits, tau, rate, seed, step, row_offset=0, o=None):
     """Direct C-ABI call of dd_sample_renoise_noalloc."""
     lib = dd.load()
     R, V = logits.shape
-    o = _outputs(R)
+    o = _outputs(R) if o is None else o
     prm = dd.SampleParams(tau, rate, seed, step, row_offset)
     code = dd.DD_BF16 if logits.dtype == torch.bfloat16 else dd.DD_F32
     st = lib.dd_sample_renoise_noalloc(
@@ -85,3 +88,44 @@ def test_noalloc_rejects_calls_beyond_its_scratch():
                                        fake, None, fake, None, None, None)
     assert st == 2  # DD_ERR_UNSUPPORTED
     assert "static scratch" in dd.last_error()
+
+
+def test_noalloc_allocates_no_device_memory():
+    w = workloads.WORKLOADS["b1_L4096"]
+    lg = workloads.logits(w, 0, device=DEV)
+    o = _outputs(lg.shape[0])
+    _noalloc_abi(lg, 1.0, 0.3, 0, 0, 0, o)           # first call: address look-up, module load
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    for step in range(3):
+        _noalloc_abi(lg, 1.0, 0.3, 0, step, 0, o)
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0, f"device free memory changed by {free0 - free1} bytes"
+
+
+def test_noalloc_size_limit_at_its_edge_and_after_rejected_calls():
+    """1927 rows of 262144 bf16 entries fit the 4 MiB scratch and match
+    dd_sample_renoise; 1928 do not.  Rejected calls (too large, NULL
+    params, a bad temperature) queue nothing, and the next call is right."""
+    lib = dd.load()
+    V = 262144
+    g = torch.Generator(device=DEV).manual_seed(7)
+    lg = (torch.randn((1928, V), generator=g, device=DEV) * 3.0).to(torch.bfloat16)
+    prm = dd.SampleParams(1.0, 0.25, 3, 1, 0)
+    o = _outputs(1928)
+    args = lambda rows, p: (ctypes.c_void_p(lg.data_ptr()), dd.DD_BF16, rows, V, V,
+                            p, ctypes.c_void_p(o["tokens"].data_ptr()), None,
+                            ctypes.c_void_p(o["conf"].data_ptr()), None, None, None)
+    assert lib.dd_sample_renoise_noalloc(*args(1928, ctypes.byref(prm))) == 2
+    assert "static scratch" in dd.last_error()
+    assert lib.dd_sample_renoise_noalloc(*args(1927, None)) == 1         # params NULL
+    assert lib.dd_sample_renoise_noalloc(*args(0, None)) == 1            # checked at rows 0 too
+    bad = dd.SampleParams(0.0, 0.25, 3, 1, 0)
+    assert lib.dd_sample_renoise_noalloc(*args(1927, ctypes.byref(bad))) == 1
+    torch.cuda.synchronize()
+    assert (o["tokens"] == -1).all()                                     # nothing ran
+    got = _noalloc_abi(lg[:1927], 1.0, 0.25, 3, 1, 0)
+    ref = dd.sample_renoise(lg[:1927], 1.0, 0.25, 3, 1, 0, outputs=_outputs(1927))
+    torch.cuda.synchronize()
+    _compare(got, ref)
