@@ -465,12 +465,42 @@ def run_soft_embed(w, reps: int = 30):
         e1.record()
         torch.cuda.synchronize()
         ts.append(e0.elapsed_time(e1))
+    # the MLP alone (dd_ffw) and the whole signal (dd_self_condition)
+    w1, b1, w2, b2 = workloads.ffw_weights(w, d, device=dev)
+    u = out.clone()
+    z = torch.empty_like(u)
+    hidden = w1.shape[1]
+    ws_f = dd.new_workspace(int(dd.load().dd_ffw_workspace(w.rows, d, hidden)), dev)
+    ws_c = dd.new_workspace(int(dd.load().dd_self_condition_workspace(w.rows, w.vocab, d,
+                                                                       hidden)), dev)
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        tt = []
+        for _ in range(reps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            tt.append(e0.elapsed_time(e1))
+        return statistics.median(tt)
+
+    ms_ffw = timed(lambda: dd.ffw(u, w1, b1, w2, b2, out=z, workspace=ws_f))
+    ms_sc = timed(lambda: dd.self_condition(lg, w.temperatures[0], E, w1, b1, w2, b2, out=z,
+                                            workspace=ws_c))
     t_wall1 = time.time()
     time.sleep(0.2)
     clocks.stop()
     dd.query_device_error(ws)
+    dd.query_device_error(ws_f)
+    dd.query_device_error(ws_c)
     ms = statistics.median(ts)
     hbm, tf_burst, tf_sus, src = _peaks()
+    ffw_flops = 4 * w.rows * d * hidden
+    ffw_bytes = 2 * (2 * d * hidden + hidden + d + 2 * w.rows * d + 2 * w.rows * hidden)
     flops = 2 * w.rows * w.vocab * d
     nbytes = (w.vocab * d + w.rows * w.vocab + w.rows * d) * 2
     gbs, tfs = nbytes / ms / 1e6, flops / ms / 1e9
@@ -485,6 +515,13 @@ def run_soft_embed(w, reps: int = 30):
         "tensor": {"achieved": tfs, "peak": tf_burst, "unit": "TFLOP/s", "frac": tfs / tf_burst,
                    "flops": flops},
         "timing": f"median of {reps} calls, CUDA events around each call",
+        "ffw": {"what": "the self-conditioning MLP GELU(u W1 + b1) W2 + b2 (dd_ffw), "
+                        f"d {d}, hidden {hidden}, synthetic weights",
+                "ms": ms_ffw, "flops": ffw_flops, "bytes": ffw_bytes,
+                "TFLOP/s": ffw_flops / ms_ffw / 1e9, "frac_tensor": ffw_flops / ms_ffw / 1e9 / tf_burst,
+                "GB/s": ffw_bytes / ms_ffw / 1e6, "frac_hbm": ffw_bytes / ms_ffw / 1e6 / hbm},
+        "self_condition": {"what": "dd_self_condition: soft embedding, then the MLP",
+                           "ms": ms_sc},
         "clocks": clocks.summary(t_wall0, t_wall1),
     }
 

@@ -35,7 +35,8 @@ EXPORTS = (
     "dd_denoise_block_graph_launch", "dd_denoise_block_graph_destroy",
     "dd_soft_embed_workspace", "dd_soft_embed", "dd_denoise_block_fp8",
     "dd_denoise_block_adaptive_graph_create", "dd_denoise_block_adaptive_graph_launch",
-    "dd_denoise_block_adaptive_graph_destroy",
+    "dd_denoise_block_adaptive_graph_destroy", "dd_ffw_workspace", "dd_ffw",
+    "dd_self_condition_workspace", "dd_self_condition", "dd_set_wait_limit_ns",
 )
 
 
@@ -121,6 +122,17 @@ def load() -> ctypes.CDLL:
     lib.dd_soft_embed_workspace.argtypes = [i32, i32, i32]
     lib.dd_soft_embed.restype = i32
     lib.dd_soft_embed.argtypes = [P, i32, i32, i32, i64, ctypes.c_float, P, i32, P, P, sz, P]
+    lib.dd_set_wait_limit_ns.restype = None
+    lib.dd_set_wait_limit_ns.argtypes = [u64]
+    lib.dd_ffw_workspace.restype = sz
+    lib.dd_ffw_workspace.argtypes = [i32, i32, i32]
+    lib.dd_ffw.restype = i32
+    lib.dd_ffw.argtypes = [P, i32, i32, i32, P, P, P, P, P, P, sz, P]
+    lib.dd_self_condition_workspace.restype = sz
+    lib.dd_self_condition_workspace.argtypes = [i32, i32, i32, i32]
+    lib.dd_self_condition.restype = i32
+    lib.dd_self_condition.argtypes = [P, i32, i32, i32, i64, ctypes.c_float, P, i32, P, P, i32, P,
+                                      P, P, P, P, sz, P]
     lib.dd_entropy_accept.restype = i32
     lib.dd_entropy_accept.argtypes = [P, P, i32, i32, i32, f32, u64, u32, u32, P, P, P]
     lib.dd_stop_check.restype = i32
@@ -406,6 +418,43 @@ def soft_embed(logits: torch.Tensor, temperature: float, emb: torch.Tensor, out=
     return out
 
 
+def ffw(u: torch.Tensor, w1: torch.Tensor, b1: torch.Tensor, w2: torch.Tensor,
+        b2: torch.Tensor, out=None, workspace=None, stream=None) -> torch.Tensor:
+    """dd_ffw: the self-conditioning MLP GELU(u w1 + b1) w2 + b2, bf16
+    [rows, d] (u [rows, d], w1 [d, h], b1 [h], w2 [h, d], b2 [d], bf16)."""
+    lib = load()
+    R, d = u.shape
+    h = w1.shape[1]
+    if out is None:
+        out = torch.empty((R, d), dtype=torch.bfloat16, device=u.device)
+    if workspace is None:
+        workspace = new_workspace(int(lib.dd_ffw_workspace(R, d, h)), u.device, stream)
+    _check(lib.dd_ffw(_ptr(u), R, d, h, _ptr(w1), _ptr(b1), _ptr(w2), _ptr(b2), _ptr(out),
+                      _ptr(workspace), workspace.numel(), _stream(stream)))
+    return out
+
+
+def self_condition(logits: torch.Tensor, temperature: float, emb: torch.Tensor,
+                   w1: torch.Tensor, b1: torch.Tensor, w2: torch.Tensor, b2: torch.Tensor,
+                   out=None, u_out=None, workspace=None, stream=None) -> torch.Tensor:
+    """dd_self_condition: z = FFW(softmax(logits / temperature) emb), bf16
+    [rows, d]; u_out (optional, bf16 [rows, d]) receives the soft embedding."""
+    lib = load()
+    R, V = logits.shape
+    d = emb.shape[1]
+    h = w1.shape[1]
+    if out is None:
+        out = torch.empty((R, d), dtype=torch.bfloat16, device=logits.device)
+    if workspace is None:
+        workspace = new_workspace(int(lib.dd_self_condition_workspace(R, V, d, h)),
+                                  logits.device, stream)
+    _check(lib.dd_self_condition(_ptr(logits), _dtype_code(logits), R, V, logits.stride(0),
+                                 float(temperature), _ptr(emb), d, _ptr(w1), _ptr(b1), h,
+                                 _ptr(w2), _ptr(b2), _ptr(out), _ptr(u_out), _ptr(workspace),
+                                 workspace.numel(), _stream(stream)))
+    return out
+
+
 class BlockGraph:
     """dd_denoise_block captured once (dd_denoise_block_graph_create) and
     replayed with one launch (launch()).  Holds every captured tensor, so the
@@ -589,6 +638,12 @@ def denoise_block_adaptive_graph(q_steps, kc_steps, vc_steps, kp, vp, cu_prefix,
 
 def query_device_error(workspace: torch.Tensor, stream=None):
     _check(load().dd_query_device_error(_ptr(workspace), _stream(stream)))
+
+
+def set_wait_limit_ns(ns: int):
+    """dd_set_wait_limit_ns: the pipeline-wait limit of the tensor-core
+    kernels launched afterwards from this thread (0 = the 1 s default)."""
+    load().dd_set_wait_limit_ns(int(ns))
 
 
 def launch_count() -> int:

@@ -245,6 +245,10 @@ dd_status run_sampler(const void* logits, dd_dtype dtype, int rows, int vocab, i
 
 void note_launch() { ++g_launches; }
 
+constexpr uint64_t kDefaultWaitNs = 1000000000ull;
+thread_local uint64_t g_wait_ns = kDefaultWaitNs;
+uint64_t pipeline_wait_ns() { return g_wait_ns; }
+
 thread_local bool g_pdl_off = false;
 bool pdl_enabled() { return !g_pdl_off; }
 
@@ -525,10 +529,12 @@ size_t dd_soft_embed_workspace(int rows, int vocab, int d) {
   return kHeaderBytes + soft_embed_scratch_bytes(rows, vocab, d);
 }
 
-dd_status dd_soft_embed(const void* logits, dd_dtype dtype, int rows, int vocab,
-                        int64_t row_stride, float temperature, const void* emb, int d, void* out,
-                        void* workspace, size_t workspace_bytes, dd_stream_t stream) {
-  g_last_error.clear();
+namespace {
+// The soft embedding's argument checks up to the tensor pointers (no device
+// work); rows == 0 passes them.
+dd_status check_soft_embed(const void* logits, dd_dtype dtype, int rows, int vocab,
+                           int64_t row_stride, float temperature, const void* emb, int d,
+                           const void* out) {
   if (dtype != DD_BF16 && dtype != DD_F32 && dtype != DD_E4M3)
     return fail(DD_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
   if (dtype != DD_BF16) return fail(DD_ERR_UNSUPPORTED, "soft embedding takes bf16 logits and E");
@@ -544,11 +550,14 @@ dd_status dd_soft_embed(const void* logits, dd_dtype dtype, int rows, int vocab,
   if (!logits || !emb || !out) return fail(DD_ERR_INVALID_ARG, "NULL tensor pointer");
   if (!aligned16(logits) || !aligned16(emb) || !aligned16(out))
     return fail(DD_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
-  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u))
-    return fail(DD_ERR_WORKSPACE, "workspace must be non-NULL and 256-byte aligned");
-  const size_t need = kHeaderBytes + soft_embed_scratch_bytes(rows, vocab, d);
-  if (workspace_bytes < need)
-    return fail(DD_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", workspace_bytes, need);
+  return DD_OK;
+}
+
+// The soft embedding's three kernels into `out`, with the workspace header
+// at `ws` and its scratch right after it.
+dd_status run_soft_embed(const void* logits, int rows, int vocab, int64_t row_stride,
+                         float temperature, const void* emb, int d, void* out, void* ws,
+                         cudaStream_t stream) {
   SoftEmbedArgs a{};
   a.logits = logits;
   a.rows = rows;
@@ -558,11 +567,133 @@ dd_status dd_soft_embed(const void* logits, dd_dtype dtype, int rows, int vocab,
   a.emb = emb;
   a.d = d;
   a.out = out;
-  a.err = static_cast<uint32_t*>(workspace);
-  a.scratch = static_cast<uint8_t*>(workspace) + kHeaderBytes;
-  cudaError_t e = launch_soft_embed(a, reinterpret_cast<cudaStream_t>(stream));
+  a.err = static_cast<uint32_t*>(ws);
+  a.scratch = static_cast<uint8_t*>(ws) + kHeaderBytes;
+  cudaError_t e = launch_soft_embed(a, stream);
   if (e != cudaSuccess) return cuda_fail(e, "soft embedding");
   return DD_OK;
+}
+}  // namespace
+
+dd_status dd_soft_embed(const void* logits, dd_dtype dtype, int rows, int vocab,
+                        int64_t row_stride, float temperature, const void* emb, int d, void* out,
+                        void* workspace, size_t workspace_bytes, dd_stream_t stream) {
+  g_last_error.clear();
+  dd_status st = check_soft_embed(logits, dtype, rows, vocab, row_stride, temperature, emb, d, out);
+  if (st != DD_OK || rows == 0) return st;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return fail(DD_ERR_WORKSPACE, "workspace must be non-NULL and 256-byte aligned");
+  const size_t need = kHeaderBytes + soft_embed_scratch_bytes(rows, vocab, d);
+  if (workspace_bytes < need)
+    return fail(DD_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", workspace_bytes, need);
+  return run_soft_embed(logits, rows, vocab, row_stride, temperature, emb, d, out, workspace,
+                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+// ---- self-conditioning MLP
+namespace {
+// Shapes the dense layers take: rows >= 0, d and hidden multiples of 16.
+dd_status check_ffw_shape(int rows, int d, int hidden) {
+  if (rows < 0) return fail(DD_ERR_INVALID_ARG, "rows=%d", rows);
+  if (d < 16 || hidden < 16) return fail(DD_ERR_INVALID_ARG, "d=%d hidden=%d", d, hidden);
+  if (d % 16 != 0 || hidden % 16 != 0)
+    return fail(DD_ERR_UNSUPPORTED, "d=%d hidden=%d (multiples of 16)", d, hidden);
+  if ((int64_t)rows > 65535LL * 128) return fail(DD_ERR_UNSUPPORTED, "rows=%d", rows);
+  return DD_OK;
+}
+
+dd_status check_ffw_ptrs(const void* w1, const void* b1, const void* w2, const void* b2,
+                         const void* out) {
+  if (!w1 || !b1 || !w2 || !b2 || !out) return fail(DD_ERR_INVALID_ARG, "NULL tensor pointer");
+  if (!aligned16(w1) || !aligned16(b1) || !aligned16(w2) || !aligned16(b2) || !aligned16(out))
+    return fail(DD_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  return DD_OK;
+}
+
+// MLP scratch: the bf16 hidden activations, then the fp32 partials of the
+// K splits (one region for both layers, which run one after the other).
+size_t ffw_scratch_bytes(int rows, int d, int hidden) {
+  return align256((size_t)rows * hidden * 2) +
+         align256(std::max(dense_partial_bytes(rows, d, hidden),
+                           dense_partial_bytes(rows, hidden, d)));
+}
+
+// The two dense layers: hid = GELU(u W1 + b1), out = hid W2 + b2; `scratch`
+// holds ffw_scratch_bytes.
+dd_status run_ffw(const void* u, int rows, int d, int hidden, const void* w1, const void* b1,
+                  const void* w2, const void* b2, void* out, void* scratch, uint32_t* err,
+                  cudaStream_t stream) {
+  void* hid = scratch;
+  void* part = static_cast<uint8_t*>(scratch) + align256((size_t)rows * hidden * 2);
+  DenseArgs l1{u, w1, b1, hid, rows, d, hidden, true, err, part};
+  cudaError_t e = launch_dense(l1, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "self-conditioning MLP, layer 1");
+  DenseArgs l2{hid, w2, b2, out, rows, hidden, d, false, err, part};
+  e = launch_dense(l2, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "self-conditioning MLP, layer 2");
+  return DD_OK;
+}
+}  // namespace
+
+size_t dd_ffw_workspace(int rows, int d, int hidden) {
+  if (rows < 0 || d < 16 || hidden < 16 || d % 16 || hidden % 16) return 0;
+  return kHeaderBytes + ffw_scratch_bytes(rows, d, hidden);
+}
+
+dd_status dd_ffw(const void* u, int rows, int d, int hidden, const void* w1, const void* b1,
+                 const void* w2, const void* b2, void* out, void* workspace,
+                 size_t workspace_bytes, dd_stream_t stream) {
+  g_last_error.clear();
+  dd_status st = check_ffw_shape(rows, d, hidden);
+  if (st != DD_OK || rows == 0) return st;
+  st = check_ffw_ptrs(w1, b1, w2, b2, out);
+  if (st != DD_OK) return st;
+  if (!u || !aligned16(u)) return fail(DD_ERR_INVALID_ARG, "u must be non-NULL and 16-byte aligned");
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return fail(DD_ERR_WORKSPACE, "workspace must be non-NULL and 256-byte aligned");
+  const size_t need = kHeaderBytes + ffw_scratch_bytes(rows, d, hidden);
+  if (workspace_bytes < need)
+    return fail(DD_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", workspace_bytes, need);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  return run_ffw(u, rows, d, hidden, w1, b1, w2, b2, out, ws + kHeaderBytes,
+                 reinterpret_cast<uint32_t*>(ws), reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t dd_self_condition_workspace(int rows, int vocab, int d, int hidden) {
+  if (rows < 0 || vocab < 1 || d < 64 || d % 64 || hidden < 16 || hidden % 16) return 0;
+  return kHeaderBytes + align256(soft_embed_scratch_bytes(rows, vocab, d)) +
+         align256((size_t)rows * d * 2) + ffw_scratch_bytes(rows, d, hidden);
+}
+
+dd_status dd_self_condition(const void* logits, dd_dtype dtype, int rows, int vocab,
+                            int64_t row_stride, float temperature, const void* emb, int d,
+                            const void* w1, const void* b1, int hidden, const void* w2,
+                            const void* b2, void* out, void* u_out, void* workspace,
+                            size_t workspace_bytes, dd_stream_t stream) {
+  g_last_error.clear();
+  // every check before the first launch
+  dd_status st = check_soft_embed(logits, dtype, rows, vocab, row_stride, temperature, emb, d,
+                                  out);
+  if (st != DD_OK) return st;
+  st = check_ffw_shape(rows, d, hidden);
+  if (st != DD_OK || rows == 0) return st;
+  st = check_ffw_ptrs(w1, b1, w2, b2, out);
+  if (st != DD_OK) return st;
+  if (u_out && !aligned16(u_out)) return fail(DD_ERR_INVALID_ARG, "u_out must be 16-byte aligned");
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return fail(DD_ERR_WORKSPACE, "workspace must be non-NULL and 256-byte aligned");
+  const size_t need = dd_self_condition_workspace(rows, vocab, d, hidden);
+  if (workspace_bytes < need)
+    return fail(DD_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", workspace_bytes, need);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const size_t se = align256(soft_embed_scratch_bytes(rows, vocab, d));
+  void* u = u_out ? u_out : ws + kHeaderBytes + se;
+  void* hid = ws + kHeaderBytes + se + align256((size_t)rows * d * 2);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  st = run_soft_embed(logits, rows, vocab, row_stride, temperature, emb, d, u, workspace, s);
+  if (st != DD_OK) return st;
+  return run_ffw(u, rows, d, hidden, w1, b1, w2, b2, out, hid, reinterpret_cast<uint32_t*>(ws),
+                 s);
 }
 
 // A captured block loop: one instantiated CUDA graph and the number of
@@ -993,6 +1124,8 @@ const char* dd_status_string(dd_status s) {
 }
 
 const char* dd_last_error(void) { return g_last_error.c_str(); }
+
+void dd_set_wait_limit_ns(uint64_t ns) { g_wait_ns = ns ? ns : kDefaultWaitNs; }
 
 uint64_t dd_launch_count(void) { return g_launches; }
 void dd_reset_launch_count(void) { g_launches = 0; }

@@ -117,6 +117,7 @@ struct TcParams {
   float* part_o;    // [slots][BM][HD], slot = (b, g, t, split)
   float* part_lse;  // [slots][BM]   log2 units
   uint32_t* err;
+  uint64_t wait_ns;  // limit of each pipeline wait (waits that drain use kWaitLimitNs)
 };
 
 __device__ __forceinline__ int cdiv(int a, int b) { return (a + b - 1) / b; }
@@ -220,12 +221,12 @@ __device__ __forceinline__ bool load_kv(Barriers* bars, uint8_t* smem, int j, in
                                         int np, int p0, int b, int C, int g,
                                         const CUtensorMap* tmKp, const CUtensorMap* tmVp,
                                         const CUtensorMap* tmKc, const CUtensorMap* tmVc,
-                                        volatile int* abort_flag) {
+                                        volatile int* abort_flag, uint64_t wait_ns) {
   using G = Lay<kF8>;
   const int st = j % G::kStages, rd = j / G::kStages;
   uint64_t* empty = v ? &bars->v_empty[st] : &bars->k_empty[st];
   uint64_t* full = v ? &bars->v_full[st] : &bars->k_full[st];
-  if (rd > 0 && !mbar_wait_bounded(empty, (rd - 1) & 1, abort_flag, kWaitLimitNs)) return false;
+  if (rd > 0 && !mbar_wait_bounded(empty, (rd - 1) & 1, abort_flag, wait_ns)) return false;
   const int k = k_begin + j;
   const CUtensorMap* map = k < np ? (v ? tmVp : tmKp) : (v ? tmVc : tmKc);
   const int row0 = k < np ? p0 + k * BN : b * C + (k - np) * BN;
@@ -307,16 +308,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       // in the order the MMAs consume them: K0, then V_j, K_{j+1}
       int kiss = 0, viss = 0;
       if (load_kv<kF8>(bars, smem, 0, 0, k_begin, np, p0, b, p.C, g, &tmKp, &tmVp, &tmKc, &tmVc,
-                  abort_flag)) {
+                  abort_flag, p.wait_ns)) {
         kiss = 1;
         for (int j = 0; j < n; ++j) {
           if (!load_kv<kF8>(bars, smem, j, 1, k_begin, np, p0, b, p.C, g, &tmKp, &tmVp, &tmKc, &tmVc,
-                       abort_flag))
+                       abort_flag, p.wait_ns))
             break;
           viss = j + 1;
           if (j + 1 < n) {
             if (!load_kv<kF8>(bars, smem, j + 1, 0, k_begin, np, p0, b, p.C, g, &tmKp, &tmVp, &tmKc,
-                         &tmVc, abort_flag))
+                         &tmVc, abort_flag, p.wait_ns))
               break;
             kiss = j + 2;
           }
@@ -346,7 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t dK = smem_desc_sw128(smem_u32(smem + G::kOffK), 16, 1024);
       const uint64_t dV = smem_desc_sw128(smem_u32(smem + G::kOffV), kF8 ? G::kTile : kHalf, 1024);
       auto wait = [&](uint64_t* bar, uint32_t parity) {
-        return __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity, abort_flag, kWaitLimitNs));
+        return __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity, abort_flag, p.wait_ns));
       };
       auto commit = [&](uint64_t* bar) {
         if (leader) tc_commit(bar);
@@ -427,7 +428,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(xbar);
     };
     auto take = [&](int ph) -> float {
-      if (!__all_sync(0xffffffffu, mbar_wait_bounded(xbar, ph & 1, abort_flag, kWaitLimitNs))) {
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(xbar, ph & 1, abort_flag, p.wait_ns))) {
         ok = false;
         return -INFINITY;
       }
@@ -474,7 +475,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int n_valid = k < np ? min(BN, L - k * BN) : min(BN, p.C - (k - np) * BN);
       // wait outcomes are made warp-uniform: tcgen05.ld/st are .sync.aligned
       if (!__all_sync(0xffffffffu,
-                      mbar_wait_bounded(&bars->s_full[q], j & 1, abort_flag, kWaitLimitNs))) {
+                      mbar_wait_bounded(&bars->s_full[q], j & 1, abort_flag, p.wait_ns))) {
         ok = false;
         break;
       }
@@ -543,7 +544,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // their partial row sums
     if (ok)
       ok = __all_sync(0xffffffffu,
-                      mbar_wait_bounded(&bars->o_done[q], 0, abort_flag, kWaitLimitNs));
+                      mbar_wait_bounded(&bars->o_done[q], 0, abort_flag, p.wait_ns));
     float lrow = l;
     if (ok) {
       post(l, n);
@@ -571,7 +572,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->staged[q]);
       if (__all_sync(0xffffffffu,
-                     mbar_wait_bounded(&bars->staged[q], 0, abort_flag, kWaitLimitNs))) {
+                     mbar_wait_bounded(&bars->staged[q], 0, abort_flag, p.wait_ns))) {
         float* dst = p.part_o + slot * BM * HD;
         const int wq = warp & 7;  // warp index within this query tile's 8
         for (int row = wq; row < BM; row += 8)
@@ -876,6 +877,7 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t stream) {
   tp.part_o = reinterpret_cast<float*>(scratch);
   tp.part_lse = reinterpret_cast<float*>(scratch + (size_t)pl.slots * BM * HD * sizeof(float));
   tp.err = a.err;
+  tp.wait_ns = pipeline_wait_ns();
 
   cudaError_t e =
       f8 ? launch_pdl(attn_tc_kernel<true>, dim3(pl.units), dim3(kThreads), Lay<true>::kSmemBytes,

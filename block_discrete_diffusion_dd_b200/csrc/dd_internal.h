@@ -2,6 +2,7 @@
 // and the kernel files.  Not part of the public interface (include/dd.h).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -131,6 +132,42 @@ struct SoftEmbedPlan {
 SoftEmbedPlan soft_embed_plan(int rows, int vocab, int d);
 size_t soft_embed_scratch_bytes(int rows, int vocab, int d);
 cudaError_t launch_soft_embed(const SoftEmbedArgs& a, cudaStream_t stream);
+
+// 2-D bf16 TMA map over [outer, inner] (row stride in elements), box
+// (box_inner, box_outer) with box_inner * 2 bytes of swizzling (64 or 128),
+// out-of-bounds elements read as zero.  False if the driver rejects it.
+bool encode_2d(CUtensorMap* m, const void* base, int64_t inner, int64_t outer, int64_t stride,
+               int box_inner, int box_outer);
+
+// One dense layer on the tensor cores (dd_ffw.cu):
+//   out[r, n] = act(sum_k x[r, k] w[k, n] + bias[n]),  act = GELU or identity
+// x bf16 [rows, K] (row stride K), w bf16 [K, N] (row stride N), bias bf16
+// [N], out bf16 [rows, N]; K and N multiples of 16, 16-byte aligned
+// pointers, validated by the ABI layer.  When K is split over CTAs, `part`
+// holds their fp32 partials.
+struct DenseArgs {
+  const void* x;
+  const void* w;
+  const void* bias;
+  void* out;
+  int rows, K, N;
+  bool gelu;
+  uint32_t* err;
+  void* part;  // fp32 partials, dense_partial_bytes(rows, K, N) (NULL when 0)
+};
+// The split of K over CTAs (device-dependent: about one wave over the SMs).
+struct DensePlan {
+  int ksteps_per_split, splits;
+};
+DensePlan dense_plan(int rows, int K, int N);
+size_t dense_partial_bytes(int rows, int K, int N);
+cudaError_t launch_dense(const DenseArgs& a, cudaStream_t stream);
+
+// Time limit of the pipeline waits (mbarrier waits that can abort) of the
+// tensor-core kernels launched from this host thread: 1 s unless changed by
+// dd_set_wait_limit_ns.  Waits that drain in-flight copies and MMAs before
+// a CTA exits always keep their own 1 s limit.
+uint64_t pipeline_wait_ns();
 
 // Launch accounting (per host thread).
 void note_launch();

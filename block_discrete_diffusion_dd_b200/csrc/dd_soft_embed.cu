@@ -75,6 +75,7 @@ struct SeParams {
   const float* lse2;     // [rows] log2-domain log-sum-exp of logits * c_log2
   float* part;           // [splits][rows][d] fp32
   uint32_t* err;
+  uint64_t wait_ns;      // limit of each pipeline wait (waits that drain use SE_WAIT_NS)
 };
 
 // ---------------------------------------------------------------- row LSE
@@ -239,7 +240,7 @@ __global__ void __launch_bounds__(SE_THREADS, 1)
       int issued = 0;
       for (int i = 0; i < nk; ++i) {
         const int s = i % SE_STAGES, rd = i / SE_STAGES;
-        if (rd > 0 && !mbar_wait_bounded(&bars->empty[s], (rd - 1) & 1, abort_flag, SE_WAIT_NS))
+        if (rd > 0 && !mbar_wait_bounded(&bars->empty[s], (rd - 1) & 1, abort_flag, p.wait_ns))
           break;
         uint8_t* st = smem + s * SE_STAGE;
         const int v0 = (ks0 + i) * SE_BK;
@@ -269,8 +270,8 @@ __global__ void __launch_bounds__(SE_THREADS, 1)
       for (int i = 0; ok && i < nk; ++i) {
         const int s = i % SE_STAGES;
         const uint32_t ph = (i / SE_STAGES) & 1;
-        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->full[s], ph, abort_flag, SE_WAIT_NS) &&
-                                         mbar_wait_bounded(&bars->pfull[s], ph, abort_flag, SE_WAIT_NS));
+        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->full[s], ph, abort_flag, p.wait_ns) &&
+                                         mbar_wait_bounded(&bars->pfull[s], ph, abort_flag, p.wait_ns));
         if (!ok) break;
         tc_fence_after();
         const uint32_t so = s * SE_STAGE;
@@ -310,7 +311,7 @@ __global__ void __launch_bounds__(SE_THREADS, 1)
     for (int i = 0; i < nk; ++i) {
       const int s = i % SE_STAGES;
       if (!__all_sync(0xffffffffu, mbar_wait_bounded(&bars->full[s], (i / SE_STAGES) & 1,
-                                                     abort_flag, SE_WAIT_NS))) {
+                                                     abort_flag, p.wait_ns))) {
         ok = false;
         break;
       }
@@ -337,7 +338,7 @@ __global__ void __launch_bounds__(SE_THREADS, 1)
     }
     const bool epilogue = warp < SE_WARP_P0 + 8;
     if (ok && nk > 0 && epilogue)
-      ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->acc_full, 0, abort_flag, SE_WAIT_NS));
+      ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->acc_full, 0, abort_flag, p.wait_ns));
     if (ok && nk > 0 && epilogue) {
       tc_fence_after();
       // TMEM lanes of this warp: 32 * (warp % 4); warps 2-5 hold tile 0,
@@ -413,6 +414,19 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+int sm_count_se() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+}  // namespace
+
 // 2-D bf16 map over [outer, inner] with a row stride in elements, box
 // (box_inner, box_outer), box_inner * 2 bytes of swizzling (64 or 128),
 // zero fill out of bounds.
@@ -430,19 +444,6 @@ bool encode_2d(CUtensorMap* m, const void* base, int64_t inner, int64_t outer, i
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
-
-int sm_count_se() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
-  }
-  return n;
-}
-
-}  // namespace
 
 // Vocabulary splits: about one wave of CTAs over the SMs, at least 16 steps
 // of 32 entries per split.
@@ -503,6 +504,7 @@ cudaError_t launch_soft_embed(const SoftEmbedArgs& a, cudaStream_t stream) {
   p.lse2 = lse2;
   p.part = part;
   p.err = a.err;
+  p.wait_ns = pipeline_wait_ns();
   e = launch_pdl(soft_embed_kernel, dim3(pl.grid_x, pl.splits, pl.grid_z), dim3(SE_THREADS),
                  SE_SMEM, stream, mL, mE, p);
   note_launch();

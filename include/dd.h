@@ -288,8 +288,8 @@ DD_API dd_status dd_denoise_block_graph_destroy(dd_block_graph graph);
  * "The mechanism", self-conditioning paragraph: the previous step's
  * predicted token distribution, pushed through the embedding matrix E, is
  * the input of a small MLP that conditions the next step).  This computes
- * the contraction; the MLP (7.8M parameters, weights not public) is not
- * part of the library:
+ * the contraction; dd_ffw is the MLP that follows it, and
+ * dd_self_condition runs both:
  *   out[r, :] = sum_v softmax(logits[r, :] / temperature)_v * E[v, :]
  * Arguments:
  *   logits       bf16 [rows, vocab] with row_stride elements between rows
@@ -311,6 +311,45 @@ DD_API dd_status dd_soft_embed(const void* logits, dd_dtype dtype, int rows, int
                                int64_t row_stride, float temperature, const void* emb, int d,
                                void* out, void* workspace, size_t workspace_bytes,
                                dd_stream_t stream);
+
+/* Self-conditioning MLP ("DiffusionGemma Technical Report", "The mechanism",
+ * self-conditioning paragraph: the soft embedding u = p0 E goes through "a
+ * small MLP (7.8M parameters)", z_t = FFW(u)).  The pages give only the
+ * size; the MLP is read as two dense layers with a GELU between them:
+ *   hid[r, :] = GELU(u[r, :] W1 + b1),   GELU(x) = x Phi(x) (erf form)
+ *   out[r, :] = hid[r, :] W2 + b2
+ * At d = 2048 and hidden = 1904 that is 7,802,784 parameters.  Both layers
+ * run on the tensor cores (bf16 operands, fp32 accumulation); the hidden
+ * activations and the output are rounded to bf16 (relative error <= 2^-8
+ * each).
+ *   u        bf16 [rows, d]
+ *   w1       bf16 [d, hidden], row-major;  b1 bf16 [hidden]
+ *   w2       bf16 [hidden, d], row-major;  b2 bf16 [d]
+ *   out      bf16 [rows, d]
+ *   workspace >= dd_ffw_workspace(rows, d, hidden) bytes, 256-byte aligned
+ *            (error word and the bf16 hidden activations)
+ * d and hidden must be multiples of 16 (>= 16), else DD_ERR_UNSUPPORTED
+ * (DD_ERR_INVALID_ARG below 16).  dd_ffw_workspace returns 0 on invalid
+ * shapes. */
+DD_API size_t dd_ffw_workspace(int rows, int d, int hidden);
+DD_API dd_status dd_ffw(const void* u, int rows, int d, int hidden, const void* w1,
+                        const void* b1, const void* w2, const void* b2, void* out,
+                        void* workspace, size_t workspace_bytes, dd_stream_t stream);
+
+/* The whole self-conditioning signal of a step: dd_soft_embed of the
+ * logits, then dd_ffw,  out = FFW(softmax(logits / temperature) E).
+ * Arguments as dd_soft_embed (logits, dtype, rows, vocab, row_stride,
+ * temperature, emb, d; d a multiple of 64) and dd_ffw (w1, b1, hidden, w2,
+ * b2, out).  u_out: bf16 [rows, d] receiving the soft embedding, or NULL
+ * (it then lives in the workspace).  Every argument is checked before the
+ * first launch.  workspace >= dd_self_condition_workspace(rows, vocab, d,
+ * hidden) bytes, 256-byte aligned; 0 on invalid shapes. */
+DD_API size_t dd_self_condition_workspace(int rows, int vocab, int d, int hidden);
+DD_API dd_status dd_self_condition(const void* logits, dd_dtype dtype, int rows, int vocab,
+                                   int64_t row_stride, float temperature, const void* emb, int d,
+                                   const void* w1, const void* b1, int hidden, const void* w2,
+                                   const void* b2, void* out, void* u_out, void* workspace,
+                                   size_t workspace_bytes, dd_stream_t stream);
 
 /* dd_sample_renoise without a workspace, for callers that may not allocate
  * device memory (code inside another framework's memory pool or fixed
@@ -458,6 +497,17 @@ DD_API const char* dd_status_string(dd_status status);
 
 /* Detail of the last failure on this host thread ("" if none). */
 DD_API const char* dd_last_error(void);
+
+/* Time limit of each pipeline wait (a wait on an mbarrier that other warps
+ * or the copy and tensor-core units complete) in the tensor-core kernels
+ * (attention, soft embedding, MLP) launched afterwards from this host
+ * thread; 0 restores the default of 1 s.  A wait that runs out latches
+ * DD_ERR_DEVICE_TIMEOUT in the call's workspace (read it with
+ * dd_query_device_error), and the kernel then waits, up to 1 s each, for
+ * its own copies and MMAs in flight, frees its tensor memory and returns;
+ * the outputs of that call are undefined.  A short limit is a test of that
+ * path (the pages have no counterpart); leave it at the default otherwise. */
+DD_API void dd_set_wait_limit_ns(uint64_t ns);
 
 /* Number of kernels the library launched on this host thread since the last
  * call to dd_reset_launch_count (for launch accounting in benchmarks). */

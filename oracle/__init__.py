@@ -45,6 +45,10 @@ Parity status per function (what pins it; tests/test_oracle_*.py):
                                (constant logits -> mean embedding, one
                                dominant logit -> its embedding row),
                                temperature scaling, linearity in E.
+  ffw / self_condition      -- pure-Python brute force with math.erf,
+                               tabulated values of the normal distribution
+                               function, closed forms (zero weights, large
+                               arguments), linearity in W2 and b2.
 
 Regression fixtures: tests/golden/*.json, written from this package alone by
 tests/golden/make_golden.py (the pages print no worked example), freeze its
@@ -447,6 +451,34 @@ def soft_embed(logits, tau: float, emb, rows=None, cols=None, v_chunk: int = 163
              else blk.astype(np.float64))
         out += p[:, v0:v0 + v_chunk] @ e
     return out
+
+
+def _gelu64(x: np.ndarray) -> np.ndarray:
+    """GELU(x) = x * Phi(x) = x (1 + erf(x / sqrt 2)) / 2, float64 (erf from
+    torch's float64 CPU routine)."""
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float64))
+    return (0.5 * t * (1.0 + torch.erf(t / np.sqrt(2.0)))).numpy()
+
+
+def ffw(u, w1, b1, w2, b2) -> np.ndarray:
+    """The self-conditioning MLP ("DiffusionGemma Technical Report"
+    (paperfeed review), "The mechanism", self-conditioning paragraph:
+    z_t = FFW(p0 E), a small MLP of 7.8M parameters).  The pages give no
+    architecture; read as two dense layers with a GELU between them:
+        z = GELU(u W1 + b1) W2 + b2
+    in float64 from the exactly decoded bf16 / float32 inputs: u [rows, d],
+    W1 [d, h], b1 [h], W2 [h, d], b2 [d]."""
+    h = _gelu64(_f64(u) @ _f64(w1) + _f64(b1))
+    return h @ _f64(w2) + _f64(b2)
+
+
+def self_condition(logits, tau: float, emb, w1, b1, w2, b2) -> np.ndarray:
+    """z = FFW(softmax(logits / tau) E): soft_embed followed by ffw, both in
+    float64 (no rounding in between)."""
+    u = soft_embed(logits, tau, emb)
+    h = _gelu64(u @ _f64(w1) + _f64(b1))
+    return h @ _f64(w2) + _f64(b2)
 
 
 # --------------------------------------------------------- the block loop

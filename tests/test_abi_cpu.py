@@ -170,6 +170,44 @@ def test_soft_embed_workspace_and_empty_call(lib):
     assert n >= 256 + 256 * 4 + 256 * 2048 * 4   # at least one split of fp32 partials
 
 
+def _ffw(lib, rows=4, d=64, h=32, ptr=FAKE, w=FAKE, ws=FAKE, ws_bytes=1 << 30):
+    return lib.dd_ffw(ptr, rows, d, h, w, w, w, w, ptr, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(d=8), 1), (dict(h=0), 1), (dict(d=72), 2), (dict(h=40), 2), (dict(rows=-1), 1),
+    (dict(ptr=None), 1), (dict(w=None), 1), (dict(w=ctypes.c_void_p((1 << 20) + 4)), 1),
+    (dict(ws=None), 3), (dict(ws_bytes=300), 3),
+])
+def test_ffw_rejects_bad_arguments(lib, kw, code):
+    assert _ffw(lib, **kw) == code
+    assert dd.last_error()
+
+
+def test_ffw_workspace_and_empty_call(lib):
+    assert _ffw(lib, rows=0, ptr=None, w=None, ws=None) == 0
+    assert lib.dd_ffw_workspace(256, 2048, 1904) >= 256 + 256 * 1904 * 2
+    assert lib.dd_ffw_workspace(256, 2048, 1900) == 0
+    n = lib.dd_self_condition_workspace(256, 262144, 2048, 1904)
+    assert n >= lib.dd_soft_embed_workspace(256, 262144, 2048) + 256 * (2048 + 1904) * 2
+    assert lib.dd_self_condition_workspace(256, 262144, 2000, 1904) == 0
+
+
+def _selfcond(lib, rows=4, vocab=100, stride=104, d=128, h=32, dtype=0, ptr=FAKE, w=FAKE,
+              u_out=None, ws=FAKE, ws_bytes=1 << 30):
+    return lib.dd_self_condition(ptr, dtype, rows, vocab, stride, 1.0, ptr, d, w, w, h, w, w, ptr,
+                                 u_out, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dtype=1), 2), (dict(d=96), 2), (dict(h=24), 2), (dict(stride=99), 1), (dict(w=None), 1),
+    (dict(u_out=ctypes.c_void_p((1 << 20) + 2)), 1), (dict(ws=None), 3), (dict(ws_bytes=512), 3),
+])
+def test_self_condition_rejects_bad_arguments(lib, kw, code):
+    assert _selfcond(lib, **kw) == code
+    assert dd.last_error()
+
+
 def test_block_graph_rejects_bad_handles(lib):
     d = _desc()
     cu = _cu([16])

@@ -216,6 +216,31 @@ def embedding(w: Workload, d: Optional[int] = None, device="cpu"):
     return _normal(w, "embedding", 0, (w.vocab, d), 1.0, device)
 
 
+# Hidden width of the self-conditioning MLP: the pages give only its size
+# (7.8M parameters).  Two dense layers d -> h -> d with biases at d = 2048
+# and h = 1904 hold 2 * 2048 * 1904 + 1904 + 2048 = 7,802,784 parameters.
+FFW_HIDDEN = 1904
+
+
+def ffw_weights(w: Workload, d: Optional[int] = None, hidden: int = FFW_HIDDEN, device="cpu"):
+    """Synthetic weights of the self-conditioning MLP in the workload's
+    dtype: W1 [d, h] ~ N(0, 1/d), b1 [h] ~ N(0, 0.1^2), W2 [h, d] ~ N(0, 1/h),
+    b2 [d] ~ N(0, 0.1^2) (fan-in scaling keeps the activations of order 1)."""
+    d = w.heads_q * w.head_dim if d is None else d
+    w1 = _normal(w, "ffw_w1", 0, (d, hidden), 1.0 / math.sqrt(d), device)
+    b1 = _normal(w, "ffw_b1", 0, (hidden,), 0.1, device)
+    w2 = _normal(w, "ffw_w2", 0, (hidden, d), 1.0 / math.sqrt(hidden), device)
+    b2 = _normal(w, "ffw_b2", 0, (d,), 0.1, device)
+    return w1, b1, w2, b2
+
+
+def ffw_input(w: Workload, rows: Optional[int] = None, d: Optional[int] = None, device="cpu"):
+    """A synthetic MLP input u [rows, d] ~ N(0, 1) (standing in for p0 E)."""
+    d = w.heads_q * w.head_dim if d is None else d
+    rows = w.rows if rows is None else rows
+    return _normal(w, "ffw_u", 0, (rows, d), 1.0, device)
+
+
 def all_steps(w: Workload, device="cpu"):
     """Per-step canvas Q/K/V and logits for every step of the workload."""
     qs, kcs, vcs, ls = [], [], [], []
