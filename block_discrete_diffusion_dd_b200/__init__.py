@@ -36,7 +36,7 @@ EXPORTS = (
     "dd_soft_embed_workspace", "dd_soft_embed", "dd_denoise_block_fp8",
     "dd_denoise_block_adaptive_graph_create", "dd_denoise_block_adaptive_graph_launch",
     "dd_denoise_block_adaptive_graph_destroy", "dd_ffw_workspace", "dd_ffw",
-    "dd_self_condition_workspace", "dd_self_condition", "dd_set_wait_limit_ns",
+    "dd_self_condition_workspace", "dd_self_condition", "dd_set_test_stall_ns",
 )
 
 
@@ -122,8 +122,8 @@ def load() -> ctypes.CDLL:
     lib.dd_soft_embed_workspace.argtypes = [i32, i32, i32]
     lib.dd_soft_embed.restype = i32
     lib.dd_soft_embed.argtypes = [P, i32, i32, i32, i64, ctypes.c_float, P, i32, P, P, sz, P]
-    lib.dd_set_wait_limit_ns.restype = None
-    lib.dd_set_wait_limit_ns.argtypes = [u64]
+    lib.dd_set_test_stall_ns.restype = None
+    lib.dd_set_test_stall_ns.argtypes = [u64]
     lib.dd_ffw_workspace.restype = sz
     lib.dd_ffw_workspace.argtypes = [i32, i32, i32]
     lib.dd_ffw.restype = i32
@@ -640,10 +640,11 @@ def query_device_error(workspace: torch.Tensor, stream=None):
     _check(load().dd_query_device_error(_ptr(workspace), _stream(stream)))
 
 
-def set_wait_limit_ns(ns: int):
-    """dd_set_wait_limit_ns: the pipeline-wait limit of the tensor-core
-    kernels launched afterwards from this thread (0 = the 1 s default)."""
-    load().dd_set_wait_limit_ns(int(ns))
+def set_test_stall_ns(ns: int):
+    """dd_set_test_stall_ns: with ns != 0 the tensor-core kernels launched
+    afterwards from this thread stall on a barrier nothing completes and
+    report DD_ERR_DEVICE_TIMEOUT after ns nanoseconds (0 turns it off)."""
+    load().dd_set_test_stall_ns(int(ns))
 
 
 def launch_count() -> int:

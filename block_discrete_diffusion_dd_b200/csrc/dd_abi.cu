@@ -246,8 +246,9 @@ dd_status run_sampler(const void* logits, dd_dtype dtype, int rows, int vocab, i
 void note_launch() { ++g_launches; }
 
 constexpr uint64_t kDefaultWaitNs = 1000000000ull;
-thread_local uint64_t g_wait_ns = kDefaultWaitNs;
-uint64_t pipeline_wait_ns() { return g_wait_ns; }
+thread_local uint64_t g_stall_ns = 0;  // 0: no test stall
+uint64_t pipeline_wait_ns() { return g_stall_ns ? g_stall_ns : kDefaultWaitNs; }
+bool pipeline_test_stall() { return g_stall_ns != 0; }
 
 thread_local bool g_pdl_off = false;
 bool pdl_enabled() { return !g_pdl_off; }
@@ -1125,7 +1126,7 @@ const char* dd_status_string(dd_status s) {
 
 const char* dd_last_error(void) { return g_last_error.c_str(); }
 
-void dd_set_wait_limit_ns(uint64_t ns) { g_wait_ns = ns ? ns : kDefaultWaitNs; }
+void dd_set_test_stall_ns(uint64_t ns) { g_stall_ns = ns; }
 
 uint64_t dd_launch_count(void) { return g_launches; }
 void dd_reset_launch_count(void) { g_launches = 0; }

@@ -62,12 +62,6 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemO = kQT * BN;     // O columns start after the S/P regions
 constexpr int kStageStride = HD + 4;       // padded fp32 row of the O staging area
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per wait
-#ifndef DD_POLY_PAIRS
-#define DD_POLY_PAIRS 0
-#endif
-// Of every 8 pairs of softmax exponentials, this many are evaluated by a
-// polynomial on the FMA pipe instead of the MUFU unit (balances the pipes).
-constexpr int kPolyPairs = DD_POLY_PAIRS;
 
 struct Barriers {
   uint64_t q_full;
@@ -76,6 +70,7 @@ struct Barriers {
   uint64_t xch[kQT][4];  // per (query tile, 32-row group): the two column halves meet
   uint64_t staged[kQT];  // per query tile: all 8 warps have staged their O rows
   uint64_t mma_final;
+  uint64_t never;  // completed by nothing: the target of the test stall
   uint32_t tmem_base;
   int abort;
   int unit_b, unit_g, unit_tp, unit_s, unit_valid, unit_nsplit, unit_slot0;
@@ -118,6 +113,7 @@ struct TcParams {
   float* part_lse;  // [slots][BM]   log2 units
   uint32_t* err;
   uint64_t wait_ns;  // limit of each pipeline wait (waits that drain use kWaitLimitNs)
+  int stall;         // test stall: one wait on `never` once the first MMAs are issued
 };
 
 __device__ __forceinline__ int cdiv(int a, int b) { return (a + b - 1) / b; }
@@ -269,6 +265,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->staged[q], 8);
     }
     mbar_init(&bars->mma_final, 1);
+    mbar_init(&bars->never, 1);
     bars->abort = 0;
     fence_mbar_init();
     resolve_unit(p, bars);
@@ -364,6 +361,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           __syncwarp();
         }
         commit(&bars->k_empty[0]);
+        // test stall: a wait nothing completes, with the first S MMAs in flight
+        if (p.stall) ok = wait(&bars->never, 0);
       }
       for (int j = 0; ok && j < n; ++j) {
         const int vst = j % G::kStages;
@@ -451,10 +450,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int e = 0; e < kKeysPerStore / 2; ++e) {
           const int c = hh * kKeysPerStore + 2 * e;
           const float2 d = __ffma2_rn(make_float2(sv[c], sv[c + 1]), sl2, nm);
-          // kPolyPairs of every 8 pairs take the FMA-pipe exponential
-          const float2 pp = (e & 7) < kPolyPairs
-                                ? exp2_poly2(d)
-                                : make_float2(ex2_approx(d.x), ex2_approx(d.y));
+          const float2 pp = make_float2(ex2_approx(d.x), ex2_approx(d.y));
           acc[e & 3] = __fadd2_rn(acc[e & 3], pp);
           if constexpr (kF8) {
             if (e & 1) w[e >> 1] = pack_e4m3x4(prev, pp);
@@ -878,6 +874,7 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t stream) {
   tp.part_lse = reinterpret_cast<float*>(scratch + (size_t)pl.slots * BM * HD * sizeof(float));
   tp.err = a.err;
   tp.wait_ns = pipeline_wait_ns();
+  tp.stall = pipeline_test_stall() ? 1 : 0;
 
   cudaError_t e =
       f8 ? launch_pdl(attn_tc_kernel<true>, dim3(pl.units), dim3(kThreads), Lay<true>::kSmemBytes,

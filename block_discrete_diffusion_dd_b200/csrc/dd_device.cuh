@@ -143,33 +143,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-// 2^x on the FMA pipe for two values at once (x <= 2^7), for the share of a
-// softmax's exponentials that should not queue on the MUFU unit.
-// Method: Cody-Waite style range reduction x = n + f with n = round(x),
-// f in [-1/2, 1/2] (adding 1.5 * 2^23 rounds to an integer in the low
-// mantissa bits), a degree-3 polynomial for 2^f whose coefficients are a
-// relative-error least-squares fit on Chebyshev nodes refined by Lawson
-// reweighting (max relative error 7.5e-5 in fp32, tested against exp2f), and
-// n re-inserted into the exponent field with one integer multiply-add.
-// Inputs below -126 are clamped there (result ~1e-38; used only where the
-// result is rounded to bf16 and summed next to terms >= 2^-8).
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  x.x = fmaxf(x.x, -126.0f);
-  x.y = fmaxf(x.y, -126.0f);
-  const float2 magic = make_float2(12582912.0f, 12582912.0f);
-  const float2 t = __fadd2_rn(x, magic);                 // low bits = round(x)
-  const float2 r = __fadd2_rn(t, make_float2(-12582912.0f, -12582912.0f));
-  const float2 f = __fadd2_rn(x, make_float2(-r.x, -r.y));  // x - round(x)
-  float2 q = __ffma2_rn(make_float2(0.055171623826026917f, 0.055171623826026917f), f,
-                        make_float2(0.2426111251115799f, 0.2426111251115799f));
-  q = __ffma2_rn(q, f, make_float2(0.6932609677314758f, 0.6932609677314758f));
-  q = __ffma2_rn(q, f, make_float2(0.9999280571937561f, 0.9999280571937561f));
-  // bits(t) << 23 == round(x) << 23 (mod 2^32): add it to q's exponent
-  const uint32_t ex = __float_as_uint(t.x) * (1u << 23) + __float_as_uint(q.x);
-  const uint32_t ey = __float_as_uint(t.y) * (1u << 23) + __float_as_uint(q.y);
-  return make_float2(__uint_as_float(ex), __uint_as_float(ey));
-}
-
 // ------------------------------------------------------------------ smem
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return (uint32_t)__cvta_generic_to_shared(p);

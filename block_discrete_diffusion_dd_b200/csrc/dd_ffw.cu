@@ -47,6 +47,7 @@ constexpr uint64_t FF_WAIT_NS = 1000000000ull;
 struct FfBars {
   uint64_t full[FF_STAGES], empty[FF_STAGES];
   uint64_t acc_full, mma_final;
+  uint64_t never;  // completed by nothing: the target of the test stall
   uint32_t tmem_base;
   int abort;
 };
@@ -61,6 +62,7 @@ struct FfParams {
   float* part;         // splits > 1: fp32 partials [splits][rows][N]
   uint32_t* err;
   uint64_t wait_ns;    // limit of each pipeline wait (waits that drain use FF_WAIT_NS)
+  int stall;           // test stall: one wait on `never` once the first MMAs are issued
 };
 
 // GELU(x) = x * Phi(x), Phi the standard normal distribution function.
@@ -92,6 +94,7 @@ __global__ void __launch_bounds__(FF_THREADS)
     }
     mbar_init(&bars->acc_full, 1);
     mbar_init(&bars->mma_final, 1);
+    mbar_init(&bars->never, 1);
     bars->abort = 0;
     fence_mbar_init();
   }
@@ -151,6 +154,11 @@ __global__ void __launch_bounds__(FF_THREADS)
         tc_commit(&bars->empty[s]);
       }
       __syncwarp();
+      // test stall: a wait nothing completes, with the first MMAs in flight
+      if (i == 0 && p.stall) {
+        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->never, 0, abort_flag, p.wait_ns));
+        if (!ok) break;
+      }
     }
     if (leader) {
       if (ok) tc_commit(&bars->acc_full);
@@ -315,6 +323,7 @@ cudaError_t launch_dense(const DenseArgs& a, cudaStream_t stream) {
   p.part = static_cast<float*>(a.part);
   p.err = a.err;
   p.wait_ns = pipeline_wait_ns();
+  p.stall = pipeline_test_stall() ? 1 : 0;
   const dim3 grid((a.N + FF_BN - 1) / FF_BN, (a.rows + FF_BM - 1) / FF_BM, pl.splits);
   e = a.gelu ? launch_pdl(dense_kernel<true>, grid, dim3(FF_THREADS), FF_SMEM, stream, mX, mW, p)
              : launch_pdl(dense_kernel<false>, grid, dim3(FF_THREADS), FF_SMEM, stream, mX, mW, p);

@@ -164,10 +164,13 @@ size_t dense_partial_bytes(int rows, int K, int N);
 cudaError_t launch_dense(const DenseArgs& a, cudaStream_t stream);
 
 // Time limit of the pipeline waits (mbarrier waits that can abort) of the
-// tensor-core kernels launched from this host thread: 1 s unless changed by
-// dd_set_wait_limit_ns.  Waits that drain in-flight copies and MMAs before
-// a CTA exits always keep their own 1 s limit.
+// tensor-core kernels launched from this host thread: 1 s unless a test
+// stall is set (dd_set_test_stall_ns).  Waits that drain in-flight copies
+// and MMAs before a CTA exits always keep their own 1 s limit.
 uint64_t pipeline_wait_ns();
+// True while a test stall is set on this host thread: each tensor-core
+// kernel then makes one pipeline wait on a barrier nothing completes.
+bool pipeline_test_stall();
 
 // Launch accounting (per host thread).
 void note_launch();

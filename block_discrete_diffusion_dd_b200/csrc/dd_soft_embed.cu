@@ -62,6 +62,7 @@ constexpr uint64_t SE_WAIT_NS = 1000000000ull;
 struct SeBars {
   uint64_t full[SE_STAGES], pfull[SE_STAGES], empty[SE_STAGES];
   uint64_t acc_full, mma_final;
+  uint64_t never;  // completed by nothing: the target of the test stall
   uint32_t tmem_base;
   int abort;
 };
@@ -76,6 +77,7 @@ struct SeParams {
   float* part;           // [splits][rows][d] fp32
   uint32_t* err;
   uint64_t wait_ns;      // limit of each pipeline wait (waits that drain use SE_WAIT_NS)
+  int stall;             // test stall: one wait on `never` once the first MMAs are issued
 };
 
 // ---------------------------------------------------------------- row LSE
@@ -218,6 +220,7 @@ __global__ void __launch_bounds__(SE_THREADS, 1)
     }
     mbar_init(&bars->acc_full, 1);
     mbar_init(&bars->mma_final, 1);
+    mbar_init(&bars->never, 1);
     bars->abort = 0;
     fence_mbar_init();
   }
@@ -285,6 +288,10 @@ __global__ void __launch_bounds__(SE_THREADS, 1)
           tc_commit(&bars->empty[s]);
         }
         __syncwarp();
+        // test stall: a wait nothing completes, with the first MMAs in flight
+        if (i == 0 && p.stall)
+          ok = __all_sync(0xffffffffu,
+                          mbar_wait_bounded(&bars->never, 0, abort_flag, p.wait_ns));
       }
       if (leader) {
         if (ok) tc_commit(&bars->acc_full);
@@ -505,6 +512,7 @@ cudaError_t launch_soft_embed(const SoftEmbedArgs& a, cudaStream_t stream) {
   p.part = part;
   p.err = a.err;
   p.wait_ns = pipeline_wait_ns();
+  p.stall = pipeline_test_stall() ? 1 : 0;
   e = launch_pdl(soft_embed_kernel, dim3(pl.grid_x, pl.splits, pl.grid_z), dim3(SE_THREADS),
                  SE_SMEM, stream, mL, mE, p);
   note_launch();

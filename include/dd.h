@@ -498,16 +498,19 @@ DD_API const char* dd_status_string(dd_status status);
 /* Detail of the last failure on this host thread ("" if none). */
 DD_API const char* dd_last_error(void);
 
-/* Time limit of each pipeline wait (a wait on an mbarrier that other warps
- * or the copy and tensor-core units complete) in the tensor-core kernels
- * (attention, soft embedding, MLP) launched afterwards from this host
- * thread; 0 restores the default of 1 s.  A wait that runs out latches
- * DD_ERR_DEVICE_TIMEOUT in the call's workspace (read it with
- * dd_query_device_error), and the kernel then waits, up to 1 s each, for
- * its own copies and MMAs in flight, frees its tensor memory and returns;
- * the outputs of that call are undefined.  A short limit is a test of that
- * path (the pages have no counterpart); leave it at the default otherwise. */
-DD_API void dd_set_wait_limit_ns(uint64_t ns);
+/* Test hook for the device-timeout path (the pages have no counterpart).
+ * Every wait of the tensor-core kernels (attention, soft embedding, MLP) on
+ * an mbarrier is bounded in time.  With ns != 0, the kernels launched
+ * afterwards from this host thread make one extra wait, once their first
+ * MMAs are in flight, on an mbarrier that nothing completes, and their
+ * pipeline waits are limited to ns nanoseconds: the wait runs out, the call
+ * latches DD_ERR_DEVICE_TIMEOUT in its workspace (read it with
+ * dd_query_device_error), and every CTA waits (up to 1 s per wait) for its
+ * own copies and MMAs in flight, frees its tensor memory and returns.  The
+ * outputs of such a call are undefined; clear the workspace
+ * (dd_workspace_init) before its next use.  ns = 0 (the default) turns the
+ * stall off. */
+DD_API void dd_set_test_stall_ns(uint64_t ns);
 
 /* Number of kernels the library launched on this host thread since the last
  * call to dd_reset_launch_count (for launch accounting in benchmarks). */
