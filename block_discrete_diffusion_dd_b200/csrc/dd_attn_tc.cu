@@ -18,15 +18,14 @@
 // log-sum-exp.
 //
 // Inside a CTA (18 warps) the two query tiles share every key tile:
-//   warps 0-7 / 8-15  softmax of query tile 0 / 1.  A query row (= one TMEM
-//              lane) is shared by two threads in two warps, one per half of
-//              the 128 key columns; they meet once per tile in shared
-//              memory to agree on the row max.  Each half reads its 64 S
-//              columns (fp32) from TMEM, runs the online softmax in fp32
-//              (log2 domain; O is rescaled only when the running max grows
-//              past a margin) and writes its half of P back (bf16 pairs in
-//              columns 0-31 / 64-95, E4M3 quads in 0-15 / 64-79) into its
-//              own half of the same TMEM region, where the P.V MMA reads it;
+//   warps 0-7 / 8-15  softmax of query tile 0 / 1.  Each warp owns 16
+//              query rows (TMEM lanes): through the 16-lane tcgen05.ld
+//              shape a row's 128 key columns sit in four threads of the
+//              warp, which reduce the row max and sum with two shuffles.
+//              They run the online softmax in fp32 (log2 domain; O is
+//              rescaled only when the running max grows past a margin) and
+//              write P back (bf16 pairs in columns 0-63, E4M3 quads in
+//              0-31) into the same TMEM region, where the P.V MMA reads it;
 //   warp 16    TMA producer: Q, then K and V tiles (rings of 128 keys, 2
 //              stages for bf16, 4 for E4M3) in the order the MMAs consume
 //              them;
@@ -67,7 +66,6 @@ struct Barriers {
   uint64_t q_full;
   uint64_t k_full[kMaxStages], k_empty[kMaxStages], v_full[kMaxStages], v_empty[kMaxStages];
   uint64_t s_full[kQT], p_full[kQT], o_done[kQT];
-  uint64_t xch[kQT][4];  // per (query tile, 32-row group): the two column halves meet
   uint64_t staged[kQT];  // per query tile: all 8 warps have staged their O rows
   uint64_t mma_final;
   uint64_t never;  // completed by nothing: the target of the test stall
@@ -94,13 +92,12 @@ struct Lay {
   static constexpr uint32_t kOffQ = 0;
   static constexpr uint32_t kOffK = kOffQ + kQT * kTile;
   static constexpr uint32_t kOffV = kOffK + kStages * kTile;
-  static constexpr uint32_t kOffX = kOffV + kStages * kTile;  // row-max exchange [q][slot][half][row]
-  static constexpr uint32_t kOffBar = kOffX + kQT * 2 * 2 * BM * 4;
+  static constexpr uint32_t kOffBar = kOffV + kStages * kTile;
   static constexpr uint32_t kSmemBytes = kOffBar + sizeof(Barriers) + 1024;
   static constexpr float kBias = kF8 ? 6.0f : 0.0f;  // log2 units
   static constexpr float kLazy = kF8 ? 2.0f : 8.0f;  // log2 units
   static_assert(kStages <= kMaxStages, "barrier arrays");
-  static_assert(kQT * BM * kStageStride * 4 <= kOffX, "O staging fits the operand buffers");
+  static_assert(kQT * BM * kStageStride * 4 <= kOffBar, "O staging fits the operand buffers");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
@@ -182,23 +179,22 @@ __device__ __forceinline__ void issue_s(uint32_t tmem, uint64_t dQ, uint64_t dK,
 }
 
 // O_q (+)= P_q V for one 128-key tile: P from tensor memory (aP), V from the
-// ring stage at descriptor bv (MN-major).  The two column halves of P sit
-// BN/2 columns apart: keys 0-63 from column 0, keys 64-127 from column 64,
-// 2 keys per column for bf16 and 4 for E4M3.
+// ring stage at descriptor bv (MN-major).  P fills the first columns of the
+// S/P region in key order, 2 keys per column for bf16 and 4 for E4M3.
 template <bool kF8>
 __device__ __forceinline__ void issue_pv(uint32_t dO, uint32_t aP, uint64_t bv, bool acc0) {
   if constexpr (kF8) {
     constexpr uint32_t idPV = idesc_e4m3_f32(BM, HD, 0, 1);
 #pragma unroll
     for (int kk = 0; kk < BN / 32; ++kk)  // 32 keys = 8 columns of P, 4 KB of V
-      tc_mma_ts_f8(dO, aP + (uint32_t)((kk >> 1) * (BN / 2) + (kk & 1) * 8),
-                   desc_at(bv, kk * 32 * HD), idPV, (acc0 || kk > 0) ? 1u : 0u);
+      tc_mma_ts_f8(dO, aP + (uint32_t)(kk * 8), desc_at(bv, kk * 32 * HD), idPV,
+                   (acc0 || kk > 0) ? 1u : 0u);
   } else {
     constexpr uint32_t idPV = idesc_bf16_f32(BM, HD, 0, 1);
 #pragma unroll
     for (int kk = 0; kk < BN / 16; ++kk)  // 16 keys = 8 columns of P, 2 KB of each half of V
-      tc_mma_ts(dO, aP + (uint32_t)((kk >> 2) * (BN / 2) + (kk & 3) * 8),
-                desc_at(bv, kk * 16 * 128), idPV, (acc0 || kk > 0) ? 1u : 0u);
+      tc_mma_ts(dO, aP + (uint32_t)(kk * 8), desc_at(bv, kk * 16 * 128), idPV,
+                (acc0 || kk > 0) ? 1u : 0u);
   }
 }
 
@@ -261,7 +257,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->s_full[q], 1);
       mbar_init(&bars->p_full[q], 8);
       mbar_init(&bars->o_done[q], 1);
-      for (int i = 0; i < 4; ++i) mbar_init(&bars->xch[q][i], 2);
       mbar_init(&bars->staged[q], 8);
     }
     mbar_init(&bars->mma_final, 1);
@@ -409,61 +404,79 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp < kSoftmaxWarps && n > 0 && (warp >> 3) < nq) {
     // ------------------------------------------------------------ softmax
-    const int q = warp >> 3, h = (warp >> 2) & 1, wl = warp & 3;
-    const int r = wl * 32 + lane;                         // query row in tile q
-    const uint32_t lane_base = (uint32_t)(wl * 32) << 16;  // TMEM lane field
+    // Warp (q, hv, wl) of query tile q reaches TMEM lane quarter wl (=
+    // warp % 4) and takes its 16-lane half hv.  Through the 16x256b shape,
+    // thread t holds rows A = 32 wl + 16 hv + t/4 and B = A + 8 and, of
+    // every 8 key columns, the two at 2 (t % 4): 32 keys of each row.  The
+    // four threads of a row reduce it with two shuffles, so the row max is
+    // known before P is formed.
+    const int q = warp >> 3, wl = warp & 3, hv = (warp >> 2) & 1;
+    const int t4 = lane & 3;
+    const int rbase = wl * 32 + hv * 16;
+    const int rA = rbase + (lane >> 2), rB = rA + 8;  // query rows in tile q
+    const uint32_t lane_base = (uint32_t)rbase << 16;  // TMEM lane field
     const uint32_t tS = tmem + lane_base + (uint32_t)(q * BN);
-    const uint32_t tO = tmem + lane_base + kTmemO + (uint32_t)(q * HD + h * (HD / 2));
-    float* xch = reinterpret_cast<float*>(smem + G::kOffX) + q * (2 * 2 * BM);
-    uint64_t* xbar = &bars->xch[q][wl];
+    const uint32_t tO = tmem + lane_base + kTmemO + (uint32_t)(q * HD);
     const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
-    float m_ref = -INFINITY, l = 0.f;
+    float mrefA = -INFINITY, mrefB = -INFINITY, lA = 0.f, lB = 0.f;
     bool ok = true;
-    // exchange a per-row value with the other column half (phase `ph`):
-    // post it, then (possibly after other work) wait for the partner's
-    auto post = [&](float v, int ph) {
-      xch[(ph & 1) * (2 * BM) + h * BM + r] = v;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(xbar);
+    auto quad_max = [](float v) {
+      v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
+      return fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));
     };
-    auto take = [&](int ph) -> float {
-      if (!__all_sync(0xffffffffu, mbar_wait_bounded(xbar, ph & 1, abort_flag, p.wait_ns))) {
-        ok = false;
-        return -INFINITY;
-      }
-      return xch[(ph & 1) * (2 * BM) + (h ^ 1) * BM + r];
+    auto quad_sum = [](float v) {
+      v += __shfl_xor_sync(0xffffffffu, v, 1);
+      return v + __shfl_xor_sync(0xffffffffu, v, 2);
     };
-    // P = 2^(s * scale_log2 - mref), packed (bf16 pairs or E4M3 quads)
-    // into columns from h*64 of the S/P region: inside this half's own S
-    // columns, so it never overwrites S the other half has yet to read;
-    // returns the partial row sum (of the unrounded P)
-    auto emit_p = [&](const float (&sv)[BN / 2], float mref) -> float {
-      const float2 nm = make_float2(-mref, -mref);
-      float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                       make_float2(0.f, 0.f)};
-      constexpr int kKeysPerStore = kF8 ? 32 : 16;  // 8 packed columns per store
+    // P = 2^(s scale_log2 - mref) for the thread's 64 scores, packed into
+    // the first BN / 2 (bf16 pairs) or BN / 4 (E4M3 quads) columns of the
+    // S/P region, where the P.V MMA reads it: this warp has loaded all of
+    // its rows' S already.  Adds the rows' partial sums of the unrounded P.
+    auto emit_p = [&](const uint32_t (&sv)[64], float ma, float mb) {
+      const float2 na = make_float2(-ma, -ma), nb = make_float2(-mb, -mb);
+      float2 sa = make_float2(0.f, 0.f), sb = make_float2(0.f, 0.f);
+      if constexpr (!kF8) {
+        uint32_t w[32];  // 16x128b: w[2i] row A, w[2i + 1] row B, column 4 i + t % 4
 #pragma unroll
-      for (int hh = 0; hh < (BN / 2) / kKeysPerStore; ++hh) {
-        uint32_t w[8];
-        float2 prev = make_float2(0.f, 0.f);
-#pragma unroll
-        for (int e = 0; e < kKeysPerStore / 2; ++e) {
-          const int c = hh * kKeysPerStore + 2 * e;
-          const float2 d = __ffma2_rn(make_float2(sv[c], sv[c + 1]), sl2, nm);
-          const float2 pp = make_float2(ex2_approx(d.x), ex2_approx(d.y));
-          acc[e & 3] = __fadd2_rn(acc[e & 3], pp);
-          if constexpr (kF8) {
-            if (e & 1) w[e >> 1] = pack_e4m3x4(prev, pp);
-            prev = pp;
-          } else {
-            w[e] = pack_bf16x2(pp.x, pp.y);
-          }
+        for (int i = 0; i < 16; ++i) {
+          const float2 da = __ffma2_rn(
+              make_float2(__uint_as_float(sv[4 * i]), __uint_as_float(sv[4 * i + 1])), sl2, na);
+          const float2 db = __ffma2_rn(
+              make_float2(__uint_as_float(sv[4 * i + 2]), __uint_as_float(sv[4 * i + 3])), sl2, nb);
+          const float2 pa = make_float2(ex2_approx(da.x), ex2_approx(da.y));
+          const float2 pb = make_float2(ex2_approx(db.x), ex2_approx(db.y));
+          sa = __fadd2_rn(sa, pa);
+          sb = __fadd2_rn(sb, pb);
+          w[2 * i] = pack_bf16x2(pa.x, pa.y);
+          w[2 * i + 1] = pack_bf16x2(pb.x, pb.y);
         }
-        tmem_st8(tS + (uint32_t)(h * (BN / 2) + hh * 8), w);
+        tmem_st16x128b_x16(tS, w);
+      } else {
+        // a 32-bit column holds 4 keys; the thread's pair and its
+        // neighbour's (thread t ^ 1) make one: the even thread stores row
+        // A's, the odd one row B's (16x64b: lane t/4 + 8 (t % 2), column
+        // 2 i + (t % 4) / 2)
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float2 da = __ffma2_rn(
+              make_float2(__uint_as_float(sv[4 * i]), __uint_as_float(sv[4 * i + 1])), sl2, na);
+          const float2 db = __ffma2_rn(
+              make_float2(__uint_as_float(sv[4 * i + 2]), __uint_as_float(sv[4 * i + 3])), sl2, nb);
+          const float2 pa = make_float2(ex2_approx(da.x), ex2_approx(da.y));
+          const float2 pb = make_float2(ex2_approx(db.x), ex2_approx(db.y));
+          sa = __fadd2_rn(sa, pa);
+          sb = __fadd2_rn(sb, pb);
+          const uint32_t ha = __nv_cvt_float2_to_fp8x2(pa, __NV_SATFINITE, __NV_E4M3);
+          const uint32_t hb = __nv_cvt_float2_to_fp8x2(pb, __NV_SATFINITE, __NV_E4M3);
+          const uint32_t oa = __shfl_xor_sync(0xffffffffu, ha, 1);
+          const uint32_t ob = __shfl_xor_sync(0xffffffffu, hb, 1);
+          w[i] = (lane & 1) ? (ob | (hb << 16)) : (ha | (oa << 16));
+        }
+        tmem_st16x64b_x16(tS, w);
       }
-      const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
-      const float2 a = __fadd2_rn(a01, a23);
-      return a.x + a.y;
+      lA += sa.x + sa.y;
+      lB += sb.x + sb.y;
     };
     int j = 0;
     for (; j < n && ok; ++j) {
@@ -476,95 +489,83 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      float sv[BN / 2];
-      {
-        uint32_t raw[BN / 2];
-        tmem_ld64(tS + (uint32_t)(h * (BN / 2)), raw);
+      uint32_t sv[64];
+      tmem_ld16x256b_x16(tS, sv);
+      if (n_valid < BN) {  // ragged last tile of the prefix or of the canvas
 #pragma unroll
-        for (int c = 0; c < BN / 2; ++c) sv[c] = __uint_as_float(raw[c]);
-      }
-      const int nv = n_valid - h * (BN / 2);  // valid columns in this half
-      if (nv < BN / 2) {  // ragged last tile of the prefix or of the canvas
-#pragma unroll
-        for (int c = 0; c < BN / 2; ++c)
-          if (c >= nv) sv[c] = -INFINITY;
-      }
-      float mx0 = sv[0], mx1 = sv[1];
-#pragma unroll
-      for (int c = 2; c < BN / 2; c += 2) {
-        mx0 = fmaxf(mx0, sv[c]);
-        mx1 = fmaxf(mx1, sv[c + 1]);
-      }
-      const float mh = fmaxf(mx0, mx1);
-      post(mh, j);
-      float lt;
-      if (j == 0) {
-        // first tile: the reference is the row max (less the bias)
-        const float mx = fmaxf(mh, take(j)) * p.scale_log2;
-        if (!ok) break;
-        m_ref = mx - G::kBias;
-        lt = emit_p(sv, m_ref);
-      } else {
-        // later tiles: P with the current reference first; the row max
-        // (the partner's post has usually arrived by then) decides, rarely,
-        // that P would exceed 2^8, so the reference rises and P is redone
-        lt = emit_p(sv, m_ref);
-        const float mx = fmaxf(mh, take(j)) * p.scale_log2;
-        if (!ok) break;
-        // lazy rescale (warp-uniform decision so tcgen05.ld/st stay
-        // converged; both halves see the same row maxima, so they decide
-        // alike); PV_q(j-1) is complete because S_q(j) is
-        if (__any_sync(0xffffffffu, mx > m_ref + (G::kLazy + G::kBias))) {
-          const float m_new = fmaxf(m_ref, mx - G::kBias);
-          const float alpha = ex2_approx(m_ref - m_new);
-          l *= alpha;
-#pragma unroll 1
-          for (int c8 = 0; c8 < HD / 16; ++c8) {
-            uint32_t raw[8];
-            tmem_ld8(tO + (uint32_t)(c8 * 8), raw);
-#pragma unroll
-            for (int c = 0; c < 8; ++c) raw[c] = __float_as_uint(__uint_as_float(raw[c]) * alpha);
-            tmem_st8(tO + (uint32_t)(c8 * 8), raw);
-          }
-          m_ref = m_new;
-          lt = emit_p(sv, m_ref);
+        for (int i = 0; i < 16; ++i) {
+          const int c = 8 * i + 2 * t4;
+          if (c >= n_valid) sv[4 * i] = sv[4 * i + 2] = __float_as_uint(-INFINITY);
+          if (c + 1 >= n_valid) sv[4 * i + 1] = sv[4 * i + 3] = __float_as_uint(-INFINITY);
         }
       }
-      l += lt;
+      float ma = fmaxf(__uint_as_float(sv[0]), __uint_as_float(sv[1]));
+      float mb = fmaxf(__uint_as_float(sv[2]), __uint_as_float(sv[3]));
+#pragma unroll
+      for (int i = 1; i < 16; ++i) {
+        ma = fmaxf(ma, fmaxf(__uint_as_float(sv[4 * i]), __uint_as_float(sv[4 * i + 1])));
+        mb = fmaxf(mb, fmaxf(__uint_as_float(sv[4 * i + 2]), __uint_as_float(sv[4 * i + 3])));
+      }
+      const float xa = quad_max(ma) * p.scale_log2, xb = quad_max(mb) * p.scale_log2;
+      if (j == 0) {
+        // first tile: the reference is the row max (less the bias)
+        mrefA = xa - G::kBias;
+        mrefB = xb - G::kBias;
+      } else if (__any_sync(0xffffffffu, xa > mrefA + (G::kLazy + G::kBias) ||
+                                             xb > mrefB + (G::kLazy + G::kBias))) {
+        // lazy rescale (rare; a warp-uniform decision so tcgen05.ld/st stay
+        // converged): PV_q(j-1) is complete because S_q(j) is
+        const float na = fmaxf(mrefA, xa - G::kBias), nb = fmaxf(mrefB, xb - G::kBias);
+        const float alA = ex2_approx(mrefA - na), alB = ex2_approx(mrefB - nb);
+        lA *= alA;
+        lB *= alB;
+#pragma unroll 1
+        for (int c16 = 0; c16 < HD / 16; ++c16) {
+          uint32_t o[8];  // 16x256b x2: o[4r], o[4r+1] row A; o[4r+2], o[4r+3] row B
+          tmem_ld16x256b_x2(tO + (uint32_t)(c16 * 16), o);
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            o[e] = __float_as_uint(__uint_as_float(o[e]) * ((e & 2) ? alB : alA));
+          tmem_st16x256b_x2(tO + (uint32_t)(c16 * 16), o);
+        }
+        mrefA = na;
+        mrefB = nb;
+      }
+      emit_p(sv, mrefA, mrefB);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->p_full[q]);
     }
-    // epilogue: O / l and the log2-domain LSE of this split; the halves add
-    // their partial row sums
+    // epilogue: O / l and the log2-domain LSE of this split
     if (ok)
       ok = __all_sync(0xffffffffu,
                       mbar_wait_bounded(&bars->o_done[q], 0, abort_flag, p.wait_ns));
-    float lrow = l;
-    if (ok) {
-      post(l, n);
-      lrow = l + take(n);
-    }
+    const float lrowA = quad_sum(lA), lrowB = quad_sum(lB);
     if (ok) {
       // O / l staged row-wise in shared memory (free now: every MMA has
       // completed), then copied out in whole 512-byte rows
       tc_fence_after();
-      const float inv = p.out_scale / lrow;
+      const float invA = p.out_scale / lrowA, invB = p.out_scale / lrowB;
       float* stage = reinterpret_cast<float*>(smem) + q * (BM * kStageStride);
-      float* srow = stage + r * kStageStride + h * (HD / 2);
+      {
+        uint32_t o[64];
+        tmem_ld16x256b_x16(tO, o);
 #pragma unroll
-      for (int c4 = 0; c4 < HD / 64; ++c4) {
-        uint32_t raw[32];
-        tmem_ld32(tO + (uint32_t)(c4 * 32), raw);
-#pragma unroll
-        for (int c = 0; c < 32; c += 4)
-          *reinterpret_cast<float4*>(srow + c4 * 32 + c) =
-              make_float4(__uint_as_float(raw[c]) * inv, __uint_as_float(raw[c + 1]) * inv,
-                          __uint_as_float(raw[c + 2]) * inv, __uint_as_float(raw[c + 3]) * inv);
+        for (int i = 0; i < 16; ++i) {
+          const int c = 8 * i + 2 * t4;
+          *reinterpret_cast<float2*>(stage + rA * kStageStride + c) =
+              make_float2(__uint_as_float(o[4 * i]) * invA, __uint_as_float(o[4 * i + 1]) * invA);
+          *reinterpret_cast<float2*>(stage + rB * kStageStride + c) =
+              make_float2(__uint_as_float(o[4 * i + 2]) * invB,
+                          __uint_as_float(o[4 * i + 3]) * invB);
+        }
       }
       const size_t slot = (size_t)slot0 + (size_t)q * nsplit;
-      if (h == 0) p.part_lse[slot * BM + r] = m_ref + __log2f(lrow);
+      if (t4 == 0) {
+        p.part_lse[slot * BM + rA] = mrefA + __log2f(lrowA);
+        p.part_lse[slot * BM + rB] = mrefB + __log2f(lrowB);
+      }
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->staged[q]);
       if (__all_sync(0xffffffffu,

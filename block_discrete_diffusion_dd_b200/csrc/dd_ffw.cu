@@ -223,8 +223,11 @@ __global__ void __launch_bounds__(FF_THREADS)
   if (warp == FF_WARP_MMA) tmem_dealloc(tmem, FF_TMEM_COLS);
 }
 
+constexpr int FF_MAX_SPLITS = 8;
+
 // out[r, n] = act(bias[n] + sum over splits, in split order, of
-// part[s][r][n]), rounded to bf16; 8 columns per thread.
+// part[s][r][n]), rounded to bf16; 8 columns per thread.  Every split's
+// values are requested before the first is added (one memory round trip).
 template <bool kGelu>
 __global__ void __launch_bounds__(256)
     dense_finish(const float* __restrict__ part, int splits, int rows, int N,
@@ -238,16 +241,24 @@ __global__ void __launch_bounds__(256)
     const int64_t r = i / n8;
     const int c = (int)(i - r * n8) * 8;
     const float* src = part + r * N + c;
-    float4 a = *reinterpret_cast<const float4*>(src);
-    float4 b = *reinterpret_cast<const float4*>(src + 4);
-    for (int s = 1; s < splits; ++s) {
-      const float* q = src + (size_t)s * rows * N;
-      const float4 x = *reinterpret_cast<const float4*>(q);
-      const float4 y = *reinterpret_cast<const float4*>(q + 4);
-      a.x += x.x; a.y += x.y; a.z += x.z; a.w += x.w;
-      b.x += y.x; b.y += y.y; b.z += y.z; b.w += y.w;
+    float4 x[FF_MAX_SPLITS], y[FF_MAX_SPLITS];
+#pragma unroll
+    for (int s = 0; s < FF_MAX_SPLITS; ++s) {
+      if (s < splits) {
+        const float* q = src + (size_t)s * rows * N;
+        x[s] = *reinterpret_cast<const float4*>(q);
+        y[s] = *reinterpret_cast<const float4*>(q + 4);
+      }
     }
     const uint4 braw = *reinterpret_cast<const uint4*>(bias + c);
+    float4 a = x[0], b = y[0];
+#pragma unroll
+    for (int s = 1; s < FF_MAX_SPLITS; ++s) {
+      if (s < splits) {
+        a.x += x[s].x; a.y += x[s].y; a.z += x[s].z; a.w += x[s].w;
+        b.x += y[s].x; b.y += y[s].y; b.z += y[s].z; b.w += y[s].w;
+      }
+    }
     float v[8] = {a.x + bf16lo(braw.x), a.y + bf16hi(braw.x), a.z + bf16lo(braw.y),
                   a.w + bf16hi(braw.y), b.x + bf16lo(braw.z), b.y + bf16hi(braw.z),
                   b.z + bf16lo(braw.w), b.w + bf16hi(braw.w)};
@@ -292,7 +303,7 @@ DensePlan dense_plan(int rows, int K, int N) {
   const int tiles = ((N + FF_BN - 1) / FF_BN) * ((rows + FF_BM - 1) / FF_BM);
   const int ksteps = (K + FF_BK - 1) / FF_BK;
   int splits = std::max(1, sm_count_ff() / std::max(1, tiles));
-  splits = std::min(splits, std::max(1, ksteps / 4));
+  splits = std::min(std::min(splits, FF_MAX_SPLITS), std::max(1, ksteps / 4));
   pl.ksteps_per_split = (ksteps + splits - 1) / splits;
   pl.splits = (ksteps + pl.ksteps_per_split - 1) / pl.ksteps_per_split;
   return pl;
