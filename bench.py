@@ -275,14 +275,14 @@ def run_ours(args, w, dist, rank, world, local_rank):
                    "parallelism": f"replicas x{world}"},
         "roofline": {"bound": "hbm", "kernel": "sampler (scan pass + row merge)",
                      "achieved": samp_gbs, "peak": hbm, "unit": "GB/s", "frac": samp_gbs / hbm,
-                     "traffic": traffic.get("sampler"), "peak_source": src,
+                     "traffic": traffic.get(f"sampler@{w.name}"), "peak_source": src,
                      "algorithmic_bytes": samp_bytes, "ms": t_samp * 1e3,
                      "alu_ceiling": _sampler_alu_ceiling(samp_gbs, clk.get("sm_mhz"))},
         "roofline_attn": {"bound": "tensor", "kernel": "canvas attention (tcgen05 + merge)",
                           "achieved": attn_tf, "peak": tf_burst, "unit": "TFLOP/s",
                           "frac": attn_tf / tf_burst, "frac_of_sustained": attn_tf / tf_sus,
                           "flops": w.attn_flops(), "ms": t_attn * 1e3,
-                          "traffic": traffic.get("attention"), "peak_source": src},
+                          "traffic": traffic.get(f"attention@{w.name}"), "peak_source": src},
         "e2e": e2e,
         "gpu_launches": int(launches),
         "clocks": clk,
@@ -427,8 +427,7 @@ def run_attn_e4m3(w, reps: int = 50):
         "ms": ms["e4m3"],
         "roofline": {"bound": "tensor", "achieved": tf8, "peak": 2 * tf_burst, "unit": "TFLOP/s",
                      "frac": tf8 / (2 * tf_burst), "flops": flops,
-                     "traffic": (_profile_traffic().get("attention_e4m3")
-                                 if w.name == "b1_L4096" else None),
+                     "traffic": _profile_traffic().get(f"attention_e4m3@{w.name}"),
                      "peak_source": f"{src} bf16 burst x 2 (nominal E4M3 / bf16 ratio)"},
         "bf16_same_workload": {"ms": ms["bf16"], "TFLOP/s": tf16, "frac": tf16 / tf_burst},
         "timing": f"median of {reps} calls, CUDA events around each call",
@@ -614,8 +613,9 @@ def _source_sha(name: str) -> str:
 def _profile_traffic() -> dict:
     """DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum)
     from the committed ncu summary profiles/traffic.txt.  A line reads
-    `<kernel> <bytes per launch> <source file> <sha256/16 of that source>`;
-    a figure taken on another version of the kernel source reads as None."""
+    `<kernel group>@<workload> <bytes per launch> <source file> <sha256/16 of
+    that source>`; a figure taken on another version of the kernel source
+    reads as None."""
     out = {}
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.txt")) as f:

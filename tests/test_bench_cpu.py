@@ -43,7 +43,7 @@ def test_profile_traffic_tracks_the_source(tmp_path, monkeypatch):
 
 def test_committed_traffic_entries_parse():
     t = bench._profile_traffic()
-    for k in ("sampler", "attention", "attention_e4m3", "soft_embed"):
+    for k in ("sampler@ragged_b8", "attention@ragged_b8", "sampler@b1_L4096"):
         assert k in t
 
 
