@@ -13,9 +13,19 @@
 // key tiles).  The key range of b is cut into 128-key tiles -- prefix tiles
 // first, then canvas tiles, each read through its own tensor map so a tile
 // never straddles the prefix/canvas boundary; the last tile of each part is
-// masked by key index.  Splits are balanced on the host so that whole waves
-// of CTAs cover the SMs; a second kernel merges the splits by their
-// log-sum-exp.
+// masked by key index.  The host picks each batch row's number of splits
+// (its tiles shared out evenly) and launches the units longest first, so
+// the SMs finish together; a second kernel merges the splits by their
+// log-sum-exp.  When the units take more than one round of the SMs, each
+// split CTA counts itself done on its (b, g, tile pair) counter with a
+// release add once its partials are written, and the merge CTAs of that
+// group poll the counter (acquire): a group is merged as soon as its own
+// splits are done -- during the tail of the attention grid, on SMs it has
+// left -- instead of after the whole grid.  The merge grid is launched as a
+// programmatic dependent, which is scheduled only once every attention CTA
+// has started, so a polling CTA never waits for a CTA that is not resident.
+// With a single round every split ends at about the same time, and the
+// merge waits for the whole grid instead (no counters).
 //
 // Inside a CTA (18 warps) the two query tiles share every key tile:
 //   warps 0-7 / 8-15  softmax of query tile 0 / 1.  Each warp owns 16
@@ -40,7 +50,11 @@
 //     may rescale O_q at that point without a further wait.
 // Every mbarrier wait is bounded in time; on expiry the CTA latches an
 // error word, drains its own asynchronous work and frees its TMEM.
+#include <algorithm>
+#include <functional>
 #include <mutex>
+#include <queue>
+#include <vector>
 
 #include "dd_device.cuh"
 #include "dd_internal.h"
@@ -101,13 +115,32 @@ struct Lay {
   static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
+// The host's split plan, passed by value (kernel parameter space).  Batch
+// rows are launched in `order`: the i-th row in that order owns the units
+// [ubase[i], ubase[i + 1]).  Row b has ns[b] key splits and its partials
+// start at slot sbase[b].  With more than kMaxPlanRows batch rows, n = 0 and
+// the kernels derive a uniform plan from TcParams::chunk instead.
+constexpr int kMaxPlanRows = 128;
+struct RowPlan {
+  int n;
+  int ubase[kMaxPlanRows + 1];
+  int order[kMaxPlanRows];
+  int sbase[kMaxPlanRows];
+  int ns[kMaxPlanRows];
+};
+
 struct TcParams {
-  int B, C, Hq, Hkv, group, T, chunk;
+  int B, C, Hq, Hkv, group, T, chunk;  // chunk: key tiles per split (uniform plan only)
   float scale_log2;  // softmax scale * log2(e), times the Q and K factors
   float out_scale;   // the V factor (1 for bf16)
   const int32_t* cu_prefix;
   float* part_o;    // [slots][BM][HD], slot = (b, g, t, split)
   float* part_lse;  // [slots][BM]   log2 units
+  // per (b, g, tile pair): splits done, and merge CTAs that have seen them
+  // all (the last one clears both for the next call); zero between calls
+  uint32_t* done;
+  uint32_t* seen;
+  int poll;  // 1: the merge polls `done` per group; 0: it waits for the grid
   uint32_t* err;
   uint64_t wait_ns;  // limit of each pipeline wait (waits that drain use kWaitLimitNs)
   int stall;         // test stall: one wait on `never` once the first MMAs are issued
@@ -115,28 +148,50 @@ struct TcParams {
 
 __device__ __forceinline__ int cdiv(int a, int b) { return (a + b - 1) / b; }
 
-// blockIdx.x -> (b, g, query-tile pair tp, split s) by walking the batch
-// rows; slot0 = partial slot of (b, g, 2 tp, s).
-__device__ void resolve_unit(const TcParams& p, Barriers* bars) {
-  int u = blockIdx.x;
-  const int nc = cdiv(p.C, BN);
+// blockIdx.x -> (b, g, query-tile pair tp, split s): a binary search of the
+// plan's unit ranges, or (uniform plan) a walk over the batch rows.
+// slot0 = partial slot of (b, g, 2 tp, s).
+__device__ void resolve_unit(const TcParams& p, const RowPlan& rp, Barriers* bars) {
   const int TP = cdiv(p.T, kQT);
-  int valid = 0, b = 0, g = 0, tp = 0, s = 0, nsplit = 1, slots = 0;
-  for (int bb = 0; bb < p.B; ++bb) {
-    const int L = p.cu_prefix[bb + 1] - p.cu_prefix[bb];
-    const int ns = cdiv(cdiv(L, BN) + nc, p.chunk);
-    const int units = p.Hkv * TP * ns;
-    if (u < units) {
-      s = u % ns;
-      tp = (u / ns) % TP;
-      g = u / (ns * TP);
-      b = bb;
-      nsplit = ns;
+  int u = blockIdx.x;
+  int valid = 0, b = 0, g = 0, tp = 0, s = 0, nsplit = 1, slot0 = 0;
+  if (rp.n > 0) {
+    if (u < rp.ubase[rp.n]) {
+      int lo = 0, hi = rp.n;  // rp.ubase[lo] <= u < rp.ubase[hi]
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (rp.ubase[mid] <= u) lo = mid;
+        else hi = mid;
+      }
+      b = rp.order[lo];
+      nsplit = rp.ns[b];
+      const int lu = u - rp.ubase[lo];
+      s = lu % nsplit;
+      tp = (lu / nsplit) % TP;
+      g = lu / (nsplit * TP);
+      slot0 = rp.sbase[b] + (g * p.T + tp * kQT) * nsplit + s;
       valid = 1;
-      break;
     }
-    u -= units;
-    slots += p.Hkv * p.T * ns;
+  } else {
+    const int nc = cdiv(p.C, BN);
+    int slots = 0;
+    for (int bb = 0; bb < p.B; ++bb) {
+      const int L = p.cu_prefix[bb + 1] - p.cu_prefix[bb];
+      const int ns = cdiv(cdiv(L, BN) + nc, p.chunk);
+      const int units = p.Hkv * TP * ns;
+      if (u < units) {
+        s = u % ns;
+        tp = (u / ns) % TP;
+        g = u / (ns * TP);
+        b = bb;
+        nsplit = ns;
+        slot0 = slots + (g * p.T + tp * kQT) * ns + s;
+        valid = 1;
+        break;
+      }
+      u -= units;
+      slots += p.Hkv * p.T * ns;
+    }
   }
   bars->unit_b = b;
   bars->unit_g = g;
@@ -144,7 +199,7 @@ __device__ void resolve_unit(const TcParams& p, Barriers* bars) {
   bars->unit_s = s;
   bars->unit_valid = valid;
   bars->unit_nsplit = nsplit;
-  bars->unit_slot0 = slots + (g * p.T + tp * kQT) * nsplit + s;
+  bars->unit_slot0 = slot0;
 }
 
 // Shared-memory descriptors are built once per CTA; an operand at byte
@@ -234,7 +289,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                    const __grid_constant__ CUtensorMap tmKp,
                    const __grid_constant__ CUtensorMap tmVp,
                    const __grid_constant__ CUtensorMap tmKc,
-                   const __grid_constant__ CUtensorMap tmVc, const TcParams p) {
+                   const __grid_constant__ CUtensorMap tmVc, const TcParams p,
+                   const __grid_constant__ RowPlan rp) {
   using G = Lay<kF8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -263,7 +319,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars->never, 1);
     bars->abort = 0;
     fence_mbar_init();
-    resolve_unit(p, bars);
+    resolve_unit(p, rp, bars);
   }
   if (warp == kWarpMMA) {
     tmem_alloc(&bars->tmem_base, kTmemCols);
@@ -281,8 +337,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int L = unit_ok ? p.cu_prefix[b + 1] - p0 : 0;
   const int np = cdiv(L, BN), nc = cdiv(p.C, BN);
   const int ntiles = np + nc;
-  const int k_begin = s * p.chunk;
-  const int n = unit_ok ? min(p.chunk, ntiles - k_begin) : 0;
+  // split s of nsplit takes tiles [s T / nsplit, (s + 1) T / nsplit) of T
+  const int k_begin = (int)((int64_t)s * ntiles / nsplit);
+  const int n = unit_ok ? (int)((int64_t)(s + 1) * ntiles / nsplit) - k_begin : 0;
   const int nq = min(kQT, p.T - tp * kQT);  // query tiles in this CTA (1 or 2)
 
   if (warp == kWarpTMA) {
@@ -583,13 +640,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // this split's partials are written (by every warp, ordered before the
+  // barrier): release them to the merge.  An aborted CTA counts too, so the
+  // merge never waits for it (its error is latched already).
+  if (p.poll && threadIdx.x == 0 && bars->unit_valid)
+    red_release_add(&p.done[(bars->unit_b * p.Hkv + bars->unit_g) * cdiv(p.T, kQT) + bars->unit_tp],
+                    1u);
   if (warp == kWarpMMA) tmem_dealloc(tmem, kTmemCols);
 }
 
 // Merge the splits of every (b, g, t) query tile: lse = log2 sum 2^lse_s,
 // O = sum_s 2^(lse_s - lse) O_s.  One warp per query row (8 rows per CTA,
-// 16 CTAs per 128-row tile); lane s holds split s's weight.
-constexpr int kCombineRowsPerCta = 8;
+// 16 CTAs per 128-row tile); lane s holds split s's weight.  kMaxS bounds
+// the splits whose rows are all requested at once (registers: kMaxS float4
+// per lane, so a small bound keeps more CTAs resident); more splits take a
+// looped path.
+constexpr int kCombineWarps = 8;  // warps per CTA of the combine kernel
 
 // Final row of the combine: O = acc / wsum (4 columns per lane) and the
 // natural-log LSE.
@@ -613,107 +679,176 @@ __device__ __forceinline__ void combine_store(const TcParams& p, TOut* __restric
     lse_out[((size_t)b * p.Hq + h) * p.C + i] = (mx + __log2f(wsum)) * 0.6931471805599453f;
 }
 
-template <typename TOut>
-__global__ void __launch_bounds__(256)
-    attn_combine_kernel(const TcParams p, int total_units, TOut* __restrict__ out,
-                        float* __restrict__ lse_out) {
-  pdl_wait();
+template <typename TOut, int kMaxS>
+__global__ void __launch_bounds__(kCombineWarps * 32, 3)
+    attn_combine_kernel(const TcParams p, const __grid_constant__ RowPlan rp, int total_units,
+                        TOut* __restrict__ out, float* __restrict__ lse_out) {
+  // polling: the group's counter orders these reads after its splits'
+  // writes (and every kernel before the attention grid has completed: each
+  // attention CTA waited for it before this grid could start)
+  if (!p.poll) pdl_wait();
   pdl_trigger();
-  const int nc = cdiv(p.C, BN);
-  constexpr int kBlocksPerTile = BM / kCombineRowsPerCta;
+  // kRows rows per warp, all of their split rows requested at once
+  constexpr int kRows = 16 / kMaxS;
+  constexpr int kBlocksPerTile = BM / (kCombineWarps * kRows);
   int q = blockIdx.x / kBlocksPerTile;  // (b, g, t) group
-  const int rbase = (blockIdx.x % kBlocksPerTile) * kCombineRowsPerCta;
+  const int groups = p.Hkv * p.T;
   int b = -1, nsplit = 0, ubase = 0;
-  for (int bb = 0; bb < p.B; ++bb) {
-    const int L = p.cu_prefix[bb + 1] - p.cu_prefix[bb];
-    const int ns = cdiv(cdiv(L, BN) + nc, p.chunk);
-    const int groups = p.Hkv * p.T;
-    if (q < groups) {
-      b = bb;
-      nsplit = ns;
-      break;
+  if (rp.n > 0) {
+    if (q < p.B * groups) {
+      b = q / groups;
+      q -= b * groups;
+      nsplit = rp.ns[b];
+      ubase = rp.sbase[b];
     }
-    q -= groups;
-    ubase += groups * ns;
+  } else {
+    const int nc = cdiv(p.C, BN);
+    for (int bb = 0; bb < p.B; ++bb) {
+      const int L = p.cu_prefix[bb + 1] - p.cu_prefix[bb];
+      const int ns = cdiv(cdiv(L, BN) + nc, p.chunk);
+      if (q < groups) {
+        b = bb;
+        nsplit = ns;
+        break;
+      }
+      q -= groups;
+      ubase += groups * ns;
+    }
   }
   if (b < 0) return;
   const int g = q / p.T, t = q % p.T;
   const int u0 = ubase + q * nsplit;
+  const int grp = (b * p.Hkv + g) * cdiv(p.T, kQT) + t / kQT;
+  // the group's merge CTAs (kBlocksPerTile per query tile of the pair) have
+  // all seen the count once the last of them has added itself to `seen`;
+  // that one clears both counters for the next call (`seen_before` is read
+  // only after this CTA's loads are in flight)
+  uint32_t seen_before = 0;
+  auto clear_if_last = [&]() {
+    const uint32_t readers = (uint32_t)(min(kQT, p.T - (t / kQT) * kQT) * kBlocksPerTile);
+    if (p.poll && threadIdx.x == 0 && seen_before == readers - 1) {
+      p.done[grp] = 0;
+      p.seen[grp] = 0;
+    }
+  };
+  if (p.poll) {
+    __shared__ int all_done;
+    if (threadIdx.x == 0) {
+      const uint64_t t0 = globaltimer_ns();
+      bool ok = true;
+      while (ld_acquire(&p.done[grp]) < (uint32_t)nsplit) {
+        if (globaltimer_ns() - t0 > p.wait_ns) {
+          atomicOr(p.err, kDevErrTimeout);
+          ok = false;
+          break;
+        }
+        __nanosleep(128);
+      }
+      all_done = ok ? 1 : 0;
+      seen_before = atomicAdd(&p.seen[grp], 1u);
+    }
+    __syncthreads();
+    if (!all_done) {
+      clear_if_last();
+      return;
+    }
+  }
   if (u0 + nsplit > total_units) {
     if (threadIdx.x == 0) atomicOr(p.err, kDevErrBounds);
+    clear_if_last();
     return;
   }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int r = rbase + warp;
-  const int pr = t * BM + r;
-  if (pr >= p.C * p.group) return;
-  if (nsplit <= 16) {
-    // common case: every split's row and LSE requested at once (one L2
-    // round trip), then the weights and the sum
-    const float lse_l = lane < nsplit ? p.part_lse[(size_t)(u0 + lane) * BM + r] : -INFINITY;
-    float4 o[16];
+  const int r0 = (blockIdx.x % kBlocksPerTile) * (kCombineWarps * kRows) + warp * kRows;
+  const int rows_valid = p.C * p.group - t * BM;  // rows of this tile that exist
+  if (nsplit <= kMaxS) {
+    // common case: every split row and LSE of the warp's rows requested at
+    // once (one L2 round trip), then the weights and the sums
+    float lse_l[kRows];
+    float4 o[kRows][kMaxS];
 #pragma unroll
-    for (int u = 0; u < 16; ++u)
-      o[u] = u < nsplit ? *reinterpret_cast<const float4*>(
-                              p.part_o + ((size_t)(u0 + u) * BM + r) * HD + lane * 4)
-                        : make_float4(0.f, 0.f, 0.f, 0.f);
-    float mx = lse_l;
+    for (int i = 0; i < kRows; ++i) {
+      const int r = r0 + i;
+      const bool rv = r < rows_valid;
+      lse_l[i] = (rv && lane < nsplit) ? __ldcg(p.part_lse + (size_t)(u0 + lane) * BM + r)
+                                       : -INFINITY;
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-    const float wl = lane < nsplit ? exp2f(lse_l - mx) : 0.f;
-    float wsum = wl;
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, off);
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int u = 0; u < 16; ++u) {
-      const float w = __shfl_sync(0xffffffffu, wl, u);  // 0 past nsplit
-      acc.x = fmaf(w, o[u].x, acc.x);
-      acc.y = fmaf(w, o[u].y, acc.y);
-      acc.z = fmaf(w, o[u].z, acc.z);
-      acc.w = fmaf(w, o[u].w, acc.w);
+      for (int u = 0; u < kMaxS; ++u)
+        o[i][u] = (rv && u < nsplit)
+                      ? __ldcg(reinterpret_cast<const float4*>(p.part_o +
+                                                               ((size_t)(u0 + u) * BM + r) * HD) +
+                               lane)
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    combine_store<TOut>(p, out, lse_out, b, g, pr, lane, acc, mx, wsum);
+    clear_if_last();
+#pragma unroll
+    for (int i = 0; i < kRows; ++i) {
+      const int r = r0 + i;
+      if (r >= rows_valid) break;
+      float mx = lse_l[i];
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1)
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+      const float wl = lane < nsplit ? exp2f(lse_l[i] - mx) : 0.f;
+      float wsum = wl;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, off);
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int u = 0; u < kMaxS; ++u) {
+        const float w = __shfl_sync(0xffffffffu, wl, u);  // 0 past nsplit
+        acc.x = fmaf(w, o[i][u].x, acc.x);
+        acc.y = fmaf(w, o[i][u].y, acc.y);
+        acc.z = fmaf(w, o[i][u].z, acc.z);
+        acc.w = fmaf(w, o[i][u].w, acc.w);
+      }
+      combine_store<TOut>(p, out, lse_out, b, g, t * BM + r, lane, acc, mx, wsum);
+    }
     return;
   }
-  // split weights, 32 splits per pass
-  float mx = -INFINITY;
-  for (int s0 = 0; s0 < nsplit; s0 += 32) {
-    const int s = s0 + lane;
-    if (s < nsplit) mx = fmaxf(mx, p.part_lse[(size_t)(u0 + s) * BM + r]);
-  }
+  clear_if_last();
+  for (int i = 0; i < kRows; ++i) {
+    const int r = r0 + i;
+    if (r >= rows_valid) break;
+    // split weights, 32 splits per pass
+    float mx = -INFINITY;
+    for (int s0 = 0; s0 < nsplit; s0 += 32) {
+      const int s = s0 + lane;
+      if (s < nsplit) mx = fmaxf(mx, __ldcg(p.part_lse + (size_t)(u0 + s) * BM + r));
+    }
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-  float wsum = 0.f;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int s0 = 0; s0 < nsplit; s0 += 32) {
-    const int s = s0 + lane;
-    const float wl = s < nsplit ? exp2f(p.part_lse[(size_t)(u0 + s) * BM + r] - mx) : 0.f;
-    float ws = wl;
+    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    float wsum = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s0 = 0; s0 < nsplit; s0 += 32) {
+      const int s = s0 + lane;
+      const float wl = s < nsplit ? exp2f(__ldcg(p.part_lse + (size_t)(u0 + s) * BM + r) - mx) : 0.f;
+      float ws = wl;
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) ws += __shfl_xor_sync(0xffffffffu, ws, off);
-    wsum += ws;
-    const int n = min(32, nsplit - s0);
-    // eight splits' rows in flight at a time (L2 latency, not bandwidth, is
-    // what a one-row-at-a-time loop waits on)
-    for (int j0 = 0; j0 < n; j0 += 8) {
-      float4 o[8];
+      for (int off = 16; off > 0; off >>= 1) ws += __shfl_xor_sync(0xffffffffu, ws, off);
+      wsum += ws;
+      const int n = min(32, nsplit - s0);
+      // eight splits' rows in flight at a time (L2 latency, not bandwidth,
+      // is what a one-row-at-a-time loop waits on)
+      for (int j0 = 0; j0 < n; j0 += 8) {
+        float4 ov[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u)
-        o[u] = j0 + u < n ? *reinterpret_cast<const float4*>(
-                                p.part_o + ((size_t)(u0 + s0 + j0 + u) * BM + r) * HD + lane * 4)
-                          : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int u = 0; u < 8; ++u)
+          ov[u] = j0 + u < n ? __ldcg(reinterpret_cast<const float4*>(
+                                   p.part_o + ((size_t)(u0 + s0 + j0 + u) * BM + r) * HD) + lane)
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const float w = __shfl_sync(0xffffffffu, wl, j0 + u);  // 0 past nsplit
-        acc.x = fmaf(w, o[u].x, acc.x);
-        acc.y = fmaf(w, o[u].y, acc.y);
-        acc.z = fmaf(w, o[u].z, acc.z);
-        acc.w = fmaf(w, o[u].w, acc.w);
+        for (int u = 0; u < 8; ++u) {
+          const float w = __shfl_sync(0xffffffffu, wl, j0 + u);  // 0 past nsplit
+          acc.x = fmaf(w, ov[u].x, acc.x);
+          acc.y = fmaf(w, ov[u].y, acc.y);
+          acc.z = fmaf(w, ov[u].z, acc.z);
+          acc.w = fmaf(w, ov[u].w, acc.w);
+        }
       }
     }
+    combine_store<TOut>(p, out, lse_out, b, g, t * BM + r, lane, acc, mx, wsum);
   }
-  combine_store<TOut>(p, out, lse_out, b, g, pr, lane, acc, mx, wsum);
 }
 
 // ----------------------------------------------------------------- host
@@ -766,44 +901,175 @@ int num_sms() {
 }
 
 struct Plan {
-  int T, chunk, units, slots, groups;
+  int T, chunk, units, slots, groups, max_ns;
+  RowPlan rp;
 };
 
-// Choose the split size (key tiles per CTA) that minimises the makespan
-// waves(units) * chunk over the SMs, plus a small charge per split for the
-// merge pass.
-Plan make_plan(const AttnArgs& a) {
+// Cost model of one CTA (measured on B200 with per-CTA %globaltimer traces):
+// about 8.5 us of fixed work -- set-up, the first S tile, the wait for the
+// last P.V and the write of 128 KB of partials -- and 1.84 us per 128-key
+// tile, so the fixed part weighs as much as kUnitFixed tiles.  The merge
+// pass reads each 64 KB partial slot once (about 13 ns per slot for the GPU
+// at ~5 TB/s, kSlotMerge tiles).
+constexpr double kUnitFixed = 4.6;
+constexpr double kSlotMerge = 0.0071;
+
+// Makespan (in key tiles) of the units of `ns` launched row by row in
+// `order`, each unit going to the SM that frees first: the hardware hands
+// out CTAs in launch order as SMs free up, one attention CTA per SM.
+double simulate(const std::vector<int>& tiles, const std::vector<int>& ns,
+                const std::vector<int>& order, int per_split, int sms) {
+  std::priority_queue<double, std::vector<double>, std::greater<double>> free_at;
+  for (int i = 0; i < sms; ++i) free_at.push(0.0);
+  double end = 0.0;
+  for (int b : order) {
+    const int t = tiles[b], n = ns[b];
+    for (int lu = 0; lu < per_split * n; ++lu) {
+      const int sp = lu % n;
+      const int len = (int)((int64_t)(sp + 1) * t / n - (int64_t)sp * t / n);
+      const double start = free_at.top();
+      free_at.pop();
+      const double fin = start + kUnitFixed + len;
+      free_at.push(fin);
+      end = std::max(end, fin);
+    }
+  }
+  return end;
+}
+
+// Rows launched longest unit first (ties: lower batch row first).
+std::vector<int> lpt_order(const std::vector<int>& tiles, const std::vector<int>& ns) {
+  std::vector<int> order(tiles.size());
+  for (size_t b = 0; b < order.size(); ++b) order[b] = (int)b;
+  auto longest = [&](int b) { return (tiles[b] + ns[b] - 1) / ns[b]; };
+  std::stable_sort(order.begin(), order.end(),
+                   [&](int x, int y) { return longest(x) > longest(y); });
+  return order;
+}
+
+// The split plan.  Every batch row b of tiles_b key tiles gets
+// ns_b = ceil(tiles_b / target) splits, for the target length (in tiles)
+// that minimises the simulated makespan plus the merge pass; rows go out
+// longest unit first.  Batches wider than kMaxPlanRows use one split length
+// for all rows (the kernels derive that plan themselves).
+Plan plan_uncached(const AttnArgs& a) {
   Plan pl{};
   const int group = a.Hq / a.Hkv;
   pl.T = (a.C * group + BM - 1) / BM;
   const int TP = (pl.T + kQT - 1) / kQT;
   const int nc = (a.C + BN - 1) / BN;
+  const int sms = num_sms();
+  pl.groups = a.B * a.Hkv * pl.T;
+  std::vector<int> tiles(a.B);
   int max_tiles = 1;
+  int64_t total = 0;
   for (int b = 0; b < a.B; ++b) {
     const int L = a.cu_prefix_host[b + 1] - a.cu_prefix_host[b];
-    max_tiles = std::max(max_tiles, (L + BN - 1) / BN + nc);
+    tiles[b] = (L + BN - 1) / BN + nc;
+    max_tiles = std::max(max_tiles, tiles[b]);
+    total += (int64_t)tiles[b] * a.Hkv * TP;
   }
-  const int sms = num_sms();
-  double best_cost = 1e300;
-  for (int chunk = 1; chunk <= max_tiles; ++chunk) {
-    int64_t units = 0, slots = 0;
-    for (int b = 0; b < a.B; ++b) {
-      const int L = a.cu_prefix_host[b + 1] - a.cu_prefix_host[b];
-      const int ns = ((L + BN - 1) / BN + nc + chunk - 1) / chunk;
-      units += (int64_t)a.Hkv * TP * ns;
-      slots += (int64_t)a.Hkv * pl.T * ns;
+  if (a.B > kMaxPlanRows) {
+    // uniform split length: waves(units) * (chunk + 2), plus a charge per
+    // split for the merge
+    double best_cost = 1e300;
+    for (int chunk = 1; chunk <= max_tiles; ++chunk) {
+      int64_t units = 0, slots = 0;
+      int max_ns = 1;
+      for (int b = 0; b < a.B; ++b) {
+        const int ns = (tiles[b] + chunk - 1) / chunk;
+        units += (int64_t)a.Hkv * TP * ns;
+        slots += (int64_t)a.Hkv * pl.T * ns;
+        max_ns = std::max(max_ns, ns);
+      }
+      const int64_t waves = (units + sms - 1) / sms;
+      const double cost = (double)waves * (chunk + 2) + 0.25 * (double)units / sms;
+      if (cost < best_cost - 1e-9) {
+        best_cost = cost;
+        pl.chunk = chunk;
+        pl.units = (int)units;
+        pl.slots = (int)slots;
+        pl.max_ns = max_ns;
+      }
     }
-    const int64_t waves = (units + sms - 1) / sms;
-    const double cost = (double)waves * (chunk + 2) + 0.25 * (double)units / sms;
+    pl.rp.n = 0;
+    return pl;
+  }
+  // candidate target lengths: each share of the longest row, and the even
+  // share of all the work over 1-4 rounds of the SMs
+  std::vector<int> cand;
+  for (int k = 1; k <= 32; ++k) cand.push_back((max_tiles + k - 1) / k);
+  for (int w = 1; w <= 4; ++w)
+    cand.push_back((int)std::max<int64_t>(1, (total + (int64_t)w * sms - 1) / ((int64_t)w * sms)));
+  std::sort(cand.begin(), cand.end());
+  cand.erase(std::unique(cand.begin(), cand.end()), cand.end());
+  double best_cost = 1e300;
+  std::vector<int> best_ns;
+  for (int target : cand) {
+    std::vector<int> ns(a.B);
+    int64_t units = 0;
+    for (int b = 0; b < a.B; ++b) {
+      ns[b] = std::min(tiles[b], std::max(1, (tiles[b] + target - 1) / target));
+      units += (int64_t)a.Hkv * TP * ns[b];
+    }
+    // more than 16 rounds of the SMs never pays; the one-split plan is
+    // always a candidate
+    if (units > 16 * (int64_t)sms && target != max_tiles) continue;
+    int64_t slots = 0;
+    for (int b = 0; b < a.B; ++b) slots += (int64_t)a.Hkv * pl.T * ns[b];
+    const double cost =
+        simulate(tiles, ns, lpt_order(tiles, ns), a.Hkv * TP, sms) + kSlotMerge * (double)slots;
     if (cost < best_cost - 1e-9) {
       best_cost = cost;
-      pl.chunk = chunk;
-      pl.units = (int)units;
-      pl.slots = (int)slots;
+      best_ns = ns;
     }
   }
-  pl.groups = a.B * a.Hkv * pl.T;
+  const std::vector<int> order = lpt_order(tiles, best_ns);
+  RowPlan& rp = pl.rp;
+  rp.n = a.B;
+  int slots = 0;
+  pl.max_ns = 1;
+  for (int b = 0; b < a.B; ++b) {
+    rp.ns[b] = best_ns[b];
+    rp.sbase[b] = slots;
+    slots += a.Hkv * pl.T * best_ns[b];
+    pl.max_ns = std::max(pl.max_ns, best_ns[b]);
+  }
+  rp.ubase[0] = 0;
+  for (int i = 0; i < a.B; ++i) {
+    rp.order[i] = order[i];
+    rp.ubase[i + 1] = rp.ubase[i] + a.Hkv * TP * best_ns[order[i]];
+  }
+  pl.units = rp.ubase[a.B];
+  pl.slots = slots;
+  pl.chunk = max_tiles;  // unused with a row plan
   return pl;
+}
+
+// The plan depends on the shape and the prefix lengths only; the last one
+// is kept per host thread (a decode loop asks for the same plan every step).
+Plan make_plan(const AttnArgs& a) {
+  struct Cache {
+    bool valid = false;
+    int B = 0, C = 0, Hq = 0, Hkv = 0, sms = 0;
+    std::vector<int32_t> cu;
+    Plan plan;
+  };
+  thread_local Cache cache;
+  const int sms = num_sms();
+  if (cache.valid && cache.B == a.B && cache.C == a.C && cache.Hq == a.Hq &&
+      cache.Hkv == a.Hkv && cache.sms == sms &&
+      std::equal(cache.cu.begin(), cache.cu.end(), a.cu_prefix_host))
+    return cache.plan;
+  cache.plan = plan_uncached(a);
+  cache.B = a.B;
+  cache.C = a.C;
+  cache.Hq = a.Hq;
+  cache.Hkv = a.Hkv;
+  cache.sms = sms;
+  cache.cu.assign(a.cu_prefix_host, a.cu_prefix_host + a.B + 1);
+  cache.valid = true;
+  return cache.plan;
 }
 
 }  // namespace
@@ -821,9 +1087,16 @@ bool attn_tc_supported(const AttnArgs& a) {
   return true;
 }
 
+// Scratch: the done/seen counters (two per (b, g, tile pair)), then the
+// partial O and LSE of every slot.
+size_t counter_bytes(const AttnArgs& a, const Plan& pl) {
+  const size_t n = (size_t)a.B * a.Hkv * ((pl.T + kQT - 1) / kQT);
+  return (2 * n * sizeof(uint32_t) + 255) & ~(size_t)255;
+}
+
 size_t attn_tc_scratch_bytes(const AttnArgs& a) {
   const Plan pl = make_plan(a);
-  return (size_t)pl.slots * BM * (HD + 1) * sizeof(float) + 256;
+  return counter_bytes(a, pl) + (size_t)pl.slots * BM * (HD + 1) * sizeof(float) + 256;
 }
 
 template <bool kF8>
@@ -871,22 +1144,39 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t stream) {
   tp.out_scale = f8 ? a.v_scale : 1.0f;
   tp.cu_prefix = a.cu_prefix;
   uint8_t* scratch = static_cast<uint8_t*>(a.scratch);
+  const size_t ncnt = (size_t)a.B * a.Hkv * ((pl.T + kQT - 1) / kQT);
+  tp.done = reinterpret_cast<uint32_t*>(scratch);
+  tp.seen = tp.done + ncnt;
+  scratch += counter_bytes(a, pl);
   tp.part_o = reinterpret_cast<float*>(scratch);
   tp.part_lse = reinterpret_cast<float*>(scratch + (size_t)pl.slots * BM * HD * sizeof(float));
   tp.err = a.err;
   tp.wait_ns = pipeline_wait_ns();
   tp.stall = pipeline_test_stall() ? 1 : 0;
+  tp.poll = pl.units > num_sms() ? 1 : 0;
 
   cudaError_t e =
       f8 ? launch_pdl(attn_tc_kernel<true>, dim3(pl.units), dim3(kThreads), Lay<true>::kSmemBytes,
-                      stream, mQ, mKp, mVp, mKc, mVc, tp)
+                      stream, mQ, mKp, mVp, mKc, mVc, tp, pl.rp)
          : launch_pdl(attn_tc_kernel<false>, dim3(pl.units), dim3(kThreads),
-                      Lay<false>::kSmemBytes, stream, mQ, mKp, mVp, mKc, mVc, tp);
+                      Lay<false>::kSmemBytes, stream, mQ, mKp, mVp, mKc, mVc, tp, pl.rp);
   note_launch();
   if (e != cudaSuccess) return e;
-  e = launch_pdl(attn_combine_kernel<__nv_bfloat16>,
-                 dim3(pl.groups * (BM / kCombineRowsPerCta)), dim3(256), 0, stream, tp,
-                 (int)pl.slots, static_cast<__nv_bfloat16*>(a.out), a.lse);
+  // kMaxS splits per row in flight, 16 / kMaxS rows per warp
+  __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out);
+  const dim3 cblock(kCombineWarps * 32);
+  auto cgrid = [&](int max_s) {
+    return dim3(pl.groups * (BM / (kCombineWarps * (16 / max_s))));
+  };
+  if (pl.max_ns <= 4)
+    e = launch_pdl(attn_combine_kernel<__nv_bfloat16, 4>, cgrid(4), cblock, 0, stream, tp, pl.rp,
+                   (int)pl.slots, out, a.lse);
+  else if (pl.max_ns <= 8)
+    e = launch_pdl(attn_combine_kernel<__nv_bfloat16, 8>, cgrid(8), cblock, 0, stream, tp, pl.rp,
+                   (int)pl.slots, out, a.lse);
+  else
+    e = launch_pdl(attn_combine_kernel<__nv_bfloat16, 16>, cgrid(16), cblock, 0, stream, tp,
+                   pl.rp, (int)pl.slots, out, a.lse);
   note_launch();
   return e;
 }

@@ -189,6 +189,19 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+// Device-scope release add and acquire load of a 32-bit counter in global
+// memory: writes ordered before the add (by this thread, or by the CTA
+// before a barrier this thread passed) are visible to a thread whose
+// acquire load reads the added value.
+__device__ __forceinline__ void red_release_add(uint32_t* p, uint32_t v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
 // Bounded wait: spins on try_wait until the phase with `parity` completes,
 // the CTA-wide abort flag is raised, or `limit_ns` elapses.  Returns false
 // (and raises the abort flag) on timeout or abort; never spins forever.

@@ -67,6 +67,29 @@ def test_tensor_core_ragged(lens, q_gain):
     print(lens, q_gain, st)
 
 
+@pytest.mark.parametrize("C,Hq,Hkv,lens", [
+    (256, 16, 8, (1536,)),     # 7 splits: merge with 8 split rows in flight per row
+    (128, 2, 1, (16384,)),     # one unit per split, about 129 splits: the looped merge
+])
+def test_tensor_core_split_counts(C, Hq, Hkv, lens):
+    q, kc, vc, kp, vp, cu = _problem(len(lens), C, Hq, Hkv, 128, lens, seed=C + Hq)
+    out, lse = _run(q, kc, vc, kp, vp, cu)
+    ref, ref_lse = oracle.canvas_attn(q, kc, vc, kp, vp, cu.numpy(), 128 ** -0.5)
+    check_attn(out, ref, torch.bfloat16)
+    np.testing.assert_allclose(lse.cpu().numpy(), ref_lse, atol=2e-2)
+
+
+def test_tensor_core_wide_batch():
+    # more batch rows than the host's per-row plan holds: the kernels then
+    # derive one split length for every row themselves
+    lens = tuple(int(x) for x in np.random.default_rng(7).integers(0, 400, 130))
+    q, kc, vc, kp, vp, cu = _problem(130, 16, 2, 1, 128, lens, seed=130)
+    out, lse = _run(q, kc, vc, kp, vp, cu)
+    ref, ref_lse = oracle.canvas_attn(q, kc, vc, kp, vp, cu.numpy(), 128 ** -0.5)
+    check_attn(out, ref, torch.bfloat16)
+    np.testing.assert_allclose(lse.cpu().numpy(), ref_lse, atol=2e-2)
+
+
 @pytest.mark.parametrize("Hq,Hkv", [(8, 8), (16, 4), (16, 2), (32, 4)])
 def test_tensor_core_head_groupings(Hq, Hkv):
     q, kc, vc, kp, vp, cu = _problem(2, 256, Hq, Hkv, 128, (200, 77), seed=Hq + Hkv)
