@@ -47,6 +47,10 @@ import workloads  # noqa: E402
 
 METRIC = "denoise steps/s per 256-token canvas"
 UNIT = "canvas-steps/s"
+# Nominal denominators, reported beside the measured ones: the benchmark spec's
+# ~8 TB/s of HBM3e and the 2.25 PFLOP/s dense bf16 datasheet figure.
+NOMINAL_HBM_GBS = 8000.0
+NOMINAL_BF16_TFLOPS = 2250.0
 N_SETS = 3
 
 
@@ -242,6 +246,17 @@ def run_ours(args, w, dist, rank, world, local_rank):
         ts.append(ev[1].elapsed_time(ev[2]))
     per = {"attn": _max_over_ranks(dist, statistics.mean(ta) / 1e3),
            "samp": _max_over_ranks(dist, statistics.mean(ts) / 1e3)}
+    # warm: the same input set replayed back to back (what stays in L2 from
+    # one call to the next is reused)
+    wa, wsm = [], []
+    for i in range(min(n2, 100)):
+        g2, ev = timed[0]
+        g2.replay()
+        torch.cuda.synchronize()
+        wa.append(ev[0].elapsed_time(ev[1]))
+        wsm.append(ev[1].elapsed_time(ev[2]))
+    warm = {"attn": _max_over_ranks(dist, statistics.mean(wa) / 1e3),
+            "samp": _max_over_ranks(dist, statistics.mean(wsm) / 1e3)}
     time.sleep(0.2)
     clocks.stop()
     dd.query_device_error(ws_attn)
@@ -277,11 +292,16 @@ def run_ours(args, w, dist, rank, world, local_rank):
                      "achieved": samp_gbs, "peak": hbm, "unit": "GB/s", "frac": samp_gbs / hbm,
                      "traffic": traffic.get(f"sampler@{w.name}"), "peak_source": src,
                      "algorithmic_bytes": samp_bytes, "ms": t_samp * 1e3,
+                     "ms_warm": warm["samp"] * 1e3,
+                     "nominal_peak": NOMINAL_HBM_GBS, "frac_of_nominal": samp_gbs / NOMINAL_HBM_GBS,
                      "alu_ceiling": _sampler_alu_ceiling(samp_gbs, clk.get("sm_mhz"))},
         "roofline_attn": {"bound": "tensor", "kernel": "canvas attention (tcgen05 + merge)",
                           "achieved": attn_tf, "peak": tf_burst, "unit": "TFLOP/s",
                           "frac": attn_tf / tf_burst, "frac_of_sustained": attn_tf / tf_sus,
+                          "nominal_peak": NOMINAL_BF16_TFLOPS,
+                          "frac_of_nominal": attn_tf / NOMINAL_BF16_TFLOPS,
                           "flops": w.attn_flops(), "ms": t_attn * 1e3,
+                          "ms_warm": warm["attn"] * 1e3,
                           "traffic": traffic.get(f"attention@{w.name}"), "peak_source": src},
         "e2e": e2e,
         "gpu_launches": int(launches),
@@ -427,9 +447,12 @@ def run_attn_e4m3(w, reps: int = 50):
         "ms": ms["e4m3"],
         "roofline": {"bound": "tensor", "achieved": tf8, "peak": 2 * tf_burst, "unit": "TFLOP/s",
                      "frac": tf8 / (2 * tf_burst), "flops": flops,
+                     "nominal_peak": 2 * NOMINAL_BF16_TFLOPS,
+                     "frac_of_nominal": tf8 / (2 * NOMINAL_BF16_TFLOPS),
                      "traffic": _profile_traffic().get(f"attention_e4m3@{w.name}"),
                      "peak_source": f"{src} bf16 burst x 2 (nominal E4M3 / bf16 ratio)"},
-        "bf16_same_workload": {"ms": ms["bf16"], "TFLOP/s": tf16, "frac": tf16 / tf_burst},
+        "bf16_same_workload": {"ms": ms["bf16"], "TFLOP/s": tf16, "frac": tf16 / tf_burst,
+                               "frac_of_nominal": tf16 / NOMINAL_BF16_TFLOPS},
         "timing": f"median of {reps} calls, CUDA events around each call",
         "clocks": clocks.summary(t_wall0, t_wall1),
     }

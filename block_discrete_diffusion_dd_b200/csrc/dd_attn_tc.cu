@@ -73,7 +73,7 @@ constexpr int kThreads = (kSoftmaxWarps + 2) * 32;
 constexpr uint32_t kHalf = 128 * 64 * 2;  // bf16: 128 rows x 64 elements (128 bytes)
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemO = kQT * BN;     // O columns start after the S/P regions
-constexpr int kStageStride = HD + 4;       // padded fp32 row of the O staging area
+constexpr int kStageWords = HD / 2 + 4;    // padded row (fp16 pairs) of the O staging area
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per wait
 
 struct Barriers {
@@ -111,15 +111,18 @@ struct Lay {
   static constexpr float kBias = kF8 ? 6.0f : 0.0f;  // log2 units
   static constexpr float kLazy = kF8 ? 2.0f : 8.0f;  // log2 units
   static_assert(kStages <= kMaxStages, "barrier arrays");
-  static_assert(kQT * BM * kStageStride * 4 <= kOffBar, "O staging fits the operand buffers");
+  static_assert(kQT * BM * kStageWords * 4 <= kOffBar, "O staging fits the operand buffers");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
 // The host's split plan, passed by value (kernel parameter space).  Batch
 // rows are launched in `order`: the i-th row in that order owns the units
-// [ubase[i], ubase[i + 1]).  Row b has ns[b] key splits and its partials
-// start at slot sbase[b].  With more than kMaxPlanRows batch rows, n = 0 and
-// the kernels derive a uniform plan from TcParams::chunk instead.
+// [ubase[i], ubase[i + 1]).  Row b has ns[b] key splits, its partials start
+// at slot sbase[b], and its prefix rows are [p0[b], p0[b] + len[b]) of the
+// packed prefix (the host's copy of cu_prefix, which also sized the prefix
+// tensor maps), so no CTA reads cu_prefix before its first copies.  With
+// more than kMaxPlanRows batch rows, n = 0 and the kernels derive a uniform
+// plan from TcParams::chunk and the device cu_prefix instead.
 constexpr int kMaxPlanRows = 128;
 struct RowPlan {
   int n;
@@ -127,6 +130,8 @@ struct RowPlan {
   int order[kMaxPlanRows];
   int sbase[kMaxPlanRows];
   int ns[kMaxPlanRows];
+  int p0[kMaxPlanRows];
+  int len[kMaxPlanRows];
 };
 
 struct TcParams {
@@ -134,8 +139,10 @@ struct TcParams {
   float scale_log2;  // softmax scale * log2(e), times the Q and K factors
   float out_scale;   // the V factor (1 for bf16)
   const int32_t* cu_prefix;
-  float* part_o;    // [slots][BM][HD], slot = (b, g, t, split)
-  float* part_lse;  // [slots][BM]   log2 units
+  // split partials, slot = (b, g, t, split): O / l of each row as fp16
+  // pairs scaled by 2^-e_row, and (log2-domain LSE, 2^e_row) per row
+  uint32_t* part_o;   // [slots][BM][HD / 2]
+  float2* part_lse;   // [slots][BM]
   // per (b, g, tile pair): splits done, and merge CTAs that have seen them
   // all (the last one clears both for the next call); zero between calls
   uint32_t* done;
@@ -147,6 +154,27 @@ struct TcParams {
 };
 
 __device__ __forceinline__ int cdiv(int a, int b) { return (a + b - 1) / b; }
+
+// 2^e as a float for e in [-126, 127] (built from the exponent field).
+__device__ __forceinline__ float pow2(int e) { return __int_as_float((127 + e) << 23); }
+
+// The scale exponent of a partial row whose largest magnitude is m: e with
+// m 2^-e in [2^14, 2^15) (below fp16's largest finite value, 65504), kept
+// within [-126, 113] so that 2^e and 2^-e are normal floats; 0 for a row of
+// zeros or a non-finite maximum.
+__device__ __forceinline__ int row_exponent(float m) {
+  if (!(m > 0.f) || !(m <= 3.4e38f)) return 0;
+  return min(113, max(-126, ilogbf(m) - 14));
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+__device__ __forceinline__ float2 unpack_f16x2(uint32_t w) {
+  return __half22float2(*reinterpret_cast<const __half2*>(&w));
+}
 
 // blockIdx.x -> (b, g, query-tile pair tp, split s): a binary search of the
 // plan's unit ranges, or (uniform plan) a walk over the batch rows.
@@ -333,8 +361,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int b = bars->unit_b, g = bars->unit_g, tp = bars->unit_tp, s = bars->unit_s;
   const bool unit_ok = bars->unit_valid != 0;
   const int nsplit = bars->unit_nsplit, slot0 = bars->unit_slot0;
-  const int p0 = unit_ok ? p.cu_prefix[b] : 0;
-  const int L = unit_ok ? p.cu_prefix[b + 1] - p0 : 0;
+  const int p0 = !unit_ok ? 0 : rp.n > 0 ? rp.p0[b] : p.cu_prefix[b];
+  const int L = !unit_ok ? 0 : rp.n > 0 ? rp.len[b] : p.cu_prefix[b + 1] - p0;
   const int np = cdiv(L, BN), nc = cdiv(p.C, BN);
   const int ntiles = np + nc;
   // split s of nsplit takes tiles [s T / nsplit, (s + 1) T / nsplit) of T
@@ -600,38 +628,53 @@ __global__ void __launch_bounds__(kThreads, 1)
                       mbar_wait_bounded(&bars->o_done[q], 0, abort_flag, p.wait_ns));
     const float lrowA = quad_sum(lA), lrowB = quad_sum(lB);
     if (ok) {
-      // O / l staged row-wise in shared memory (free now: every MMA has
-      // completed), then copied out in whole 512-byte rows
+      // O / l in fp16 pairs, each row scaled by a power of two 2^-e that
+      // puts its largest magnitude in [2^14, 2^15): 11 significant bits
+      // against the row maximum, whatever V's range, in half the bytes of
+      // fp32.  Staged row-wise in shared memory (free now: every MMA has
+      // completed; rows 68 words apart, so a warp's 32-bit stores hit 32
+      // different banks), then copied out in whole 256-byte rows.
       tc_fence_after();
       const float invA = p.out_scale / lrowA, invB = p.out_scale / lrowB;
-      float* stage = reinterpret_cast<float*>(smem) + q * (BM * kStageStride);
+      uint32_t* stage = reinterpret_cast<uint32_t*>(smem) + q * (BM * kStageWords);
+      const size_t slot = (size_t)slot0 + (size_t)q * nsplit;
       {
         uint32_t o[64];
         tmem_ld16x256b_x16(tO, o);
+        float mA = 0.f, mB = 0.f;
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const int c = 8 * i + 2 * t4;
-          *reinterpret_cast<float2*>(stage + rA * kStageStride + c) =
-              make_float2(__uint_as_float(o[4 * i]) * invA, __uint_as_float(o[4 * i + 1]) * invA);
-          *reinterpret_cast<float2*>(stage + rB * kStageStride + c) =
-              make_float2(__uint_as_float(o[4 * i + 2]) * invB,
-                          __uint_as_float(o[4 * i + 3]) * invB);
+          mA = fmaxf(mA, fmaxf(fabsf(__uint_as_float(o[4 * i])), fabsf(__uint_as_float(o[4 * i + 1]))));
+          mB = fmaxf(mB, fmaxf(fabsf(__uint_as_float(o[4 * i + 2])),
+                               fabsf(__uint_as_float(o[4 * i + 3]))));
         }
-      }
-      const size_t slot = (size_t)slot0 + (size_t)q * nsplit;
-      if (t4 == 0) {
-        p.part_lse[slot * BM + rA] = mrefA + __log2f(lrowA);
-        p.part_lse[slot * BM + rB] = mrefB + __log2f(lrowB);
+        mA = quad_max(mA) * invA;
+        mB = quad_max(mB) * invB;
+        const int eA = row_exponent(mA), eB = row_exponent(mB);
+        const float sA = invA * pow2(-eA), sB = invB * pow2(-eB);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int w = 4 * i + t4;  // columns 8 i + 2 t4, + 1
+          stage[rA * kStageWords + w] =
+              pack_f16x2(__uint_as_float(o[4 * i]) * sA, __uint_as_float(o[4 * i + 1]) * sA);
+          stage[rB * kStageWords + w] =
+              pack_f16x2(__uint_as_float(o[4 * i + 2]) * sB, __uint_as_float(o[4 * i + 3]) * sB);
+        }
+        if (t4 == 0) {
+          p.part_lse[slot * BM + rA] = make_float2(mrefA + __log2f(lrowA), pow2(eA));
+          p.part_lse[slot * BM + rB] = make_float2(mrefB + __log2f(lrowB), pow2(eB));
+        }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->staged[q]);
       if (__all_sync(0xffffffffu,
                      mbar_wait_bounded(&bars->staged[q], 0, abort_flag, p.wait_ns))) {
-        float* dst = p.part_o + slot * BM * HD;
+        uint32_t* dst = p.part_o + slot * BM * (HD / 2);
         const int wq = warp & 7;  // warp index within this query tile's 8
-        for (int row = wq; row < BM; row += 8)
-          *reinterpret_cast<float4*>(dst + row * HD + lane * 4) =
-              *reinterpret_cast<const float4*>(stage + row * kStageStride + lane * 4);
+        // two rows per warp instruction, 16 bytes per lane
+        for (int row = 2 * wq + (lane >> 4); row < BM; row += 16)
+          *reinterpret_cast<uint4*>(dst + row * (HD / 2) + (lane & 15) * 4) =
+              *reinterpret_cast<const uint4*>(stage + row * kStageWords + (lane & 15) * 4);
       }
     }
   }
@@ -764,43 +807,45 @@ __global__ void __launch_bounds__(kCombineWarps * 32, 3)
   if (nsplit <= kMaxS) {
     // common case: every split row and LSE of the warp's rows requested at
     // once (one L2 round trip), then the weights and the sums
-    float lse_l[kRows];
-    float4 o[kRows][kMaxS];
+    float2 lse_l[kRows];    // lane s: split s's (LSE, row scale)
+    uint2 o[kRows][kMaxS];  // 4 fp16 columns per lane
 #pragma unroll
     for (int i = 0; i < kRows; ++i) {
       const int r = r0 + i;
       const bool rv = r < rows_valid;
       lse_l[i] = (rv && lane < nsplit) ? __ldcg(p.part_lse + (size_t)(u0 + lane) * BM + r)
-                                       : -INFINITY;
+                                       : make_float2(-INFINITY, 0.f);
 #pragma unroll
       for (int u = 0; u < kMaxS; ++u)
         o[i][u] = (rv && u < nsplit)
-                      ? __ldcg(reinterpret_cast<const float4*>(p.part_o +
-                                                               ((size_t)(u0 + u) * BM + r) * HD) +
+                      ? __ldcg(reinterpret_cast<const uint2*>(
+                                   p.part_o + ((size_t)(u0 + u) * BM + r) * (HD / 2)) +
                                lane)
-                      : make_float4(0.f, 0.f, 0.f, 0.f);
+                      : make_uint2(0u, 0u);
     }
     clear_if_last();
 #pragma unroll
     for (int i = 0; i < kRows; ++i) {
       const int r = r0 + i;
       if (r >= rows_valid) break;
-      float mx = lse_l[i];
+      float mx = lse_l[i].x;
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1)
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-      const float wl = lane < nsplit ? exp2f(lse_l[i] - mx) : 0.f;
+      const float wl = lane < nsplit ? exp2f(lse_l[i].x - mx) : 0.f;
+      const float wo = wl * lse_l[i].y;  // the weight of the scaled fp16 row
       float wsum = wl;
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, off);
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
       for (int u = 0; u < kMaxS; ++u) {
-        const float w = __shfl_sync(0xffffffffu, wl, u);  // 0 past nsplit
-        acc.x = fmaf(w, o[i][u].x, acc.x);
-        acc.y = fmaf(w, o[i][u].y, acc.y);
-        acc.z = fmaf(w, o[i][u].z, acc.z);
-        acc.w = fmaf(w, o[i][u].w, acc.w);
+        const float w = __shfl_sync(0xffffffffu, wo, u);  // 0 past nsplit
+        const float2 a = unpack_f16x2(o[i][u].x), c = unpack_f16x2(o[i][u].y);
+        acc.x = fmaf(w, a.x, acc.x);
+        acc.y = fmaf(w, a.y, acc.y);
+        acc.z = fmaf(w, c.x, acc.z);
+        acc.w = fmaf(w, c.y, acc.w);
       }
       combine_store<TOut>(p, out, lse_out, b, g, t * BM + r, lane, acc, mx, wsum);
     }
@@ -814,7 +859,7 @@ __global__ void __launch_bounds__(kCombineWarps * 32, 3)
     float mx = -INFINITY;
     for (int s0 = 0; s0 < nsplit; s0 += 32) {
       const int s = s0 + lane;
-      if (s < nsplit) mx = fmaxf(mx, __ldcg(p.part_lse + (size_t)(u0 + s) * BM + r));
+      if (s < nsplit) mx = fmaxf(mx, __ldcg(p.part_lse + (size_t)(u0 + s) * BM + r).x);
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
@@ -822,7 +867,10 @@ __global__ void __launch_bounds__(kCombineWarps * 32, 3)
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int s0 = 0; s0 < nsplit; s0 += 32) {
       const int s = s0 + lane;
-      const float wl = s < nsplit ? exp2f(__ldcg(p.part_lse + (size_t)(u0 + s) * BM + r) - mx) : 0.f;
+      const float2 ls = s < nsplit ? __ldcg(p.part_lse + (size_t)(u0 + s) * BM + r)
+                                   : make_float2(-INFINITY, 0.f);
+      const float wl = s < nsplit ? exp2f(ls.x - mx) : 0.f;
+      const float wo = wl * ls.y;  // the weight of the scaled fp16 row
       float ws = wl;
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) ws += __shfl_xor_sync(0xffffffffu, ws, off);
@@ -831,19 +879,21 @@ __global__ void __launch_bounds__(kCombineWarps * 32, 3)
       // eight splits' rows in flight at a time (L2 latency, not bandwidth,
       // is what a one-row-at-a-time loop waits on)
       for (int j0 = 0; j0 < n; j0 += 8) {
-        float4 ov[8];
+        uint2 ov[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u)
-          ov[u] = j0 + u < n ? __ldcg(reinterpret_cast<const float4*>(
-                                   p.part_o + ((size_t)(u0 + s0 + j0 + u) * BM + r) * HD) + lane)
-                             : make_float4(0.f, 0.f, 0.f, 0.f);
+          ov[u] = j0 + u < n ? __ldcg(reinterpret_cast<const uint2*>(
+                                   p.part_o + ((size_t)(u0 + s0 + j0 + u) * BM + r) * (HD / 2)) +
+                               lane)
+                             : make_uint2(0u, 0u);
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-          const float w = __shfl_sync(0xffffffffu, wl, j0 + u);  // 0 past nsplit
-          acc.x = fmaf(w, ov[u].x, acc.x);
-          acc.y = fmaf(w, ov[u].y, acc.y);
-          acc.z = fmaf(w, ov[u].z, acc.z);
-          acc.w = fmaf(w, ov[u].w, acc.w);
+          const float w = __shfl_sync(0xffffffffu, wo, j0 + u);  // 0 past nsplit
+          const float2 a = unpack_f16x2(ov[u].x), c = unpack_f16x2(ov[u].y);
+          acc.x = fmaf(w, a.x, acc.x);
+          acc.y = fmaf(w, a.y, acc.y);
+          acc.z = fmaf(w, c.x, acc.z);
+          acc.w = fmaf(w, c.y, acc.w);
         }
       }
     }
@@ -904,6 +954,11 @@ struct Plan {
   int T, chunk, units, slots, groups, max_ns;
   RowPlan rp;
 };
+
+// The attention kernel's parameters (five tensor maps, TcParams, RowPlan)
+// stay within the classic 4 KB kernel-parameter space.
+static_assert(5 * sizeof(CUtensorMap) + sizeof(TcParams) + sizeof(RowPlan) <= 4096,
+              "kernel parameters");
 
 // Cost model of one CTA (measured on B200 with per-CTA %globaltimer traces):
 // about 8.5 us of fixed work -- set-up, the first S tile, the wait for the
@@ -1031,6 +1086,8 @@ Plan plan_uncached(const AttnArgs& a) {
   pl.max_ns = 1;
   for (int b = 0; b < a.B; ++b) {
     rp.ns[b] = best_ns[b];
+    rp.p0[b] = a.cu_prefix_host[b];
+    rp.len[b] = a.cu_prefix_host[b + 1] - a.cu_prefix_host[b];
     rp.sbase[b] = slots;
     slots += a.Hkv * pl.T * best_ns[b];
     pl.max_ns = std::max(pl.max_ns, best_ns[b]);
@@ -1096,7 +1153,7 @@ size_t counter_bytes(const AttnArgs& a, const Plan& pl) {
 
 size_t attn_tc_scratch_bytes(const AttnArgs& a) {
   const Plan pl = make_plan(a);
-  return counter_bytes(a, pl) + (size_t)pl.slots * BM * (HD + 1) * sizeof(float) + 256;
+  return counter_bytes(a, pl) + (size_t)pl.slots * BM * (HD * 2 + sizeof(float2)) + 256;
 }
 
 template <bool kF8>
@@ -1148,8 +1205,8 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t stream) {
   tp.done = reinterpret_cast<uint32_t*>(scratch);
   tp.seen = tp.done + ncnt;
   scratch += counter_bytes(a, pl);
-  tp.part_o = reinterpret_cast<float*>(scratch);
-  tp.part_lse = reinterpret_cast<float*>(scratch + (size_t)pl.slots * BM * HD * sizeof(float));
+  tp.part_o = reinterpret_cast<uint32_t*>(scratch);
+  tp.part_lse = reinterpret_cast<float2*>(scratch + (size_t)pl.slots * BM * HD * 2);
   tp.err = a.err;
   tp.wait_ns = pipeline_wait_ns();
   tp.stall = pipeline_test_stall() ? 1 : 0;

@@ -79,6 +79,20 @@ def test_tensor_core_split_counts(C, Hq, Hkv, lens):
     np.testing.assert_allclose(lse.cpu().numpy(), ref_lse, atol=2e-2)
 
 
+@pytest.mark.parametrize("v_gain", [1e5, 1e-6])
+def test_tensor_core_value_range(v_gain):
+    # split partials are stored as fp16 scaled per row by a power of two: V
+    # far above fp16's range (65504) and far below its normal range must
+    # come through with the relative accuracy of unit-scale V
+    q, kc, vc, kp, vp, cu = _problem(2, 256, 16, 8, 128, (300, 1000), seed=11)
+    vc = (vc.float() * v_gain).to(torch.bfloat16)
+    vp = (vp.float() * v_gain).to(torch.bfloat16)
+    out, lse = _run(q, kc, vc, kp, vp, cu)
+    ref, ref_lse = oracle.canvas_attn(q, kc, vc, kp, vp, cu.numpy(), 128 ** -0.5)
+    check_attn(out, ref, torch.bfloat16, max_abs=2e-2 * v_gain)
+    np.testing.assert_allclose(lse.cpu().numpy(), ref_lse, atol=2e-2)
+
+
 def test_tensor_core_wide_batch():
     # more batch rows than the host's per-row plan holds: the kernels then
     # derive one split length for every row themselves
