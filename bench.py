@@ -302,6 +302,12 @@ def run_ours(args, w, dist, rank, world, local_rank):
                           "frac_of_nominal": attn_tf / NOMINAL_BF16_TFLOPS,
                           "flops": w.attn_flops(), "ms": t_attn * 1e3,
                           "ms_warm": warm["attn"] * 1e3,
+                          # the step time less the sampler's: the event records
+                          # between the two calls in `ms` stop the attention
+                          # launch from overlapping the previous kernel's tail
+                          "ms_marginal": (ms_per_step / 1e3 - t_samp) * 1e3,
+                          "frac_marginal": (w.attn_flops() / (ms_per_step / 1e3 - t_samp) / 1e12
+                                            / tf_burst) if ms_per_step / 1e3 > t_samp else None,
                           "traffic": traffic.get(f"attention@{w.name}"), "peak_source": src},
         "e2e": e2e,
         "gpu_launches": int(launches),

@@ -722,7 +722,7 @@ __device__ __forceinline__ void combine_store(const TcParams& p, TOut* __restric
     lse_out[((size_t)b * p.Hq + h) * p.C + i] = (mx + __log2f(wsum)) * 0.6931471805599453f;
 }
 
-template <typename TOut, int kMaxS>
+template <typename TOut, int kMaxS, int kRows>
 __global__ void __launch_bounds__(kCombineWarps * 32, 3)
     attn_combine_kernel(const TcParams p, const __grid_constant__ RowPlan rp, int total_units,
                         TOut* __restrict__ out, float* __restrict__ lse_out) {
@@ -732,7 +732,7 @@ __global__ void __launch_bounds__(kCombineWarps * 32, 3)
   if (!p.poll) pdl_wait();
   pdl_trigger();
   // kRows rows per warp, all of their split rows requested at once
-  constexpr int kRows = 16 / kMaxS;
+  static_assert(kMaxS * kRows <= 24 && BM % (kCombineWarps * kRows) == 0, "merge shape");
   constexpr int kBlocksPerTile = BM / (kCombineWarps * kRows);
   int q = blockIdx.x / kBlocksPerTile;  // (b, g, t) group
   const int groups = p.Hkv * p.T;
@@ -1219,20 +1219,22 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t stream) {
                       Lay<false>::kSmemBytes, stream, mQ, mKp, mVp, mKc, mVc, tp, pl.rp);
   note_launch();
   if (e != cudaSuccess) return e;
-  // kMaxS splits per row in flight, 16 / kMaxS rows per warp
+  // kMaxS splits of kRows rows per warp in flight (kMaxS * kRows <= 24
+  // 8-byte loads per lane), so that the merge grid is about one wave
   __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out);
   const dim3 cblock(kCombineWarps * 32);
-  auto cgrid = [&](int max_s) {
-    return dim3(pl.groups * (BM / (kCombineWarps * (16 / max_s))));
-  };
+  auto cgrid = [&](int rows) { return dim3(pl.groups * (BM / (kCombineWarps * rows))); };
   if (pl.max_ns <= 4)
-    e = launch_pdl(attn_combine_kernel<__nv_bfloat16, 4>, cgrid(4), cblock, 0, stream, tp, pl.rp,
-                   (int)pl.slots, out, a.lse);
+    e = launch_pdl(attn_combine_kernel<__nv_bfloat16, 4, 4>, cgrid(4), cblock, 0, stream, tp,
+                   pl.rp, (int)pl.slots, out, a.lse);
   else if (pl.max_ns <= 8)
-    e = launch_pdl(attn_combine_kernel<__nv_bfloat16, 8>, cgrid(8), cblock, 0, stream, tp, pl.rp,
-                   (int)pl.slots, out, a.lse);
+    e = launch_pdl(attn_combine_kernel<__nv_bfloat16, 8, 2>, cgrid(2), cblock, 0, stream, tp,
+                   pl.rp, (int)pl.slots, out, a.lse);
+  else if (pl.max_ns <= 12)
+    e = launch_pdl(attn_combine_kernel<__nv_bfloat16, 12, 2>, cgrid(2), cblock, 0, stream, tp,
+                   pl.rp, (int)pl.slots, out, a.lse);
   else
-    e = launch_pdl(attn_combine_kernel<__nv_bfloat16, 16>, cgrid(16), cblock, 0, stream, tp,
+    e = launch_pdl(attn_combine_kernel<__nv_bfloat16, 16, 1>, cgrid(1), cblock, 0, stream, tp,
                    pl.rp, (int)pl.slots, out, a.lse);
   note_launch();
   return e;

@@ -68,7 +68,9 @@ def test_tensor_core_ragged(lens, q_gain):
 
 
 @pytest.mark.parametrize("C,Hq,Hkv,lens", [
-    (256, 16, 8, (1536,)),     # 7 splits: merge with 8 split rows in flight per row
+    (256, 16, 8, (1536,)),     # 7 splits: the merge shape for up to 8 splits
+    (256, 16, 8, (4096,)),     # 9 splits: up to 12
+    (256, 8, 4, (1408,)),      # 13 splits: up to 16
     (128, 2, 1, (16384,)),     # one unit per split, about 129 splits: the looped merge
 ])
 def test_tensor_core_split_counts(C, Hq, Hkv, lens):
