@@ -33,11 +33,15 @@
  *     first use.  The sampler keeps a small state in it (a work counter and
  *     per-row maxima) and per-chunk records, all of which every completed
  *     call leaves cleared, so sampler calls of any shape may share a
- *     workspace.  A dd_denoise_block or dd_denoise_block_adaptive workspace
- *     also holds attention scratch that calls do not clear: it serves one
- *     geometry (batch, canvas, heads, prefix lengths, vocabulary); clear it
- *     with dd_workspace_init before using it for another.  After a call
- *     that failed on the device, clear the workspace again.
+ *     workspace.  The attention path keeps a pair of counters per (batch
+ *     row, kv head, query-tile pair) at the start of its scratch (split
+ *     partials done, merge CTAs that have seen them), which every completed
+ *     call also leaves cleared; its split partials are not cleared and are
+ *     laid out for one geometry.  So a dd_denoise_block or
+ *     dd_denoise_block_adaptive workspace serves one geometry (batch,
+ *     canvas, heads, prefix lengths, vocabulary); clear it with
+ *     dd_workspace_init before using it for another.  After a call that
+ *     failed on the device, clear the workspace again.
  *   - There is no CPU fallback: if the CUDA kernels cannot run, calls fail.
  */
 #ifndef DD_H_
@@ -109,8 +113,12 @@ DD_API size_t dd_canvas_attn_workspace(const dd_attn_desc* desc, const int32_t* 
  *   v_prefix     same
  *   cu_prefix    device int32 [B+1], cu_prefix[0] = 0, non-decreasing;
  *                L_b = cu_prefix[b+1] - cu_prefix[b] may be 0
- *   cu_prefix_host  host copy of the same values (used to plan the launch;
- *                the two must agree, which is not checked on the device)
+ *   cu_prefix_host  host copy of the same values.  It plans the launch and,
+ *                for batches of up to 128 rows, carries each row's prefix
+ *                offset into the kernels, which then address the prefix
+ *                with it; wider batches read cu_prefix on the device.  The
+ *                two must agree, which is not checked (reads stay inside
+ *                the prefix tensor, whose extent is cu_prefix_host[B])
  *   out          [B, C, Hq, D], element type = desc->dtype
  *   lse          optional fp32 [B, Hq, C]: natural-log sum of exp of scores
  *   workspace    >= dd_canvas_attn_workspace(...) bytes, 256-byte aligned
