@@ -962,10 +962,13 @@ static_assert(5 * sizeof(CUtensorMap) + sizeof(TcParams) + sizeof(RowPlan) <= 40
 
 // Cost model of one CTA (measured on B200 with per-CTA %globaltimer traces):
 // about 8.5 us of fixed work -- set-up, the first S tile, the wait for the
-// last P.V and the write of 128 KB of partials -- and 1.84 us per 128-key
-// tile, so the fixed part weighs as much as kUnitFixed tiles.  The merge
-// pass reads each 64 KB partial slot once (about 13 ns per slot for the GPU
-// at ~5 TB/s, kSlotMerge tiles).
+// last P.V and the write of its split partials (128 KB per CTA when they
+// were fp32; the fp16 partials take about 1.5 us off, which changes none of
+// the plans of the workloads measured here) -- and 1.84 us per 128-key tile,
+// so the fixed part weighs as much as kUnitFixed tiles.  The merge pass
+// reads each partial slot once: kSlotMerge tiles per slot for the GPU (set
+// for a 64 KB fp32 slot at ~5 TB/s; the fp16 slots are half that, which
+// again changes none of those plans).
 constexpr double kUnitFixed = 4.6;
 constexpr double kSlotMerge = 0.0071;
 

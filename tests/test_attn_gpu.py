@@ -161,6 +161,43 @@ def test_full_workloads_sampled(name):
     print(name, st)
 
 
+def test_multi_round_merge_repeats_and_replays():
+    # The ragged batch takes more than one round of the SMs (240 CTAs), so
+    # its split merge polls per-group counters in the workspace that every
+    # call must leave cleared: repeated calls on one workspace, and replays
+    # of one captured call, give the same bits.
+    w = workloads.WORKLOADS["ragged_b8"]
+    q, kc, vc = workloads.canvas_qkv(w, 0, device=DEV)
+    kp, vp, cu = workloads.prefix_kv(w, device=DEV)
+    cud = cu.to(DEV)
+    desc = dd.attn_desc(q, kc, w.scale)
+    ws = dd.new_workspace(dd.canvas_attn_workspace_bytes(desc, cu.numpy()))
+    out = torch.empty_like(q)
+
+    def call():
+        dd.canvas_attn(q, kc, vc, kp, vp, cud, cu, scale=w.scale, out=out, workspace=ws)
+
+    outs = []
+    for _ in range(3):
+        call()
+        outs.append(out.clone())
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(graph, stream=side):
+            call()
+    torch.cuda.current_stream().wait_stream(side)
+    for _ in range(2):
+        out.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+        outs.append(out.clone())
+    dd.query_device_error(ws)
+    for o in outs[1:]:
+        assert torch.equal(o, outs[0])
+
+
 def test_no_device_error_latched():
     q, kc, vc, kp, vp, cu = _problem(1, 256, 16, 8, 128, (1000,), seed=4)
     desc = dd.attn_desc(q, kc)
