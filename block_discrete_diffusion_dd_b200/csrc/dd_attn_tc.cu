@@ -693,11 +693,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // Merge the splits of every (b, g, t) query tile: lse = log2 sum 2^lse_s,
-// O = sum_s 2^(lse_s - lse) O_s.  One warp per query row (8 rows per CTA,
-// 16 CTAs per 128-row tile); lane s holds split s's weight.  kMaxS bounds
-// the splits whose rows are all requested at once (registers: kMaxS float4
-// per lane, so a small bound keeps more CTAs resident); more splits take a
-// looped path.
+// O = sum_s 2^(lse_s - lse) 2^e_s O_s, O_s the split's scaled fp16 row.
+// Each warp takes kRows query rows (kCombineWarps warps per CTA); lane s
+// holds split s's weight, and lane l the row's columns 4 l .. 4 l + 3.
+// kMaxS bounds the splits whose rows are all requested at once (kRows x
+// kMaxS 8-byte loads per lane, at most 24, so that the grid is about one
+// wave); more splits take a looped path.
 constexpr int kCombineWarps = 8;  // warps per CTA of the combine kernel
 
 // Final row of the combine: O = acc / wsum (4 columns per lane) and the
